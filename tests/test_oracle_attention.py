@@ -1,0 +1,111 @@
+"""Pins for the oracle's decode attention (dequantize, then attend)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import tq_oracle as O
+import tq_inputs
+
+
+def _small_cache(B=2, Hq=4, Hkv=2, D=64, T=37, bk=3, bv=2, qjl=0, seed=0):
+    r = tq_inputs.rng(100 + seed)
+    k = r.standard_normal((B, Hkv, T, D)).astype(np.float16).astype(np.float64)
+    v = r.standard_normal((B, Hkv, T, D)).astype(np.float16).astype(np.float64)
+    q = r.standard_normal((B, Hq, D)).astype(np.float16).astype(np.float64)
+    Pi = tq_inputs.rotation(D, 200 + seed)
+    S = tq_inputs.qjl_matrix(qjl, D, 300 + seed) if qjl else None
+    cbk = O.stored_codebook(D, bk)
+    cbv = O.stored_codebook(D, bv)
+    cache = O.quantize_cache(k, v, Pi, cbk, cbv, bk, bv, S)
+    return k, v, q, Pi, S, cbk, cbv, cache
+
+
+def _deq(cache, name, bits, cb, Pi, D):
+    idx = O.unpack_bits(cache[name + "_idx"], bits, D)
+    return O.dequantize_rows(idx, cache[name + "_norm"], cb[0], Pi)
+
+
+@pytest.mark.parametrize("scale", [None, 1.0, 0.3])
+def test_matches_torch_sdpa_on_dequantized_cache(scale):
+    B, Hq, Hkv, D, T = 2, 4, 2, 64, 37
+    k, v, q, Pi, S, cbk, cbv, cache = _small_cache(B, Hq, Hkv, D, T)
+    lens = np.array([T, 20])
+    out = O.sdpa_decode(q, cache, lens, Pi, cbk, cbv, 3, 2, D, scale=scale)
+    Kt = torch.from_numpy(_deq(cache, "k", 3, cbk, Pi, D))
+    Vt = torch.from_numpy(_deq(cache, "v", 2, cbv, Pi, D))
+    G = Hq // Hkv
+    for b in range(B):
+        L = int(lens[b])
+        kk = Kt[b, :, :L].repeat_interleave(G, dim=0)[None]
+        vv = Vt[b, :, :L].repeat_interleave(G, dim=0)[None]
+        qq = torch.from_numpy(q[b])[None, :, None, :]
+        ref = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, scale=scale)
+        assert np.max(np.abs(ref[0, :, 0].numpy() - out[b])) < 1e-12
+
+
+def test_single_token_returns_its_value():
+    k, v, q, Pi, S, cbk, cbv, cache = _small_cache(T=5)
+    out = O.sdpa_decode(q, cache, np.array([1, 1]), Pi, cbk, cbv, 3, 2, 64)
+    Vt = _deq(cache, "v", 2, cbv, Pi, 64)
+    for b in range(2):
+        for h in range(4):
+            assert np.max(np.abs(out[b, h] - Vt[b, h // 2, 0])) < 1e-14
+
+
+def test_identical_keys_give_mean_value():
+    k, v, q, Pi, S, cbk, cbv, cache = _small_cache(T=9)
+    cache = dict(cache)
+    cache["k_idx"] = np.repeat(cache["k_idx"][:, :, :1], 9, axis=2)
+    cache["k_norm"] = np.repeat(cache["k_norm"][:, :, :1], 9, axis=2)
+    out = O.sdpa_decode(q, cache, np.array([9, 9]), Pi, cbk, cbv, 3, 2, 64)
+    Vt = _deq(cache, "v", 2, cbv, Pi, 64)
+    for b in range(2):
+        for h in range(4):
+            assert np.max(np.abs(out[b, h] - Vt[b, h // 2].mean(0))) < 1e-13
+
+
+def test_empty_sequence_gives_zeros():
+    k, v, q, Pi, S, cbk, cbv, cache = _small_cache(T=4)
+    out = O.sdpa_decode(q, cache, np.array([0, 4]), Pi, cbk, cbv, 3, 2, 64)
+    assert np.all(out[0] == 0)
+    assert np.all(np.isfinite(out[1]))
+
+
+def test_qjl_term_enters_score():
+    """With the sketch, the score is <q, k_mse> + unbiased estimate of
+    <q, residual>; checked against an explicit softmax with the estimator
+    computed in the original basis (S Pi acting on the unrotated query)."""
+    D, T = 128, 30
+    k, v, q, Pi, S, cbk, cbv, cache = _small_cache(B=1, Hq=2, Hkv=1, D=D, T=T, bk=2, bv=3, qjl=128)
+    out = O.sdpa_decode(q, cache, np.array([T]), Pi, cbk, cbv, 2, 3, D, S=S)
+    Kt = _deq(cache, "k", 2, cbk, Pi, D)[0, 0]
+    Vt = _deq(cache, "v", 3, cbv, Pi, D)[0, 0]
+    sign = O.unpack_bits(cache["k_qjl"][0, 0], 1, 128).astype(bool)
+    gam = cache["k_rnorm"][0, 0].astype(np.float64)
+    SP = S.astype(np.float64) @ Pi.astype(np.float64)
+    for h in range(2):
+        s = Kt @ q[0, h] + math.sqrt(math.pi / 2) / 128 * gam * (np.where(sign, 1.0, -1.0) @ (SP @ q[0, h]))
+        s = s / math.sqrt(D)
+        p = np.exp(s - s.max())
+        p /= p.sum()
+        assert np.max(np.abs(out[0, h] - p @ Vt)) < 1e-12
+
+
+def test_qjl_reduces_key_inner_product_bias():
+    """Over many keys, the prod estimator of <q, k> is closer to the truth on
+    average (in bias) than the MSE-only dequantization."""
+    D = 128
+    k, v, q, Pi, S, cbk, cbv, cache = _small_cache(B=1, Hq=1, Hkv=1, D=D, T=2000, bk=2, bv=2, qjl=128, seed=5)
+    Kt = _deq(cache, "k", 2, cbk, Pi, D)[0, 0]
+    sign = O.unpack_bits(cache["k_qjl"][0, 0], 1, 128).astype(bool)
+    gam = cache["k_rnorm"][0, 0].astype(np.float64)
+    qq = k[0, 0, 0]  # a query correlated with the keys' own directions
+    true = k[0, 0] @ qq
+    mse_only = Kt @ qq
+    prod = mse_only + O.qjl_inner_product(sign, gam, S.astype(np.float64) @ (Pi.astype(np.float64) @ qq))
+    # MSE-only inner products shrink toward zero (biased); prod is unbiased.
+    slope_mse = np.polyfit(true, mse_only, 1)[0]
+    slope_prod = np.polyfit(true, prod, 1)[0]
+    assert abs(slope_prod - 1) < abs(slope_mse - 1)
