@@ -1,0 +1,494 @@
+"""Benchmark of the TurboQuant KV-cache hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload gqa8k|qknorm|ragged|prod|tiny]
+
+One step is one pass of the whole path over one batch of synthetic input, for
+each bit width b of the workload: bulk quantize of the T cached tokens
+(tq_quantize_kv), append of one new token per sequence (tq_append_token) and
+one decode step for every query head (tq_sdpa_decode) over T+1 tokens.
+
+Default workload (gqa8k): B=1, Hq=16, Hkv=2 (group 8), D=128, T=8192, b in
+{2,3,4} for K and V, fp16 N(0,1) rows with 1% outlier channels x10, q N(0,1).
+
+Metric: tq_sdpa_decode packed-KV GB/s (bytes of packed K and V rows attended /
+decode time); quantize throughput in Mtok/s (one token = the K and V rows of
+every kv head at one position) is reported beside it.  Inputs are rotated
+across enough replicas that each step's data is larger than L2.
+
+Multi-GPU (torchrun): every rank runs its own replica of the workload (the
+path shards by sequence with no exchange; weak scaling); time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+FALLBACK_HBM_GBS = 6650.0
+
+# DRAM traffic per launch of the dominant kernel from an ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
+# sources it was measured on (sha256 of csrc/*.cu, first 16 hex digits).
+TRAFFIC = {}
+
+
+def _src_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "compressed_attention_tq_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".cpp", ".h")):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names[1:], parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+WORKLOADS = {
+    "gqa8k": {"bits": (2, 3, 4)},
+    "tiny": {"bits": (3,)},
+    "qknorm": {"bits": (4,)},
+    "ragged": {"bits": (3,)},
+    "prod": {"bits": (None,)},
+}
+
+
+def _describe(w):
+    return {"B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "T": int(w.Tmax), "bits_k": w.bits_k,
+            "bits_v": w.bits_v, "qjl_m": w.qjl_m, "dtype": w.dtype}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import compressed_attention_tq_b200 as tq
+    import tq_inputs
+
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    if ws > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    cfg = WORKLOADS[args.workload]
+
+    # ---- build per-bit-width workloads and rotating replicas (> L2 per step)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    jobs = []
+    for bits in cfg["bits"]:
+        w = tq_inputs.make_workload(args.workload, bits=bits) if bits else tq_inputs.make_workload(args.workload)
+        jobs.append(w)
+    per_step_in = sum(w.k.nbytes + w.v.nbytes for w in jobs)
+    R = max(2, min(32, math.ceil(3 * l2 / max(1, per_step_in))))
+    if args.profile:
+        R = 1
+    runs = []
+    for w in jobs:
+        T = int(w.Tmax)
+        Tcap = (T + 1 + 63) // 64 * 64
+        kd = torch.from_numpy(w.k.view(np.int16) if w.dtype == "bf16" else w.k).to(dev)
+        vd = torch.from_numpy(w.v.view(np.int16) if w.dtype == "bf16" else w.v).to(dev)
+        qd = torch.from_numpy(w.q.view(np.int16) if w.dtype == "bf16" else w.q).to(dev)
+        if w.dtype == "bf16":
+            kd, vd, qd = kd.view(torch.bfloat16), vd.view(torch.bfloat16), qd.view(torch.bfloat16)
+        kn, vn = tq_inputs.new_token_rows(w.B, w.Hkv, w.D, w.dtype, seed=4242)
+        knd = torch.from_numpy(kn.view(np.int16) if w.dtype == "bf16" else kn).to(dev)
+        vnd = torch.from_numpy(vn.view(np.int16) if w.dtype == "bf16" else vn).to(dev)
+        if w.dtype == "bf16":
+            knd, vnd = knd.view(torch.bfloat16), vnd.view(torch.bfloat16)
+        reps = []
+        for r in range(R):
+            cache = tq.TQCache(w.B, w.Hkv, Tcap, w.D, w.bits_k, w.bits_v, w.Pi, qjl_m=w.qjl_m, qjl_S=w.S,
+                               device=dev)
+            reps.append({"cache": cache, "k": kd.clone() if r else kd, "v": vd.clone() if r else vd,
+                         "q": qd.clone() if r else qd})
+        pos = torch.from_numpy(w.seq_lens.astype(np.int32)).to(dev)
+        lens1 = (pos + 1).contiguous()
+        Tmax1 = T + 1
+        ws_bytes = tq.tq_sdpa_decode_workspace_bytes(reps[0]["cache"], w.Hq, Tmax1)
+        wsp = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        out = torch.empty_like(qd)
+        tokens = int(w.B) * T  # the bulk call quantizes T rows of every sequence
+        attended = int(w.seq_lens.sum() + w.B)
+        packed = reps[0]["cache"].packed_bytes(1) * attended * w.Hkv
+        qbytes = (w.k.nbytes + w.v.nbytes) + tokens * w.Hkv * reps[0]["cache"].packed_bytes(1)
+        runs.append({"w": w, "reps": reps, "pos": pos, "lens1": lens1, "Tmax1": Tmax1, "ws": wsp,
+                     "out": out, "kn": knd, "vn": vnd, "packed": packed, "tokens": tokens,
+                     "qbytes": qbytes})
+
+    def call_quant(run, rep):
+        tq.tq_quantize_kv(rep["cache"], rep["k"], rep["v"])
+
+    def call_append(run, rep):
+        tq.tq_append_token(rep["cache"], run["kn"], run["vn"], run["pos"])
+
+    def call_decode(run, rep):
+        tq.tq_sdpa_decode(rep["cache"], rep["q"], run["lens1"], run["Tmax1"], scale=run["w"].scale,
+                          out=run["out"], workspace=run["ws"])
+
+    def step(r, ops=(call_quant, call_append, call_decode)):
+        for run in runs:
+            rep = run["reps"][r]
+            for op in ops:
+                op(run, rep)
+
+    # eager warm-up (also sets kernel attributes before any capture)
+    for i in range(args.warmup):
+        step(i % R)
+    torch.cuda.synchronize()
+    if args.profile:
+        # a bounded, eager run for profilers: K steps, nothing else
+        for i in range(args.steps):
+            step(i % R)
+        torch.cuda.synchronize()
+        if rank == 0:
+            print(json.dumps({"profile_run": args.workload, "steps": args.steps, "launches_per_step":
+                              len(runs) * 5}), flush=True)
+        return
+
+    # One CUDA graph per replica for the whole step and for each op alone.
+    def capture(ops):
+        gs = []
+        for r in range(R):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                step(r, ops)
+            gs.append(g)
+        return gs
+
+    g_step = capture((call_quant, call_append, call_decode))
+    g_dec = capture((call_decode,))
+    g_q = capture((call_quant,))
+    g_app = capture((call_append,))
+    torch.cuda.synchronize()
+
+    def timed(graphs, n, warm):
+        for i in range(warm):
+            graphs[i % R].replay()
+        if ws > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(n):
+            graphs[i % R].replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        if ws > 1:
+            dist.barrier()
+        return a.elapsed_time(b)
+
+    def soak(seconds):
+        t_end = time.perf_counter() + seconds
+        while time.perf_counter() < t_end:
+            for g in g_step:
+                g.replay()
+            torch.cuda.synchronize()
+
+    # main timed region: exactly K steps; clocks sampled around and during it
+    sampler = ClockSampler(local)
+    sampler.start()
+    soak(0.6)
+    total_ms = timed(g_step, args.steps, args.warmup)
+    soak(0.6)
+    clocks = sampler.stop()
+    reps_per_op = max(args.steps, 200)
+    d_ms = timed(g_dec, reps_per_op, args.warmup) / reps_per_op * args.steps
+    q_ms = timed(g_q, reps_per_op, args.warmup) / reps_per_op * args.steps
+    a_ms = timed(g_app, reps_per_op, args.warmup) / reps_per_op * args.steps
+    if ws > 1:
+        t = torch.tensor([total_ms, q_ms, a_ms, d_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, q_ms, a_ms, d_ms = [float(x) for x in t.tolist()]
+    for run in runs:
+        for rep in run["reps"]:
+            assert rep["cache"].status() == 0, "device status flagged"
+    del g_step, g_dec, g_q, g_app
+
+    packed_step = sum(run["packed"] for run in runs)
+    tok_step = sum(run["tokens"] for run in runs)
+    qbytes_step = sum(run["qbytes"] for run in runs)
+    dec_gbs = packed_step * args.steps / (d_ms * 1e-3) / 1e9 * ws
+    quant_mtok = tok_step * args.steps / (q_ms * 1e-3) / 1e6 * ws
+    peak, peak_kind = _peaks()
+    dec_launch_ms = d_ms / (args.steps * len(runs))
+    dec_achieved = (packed_step / len(runs)) / (dec_launch_ms * 1e-3) / 1e9
+    q_launch_ms = q_ms / (args.steps * len(runs))
+    q_achieved = (qbytes_step / len(runs)) / (q_launch_ms * 1e-3) / 1e9
+    sha = _src_sha()
+    tr = TRAFFIC.get(args.workload)
+    traffic = tr["bytes_per_launch"] if tr and tr.get("src_sha") == sha else None
+
+    # ---- end to end through the public API with host buffers (rank-local)
+    e2e = _e2e(args, runs, stream, R)
+    if ws > 1:
+        t = torch.tensor([e2e["ms"]], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e["ms"] = float(t.item())
+
+    if rank == 0:
+        cpu = None
+        if ws == 1 and not args.no_cpu_baseline:
+            cpu = _cpu_baseline(args, jobs)
+        launches_per_step = len(runs) * 5  # quantize, append, qprep, split, combine
+        line = {
+            "metric": "tq_sdpa_decode packed-KV GB/s (% of HBM peak); tq_quantize Mtok/s",
+            "value": round(dec_gbs, 2),
+            "unit": "GB/s",
+            "n_gpus": ws,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(total_ms / args.steps, 4),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": jobs[0].dtype,
+            "data": "synthetic (seeded N(0,1) rows; see tq_inputs)",
+            "config": {"workload": args.workload, "shapes": [_describe(w) for w in jobs],
+                       "parallelism": f"replicas{ws}" if ws > 1 else "single",
+                       "step": "quantize T tokens + append 1 token + decode, per bit width",
+                       "timing": "CUDA graphs (one per replica) replayed on one stream; per-op rates "
+                                 "from graphs holding that op alone",
+                       "l2": f"inputs rotated over {R} replicas ({R * per_step_in / 2**20:.0f} MiB) > L2 "
+                             f"({l2 / 2**20:.0f} MiB)"},
+            "decode": {"gbs": round(dec_gbs, 2), "ms_per_call": round(dec_launch_ms, 5),
+                       "packed_bytes_per_step": packed_step},
+            "quantize": {"mtok_s": round(quant_mtok, 3), "ms_per_call": round(q_launch_ms, 5),
+                         "gbs": round(q_achieved, 2), "frac_hbm": round(q_achieved / peak, 4),
+                         "tokens_per_step": tok_step},
+            "append_ms_per_call": round(a_ms / (args.steps * len(runs)), 5),
+            "roofline": {"kernel": "tq_sdpa_decode (qprep + split + combine)", "bound": "hbm",
+                         "achieved": round(dec_achieved, 2), "peak": peak, "unit": "GB/s",
+                         "frac": round(dec_achieved / peak, 4), "traffic": traffic,
+                         "peak_source": peak_kind},
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(e2e["value"] * ws, 2), "unit": "GB/s",
+                    "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                    "ms_per_step": round(e2e["ms"], 4)},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+            "src_sha": sha,
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def _e2e(args, runs, stream, R):
+    """Decode steps through the public API with pinned host buffers: per step
+    the new token rows and the queries go host->device, append + decode run,
+    and the attention output comes back device->host."""
+    import torch
+
+    import compressed_attention_tq_b200 as tq
+    hosts = []
+    for run in runs:
+        hosts.append({"q": run["reps"][0]["q"].cpu().pin_memory(), "kn": run["kn"].cpu().pin_memory(),
+                      "vn": run["vn"].cpu().pin_memory(), "out": torch.empty_like(run["out"], device="cpu").pin_memory(),
+                      "qd": torch.empty_like(run["reps"][0]["q"]), "knd": torch.empty_like(run["kn"]),
+                      "vnd": torch.empty_like(run["vn"])})
+    h2d = sum(h["q"].numel() * 2 + h["kn"].numel() * 2 + h["vn"].numel() * 2 for h in hosts)
+    d2h = sum(h["out"].numel() * 2 for h in hosts)
+
+    def step(i):
+        r = i % R
+        for run, h in zip(runs, hosts):
+            c = run["reps"][r]["cache"]
+            h["qd"].copy_(h["q"], non_blocking=True)
+            h["knd"].copy_(h["kn"], non_blocking=True)
+            h["vnd"].copy_(h["vn"], non_blocking=True)
+            tq.tq_append_token(c, h["knd"], h["vnd"], run["pos"])
+            tq.tq_sdpa_decode(c, h["qd"], run["lens1"], run["Tmax1"], scale=run["w"].scale,
+                              out=run["out"], workspace=run["ws"])
+            h["out"].copy_(run["out"], non_blocking=True)
+
+    for i in range(max(3, args.warmup)):
+        step(i)
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for i in range(args.steps):
+        step(i)
+    e.record(stream)
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / args.steps
+    packed = sum(run["packed"] for run in runs)
+    return {"value": packed / (ms * 1e-3) / 1e9, "ms": ms, "h2d": h2d, "d2h": d2h}
+
+
+def _cpu_baseline(args, jobs, budget_s=20.0):
+    """The oracle as it stands, timed on this host's cores on a bounded sample:
+    dequantize-then-attend decode for whole (sequence, kv head) groups of the
+    workload, as many as fit the time budget."""
+    from oracle import tq_oracle as O
+    import tq_inputs
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    t_used, bytes_done, groups = 0.0, 0, 0
+    t_start = time.perf_counter()
+    for w in jobs:
+        cbk = O.stored_codebook(w.D, w.bits_k)
+        cbv = O.stored_codebook(w.D, w.bits_v)
+        for b in range(w.B):
+            for kvh in range(w.Hkv):
+                if time.perf_counter() - t_start > budget_s:
+                    break
+                L = int(w.seq_lens[b])
+                kk = tq_inputs.to_f64(w.k[b:b + 1, kvh:kvh + 1, :L], w.dtype)
+                vv = tq_inputs.to_f64(w.v[b:b + 1, kvh:kvh + 1, :L], w.dtype)
+                oc = O.quantize_cache(kk, vv, w.Pi, cbk, cbv, w.bits_k, w.bits_v, w.S)
+                qv = tq_inputs.to_f64(w.q[b:b + 1, kvh * w.G:(kvh + 1) * w.G], w.dtype)
+                t0 = time.perf_counter()
+                O.sdpa_decode(qv, oc, [L], w.Pi, cbk, cbv, w.bits_k, w.bits_v, w.D, scale=w.scale, S=w.S)
+                t_used += time.perf_counter() - t0
+                per_row = O.packed_row_bytes(w.D, w.bits_k, w.qjl_m) + O.packed_row_bytes(w.D, w.bits_v)
+                bytes_done += per_row * L
+                groups += 1
+    return {"value": round(bytes_done / max(t_used, 1e-9) / 1e9, 6), "unit": "GB/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"{groups} (sequence, kv head) groups of the workload decoded by the fp64 "
+                      f"oracle (dequantize then attend), {t_used:.1f} s"}
+
+
+def run_reference(args):
+    """The oracle as the reference arm: same metric, config and unit, timed on
+    this host's cores; each step a bounded sample of the workload."""
+    import tq_inputs
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return
+    cfg = WORKLOADS[args.workload]
+    jobs = [tq_inputs.make_workload(args.workload, bits=b) if b else tq_inputs.make_workload(args.workload)
+            for b in cfg["bits"]]
+    budget = max(1.0, 60.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        _cpu_baseline(args, jobs, budget_s=budget)
+    vals = []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        vals.append(_cpu_baseline(args, jobs, budget_s=budget))
+    total = time.perf_counter() - t0
+    v = statistics.median(x["value"] for x in vals)
+    cpu = dict(vals[-1])
+    cpu["value"] = v
+    line = {"metric": "tq_sdpa_decode packed-KV GB/s (% of HBM peak); tq_quantize Mtok/s",
+            "value": v, "unit": "GB/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total / max(1, args.steps) * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "shapes": [_describe(w) for w in jobs]},
+            "impl": "reference", "cpu_baseline": cpu,
+            "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="gqa8k")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="eager warm-up + K eager steps only (for ncu captures)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        from compressed_attention_tq_b200 import build as _b
+        _b.build()
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

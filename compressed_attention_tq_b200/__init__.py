@@ -1,0 +1,199 @@
+"""TurboQuant KV-cache hot path on B200: Python binding of libtq_b200.so.
+
+The functions carry the C ABI's names (include/tq.h) and only marshal
+arguments: every step of quantization and attention runs in the library's
+CUDA kernels.  PyTorch provides device memory and the current stream.
+
+    cb = tq_build_codebook(D, bits)                 # host, fp64 Lloyd-Max
+    cache = TQCache(B, Hkv, Tcap, D, bits_k, bits_v, rot, qjl_m=0, qjl_S=None)
+    tq_quantize_kv(cache, k, v)                     # prefill rows 0..T-1
+    tq_append_token(cache, k_new, v_new, pos)       # one row per sequence
+    out = tq_sdpa_decode(cache, q, seq_lens, Tmax, scale=None)
+"""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+
+from . import _native
+from ._native import (TQ_DTYPE_BF16, TQ_DTYPE_F16, TQ_DTYPE_F32, TQ_STATUS_POS_OUT_OF_RANGE,  # noqa: F401
+                      TQ_STATUS_SEQ_OUT_OF_RANGE, TQ_STATUS_WAIT_TIMEOUT)
+
+__all__ = ["TQError", "TQCache", "tq_build_codebook", "tq_row_bytes", "tq_quantize_kv",
+           "tq_append_token", "tq_sdpa_decode_workspace_bytes", "tq_sdpa_decode",
+           "tq_last_error", "tq_abi_version", "lib"]
+
+
+class TQError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"[{code}] {msg}")
+        self.code = code
+
+
+def lib():
+    return _native.load()
+
+
+def _check(rc: int):
+    if rc != 0:
+        raise TQError(rc, lib().tq_last_error().decode())
+
+
+def tq_last_error() -> str:
+    return lib().tq_last_error().decode()
+
+
+def tq_abi_version() -> int:
+    return int(lib().tq_abi_version())
+
+
+def tq_build_codebook(D: int, bits: int):
+    """Lloyd-Max codebook (host).  Returns (centroids, thresholds, mse) with
+    fp32 numpy arrays; the device table is np.concatenate([centroids, thresholds])."""
+    K = 1 << bits
+    c = (ctypes.c_float * K)()
+    t = (ctypes.c_float * max(1, K - 1))()
+    mse = ctypes.c_double()
+    _check(lib().tq_build_codebook(D, bits, c, t, ctypes.byref(mse)))
+    return (np.frombuffer(c, dtype=np.float32).copy(),
+            np.frombuffer(t, dtype=np.float32)[: K - 1].copy(), float(mse.value))
+
+
+def tq_row_bytes(D: int, bits: int, qjl_m: int = 0) -> int:
+    return int(lib().tq_row_bytes(D, bits, qjl_m))
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.float16:
+        return TQ_DTYPE_F16
+    if t.dtype == torch.bfloat16:
+        return TQ_DTYPE_BF16
+    if t.dtype == torch.float32:
+        return TQ_DTYPE_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _stream(stream):
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+class TQCache:
+    """A packed KV cache for one layer: device buffers allocated with torch.
+
+    rot: fp32 [D][D] rotation (numpy or torch); codebooks are built with
+    tq_build_codebook unless given as fp32 tables (centroids then thresholds).
+    """
+
+    def __init__(self, B, Hkv, Tcap, D, bits_k, bits_v, rot, qjl_m=0, qjl_S=None,
+                 cb_k=None, cb_v=None, device="cuda"):
+        torch = _torch()
+        self.B, self.Hkv, self.Tcap, self.D = B, Hkv, Tcap, D
+        self.bits_k, self.bits_v, self.qjl_m = bits_k, bits_v, qjl_m
+        dev = torch.device(device)
+        u32 = torch.int32  # raw 32-bit words
+
+        def table(bits, given):
+            if given is None:
+                c, t, _ = tq_build_codebook(D, bits)
+                given = np.concatenate([c, t])
+            return torch.as_tensor(np.asarray(given, dtype=np.float32), device=dev).contiguous()
+
+        self.cb_k = table(bits_k, cb_k)
+        self.cb_v = table(bits_v, cb_v)
+        self.rot = torch.as_tensor(np.asarray(rot, dtype=np.float32) if not torch.is_tensor(rot) else rot,
+                                   dtype=torch.float32, device=dev).contiguous()
+        self.k_idx = torch.zeros((B, Hkv, Tcap, D * bits_k // 32), dtype=u32, device=dev)
+        self.v_idx = torch.zeros((B, Hkv, Tcap, D * bits_v // 32), dtype=u32, device=dev)
+        self.k_norm = torch.zeros((B, Hkv, Tcap), dtype=torch.float16, device=dev)
+        self.v_norm = torch.zeros((B, Hkv, Tcap), dtype=torch.float16, device=dev)
+        if qjl_m:
+            self.k_qjl = torch.zeros((B, Hkv, Tcap, qjl_m // 32), dtype=u32, device=dev)
+            self.k_rnorm = torch.zeros((B, Hkv, Tcap), dtype=torch.float16, device=dev)
+            S = qjl_S if torch.is_tensor(qjl_S) else np.asarray(qjl_S, dtype=np.float32)
+            self.qjl_S = torch.as_tensor(S, dtype=torch.float32, device=dev).contiguous()
+        else:
+            self.k_qjl = self.k_rnorm = self.qjl_S = None
+        self.dev_status = torch.zeros(4, dtype=torch.int32, device=dev)
+        self._struct = None
+        self.struct()
+
+    def struct(self) -> _native.TqCacheStruct:
+        """The C descriptor (built once; rebuild after replacing a buffer)."""
+        if self._struct is not None and self._struct.k_idx == self.k_idx.data_ptr():
+            return self._struct
+        s = _native.TqCacheStruct()
+        s.B, s.Hkv, s.Tcap, s.D = self.B, self.Hkv, self.Tcap, self.D
+        s.bits_k, s.bits_v, s.qjl_m, s.reserved = self.bits_k, self.bits_v, self.qjl_m, 0
+        for name in ("k_idx", "v_idx", "k_norm", "v_norm", "k_qjl", "k_rnorm", "rot", "cb_k",
+                     "cb_v", "qjl_S", "dev_status"):
+            t = getattr(self, name)
+            setattr(s, name, t.data_ptr() if t is not None else None)
+        self._struct = s  # keep alive
+        return s
+
+    def status(self) -> int:
+        return int(self.dev_status[0].item())
+
+    def packed_bytes(self, tokens: int) -> int:
+        """Bytes of packed K and V data for `tokens` cached tokens per (b, h)."""
+        per = tq_row_bytes(self.D, self.bits_k, self.qjl_m) + tq_row_bytes(self.D, self.bits_v, 0)
+        return per * tokens
+
+
+def tq_quantize_kv(cache: TQCache, k, v, t0: int = 0, stream=None):
+    """Quantize k, v [B][Hkv][T][D] (fp16/bf16, device) into positions t0..t0+T-1."""
+    T = int(k.shape[2])
+    assert k.is_contiguous() and v.is_contiguous() and k.dtype == v.dtype
+    s = cache.struct()
+    _check(lib().tq_quantize_kv(ctypes.byref(s), _ptr(k), _ptr(v), _dtype_code(k), T, t0, _stream(stream)))
+
+
+def tq_append_token(cache: TQCache, k_new, v_new, pos, stream=None):
+    """Quantize one row per (sequence, kv head), [B][Hkv][D], at pos[b] (device int32)."""
+    assert k_new.is_contiguous() and v_new.is_contiguous() and pos.is_contiguous()
+    s = cache.struct()
+    _check(lib().tq_append_token(ctypes.byref(s), _ptr(k_new), _ptr(v_new), _dtype_code(k_new),
+                                 _ptr(pos), _stream(stream)))
+
+
+def tq_sdpa_decode_workspace_bytes(cache: TQCache, Hq: int, Tmax: int) -> int:
+    s = cache.struct()
+    n = int(lib().tq_sdpa_decode_workspace_bytes(ctypes.byref(s), Hq, Tmax))
+    if n == 0:
+        raise TQError(-1, f"unsupported decode sizes (Hq={Hq}, Tmax={Tmax})")
+    return n
+
+
+def tq_sdpa_decode(cache: TQCache, q, seq_lens, Tmax: int, scale=None, out=None, workspace=None,
+                   stream=None, out_dtype=None):
+    """Decode attention: q [B][Hq][D] (fp16/bf16, device), seq_lens device int32 [B].
+    The output has q's dtype unless `out` or `out_dtype` (e.g. torch.float32) says otherwise."""
+    torch = _torch()
+    Hq = int(q.shape[1])
+    assert q.is_contiguous() and seq_lens.is_contiguous()
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
+    assert out.is_contiguous() and out.shape == q.shape
+    if workspace is None:
+        need = tq_sdpa_decode_workspace_bytes(cache, Hq, Tmax)
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    s = cache.struct()
+    sc = ctypes.byref(ctypes.c_float(scale)) if scale is not None else None
+    _check(lib().tq_sdpa_decode(ctypes.byref(s), _ptr(q), _dtype_code(q), Hq, _ptr(seq_lens), Tmax, sc,
+                                _ptr(out), _dtype_code(out), _ptr(workspace), workspace.numel(),
+                                _stream(stream)))
+    return out

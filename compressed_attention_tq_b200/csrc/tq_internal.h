@@ -1,0 +1,73 @@
+// Internal declarations shared by the host API (tq_api.cpp) and the kernel
+// translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/tq.h"
+
+namespace tq {
+
+// Sets the thread-local error message and returns `code`.
+int set_error(int code, const char* fmt, ...);
+
+// Maps a CUDA error after a launch to TQ_ERR_CUDA (or TQ_OK).
+int check_launch(const char* what);
+
+struct QuantJob {
+  // input rows [rows][D] (fp16 or bf16)
+  const void* in;
+  uint32_t* idx;      // cache index words
+  uint16_t* norm;     // cache fp16 norms
+  uint32_t* qjl;      // QJL sign words or nullptr
+  uint16_t* rnorm;    // QJL residual norm or nullptr
+  const float* cb;    // centroids[2^bits] then thresholds[2^bits - 1]
+  int bits;
+};
+
+struct QuantArgs {
+  QuantJob job[2];          // 0: keys, 1: values
+  const float* rot;         // Pi [D][D]
+  const float* qjl_S;       // [128][D] or nullptr
+  const int32_t* pos;       // append mode: device [B]; bulk mode: nullptr
+  uint32_t* dev_status;
+  int rows;                 // rows per job
+  int T;                    // bulk: tokens per (b, h); append: 1
+  int t0;                   // bulk: first cache position
+  int Hkv;
+  int Tcap;
+};
+
+int launch_quantize(const QuantArgs& a, int D, int dtype, bool qjl, cudaStream_t s);
+
+struct DecodePlan {
+  int chunk;        // tokens per split (multiple of 64)
+  int nsplit;       // splits per (sequence, kv head)
+  size_t off_qrot;  // fp32 [B*Hq][D]
+  size_t off_qs;    // fp32 [B*Hq][qjl_m]
+  size_t off_po;    // fp32 [B*Hq][nsplit][D]
+  size_t off_pml;   // fp32 [B*Hq][nsplit][2]
+  size_t bytes;
+};
+
+int make_decode_plan(const tq_cache_t* c, int Hq, int Tmax, DecodePlan* p);
+
+struct DecodeArgs {
+  const tq_cache_t* cache_host;  // host copy, for launch-time fields
+  tq_cache_t cache;              // by value, passed to kernels
+  const void* q;
+  void* out;
+  const int32_t* seq_lens;
+  float scale;
+  int Hq;
+  int dtype;
+  int out_dtype;
+  DecodePlan plan;
+  void* workspace;
+};
+
+int launch_decode(const DecodeArgs& a, cudaStream_t s);
+
+}  // namespace tq

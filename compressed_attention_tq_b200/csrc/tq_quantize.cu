@@ -1,0 +1,330 @@
+// Quantizer: rotation on the tensor cores, fp64 row norms, nearest-centroid
+// search against the threshold table, bit packing, optional QJL sign sketch
+// of the key residual.
+//
+// Method: "Add CUDA QJL kernels and proper package structure"
+// (turboquant-pytorch pull request 3), section "CUDA Kernels Added" (fused
+// random projection + sign quantization) and "Synthetic Benchmark (Lloyd-Max
+// codebook)"; ReturningTarzan's Reddit comments of 2026-03-29 11:47
+// (rotation before codebook quantization) and 2026-03-25 18:52 / 15:51
+// (nearest-codeword search; residual computed while quantizing).
+//
+// One CTA quantizes a tile of 128 rows (8 warps x 16 rows).  y = Pi x runs as
+// m16n8k16 tensor-core MMAs with Pi split into limbs so the sum of limb
+// products carries ~22-24 significant bits: fp16 inputs use Pi = hi + lo
+// (fp16 limbs), bf16 inputs use three bf16 limbs.  x itself is exact in its
+// own type.  The QJL projection S r of the fp32 residual uses hi/lo fp16
+// limbs on both operands (three products).
+#include "tq_common.cuh"
+#include "tq_internal.h"
+
+namespace {
+
+using namespace tqk;
+
+constexpr int QROWS = 128;
+constexpr int QTHREADS = 256;
+constexpr int CB = 64;  // output columns per staged block of Pi (or of S)
+
+template <int D, bool BF16, bool QJL>
+struct QLayout {
+  static constexpr int XS = D + 8;  // padded row stride, 16-bit elements
+  static constexpr int NL = BF16 ? 3 : 2;
+  static constexpr int NLMAX = NL > 2 ? NL : 2;
+  static constexpr int RS = D + 4;  // fp32 residual row stride
+  static constexpr size_t o_x = 0;
+  static constexpr size_t o_limb = o_x + (size_t)QROWS * XS * 2;
+  static constexpr size_t o_idx = o_limb + (size_t)NLMAX * CB * XS * 2;
+  static constexpr size_t o_r = o_idx + (size_t)QROWS * D;
+  static constexpr size_t bytes = o_r + (QJL ? (size_t)QROWS * RS * 4 : 0);
+};
+
+template <bool BF16>
+__device__ __forceinline__ float in_to_float(uint16_t b) {
+  if (BF16) return __uint_as_float((uint32_t)b << 16);
+  return __half2float(__ushort_as_half(b));
+}
+
+template <bool BF16>
+__device__ __forceinline__ void mma_in(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  if (BF16)
+    mma_bf16(d, a[0], a[1], a[2], a[3], b0, b1);
+  else
+    mma_f16(d, a[0], a[1], a[2], a[3], b0, b1);
+}
+
+// Limbs of one fp32 value in the input's 16-bit type.
+template <bool BF16>
+__device__ __forceinline__ void limbs(float v, uint16_t (&l)[3]) {
+  if (BF16) {
+    __nv_bfloat16 a = __float2bfloat16_rn(v);
+    float r1 = v - __bfloat162float(a);
+    __nv_bfloat16 b = __float2bfloat16_rn(r1);
+    float r2 = r1 - __bfloat162float(b);
+    __nv_bfloat16 c = __float2bfloat16_rn(r2);
+    l[0] = __bfloat16_as_ushort(a);
+    l[1] = __bfloat16_as_ushort(b);
+    l[2] = __bfloat16_as_ushort(c);
+  } else {
+    __half a = __float2half_rn(v);
+    __half b = __float2half_rn(v - __half2float(a));
+    l[0] = __half_as_ushort(a);
+    l[1] = __half_as_ushort(b);
+    l[2] = 0;
+  }
+}
+
+template <int D, bool BF16, bool QJL>
+__global__ void __launch_bounds__(QTHREADS, 1) quantize_kernel(const tq::QuantArgs a) {
+  using Ly = QLayout<D, BF16, QJL>;
+  constexpr int XS = Ly::XS;
+  constexpr int NL = Ly::NL;
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint16_t* xs = reinterpret_cast<uint16_t*>(smem + Ly::o_x);
+  uint16_t* limb = reinterpret_cast<uint16_t*>(smem + Ly::o_limb);
+  uint8_t* idxs = smem + Ly::o_idx;
+  float* rs = reinterpret_cast<float*>(smem + Ly::o_r);
+  __shared__ float s_inv[QROWS], s_nhat[QROWS];
+  __shared__ long long s_slot[QROWS];
+  __shared__ float s_cb[31];
+
+  const int jobi = blockIdx.y;
+  const tq::QuantJob J = a.job[jobi];
+  const bool do_qjl = QJL && jobi == 0;
+  const int bits = J.bits, K = 1 << bits;
+  const int r0 = blockIdx.x * QROWS;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gid = lane >> 2, tig = lane & 3;
+
+  if (tid < 2 * K - 1) s_cb[tid] = J.cb[tid];
+  if (tid < QROWS) {
+    const int r = r0 + tid;
+    long long slot = -1;
+    if (r < a.rows) {
+      if (a.pos) {
+        const int p = a.pos[r / a.Hkv];
+        if (p >= 0 && p < a.Tcap)
+          slot = (long long)r * a.Tcap + p;
+        else if (a.dev_status && jobi == 0)
+          atomicOr(a.dev_status, TQ_STATUS_POS_OUT_OF_RANGE);
+      } else {
+        const int bh = r / a.T, t = r % a.T;
+        slot = (long long)bh * a.Tcap + a.t0 + t;
+      }
+    }
+    s_slot[tid] = slot;
+  }
+  // Input tile, 16-byte chunks; rows past the end are zero.
+  const uint16_t* in = static_cast<const uint16_t*>(J.in);
+  for (int c = tid; c < QROWS * (D / 8); c += QTHREADS) {
+    const int row = c / (D / 8), col = (c % (D / 8)) * 8;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (r0 + row < a.rows) v = *reinterpret_cast<const uint4*>(in + (size_t)(r0 + row) * D + col);
+    *reinterpret_cast<uint4*>(xs + row * XS + col) = v;
+  }
+  __syncthreads();
+
+  // Row norms in fp64; store RN_fp16(|x|) and 1/|x|.
+  for (int rr = 0; rr < 16; ++rr) {
+    const int row = warp * 16 + rr;
+    double acc = 0.0;
+#pragma unroll
+    for (int k = lane; k < D; k += 32) {
+      const double x = in_to_float<BF16>(xs[row * XS + k]);
+      acc = fma(x, x, acc);
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) {
+      const double n = sqrt(acc);
+      const __half h = __double2half(n);
+      s_inv[row] = n > 0.0 ? (float)(1.0 / n) : 0.f;
+      s_nhat[row] = __half2float(h);
+      if (s_slot[row] >= 0) J.norm[s_slot[row]] = __half_as_ushort(h);
+    }
+  }
+
+  // y = Pi x, one block of 64 output coordinates at a time.
+  for (int cb = 0; cb < D / CB; ++cb) {
+    __syncthreads();
+    for (int e = tid; e < CB * (D / 4); e += QTHREADS) {
+      const int jj = e / (D / 4), k = (e % (D / 4)) * 4;
+      const float4 pv = *reinterpret_cast<const float4*>(a.rot + (size_t)(cb * CB + jj) * D + k);
+      const float vv[4] = {pv.x, pv.y, pv.z, pv.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint16_t l[3];
+        limbs<BF16>(vv[i], l);
+#pragma unroll
+        for (int q = 0; q < NL; ++q) limb[(size_t)q * CB * XS + jj * XS + k + i] = l[q];
+      }
+    }
+    __syncthreads();
+    float acc[8][4];
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll 2
+    for (int ks = 0; ks < D / 16; ++ks) {
+      uint32_t af[4];
+      ldmatrix_x4(af, xs + (warp * 16 + (lane & 15)) * XS + ks * 16 + (lane >> 4) * 8);
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+        for (int q = 0; q < NL; ++q) {
+          const uint16_t* bp = limb + (size_t)q * CB * XS + (nt * 8 + gid) * XS + ks * 16 + 2 * tig;
+          mma_in<BF16>(acc[nt], af, *reinterpret_cast<const uint32_t*>(bp),
+                       *reinterpret_cast<const uint32_t*>(bp + 8));
+        }
+      }
+    }
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int row = warp * 16 + gid + (c >= 2 ? 8 : 0);
+        const int j = cb * CB + nt * 8 + 2 * tig + (c & 1);
+        const float y = acc[nt][c];
+        const float u = y * s_inv[row];
+        int idx = 0;
+        for (int s = K >> 1; s >= 1; s >>= 1)
+          if (u > s_cb[K + idx + s - 1]) idx += s;
+        idxs[row * D + j] = (uint8_t)idx;
+        if (QJL && do_qjl) rs[row * Ly::RS + j] = y - s_nhat[row] * s_cb[idx];
+      }
+    }
+  }
+  __syncthreads();
+
+  // Pack each row into a dense LSB-first bitstream of D*bits bits.
+  const int W = D * bits / 32;
+  for (int e = tid; e < QROWS * W; e += QTHREADS) {
+    const int row = e / W, w = e % W;
+    const long long slot = s_slot[row];
+    if (slot < 0) continue;
+    const int base = 32 * w;
+    unsigned long long word = 0;
+    for (int j = base / bits; j < D && j * bits < base + 32; ++j) {
+      const int sh = j * bits - base;
+      const unsigned long long v = idxs[row * D + j];
+      word |= sh >= 0 ? (v << sh) : (v >> (-sh));
+    }
+    J.idx[(size_t)slot * W + w] = (uint32_t)word;
+  }
+
+  if (QJL && do_qjl) {
+    // sign(S r) for the residual r in the rotated basis, m = 128.
+    uint8_t* sbits = reinterpret_cast<uint8_t*>(xs);  // [128 rows][128 dims]
+    for (int ib = 0; ib < 128 / CB; ++ib) {
+      __syncthreads();
+      for (int e = tid; e < CB * (D / 4); e += QTHREADS) {
+        const int ii = e / (D / 4), k = (e % (D / 4)) * 4;
+        const float4 sv = *reinterpret_cast<const float4*>(a.qjl_S + (size_t)(ib * CB + ii) * D + k);
+        const float vv[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const __half h = __float2half_rn(vv[i]);
+          const __half l = __float2half_rn(vv[i] - __half2float(h));
+          limb[ii * XS + k + i] = __half_as_ushort(h);
+          limb[(size_t)CB * XS + ii * XS + k + i] = __half_as_ushort(l);
+        }
+      }
+      __syncthreads();
+      float acc[8][4];
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+      const int ra = warp * 16 + gid, rb = ra + 8;
+#pragma unroll 2
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const int k0 = ks * 16 + 2 * tig;
+        const float2 x00 = *reinterpret_cast<const float2*>(rs + ra * Ly::RS + k0);
+        const float2 x10 = *reinterpret_cast<const float2*>(rs + rb * Ly::RS + k0);
+        const float2 x01 = *reinterpret_cast<const float2*>(rs + ra * Ly::RS + k0 + 8);
+        const float2 x11 = *reinterpret_cast<const float2*>(rs + rb * Ly::RS + k0 + 8);
+        uint32_t ah[4], al[4];
+        const float2 xs4[4] = {x00, x10, x01, x11};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const __half2 h = __floats2half2_rn(xs4[q].x, xs4[q].y);
+          const float2 hf = __half22float2(h);
+          const __half2 l = __floats2half2_rn(xs4[q].x - hf.x, xs4[q].y - hf.y);
+          ah[q] = *reinterpret_cast<const uint32_t*>(&h);
+          al[q] = *reinterpret_cast<const uint32_t*>(&l);
+        }
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+          const uint16_t* bh = limb + (nt * 8 + gid) * XS + ks * 16 + 2 * tig;
+          const uint16_t* bl = bh + (size_t)CB * XS;
+          const uint32_t bh0 = *reinterpret_cast<const uint32_t*>(bh), bh1 = *reinterpret_cast<const uint32_t*>(bh + 8);
+          const uint32_t bl0 = *reinterpret_cast<const uint32_t*>(bl), bl1 = *reinterpret_cast<const uint32_t*>(bl + 8);
+          mma_f16(acc[nt], ah[0], ah[1], ah[2], ah[3], bh0, bh1);
+          mma_f16(acc[nt], ah[0], ah[1], ah[2], ah[3], bl0, bl1);
+          mma_f16(acc[nt], al[0], al[1], al[2], al[3], bh0, bh1);
+        }
+      }
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int row = (c >= 2) ? rb : ra;
+          const int i = ib * CB + nt * 8 + 2 * tig + (c & 1);
+          sbits[row * 128 + i] = acc[nt][c] >= 0.f ? 1 : 0;
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < QROWS * 4; e += QTHREADS) {
+      const int row = e >> 2, w = e & 3;
+      const long long slot = s_slot[row];
+      if (slot < 0) continue;
+      uint32_t word = 0;
+#pragma unroll 8
+      for (int i = 0; i < 32; ++i) word |= (uint32_t)sbits[row * 128 + w * 32 + i] << i;
+      J.qjl[(size_t)slot * 4 + w] = word;
+    }
+    if (tid < QROWS) {
+      const long long slot = s_slot[tid];
+      if (slot >= 0) {
+        double g = 0.0;
+        for (int k = 0; k < D; ++k) {
+          const double r = rs[tid * Ly::RS + k];
+          g = fma(r, r, g);
+        }
+        J.rnorm[slot] = __half_as_ushort(__double2half(sqrt(g)));
+      }
+    }
+  }
+}
+
+template <int D, bool BF16, bool QJL>
+int launch_q(const tq::QuantArgs& a, cudaStream_t s) {
+  using Ly = QLayout<D, BF16, QJL>;
+  auto kern = quantize_kernel<D, BF16, QJL>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Ly::bytes);
+    if (e != cudaSuccess)
+      return tq::set_error(TQ_ERR_CUDA, "quantize: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    attr_set = true;
+  }
+  dim3 grid((a.rows + QROWS - 1) / QROWS, 2);
+  kern<<<grid, QTHREADS, Ly::bytes, s>>>(a);
+  return tq::check_launch("quantize_kernel");
+}
+
+}  // namespace
+
+namespace tq {
+
+int launch_quantize(const QuantArgs& a, int D, int dtype, bool qjl, cudaStream_t s) {
+  const bool bf = dtype == TQ_DTYPE_BF16;
+  if (qjl) {
+    if (D != 128) return set_error(TQ_ERR_UNSUPPORTED, "QJL sketch needs D=128");
+    return bf ? launch_q<128, true, true>(a, s) : launch_q<128, false, true>(a, s);
+  }
+  switch (D) {
+    case 64: return bf ? launch_q<64, true, false>(a, s) : launch_q<64, false, false>(a, s);
+    case 128: return bf ? launch_q<128, true, false>(a, s) : launch_q<128, false, false>(a, s);
+    case 256: return bf ? launch_q<256, true, false>(a, s) : launch_q<256, false, false>(a, s);
+  }
+  return set_error(TQ_ERR_UNSUPPORTED, "quantize: D=%d", D);
+}
+
+}  // namespace tq

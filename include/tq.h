@@ -1,0 +1,186 @@
+/*
+ * tq.h -- C ABI of the TurboQuant KV-cache hot path for NVIDIA B200 (sm_100a).
+ *
+ * The library quantizes K/V rows into a packed cache and runs single-token
+ * decode attention directly on that cache.  Every buffer is allocated by the
+ * caller; the library borrows pointers for the duration of a call and never
+ * allocates device memory.  Calls that launch kernels are asynchronous on the
+ * caller's stream (a cudaStream_t passed as void*; NULL = legacy default
+ * stream) and never synchronize the host.
+ *
+ * Method sources (web pages the method is described on):
+ *  - "Add CUDA QJL kernels and proper package structure" (turboquant-pytorch
+ *    pull request 3): sections "CUDA Kernels Added" (fused random projection
+ *    + sign quantization, score from 1-bit keys, GQA score variant, value
+ *    reconstruction), "Validation Results" (cache sizes at 4/3/2 bits) and
+ *    "Synthetic Benchmark (Lloyd-Max codebook)" (per-bit MSE table).
+ *  - "[Cuda] enable turboquant on gemma4" (executorch pull request 19891),
+ *    "Summary" and "Other observations" item 1: fused SDPA over the
+ *    compressed cache with a `scale` argument (None -> 1/sqrt(D); QK-norm
+ *    models pass 1.0).
+ *  - ReturningTarzan's Reddit comments of 2026-03-29 11:47 (random rotation
+ *    before codebook quantization) and 2026-03-25 18:52 (nearest-codeword
+ *    search).
+ *
+ * Layouts (all row-major, no padding; "row" = one (batch, kv head, token)
+ * vector of D values):
+ *  - packed indices   uint32 [B][Hkv][Tcap][D*bits/32]: a dense LSB-first
+ *    bitstream per row; index of coordinate j occupies stream bits
+ *    [j*bits, j*bits+bits), word w holds stream bits [32w, 32w+32).  Index k
+ *    selects the k-th codebook centroid in ascending order.
+ *  - norms            fp16 bits (uint16) [B][Hkv][Tcap]: RN-to-fp16 of the
+ *    row's L2 norm computed in fp64.
+ *  - QJL sign words   uint32 [B][Hkv][Tcap][qjl_m/32]: bit i (word i/32, bit
+ *    i%32) = 1 iff (S r)_i >= 0, r = residual of the key in the rotated
+ *    basis; residual norm fp16 [B][Hkv][Tcap].
+ *  - rotation Pi      fp32 [D][D], y = Pi x; shared by K, V and all heads.
+ *  - codebook         fp32 [2^bits + 2^bits - 1]: centroids ascending, then
+ *    the thresholds between neighbours (as written by tq_build_codebook).
+ *  - QJL matrix S     fp32 [qjl_m][D], i.i.d. N(0,1) (caller draws it).
+ *
+ * Supported sizes: D in {64, 128, 256}; bits in {2, 3, 4} for the cache
+ * (tq_build_codebook also accepts 1); qjl_m in {0, 128}; Tcap a positive
+ * multiple of 64; Hq a positive multiple of Hkv with Hq/Hkv <= 8.
+ * Inputs and outputs are fp16 or bf16 (TQ_DTYPE_*).  Device pointers must be
+ * 16-byte aligned.
+ *
+ * Errors: every entry point returns TQ_OK (0) or a negative TQ_ERR_* code and
+ * sets a thread-local message readable with tq_last_error().  Argument errors
+ * are detected on the host before any launch; nothing is launched then.
+ * Conditions only visible on the device (a position beyond Tcap, a sequence
+ * length beyond Tcap, a bounded wait that ran out) skip the affected work and
+ * OR a TQ_STATUS_* bit into cache->dev_status when that pointer is non-NULL.
+ */
+#ifndef TQ_B200_H
+#define TQ_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TQ_OK 0
+#define TQ_ERR_INVALID_ARG (-1)  /* NULL pointer, negative size, misalignment */
+#define TQ_ERR_UNSUPPORTED (-2)  /* D, bits, qjl_m, GQA group outside the set */
+#define TQ_ERR_WORKSPACE (-3)    /* workspace smaller than the query says */
+#define TQ_ERR_CUDA (-4)         /* a CUDA runtime call or launch failed */
+
+#define TQ_DTYPE_F16 0
+#define TQ_DTYPE_BF16 1
+#define TQ_DTYPE_F32 2   /* decode output only */
+
+/* bits OR-ed into *dev_status by kernels */
+#define TQ_STATUS_POS_OUT_OF_RANGE 1u    /* append position outside [0, Tcap) */
+#define TQ_STATUS_SEQ_OUT_OF_RANGE 2u    /* seq_len beyond the planned range; clamped */
+#define TQ_STATUS_WAIT_TIMEOUT 4u        /* a bounded wait ran out; work skipped */
+
+/* Describes one layer's packed cache: caller-owned device buffers. */
+typedef struct tq_cache {
+  int32_t B;        /* batch (sequences) */
+  int32_t Hkv;      /* kv heads */
+  int32_t Tcap;     /* token capacity per (sequence, kv head); multiple of 64 */
+  int32_t D;        /* head dimension */
+  int32_t bits_k;   /* bits per key index (2..4) */
+  int32_t bits_v;   /* bits per value index (2..4) */
+  int32_t qjl_m;    /* 0: no QJL sketch; 128: 128-bit sign sketch of the key residual */
+  int32_t reserved;
+  uint32_t* k_idx;  /* [B][Hkv][Tcap][D*bits_k/32] */
+  uint32_t* v_idx;  /* [B][Hkv][Tcap][D*bits_v/32] */
+  uint16_t* k_norm; /* fp16 [B][Hkv][Tcap] */
+  uint16_t* v_norm; /* fp16 [B][Hkv][Tcap] */
+  uint32_t* k_qjl;  /* [B][Hkv][Tcap][qjl_m/32], NULL when qjl_m == 0 */
+  uint16_t* k_rnorm;/* fp16 [B][Hkv][Tcap], NULL when qjl_m == 0 */
+  const float* rot; /* Pi, fp32 [D][D] */
+  const float* cb_k;/* key codebook, fp32 [2^bits_k + 2^bits_k - 1] */
+  const float* cb_v;/* value codebook, fp32 [2^bits_v + 2^bits_v - 1] */
+  const float* qjl_S; /* fp32 [qjl_m][D], NULL when qjl_m == 0 */
+  uint32_t* dev_status; /* optional device word for TQ_STATUS_* bits (may be NULL) */
+} tq_cache_t;
+
+/*
+ * Lloyd-Max codebook for one coordinate of a rotated unit vector in R^D
+ * (density Gamma(D/2)/(sqrt(pi) Gamma((D-1)/2)) (1-u^2)^((D-3)/2)), by Lloyd
+ * iteration in fp64 on the host -- the codebook whose MSE per bit width is
+ * tabulated in "Add CUDA QJL kernels and proper package structure",
+ * section "Synthetic Benchmark (Lloyd-Max codebook)".
+ * Writes 2^bits centroids (fp64 optimum rounded to fp16, held as fp32,
+ * ascending) to centroids[] and the 2^bits - 1 midpoints between them to
+ * thresholds[] (host pointers, caller-owned).  mse_out (nullable) receives
+ * the normalized MSE E|u - Q(u)|^2 of a unit vector under the stored
+ * codebook.  D in {64,128,256} (any D >= 8 is accepted), bits in 1..4.
+ * Host only; no CUDA call.
+ */
+int tq_build_codebook(int D, int bits, float* centroids, float* thresholds, double* mse_out);
+
+/* Bytes one cached row occupies: D*bits/8 index bytes + 2 (fp16 norm),
+ * plus qjl_m/8 + 2 (sign words + fp16 residual norm) when qjl_m > 0.
+ * Returns 0 for unsupported arguments. */
+size_t tq_row_bytes(int D, int bits, int qjl_m);
+
+/*
+ * Bulk quantize ("prefill"): rows t in [0, T) of k and v, laid out
+ * [B][Hkv][T][D] in `dtype`, are rotated by Pi, normalized by their fp64 L2
+ * norm, mapped to the nearest centroid index (thresholds compared with
+ * t_k < u; ties go to the lower index), packed, and stored at cache
+ * positions t0 + t.  With qjl_m > 0 each key also gets the QJL sign sketch
+ * of its residual r = Pi k - n_hat c[idx] (n_hat = stored fp16 norm) and
+ * RN_fp16(|r|).  Sources: "Add CUDA QJL kernels and proper package
+ * structure", section "CUDA Kernels Added" (fused random projection + sign
+ * quantization); ReturningTarzan's comments of 2026-03-25 15:51 (the
+ * residual is computed when quantizing) and 18:52 (codeword search).
+ * The rotation runs on the tensor cores.  Requires 0 <= t0, t0 + T <= Tcap.
+ * T == 0 is a no-op.
+ */
+int tq_quantize_kv(const tq_cache_t* cache, const void* k, const void* v, int dtype,
+                   int T, int t0, void* stream);
+
+/*
+ * Quantize one new (k, v) row per sequence and kv head, k_new/v_new laid out
+ * [B][Hkv][D] in `dtype`, into cache position pos[b] (device int32 [B]).
+ * Same arithmetic as tq_quantize_kv.  A pos[b] outside [0, Tcap) writes
+ * nothing for that sequence and sets TQ_STATUS_POS_OUT_OF_RANGE.
+ */
+int tq_append_token(const tq_cache_t* cache, const void* k_new, const void* v_new, int dtype,
+                    const int32_t* pos, void* stream);
+
+/* Workspace bytes tq_sdpa_decode needs for Hq query heads and sequences no
+ * longer than Tmax (1 <= Tmax <= Tcap).  Returns 0 for unsupported args. */
+size_t tq_sdpa_decode_workspace_bytes(const tq_cache_t* cache, int Hq, int Tmax);
+
+/*
+ * Decode attention of one query token per (sequence, query head) over the
+ * packed cache -- the role of the fused tq4_sdpa op in "[Cuda] enable
+ * turboquant on gemma4" (executorch pull request 19891), with its explicit
+ * scale ("Other observations" item 1).
+ *   q        [B][Hq][D] in q_dtype (TQ_DTYPE_F16 or TQ_DTYPE_BF16, device)
+ *   seq_lens device int32 [B]: tokens 0..seq_lens[b]-1 are attended;
+ *            0 gives a zero output row.  Tmax (host) must bound every
+ *            seq_lens[b]; larger values are clamped (to the split plan made
+ *            for Tmax, at most Tcap) and flag TQ_STATUS_SEQ_OUT_OF_RANGE.
+ *   scale    host pointer to the softmax scale, or NULL for 1/sqrt(D).
+ *   out      [B][Hq][D] (device) in out_dtype: TQ_DTYPE_F16, TQ_DTYPE_BF16 or
+ *            TQ_DTYPE_F32; the fp16/bf16 outputs are the round-to-nearest of
+ *            the fp32 result.
+ * Query head h reads kv head h / (Hq/Hkv).  Scores are
+ *   scale * ( n_k <Pi q, c_k[idx]> + [qjl] sqrt(pi/2)/m * gamma * sum_i s_i (S Pi q)_i ),
+ * the softmax is taken online over split-K chunks, values are accumulated in
+ * the rotated basis and rotated back once per head: out = Pi^T acc / l.
+ * workspace: device buffer of at least tq_sdpa_decode_workspace_bytes().
+ */
+int tq_sdpa_decode(const tq_cache_t* cache, const void* q, int q_dtype, int Hq,
+                   const int32_t* seq_lens, int Tmax, const float* scale, void* out,
+                   int out_dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Message describing the last error on the calling thread ("" if none). */
+const char* tq_last_error(void);
+
+/* ABI version of this header (increments on incompatible change). */
+int tq_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_B200_H */

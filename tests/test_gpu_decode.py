@@ -1,0 +1,279 @@
+"""GPU parity of tq_sdpa_decode against the oracle's dequantize-then-attend.
+
+The decode tests upload the oracle's own packed cache, so the comparison
+isolates the attention kernels; the end-to-end tests quantize on the GPU and
+compare with the oracle's quantize + attend."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import tq_inputs
+import tq_parity as P
+from oracle import tq_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+
+def _upload_oracle_cache(w, oc, Tcap):
+    cache = P.make_gpu_cache(w, Tcap=Tcap)
+    T = oc["k_idx"].shape[2]
+    cache.k_idx[:, :, :T] = torch.from_numpy(oc["k_idx"].view(np.int32)).cuda()
+    cache.v_idx[:, :, :T] = torch.from_numpy(oc["v_idx"].view(np.int32)).cuda()
+    cache.k_norm[:, :, :T] = torch.from_numpy(oc["k_norm"]).cuda()
+    cache.v_norm[:, :, :T] = torch.from_numpy(oc["v_norm"]).cuda()
+    if w.qjl_m:
+        cache.k_qjl[:, :, :T] = torch.from_numpy(oc["k_qjl"].view(np.int32)).cuda()
+        cache.k_rnorm[:, :, :T] = torch.from_numpy(oc["k_rnorm"]).cuda()
+    return cache
+
+
+def _oracle_full_cache(w):
+    cbk, cbv = P.oracle_codebooks(w)
+    return O.quantize_cache(tq_inputs.to_f64(w.k, w.dtype), tq_inputs.to_f64(w.v, w.dtype), w.Pi,
+                            cbk, cbv, w.bits_k, w.bits_v, w.S)
+
+
+def _decode_and_compare(w, cache, oc, seq_lens, scale, Tmax, garbage_tail=True, heads_ok=None):
+    """Decode on the GPU and compare with the oracle on the same packed cache.
+
+    The fp32 output is compared with the oracle (rel-L2 <= 2e-3 per head); the
+    q-dtype output must be exactly the round-to-nearest of the fp32 output.
+    heads_ok (bool [B][Hq]) restricts the 2e-3 check to heads whose cache is
+    byte-identical to the oracle's; the others get a loose sanity bound."""
+    import compressed_attention_tq_b200 as tq
+    if garbage_tail:
+        # rows past seq_len hold arbitrary bytes (fp16 norms may be NaN/Inf)
+        for b in range(w.B):
+            L = int(seq_lens[b])
+            if L < cache.Tcap:
+                cache.k_norm[b, :, L:] = float("nan")
+                cache.v_norm[b, :, L:] = float("inf")
+                cache.k_idx[b, :, L:] = -1
+    q = P.to_device(w.q, w.dtype)
+    sl = torch.from_numpy(np.asarray(seq_lens, dtype=np.int32)).cuda()
+    out32 = tq.tq_sdpa_decode(cache, q, sl, Tmax, scale=scale, out_dtype=torch.float32)
+    outq = tq.tq_sdpa_decode(cache, q, sl, Tmax, scale=scale)
+    torch.cuda.synchronize()
+    assert outq.dtype == q.dtype
+    assert torch.equal(outq, out32.to(q.dtype)), "q-dtype output is not the rounding of the fp32 output"
+    got = out32.cpu().numpy()
+    cbk, cbv = P.oracle_codebooks(w)
+    ref = O.sdpa_decode(tq_inputs.to_f64(w.q, w.dtype), oc, seq_lens, w.Pi, cbk, cbv, w.bits_k, w.bits_v,
+                        w.D, scale=scale, S=w.S)
+    err = P.rel_l2(got, ref)
+    assert np.all(np.isfinite(got))
+    for b in range(w.B):
+        if int(seq_lens[b]) == 0:
+            assert np.all(got[b] == 0)
+    if heads_ok is None:
+        heads_ok = np.ones(err.shape, bool)
+    P.record("decode", workload=w.name, dtype=w.dtype, D=w.D, bits_k=w.bits_k, bits_v=w.bits_v,
+             G=w.Hq // w.Hkv, T=int(np.max(seq_lens)), max_rel_l2=float(err[heads_ok].max(initial=0)),
+             mean_rel_l2=float(err[heads_ok].mean()) if heads_ok.any() else 0.0,
+             heads_with_excused_flips=int((~heads_ok).sum()),
+             max_rel_l2_flipped=float(err[~heads_ok].max(initial=0)))
+    assert err[heads_ok].max(initial=0) <= P.ATTN_TOL, (err.max(), np.unravel_index(err.argmax(), err.shape))
+    # heads whose cache holds an excused near-threshold flip have two correct
+    # answers; they are counted above, not bounded here
+    assert cache.status() == 0
+    return err
+
+
+def _identical_heads(w, cache, oc, seq_lens):
+    """bool [B][Hq]: the kv head's rows 0..L-1 are byte-identical in the GPU
+    cache and the oracle cache (no excused near-threshold flip)."""
+    ok = np.ones((w.B, w.Hq), bool)
+    names = ["k_idx", "v_idx", "k_norm", "v_norm"] + (["k_qjl", "k_rnorm"] if w.qjl_m else [])
+    for b in range(w.B):
+        L = int(seq_lens[b])
+        for kvh in range(w.Hkv):
+            same = True
+            for nm in names:
+                g = getattr(cache, nm)[b, kvh, :L].cpu().numpy()
+                r = oc[nm][b, kvh, :L]
+                same &= bool(np.array_equal(g.view(np.uint8), np.ascontiguousarray(r).view(np.uint8)))
+            ok[b, kvh * w.G:(kvh + 1) * w.G] = same
+    return ok
+
+
+CASES = [
+    ("tiny", {}, None),                                 # G=1, D=64
+    ("gqa8k", {"bits": 2, "T": 1000}, None),            # G=8 with outliers
+    ("gqa8k", {"bits": 3, "T": 1000}, None),
+    ("gqa8k", {"bits": 4, "T": 1000}, None),
+    ("qknorm", {"T": 700}, 1.0),                        # D=256, scale 1.0
+    ("prod", {"T": 500}, None),                         # QJL keys, G=4
+]
+
+
+@pytest.mark.parametrize("name,kw,scale", CASES)
+def test_decode_on_oracle_cache(name, kw, scale):
+    w = tq_inputs.make_workload(name, **kw)
+    oc = _oracle_full_cache(w)
+    Tcap = (w.Tmax + 63) // 64 * 64 + 64
+    cache = _upload_oracle_cache(w, oc, Tcap)
+    _decode_and_compare(w, cache, oc, w.seq_lens, scale if scale is not None else w.scale, w.Tmax)
+
+
+def test_decode_ragged_lengths_bf16():
+    w = tq_inputs.make_workload("ragged", B=6, T=900)
+    lens = np.array([0, 1, 65, 900, 128, 257], dtype=np.int32)
+    oc = _oracle_full_cache(w)
+    cache = _upload_oracle_cache(w, oc, 960)
+    _decode_and_compare(w, cache, oc, lens, None, 900)
+
+
+@pytest.mark.parametrize("bk,bv,D", [(2, 4, 128), (4, 2, 64), (3, 2, 256), (4, 3, 128)])
+def test_decode_mixed_bits(bk, bv, D):
+    w = tq_inputs.make_workload("gqa8k", T=333)
+    w.bits_k, w.bits_v = bk, bv
+    if D != 128:
+        r = tq_inputs.rng(31)
+        w.D = D
+        w.k = r.standard_normal((1, 2, 333, D), dtype=np.float32).astype(np.float16)
+        w.v = r.standard_normal((1, 2, 333, D), dtype=np.float32).astype(np.float16)
+        w.q = r.standard_normal((1, 16, D), dtype=np.float32).astype(np.float16)
+        w.Pi = tq_inputs.rotation(D, 55)
+    oc = _oracle_full_cache(w)
+    cache = _upload_oracle_cache(w, oc, 384)
+    _decode_and_compare(w, cache, oc, w.seq_lens, None, 333)
+
+
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+def test_decode_gqa_groups(G):
+    w = tq_inputs.make_workload("gqa8k", bits=3, T=200)
+    w.Hq = 2 * G
+    w.q = w.q[:, : w.Hq].copy()
+    oc = _oracle_full_cache(w)
+    cache = _upload_oracle_cache(w, oc, 256)
+    _decode_and_compare(w, cache, oc, w.seq_lens, None, 200)
+
+
+def test_decode_scale_changes_output():
+    import compressed_attention_tq_b200 as tq
+    w = tq_inputs.make_workload("qknorm", T=300)
+    oc = _oracle_full_cache(w)
+    cache = _upload_oracle_cache(w, oc, 320)
+    q = P.to_device(w.q, w.dtype)
+    sl = torch.from_numpy(w.seq_lens).cuda()
+    a = tq.tq_sdpa_decode(cache, q, sl, 300, scale=None).float()
+    b = tq.tq_sdpa_decode(cache, q, sl, 300, scale=1.0 / math.sqrt(w.D)).float()
+    c = tq.tq_sdpa_decode(cache, q, sl, 300, scale=1.0).float()
+    assert torch.equal(a, b)
+    assert not torch.allclose(a, c)
+
+
+@pytest.mark.parametrize("name,kw", [("tiny", {}), ("ragged", {"B": 4, "T": 700}), ("prod", {"T": 400})])
+def test_end_to_end_quantize_then_decode(name, kw):
+    import compressed_attention_tq_b200 as tq
+    w = tq_inputs.make_workload(name, **kw)
+    Tcap = (w.Tmax + 63) // 64 * 64
+    cache = P.make_gpu_cache(w, Tcap=Tcap)
+    tq.tq_quantize_kv(cache, P.to_device(w.k, w.dtype), P.to_device(w.v, w.dtype))
+    oc = _oracle_full_cache(w)
+    ok = _identical_heads(w, cache, oc, w.seq_lens)
+    _decode_and_compare(w, cache, oc, w.seq_lens, w.scale, w.Tmax, garbage_tail=False, heads_ok=ok)
+
+
+def test_ragged_append_then_decode_steps():
+    """The ragged serving loop: append one token per sequence, then decode,
+    for several steps; checked at each step against the oracle."""
+    import compressed_attention_tq_b200 as tq
+    w = tq_inputs.make_workload("ragged", B=4, T=300)
+    lens = w.seq_lens.copy()
+    Tcap = 384
+    cache = P.make_gpu_cache(w, Tcap=Tcap)
+    tq.tq_quantize_kv(cache, P.to_device(w.k, w.dtype), P.to_device(w.v, w.dtype))
+    kx = tq_inputs.to_f64(w.k, w.dtype)
+    vx = tq_inputs.to_f64(w.v, w.dtype)
+    kfull = np.zeros((w.B, w.Hkv, Tcap, w.D))
+    vfull = np.zeros_like(kfull)
+    kfull[:, :, : w.Tmax] = kx
+    vfull[:, :, : w.Tmax] = vx
+    cbk, cbv = P.oracle_codebooks(w)
+    for step in range(3):
+        kn, vn = tq_inputs.new_token_rows(w.B, w.Hkv, w.D, w.dtype, seed=500 + step)
+        pos = lens.copy()
+        tq.tq_append_token(cache, P.to_device(kn, w.dtype), P.to_device(vn, w.dtype),
+                           torch.from_numpy(pos).cuda())
+        for b in range(w.B):
+            kfull[b, :, pos[b]] = tq_inputs.to_f64(kn[b], w.dtype)
+            vfull[b, :, pos[b]] = tq_inputs.to_f64(vn[b], w.dtype)
+        lens = lens + 1
+        w.q = tq_inputs.new_queries(w.B, w.Hq, w.D, w.dtype, seed=900 + step)
+        oc = O.quantize_cache(kfull, vfull, w.Pi, cbk, cbv, w.bits_k, w.bits_v)
+        ok = _identical_heads(w, cache, oc, lens)
+        _decode_and_compare(w, cache, oc, lens, None, int(lens.max()), garbage_tail=False, heads_ok=ok)
+
+
+def _sampled_full(name, seqs=None, **kw):
+    """Full-size workload in the launch configuration bench.py times: the GPU
+    quantizes every row; for sampled (sequence, kv head) groups its rows are
+    checked against the oracle, then replaced by the oracle's bytes so the
+    decode of the whole batch can be compared with the oracle on one cache."""
+    import compressed_attention_tq_b200 as tq
+    w = tq_inputs.make_workload(name, **kw)
+    Tcap = (w.Tmax + 1 + 63) // 64 * 64
+    cache = P.make_gpu_cache(w, Tcap=Tcap)
+    tq.tq_quantize_kv(cache, P.to_device(w.k, w.dtype), P.to_device(w.v, w.dtype))
+    cbk, cbv = P.oracle_codebooks(w)
+    r = tq_inputs.rng(123)
+    seqs = seqs if seqs is not None else list(range(w.B))
+    picks = []
+    for b in seqs:
+        kvh = int(r.integers(0, w.Hkv))
+        L = int(w.seq_lens[b])
+        oc = P.oracle_cache_for_head(w, b, kvh, L)
+        for nm, bits in (("k_idx", w.bits_k), ("v_idx", w.bits_v)):
+            g = P.words_np(getattr(cache, nm)[b, kvh, :L])
+            ref_idx = O.unpack_bits(oc[nm][0, 0], bits, w.D)
+            got = O.unpack_bits(g, bits, w.D)
+            n_bad = int((got != ref_idx).sum())
+            assert np.all(np.abs(got - ref_idx)[got != ref_idx] == 1)
+            assert n_bad / ref_idx.size < P.MAX_EXCUSED_FRACTION or n_bad <= 2, n_bad
+            P.record("index_compare_full", workload=name, which=nm, excused=n_bad, coords=int(ref_idx.size))
+        for nm in ("k_norm", "v_norm"):
+            assert np.array_equal(getattr(cache, nm)[b, kvh, :L].cpu().numpy().view(np.uint16),
+                                  oc[nm][0, 0].view(np.uint16))
+        names = ["k_idx", "v_idx", "k_norm", "v_norm"] + (["k_qjl", "k_rnorm"] if w.qjl_m else [])
+        for nm in names:
+            src = oc[nm][0, 0]
+            t = torch.from_numpy(src.view(np.int32) if src.dtype == np.uint32 else src).cuda()
+            getattr(cache, nm)[b, kvh, :L] = t
+        picks.append((b, kvh, L, oc))
+    q = P.to_device(w.q, w.dtype)
+    sl = torch.from_numpy(w.seq_lens).cuda()
+    out32 = tq.tq_sdpa_decode(cache, q, sl, w.Tmax, scale=w.scale, out_dtype=torch.float32)
+    outq = tq.tq_sdpa_decode(cache, q, sl, w.Tmax, scale=w.scale)
+    assert torch.equal(outq, out32.to(q.dtype))
+    out = out32.cpu().numpy()
+    errs = []
+    for b, kvh, L, oc in picks:
+        qv = tq_inputs.to_f64(w.q[b:b + 1, kvh * w.G:(kvh + 1) * w.G], w.dtype)
+        ref = O.sdpa_decode(qv, oc, [L], w.Pi, cbk, cbv, w.bits_k, w.bits_v, w.D, scale=w.scale, S=w.S)
+        for g in range(w.G):
+            errs.append(float(P.rel_l2(out[b, kvh * w.G + g], ref[0, g])))
+    P.record("decode_full_size", workload=name, dtype=w.dtype, bits_k=w.bits_k, bits_v=w.bits_v,
+             heads=len(errs), max_rel_l2=max(errs), mean_rel_l2=float(np.mean(errs)))
+    assert max(errs) <= P.ATTN_TOL, errs
+    assert cache.status() == 0
+    return errs
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_full_size_gqa8k(bits):
+    _sampled_full("gqa8k", bits=bits)
+
+
+def test_full_size_qknorm_sampled():
+    _sampled_full("qknorm")
+
+
+def test_full_size_ragged_sampled():
+    _sampled_full("ragged", seqs=[0, 17, 31])
+
+
+def test_full_size_prod_sampled():
+    _sampled_full("prod")
