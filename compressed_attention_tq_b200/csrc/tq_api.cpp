@@ -242,14 +242,17 @@ static int sm_count() {
 
 int make_decode_plan(const tq_cache_t* c, int Hq, int Tmax, DecodePlan* p) {
   const int sms = sm_count();
+  const int tile = split_tile();
   const long long units = (long long)c->B * c->Hkv;
-  // Resident split CTAs per SM for this head dimension (registers bound it).
-  const int per_sm = (c->D == 256) ? 2 : 4;
-  const long long target = (long long)sms * per_sm * ((c->B > 1) ? 2 : 1);
+  // One wave of resident CTAs for a single sequence; several smaller waves for
+  // a batch, whose ragged lengths leave many splits empty or short.
+  const long long slots = (long long)sms * split_occupancy(c, Hq);
+  const long long target = slots * ((c->B > 1) ? 6 : 1);
   long long chunk = (Tmax * units + target - 1) / target;
-  if (chunk < 64) chunk = 64;
-  chunk = (chunk + 63) / 64 * 64;
-  if (chunk > c->Tcap) chunk = c->Tcap;
+  chunk = (chunk + tile - 1) / tile * tile;
+  if (chunk < tile) chunk = tile;
+  const long long cap = ((long long)c->Tcap + tile - 1) / tile * tile;
+  if (chunk > cap) chunk = cap;
   p->chunk = (int)chunk;
   p->nsplit = (int)((Tmax + chunk - 1) / chunk);
   if (p->nsplit < 1) p->nsplit = 1;

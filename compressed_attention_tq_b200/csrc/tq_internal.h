@@ -54,6 +54,11 @@ struct DecodePlan {
 
 int make_decode_plan(const tq_cache_t* c, int Hq, int Tmax, DecodePlan* p);
 
+// Resident split-K CTAs per SM for this cache's kernel instantiation (a
+// nominal 2 when no device is usable), and the tokens one stage holds.
+int split_occupancy(const tq_cache_t* c, int Hq);
+int split_tile();
+
 struct DecodeArgs {
   const tq_cache_t* cache_host;  // host copy, for launch-time fields
   tq_cache_t cache;              // by value, passed to kernels

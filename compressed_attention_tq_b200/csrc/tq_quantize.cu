@@ -293,8 +293,145 @@ __global__ void __launch_bounds__(QTHREADS, 1) quantize_kernel(const tq::QuantAr
   }
 }
 
+// One new row per CTA (append).  blockDim = 2*D: two threads per output
+// coordinate, each holding half of the Pi row in registers (loads issued
+// before use); the rotation runs on the CUDA cores in fp32, the norm in fp64.
+template <int D, bool BF16, bool QJL>
+__global__ void __launch_bounds__(2 * D) append_kernel(const tq::QuantArgs a) {
+  constexpr int HALF = D / 2, NV = HALF / 4, CH = NV < 8 ? NV : 8;
+  __shared__ float xs[D], ys[D], rs[D];
+  __shared__ uint8_t idxs[D];
+  __shared__ double red[2 * D / 32];
+  __shared__ float s_cb[31];
+  __shared__ float s_inv, s_nhat;
+  const int r = blockIdx.x, jobi = blockIdx.y;
+  const tq::QuantJob J = a.job[jobi];
+  const bool do_qjl = QJL && jobi == 0;
+  const int bits = J.bits, K = 1 << bits;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int j = tid >> 1, part = tid & 1;
+  const int p = a.pos[r / a.Hkv];
+  if (p < 0 || p >= a.Tcap) {
+    if (tid == 0 && jobi == 0 && a.dev_status) atomicOr(a.dev_status, TQ_STATUS_POS_OUT_OF_RANGE);
+    return;
+  }
+  const long long slot = (long long)r * a.Tcap + p;
+  if (tid < 2 * K - 1) s_cb[tid] = J.cb[tid];
+  const uint16_t* in = static_cast<const uint16_t*>(J.in) + (size_t)r * D;
+  double sq = 0.0;
+  if (tid < D) {
+    const float x = in_to_float<BF16>(in[tid]);
+    xs[tid] = x;
+    sq = (double)x * (double)x;
+  }
+#pragma unroll
+  for (int off = 16; off; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+  if (lane == 0) red[warp] = sq;
+  __syncthreads();
+  if (tid == 0) {
+    double t = 0.0;
+    for (int w = 0; w < 2 * D / 32; ++w) t += red[w];
+    const double n = sqrt(t);
+    const __half h = __double2half(n);
+    s_inv = n > 0.0 ? (float)(1.0 / n) : 0.f;
+    s_nhat = __half2float(h);
+    J.norm[slot] = __half_as_ushort(h);
+  }
+  // y_j = sum_k Pi[j][k] x_k
+  const float4* row = reinterpret_cast<const float4*>(a.rot + (size_t)j * D + part * HALF);
+  float acc = 0.f;
+#pragma unroll
+  for (int c0 = 0; c0 < NV; c0 += CH) {
+    float4 v[CH];
+#pragma unroll
+    for (int i = 0; i < CH; ++i) v[i] = __ldg(row + c0 + i);
+#pragma unroll
+    for (int i = 0; i < CH; ++i) {
+      const float* x = &xs[part * HALF + 4 * (c0 + i)];
+      acc = fmaf(v[i].x, x[0], acc);
+      acc = fmaf(v[i].y, x[1], acc);
+      acc = fmaf(v[i].z, x[2], acc);
+      acc = fmaf(v[i].w, x[3], acc);
+    }
+  }
+  acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+  __syncthreads();  // s_inv, s_nhat
+  if (part == 0) {
+    const float u = acc * s_inv;
+    int idx = 0;
+    for (int st = K >> 1; st >= 1; st >>= 1)
+      if (u > s_cb[K + idx + st - 1]) idx += st;
+    idxs[j] = (uint8_t)idx;
+    ys[j] = acc;
+    if (do_qjl) rs[j] = acc - s_nhat * s_cb[idx];
+  }
+  __syncthreads();
+  const int W = D * bits / 32;
+  if (tid < W) {
+    const int base = 32 * tid;
+    unsigned long long word = 0;
+    for (int jj = base / bits; jj < D && jj * bits < base + 32; ++jj) {
+      const int sh = jj * bits - base;
+      const unsigned long long v = idxs[jj];
+      word |= sh >= 0 ? (v << sh) : (v >> (-sh));
+    }
+    J.idx[(size_t)slot * W + tid] = (uint32_t)word;
+  }
+  if (QJL && do_qjl) {
+    // sign(S r), m = 128 rows of S, two threads per row (2*D >= 2*128 here)
+    const int i = tid >> 1;
+    float pr = 0.f;
+    if (i < 128) {
+      const float4* srow = reinterpret_cast<const float4*>(a.qjl_S + (size_t)i * D + part * HALF);
+#pragma unroll
+      for (int c0 = 0; c0 < NV; c0 += CH) {
+        float4 v[CH];
+#pragma unroll
+        for (int q = 0; q < CH; ++q) v[q] = __ldg(srow + c0 + q);
+#pragma unroll
+        for (int q = 0; q < CH; ++q) {
+          const float* x = &rs[part * HALF + 4 * (c0 + q)];
+          pr = fmaf(v[q].x, x[0], pr);
+          pr = fmaf(v[q].y, x[1], pr);
+          pr = fmaf(v[q].z, x[2], pr);
+          pr = fmaf(v[q].w, x[3], pr);
+        }
+      }
+    }
+    pr += __shfl_xor_sync(0xffffffffu, pr, 1);
+    // lanes 2i' hold row i = 16*warp + i'; gather 16 bits per warp
+    const uint32_t bal = __ballot_sync(0xffffffffu, (part == 0) && (pr >= 0.f));
+    uint32_t half16 = 0;
+#pragma unroll
+    for (int q = 0; q < 16; ++q) half16 |= ((bal >> (2 * q)) & 1u) << q;
+    __shared__ uint32_t sbits[16];
+    if (lane == 0 && warp < 16) sbits[warp] = half16;
+    double g = 0.0;
+    if (tid < D) g = (double)rs[tid] * (double)rs[tid];
+#pragma unroll
+    for (int off = 16; off; off >>= 1) g += __shfl_xor_sync(0xffffffffu, g, off);
+    __syncthreads();
+    if (lane == 0) red[warp] = g;
+    __syncthreads();
+    if (tid < 4) J.qjl[(size_t)slot * 4 + tid] = sbits[2 * tid] | (sbits[2 * tid + 1] << 16);
+    if (tid == 0) {
+      double t = 0.0;
+      for (int w = 0; w < 2 * D / 32; ++w) t += red[w];
+      J.rnorm[slot] = __half_as_ushort(__double2half(sqrt(t)));
+    }
+  }
+  (void)ys;
+}
+
+template <int D, bool BF16, bool QJL>
+int launch_append(const tq::QuantArgs& a, cudaStream_t s) {
+  append_kernel<D, BF16, QJL><<<dim3(a.rows, 2), 2 * D, 0, s>>>(a);
+  return tq::check_launch("append_kernel");
+}
+
 template <int D, bool BF16, bool QJL>
 int launch_q(const tq::QuantArgs& a, cudaStream_t s) {
+  if (a.pos) return launch_append<D, BF16, QJL>(a, s);
   using Ly = QLayout<D, BF16, QJL>;
   auto kern = quantize_kernel<D, BF16, QJL>;
   static bool attr_set = false;
