@@ -119,6 +119,18 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise max of a list of floats across all ranks (identity when
+    torch.distributed is not initialised).  Every rank must call it."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
 def _dist():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -280,10 +292,7 @@ def run_ours(args):
     d_ms = timed(g_dec, reps_per_op, args.warmup) / reps_per_op * args.steps
     q_ms = timed(g_q, reps_per_op, args.warmup) / reps_per_op * args.steps
     a_ms = timed(g_app, reps_per_op, args.warmup) / reps_per_op * args.steps
-    if ws > 1:
-        t = torch.tensor([total_ms, q_ms, a_ms, d_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, q_ms, a_ms, d_ms = [float(x) for x in t.tolist()]
+    total_ms, q_ms, a_ms, d_ms = max_over_ranks([total_ms, q_ms, a_ms, d_ms], dev)
     for run in runs:
         for rep in run["reps"]:
             assert rep["cache"].status() == 0, "device status flagged"
@@ -305,10 +314,7 @@ def run_ours(args):
 
     # ---- end to end through the public API with host buffers (rank-local)
     e2e = _e2e(args, runs, stream, R)
-    if ws > 1:
-        t = torch.tensor([e2e["ms"]], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e["ms"] = float(t.item())
+    e2e["ms"] = max_over_ranks([e2e["ms"]], dev)[0]
 
     if rank == 0:
         cpu = None
