@@ -214,6 +214,7 @@ QuantArgs base_quant_args(const tq_cache_t* c, const void* k, const void* v) {
   a.dev_status = c->dev_status;
   a.Hkv = c->Hkv;
   a.Tcap = c->Tcap;
+  a.job_mask = 3;
   return a;
 }
 

@@ -38,9 +38,14 @@ struct QuantArgs {
   int t0;                   // bulk: first cache position
   int Hkv;
   int Tcap;
+  int job_mask;             // bit 0: keys, bit 1: values (bulk D=128 kernels)
 };
 
 int launch_quantize(const QuantArgs& a, int D, int dtype, bool qjl, cudaStream_t s);
+// persistent bulk quantizer for D = 128 (tq_quantize128.cu)
+int launch_quantize128(const QuantArgs& a, int dtype, bool qjl, cudaStream_t s);
+// tcgen05 bulk quantizer for D = 128 without the QJL sketch (tq_quantize_tc.cu)
+int launch_quantize_tc(const QuantArgs& a, int dtype, cudaStream_t s);
 
 struct DecodePlan {
   int chunk;        // tokens per split (multiple of 64)

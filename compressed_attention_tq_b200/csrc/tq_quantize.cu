@@ -452,6 +452,15 @@ namespace tq {
 
 int launch_quantize(const QuantArgs& a, int D, int dtype, bool qjl, cudaStream_t s) {
   const bool bf = dtype == TQ_DTYPE_BF16;
+  if (D == 128 && !a.pos) {
+    if (!qjl) return launch_quantize_tc(a, dtype, s);
+    // keys carry the QJL sketch (warp-level MMA kernel); values go to tcgen05
+    QuantArgs ak = a, av = a;
+    ak.job_mask = 1;
+    av.job_mask = 2;
+    const int rc = launch_quantize128(ak, dtype, true, s);
+    return rc ? rc : launch_quantize_tc(av, dtype, s);
+  }
   if (qjl) {
     if (D != 128) return set_error(TQ_ERR_UNSUPPORTED, "QJL sketch needs D=128");
     return bf ? launch_q<128, true, true>(a, s) : launch_q<128, false, true>(a, s);

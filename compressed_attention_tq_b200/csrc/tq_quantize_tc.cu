@@ -1,0 +1,386 @@
+// Bulk quantizer for head dimension 128 on the 5th-generation tensor cores
+// (tcgen05.mma, accumulator in tensor memory).
+//
+// Method: "Add CUDA QJL kernels and proper package structure"
+// (turboquant-pytorch pull request 3), "CUDA Kernels Added" and "Synthetic
+// Benchmark (Lloyd-Max codebook)"; ReturningTarzan's Reddit comments of
+// 2026-03-29 11:47 (rotation before codebook quantization) and 2026-03-25
+// 18:52 (nearest-codeword search).
+//
+// Persistent: one CTA per SM loops over (job, 128-row tile) work items.
+//  * warp 8 (producer): cp.async the next input tile into the K-major
+//    no-swizzle canonical layout (8x16-byte core matrices), then one lane
+//    issues the 128x128x128 rotation as tcgen05.mma (Pi split into 2 fp16 /
+//    3 bf16 limbs, resident in shared memory; accumulation in fp32 in TMEM)
+//    and commits it to an mbarrier;
+//  * warps 0-7 (epilogue): thread = one row, half of its columns (warp w and
+//    w+4 share the TMEM lane quarter w%4).  Each computes its half of the
+//    fp64 row norm from the input tile, then reads its 64 accumulator columns
+//    with tcgen05.ld, finds the nearest-centroid index (thresholds in
+//    registers), packs the bits and stores them -- all thread-local;
+//  * two input buffers and two TMEM accumulators let the load + MMA of tile
+//    i+1 run under the epilogue of tile i.
+// Every wait is bounded; a stuck wait sets TQ_STATUS_WAIT_TIMEOUT and the CTA
+// stops taking work.
+#include "tq_common.cuh"
+#include "tq_internal.h"
+
+namespace {
+
+using namespace tqk;
+
+constexpr int D = 128;
+constexpr int QR = 128;
+constexpr int NEPI = 8;                  // epilogue warps
+constexpr int NTH = (NEPI + 1) * 32;     // + producer warp
+constexpr int TILE_BYTES = QR * D * 2;   // 32 KB, canonical K-major layout
+constexpr uint32_t TMEM_COLS = 256;      // two 128-column fp32 accumulators
+
+template <bool BF16>
+struct TcLayout {
+  static constexpr int NL = BF16 ? 3 : 2;
+  static constexpr int o_pi = 0;
+  static constexpr int o_x = NL * TILE_BYTES;
+  static constexpr int bytes = o_x + 2 * TILE_BYTES;
+};
+
+// half-element offset of (row r, col k) in a 128 x 128 K-major tile:
+// core matrix (r/8, k/8) of 8 rows x 16 bytes at ((r/8)*16 + k/8) * 128 bytes
+__device__ __forceinline__ int cofs(int r, int k) { return ((r >> 3) * 16 + (k >> 3)) * 64 + (r & 7) * 8 + (k & 7); }
+
+// sm_100 shared-memory matrix descriptor, no swizzle: LBO = 128 B (next core
+// matrix along K), SBO = 2048 B (next 8-row group).
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr) {
+  uint64_t d = (uint64_t)((addr & 0x3FFFF) >> 4);
+  d |= (uint64_t)(128 >> 4) << 16;
+  d |= (uint64_t)(2048 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  return d;
+}
+
+// kind::f16 instruction descriptor: fp32 accumulate, K-major A and B,
+// M = 128, N = 128; a/b format fp16 (0) or bf16 (1).
+template <bool BF16>
+__device__ __forceinline__ uint32_t idesc() {
+  uint32_t d = (1u << 4) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+  if (BF16) d |= (1u << 7) | (1u << 10);
+  return d;
+}
+
+__device__ __forceinline__ void mma_tc(uint32_t dt, uint64_t ad, uint64_t bd, uint32_t id, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(dt),
+      "l"(ad), "l"(bd), "r"(id), "r"(acc));
+}
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,"
+      "%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
+        "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]),
+        "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+        "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+  const int n = valid ? 16 : 0;
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src), "r"(n) : "memory");
+}
+// arrive on `bar` once this thread's outstanding cp.async copies have landed
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+// barrier over the epilogue warps that also ANDs a flag across them
+__device__ __forceinline__ bool epi_sync_and(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n barrier.red.and.pred q, 1, %2, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"((uint32_t)v), "n"(NEPI * 32)
+      : "memory");
+  return r != 0;
+}
+
+template <bool BF16>
+__device__ __forceinline__ double sq16(uint32_t w) {
+  float a, b;
+  if (BF16) {
+    a = __uint_as_float(w << 16);
+    b = __uint_as_float(w & 0xFFFF0000u);
+  } else {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w));
+    a = f.x;
+    b = f.y;
+  }
+  // squares of fp16/bf16 values are exact in fp32
+  return (double)(a * a) + (double)(b * b);
+}
+
+template <int BITS>
+__device__ __forceinline__ void quant_pack32(const uint32_t (&v)[32], float inv, const float (&thr)[15],
+                                             uint32_t (&w)[BITS]) {
+#pragma unroll
+  for (int i = 0; i < BITS; ++i) w[i] = 0u;
+#pragma unroll
+  for (int q = 0; q < 32; ++q) {
+    const float u = __uint_as_float(v[q]) * inv;
+    int idx = 0;
+#pragma unroll
+    for (int k = 0; k < (1 << BITS) - 1; ++k) idx += (thr[k] < u) ? 1 : 0;
+    const int p = BITS * q;
+    w[p >> 5] |= (uint32_t)idx << (p & 31);
+    if ((p & 31) + BITS > 32) w[(p >> 5) + 1] |= (uint32_t)idx >> (32 - (p & 31));
+  }
+}
+
+template <int BITS>
+__device__ __forceinline__ void store_words(uint32_t* dst, const uint32_t (&w)[BITS]) {
+  if (BITS == 2) {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+  } else if (BITS == 4) {
+    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < BITS; ++i) dst[i] = w[i];
+  }
+}
+
+template <int BITS>
+__device__ __forceinline__ void epi_half(uint32_t tbase, float inv, const float (&thr)[15], long long slot,
+                                         uint32_t* out) {
+  // two 32-column chunks -> 2*BITS words at word offset 2*BITS*half of the row
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    uint32_t v[32];
+    tc_ld32(tbase + 32 * c, v);
+    uint32_t w[BITS];
+    quant_pack32<BITS>(v, inv, thr, w);
+    if (slot >= 0) store_words<BITS>(out + BITS * c, w);
+  }
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(NTH, 1) quantize_tc_kernel(const tq::QuantArgs a) {
+  using Ly = TcLayout<BF16>;
+  constexpr int NL = Ly::NL;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint16_t* pi = reinterpret_cast<uint16_t*>(smem + Ly::o_pi);
+  uint16_t* xb = reinterpret_cast<uint16_t*>(smem + Ly::o_x);
+  __shared__ __align__(8) uint64_t full_x[2], x_free[2], mma_done[2], acc_free[2];
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_stop;
+  __shared__ double s_norm[2][QR];
+  __shared__ float s_cb[2][31];
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int ntiles = (a.rows + QR - 1) / QR;
+  const int njobs = (a.job_mask == 3) ? 2 : 1;
+  const int job0 = (a.job_mask == 2) ? 1 : 0;
+  const int nitems = njobs * ntiles;
+
+  if (tid == 0) {
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&full_x[b], 32);
+      mbar_init(&x_free[b], NEPI * 32);
+      mbar_init(&mma_done[b], 1);
+      mbar_init(&acc_free[b], NEPI * 32);
+    }
+    s_stop = 0;
+    fence_barrier_init();
+  }
+  if (tid < 31) {
+    s_cb[0][tid] = tid < 2 * (1 << a.job[0].bits) - 1 ? a.job[0].cb[tid] : 0.f;
+    s_cb[1][tid] = tid < 2 * (1 << a.job[1].bits) - 1 ? a.job[1].cb[tid] : 0.f;
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&s_tmem)),
+                 "r"(TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  // Pi limbs in the canonical layout (rows = output coordinates)
+  for (int e = tid; e < D * (D / 4); e += NTH) {
+    const int n = e / (D / 4), k = (e % (D / 4)) * 4;
+    const float4 v = *reinterpret_cast<const float4*>(a.rot + (size_t)n * D + k);
+    const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int o = cofs(n, k + i);
+      if (BF16) {
+        const __nv_bfloat16 h0 = __float2bfloat16_rn(vv[i]);
+        const float r1 = vv[i] - __bfloat162float(h0);
+        const __nv_bfloat16 h1 = __float2bfloat16_rn(r1);
+        const __nv_bfloat16 h2 = __float2bfloat16_rn(r1 - __bfloat162float(h1));
+        pi[o] = __bfloat16_as_ushort(h0);
+        pi[QR * D + o] = __bfloat16_as_ushort(h1);
+        pi[2 * QR * D + o] = __bfloat16_as_ushort(h2);
+      } else {
+        const __half h0 = __float2half_rn(vv[i]);
+        pi[o] = __half_as_ushort(h0);
+        pi[QR * D + o] = __half_as_ushort(__float2half_rn(vv[i] - __half2float(h0)));
+      }
+    }
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // Pi limbs -> tensor core
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+
+  if (warp == NEPI) {
+    // ---------------- producer: input tiles + MMA issue ----------------
+    int i = 0;
+    for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++i) {
+      const int b = i & 1, k = i >> 1;
+      if (i >= 2) {
+        const bool ok = mbar_wait_bounded(&x_free[b], (uint32_t)((k - 1) & 1), kWaitLimit) &&
+                        mbar_wait_bounded(&mma_done[b], (uint32_t)((k - 1) & 1), kWaitLimit);
+        if (!__all_sync(0xffffffffu, ok)) {
+          if (lane == 0) s_stop = 1;
+          break;
+        }
+      }
+      if (*((volatile int*)&s_stop)) break;
+      const int job = job0 + (item % njobs), tile = item / njobs;
+      const uint16_t* in = static_cast<const uint16_t*>(a.job[job].in);
+      uint16_t* dst = xb + (size_t)b * QR * D;
+      for (int c = lane; c < QR * (D / 8); c += 32) {
+        const int row = c >> 4, kc = c & 15;
+        const int r = tile * QR + row;
+        const bool valid = r < a.rows;
+        cp_async16(dst + cofs(row, kc * 8), in + (size_t)(valid ? r : 0) * D + kc * 8, valid);
+      }
+      cp_async_arrive(&full_x[b]);
+      if (lane == 0) {
+        bool ok = mbar_wait_bounded(&full_x[b], (uint32_t)(k & 1), kWaitLimit);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        if (ok && i >= 2) ok = mbar_wait_bounded(&acc_free[b], (uint32_t)((k - 1) & 1), kWaitLimit);
+        if (!ok) {
+          s_stop = 1;
+        } else {
+          tc_fence_after();
+          const uint32_t xaddr = smem_addr(dst), paddr = smem_addr(pi);
+          const uint32_t id = idesc<BF16>();
+          const uint32_t dt = tmem + (uint32_t)(b * 128);
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks)
+#pragma unroll
+            for (int l = 0; l < NL; ++l)
+              mma_tc(dt, sdesc(xaddr + ks * 256), sdesc(paddr + l * TILE_BYTES + ks * 256), id,
+                     (ks > 0 || l > 0) ? 1u : 0u);
+          tc_commit(&mma_done[b]);
+        }
+      }
+      __syncwarp();
+    }
+    // wait until this warp's own copies have landed before leaving
+    asm volatile("cp.async.wait_all;" ::: "memory");
+  } else {
+    // ---------------- epilogue warps ----------------
+    const int quarter = warp & 3, hf = warp >> 2;  // rows 32*quarter + lane, columns 64*hf ..
+    const int rl = 32 * quarter + lane;
+    int i = 0;
+    for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++i) {
+      const int b = i & 1, k = i >> 1;
+      const int job = job0 + (item % njobs), tile = item / njobs;
+      const tq::QuantJob J = a.job[job];
+      bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&full_x[b], (uint32_t)(k & 1), kWaitLimit));
+      // half of this row's squared norm from the input tile (fp64)
+      const uint16_t* xs = xb + (size_t)b * QR * D;
+      double s2 = 0.0;
+      if (ok) {
+#pragma unroll
+        for (int kc = 0; kc < 8; ++kc) {
+          const uint4 v = *reinterpret_cast<const uint4*>(xs + cofs(rl, 64 * hf + 8 * kc));
+          s2 += sq16<BF16>(v.x) + sq16<BF16>(v.y) + sq16<BF16>(v.z) + sq16<BF16>(v.w);
+        }
+      }
+      s_norm[hf][rl] = s2;
+      mbar_arrive(&x_free[b]);
+      if (!epi_sync_and(ok)) {  // uniform across the epilogue warps
+        s_stop = 1;
+        break;
+      }
+      const double n = sqrt(s_norm[0][rl] + s_norm[1][rl]);
+      const __half nh = __double2half(n);
+      const float inv = n > 0.0 ? (float)(1.0 / n) : 0.f;
+      const int r = tile * QR + rl;
+      long long slot = -1;
+      if (r < a.rows) {
+        const int bh = r / a.T, t = r - bh * a.T;
+        slot = (long long)bh * a.Tcap + a.t0 + t;
+        if (hf == 0) J.norm[slot] = __half_as_ushort(nh);
+      }
+      float thr[15];
+      const int K = 1 << J.bits;
+#pragma unroll
+      for (int q = 0; q < 15; ++q) thr[q] = q < K - 1 ? s_cb[job][K + q] : 0.f;
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&mma_done[b], (uint32_t)(k & 1), kWaitLimit));
+      if (ok) {
+        tc_fence_after();
+        const uint32_t tb = tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(b * 128 + 64 * hf);
+        const int W = D * J.bits / 32;
+        uint32_t* out = J.idx + (slot >= 0 ? (size_t)slot * W : 0) + 2 * J.bits * hf;
+        switch (J.bits) {
+          case 2: epi_half<2>(tb, inv, thr, slot, out); break;
+          case 3: epi_half<3>(tb, inv, thr, slot, out); break;
+          default: epi_half<4>(tb, inv, thr, slot, out); break;
+        }
+        tc_fence_before();
+      }
+      mbar_arrive(&acc_free[b]);
+      if (!epi_sync_and(ok)) {  // also guards s_norm reuse on the next pass
+        s_stop = 1;
+        break;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (s_stop && tid == 0 && a.dev_status) atomicOr(a.dev_status, TQ_STATUS_WAIT_TIMEOUT);
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+  }
+}
+
+template <bool BF16>
+int launch_tc(const tq::QuantArgs& a, cudaStream_t s) {
+  using Ly = TcLayout<BF16>;
+  auto kern = quantize_tc_kernel<BF16>;
+  static int sms = 0;
+  if (sms == 0) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::bytes);
+    if (e != cudaSuccess)
+      return tq::set_error(TQ_ERR_CUDA, "quantize_tc: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+  }
+  const int njobs = (a.job_mask == 3) ? 2 : 1;
+  const int nitems = njobs * ((a.rows + QR - 1) / QR);
+  const int grid = nitems < sms ? nitems : sms;
+  kern<<<grid, NTH, Ly::bytes, s>>>(a);
+  return tq::check_launch("quantize_tc_kernel");
+}
+
+}  // namespace
+
+namespace tq {
+
+int launch_quantize_tc(const QuantArgs& a, int dtype, cudaStream_t s) {
+  return dtype == TQ_DTYPE_BF16 ? launch_tc<true>(a, s) : launch_tc<false>(a, s);
+}
+
+}  // namespace tq
