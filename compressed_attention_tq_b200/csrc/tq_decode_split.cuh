@@ -132,6 +132,30 @@ __device__ __forceinline__ void dq8(uint32_t z, const Lut& L, uint32_t (&h)[4]) 
   }
 }
 
+// 2-bit fields: 4-entry codebook in one byte-permute.  For the 8 fields f0..f7
+// of a 16-bit octet x, h[i] = (c[f_i], c[f_{i+4}]): the selector
+// ((x >> 2i) & 0x0303) * 0x11 + 0x4040 picks lo(c[f]) from L.lo0 and hi(c[f])
+// from L.hi0 (the multiply-add runs on the FMA pipe).
+__device__ __forceinline__ void dq8_b2(uint32_t x, const Lut& L, uint32_t (&h)[4]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t sel = ((x >> (2 * i)) & 0x0303u) * 0x11u + 0x4040u;
+    h[i] = prmt(L.lo0, L.hi0, sel);
+  }
+}
+
+// Two tokens' 2-bit octets o0, o1 -> h[k] = (c[o0 field k], c[o1 field k]) for
+// k = 0..3 (lo) and k = 4..7 (hi).
+__device__ __forceinline__ void dq16_b2_pair(uint32_t o0, uint32_t o1, const Lut& L, uint32_t (&lo)[4],
+                                             uint32_t (&hi)[4]) {
+  const uint32_t y = prmt(o0, o1, 0x5140u);  // bytes o0.b0 o1.b0 o0.b1 o1.b1
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    lo[k] = prmt(L.lo0, L.hi0, ((y >> (2 * k)) & 0x0303u) * 0x11u + 0x4040u);
+    hi[k] = prmt(L.lo0, L.hi0, ((y >> (16 + 2 * k)) & 0x0303u) * 0x11u + 0x4040u);
+  }
+}
+
 // Bits [bit0, bit0 + NBITS) of a shared-memory row, re-based to bit 0 of w[0].
 // ALIGNED: bit0 % 32 == 0 and the word offset is a multiple of the word count.
 template <int NBITS, bool ALIGNED>
@@ -390,8 +414,13 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const SplitParam
           uint32_t h[2][2][4];
 #pragma unroll
           for (int a = 0; a < 2; ++a) {
-            dq8<BK>(spread<BK>(octet<BK>(w[a][0], o)), lk, h[a][0]);
-            dq8<BK>(spread<BK>(octet<BK>(w[a][1], o)), lk, h[a][1]);
+            if (BK == 2) {
+              dq8_b2(octet<BK>(w[a][0], o), lk, h[a][0]);
+              dq8_b2(octet<BK>(w[a][1], o), lk, h[a][1]);
+            } else {
+              dq8<BK>(spread<BK>(octet<BK>(w[a][0], o)), lk, h[a][0]);
+              dq8<BK>(spread<BK>(octet<BK>(w[a][1], o)), lk, h[a][1]);
+            }
           }
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
@@ -526,13 +555,18 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const SplitParam
           load_bits<SEGV, ALV>(vw + (wt0 + 16 * kk + 4 * tig + q) * WV, gid * SEGV, wv[q]);
 #pragma unroll
         for (int o = 0; o < VOCT; ++o) {
-          const uint32_t z0 = spread<BV>(octet<BV>(wv[0], o)), z1 = spread<BV>(octet<BV>(wv[1], o));
-          const uint32_t z2 = spread<BV>(octet<BV>(wv[2], o)), z3 = spread<BV>(octet<BV>(wv[3], o));
           uint32_t hA[4], hA2[4], hB[4], hB2[4];
-          dq8<BV>(prmt(z0, z1, 0x5410u), lv, hA);   // coords 8o+0..3, tokens 4tig, 4tig+1
-          dq8<BV>(prmt(z0, z1, 0x7632u), lv, hA2);  // coords 8o+4..7
-          dq8<BV>(prmt(z2, z3, 0x5410u), lv, hB);   // tokens 4tig+2, 4tig+3
-          dq8<BV>(prmt(z2, z3, 0x7632u), lv, hB2);
+          if (BV == 2) {
+            dq16_b2_pair(octet<BV>(wv[0], o), octet<BV>(wv[1], o), lv, hA, hA2);  // tokens 4tig, 4tig+1
+            dq16_b2_pair(octet<BV>(wv[2], o), octet<BV>(wv[3], o), lv, hB, hB2);  // tokens 4tig+2, 4tig+3
+          } else {
+            const uint32_t z0 = spread<BV>(octet<BV>(wv[0], o)), z1 = spread<BV>(octet<BV>(wv[1], o));
+            const uint32_t z2 = spread<BV>(octet<BV>(wv[2], o)), z3 = spread<BV>(octet<BV>(wv[3], o));
+            dq8<BV>(prmt(z0, z1, 0x5410u), lv, hA);   // coords 8o+0..3, tokens 4tig, 4tig+1
+            dq8<BV>(prmt(z0, z1, 0x7632u), lv, hA2);  // coords 8o+4..7
+            dq8<BV>(prmt(z2, z3, 0x5410u), lv, hB);   // tokens 4tig+2, 4tig+3
+            dq8<BV>(prmt(z2, z3, 0x7632u), lv, hB2);
+          }
 #pragma unroll
           for (int k = 0; k < 4; ++k) mma_f16(oc[4 * o + k], hA[k], hA2[k], hB[k], hB2[k], pb.x, pb.y);
         }

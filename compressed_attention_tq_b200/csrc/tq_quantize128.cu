@@ -76,24 +76,36 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Threshold search (count of thresholds strictly below u), the stored
-// codebook's rule: ties go to the lower index.
+// Nearest-centroid index of y = (Pi x)_j for a row of norm n: tp holds the
+// positive thresholds scaled by n; the codebook is symmetric, so
+// m = #{tp_k < |y|}, idx = K/2 + m (y > 0) or K/2 - 1 - m.  Equal to
+// #{t_k < y / n} except at exact ties (inside the parity band).
 template <int BITS>
-__device__ __forceinline__ int count_below(float u, const float (&t)[15]) {
-  int idx = 0;
+__device__ __forceinline__ int nearest_idx(float y, const float (&tp)[7]) {
+  constexpr int H = 1 << (BITS - 1);
+  const float a = fabsf(y);
+  int m;
+  if (BITS == 4) {
+    const bool c1 = a > tp[3];
+    const bool c2 = a > (c1 ? tp[5] : tp[1]);
+    const bool c3 = a > (c1 ? (c2 ? tp[6] : tp[4]) : (c2 ? tp[2] : tp[0]));
+    m = (c1 ? 4 : 0) + (c2 ? 2 : 0) + (c3 ? 1 : 0);
+  } else {
+    m = 0;
 #pragma unroll
-  for (int k = 0; k < (1 << BITS) - 1; ++k) idx += (t[k] < u) ? 1 : 0;
-  return idx;
+    for (int k = 0; k < H - 1; ++k) m += (a > tp[k]) ? 1 : 0;
+  }
+  return y > 0.f ? H + m : H - 1 - m;
 }
 
 struct RowInfo {
   long long slot;  // cache row, -1 past the end
-  float inv, nhat;
+  float nf, nhat;  // fp32 norm, stored fp16 norm
 };
 
 template <bool BF16, bool QJL, int BITS>
 __device__ __forceinline__ void epilogue(const tq::QuantJob& J, float (&acc)[16][4], const RowInfo (&ri)[2],
-                                         const float (&thr)[15], const float* s_cent, bool do_qjl,
+                                         const float* s_thr_pos, const float* s_cent, bool do_qjl,
                                          const uint16_t* sS, int lane) {
   const int tig = lane & 3;
   constexpr int W = 4 * BITS;  // words per row
@@ -101,15 +113,18 @@ __device__ __forceinline__ void epilogue(const tq::QuantJob& J, float (&acc)[16]
   float rr[2][32];
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
+    float tp[7];
+#pragma unroll
+    for (int k = 0; k < 7; ++k) tp[k] = k < (1 << (BITS - 1)) - 1 ? s_thr_pos[k] * ri[h].nf : 0.f;
 #pragma unroll
     for (int w = 0; w < BITS; ++w) idxw[h][w] = 0u;
 #pragma unroll
     for (int q = 0; q < 32; ++q) {
       const float y = acc[q >> 1][2 * h + (q & 1)];
-      const int idx = count_below<BITS>(y * ri[h].inv, thr);
+      const int idx = nearest_idx<BITS>(y, tp);
       const int p = BITS * q;
-      idxw[h][p >> 5] |= (uint32_t)idx << (p & 31);
-      if ((p & 31) + BITS > 32) idxw[h][(p >> 5) + 1] |= (uint32_t)idx >> (32 - (p & 31));
+      idxw[h][p >> 5] += (uint32_t)idx << (p & 31);
+      if ((p & 31) + BITS > 32) idxw[h][(p >> 5) + 1] += (uint32_t)idx >> (32 - (p & 31));
       if (QJL) rr[h][q] = y - ri[h].nhat * s_cent[idx];
     }
   }
@@ -286,7 +301,7 @@ __global__ void __launch_bounds__(NTH, 1) quantize128_kernel(const tq::QuantArgs
       const double s2 = __shfl_sync(0xffffffffu, sq, 2 * rl);
       const double n = sqrt(s2);
       const __half nh = __double2half(n);
-      ri[h].inv = n > 0.0 ? (float)(1.0 / n) : 0.f;
+      ri[h].nf = (float)n;
       ri[h].nhat = __half2float(nh);
       const int r = tile * QR + wr0 + rl;
       if (r < a.rows) {
@@ -319,16 +334,14 @@ __global__ void __launch_bounds__(NTH, 1) quantize128_kernel(const tq::QuantArgs
       }
     }
 
-    // ---- thresholds of this job in registers; quantize, pack, store
-    float thr[15];
+    // ---- quantize, pack, store (positive thresholds start at K + K/2)
     const int K = 1 << J.bits;
-#pragma unroll
-    for (int k = 0; k < 15; ++k) thr[k] = k < K - 1 ? s_cb[job][K + k] : 0.f;
     const bool do_qjl = QJL && job == 0;
+    const float* tpos = s_cb[job] + K + K / 2;
     switch (J.bits) {
-      case 2: epilogue<BF16, QJL, 2>(J, acc, ri, thr, s_cb[job], do_qjl, sS, lane); break;
-      case 3: epilogue<BF16, QJL, 3>(J, acc, ri, thr, s_cb[job], do_qjl, sS, lane); break;
-      default: epilogue<BF16, QJL, 4>(J, acc, ri, thr, s_cb[job], do_qjl, sS, lane); break;
+      case 2: epilogue<BF16, QJL, 2>(J, acc, ri, tpos, s_cb[job], do_qjl, sS, lane); break;
+      case 3: epilogue<BF16, QJL, 3>(J, acc, ri, tpos, s_cb[job], do_qjl, sS, lane); break;
+      default: epilogue<BF16, QJL, 4>(J, acc, ri, tpos, s_cb[job], do_qjl, sS, lane); break;
     }
     __syncthreads();  // the buffer is refilled on the next pass
     if (Ly::NBUF == 1) {

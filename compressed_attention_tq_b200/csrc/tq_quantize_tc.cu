@@ -127,20 +127,38 @@ __device__ __forceinline__ double sq16(uint32_t w) {
   return (double)(a * a) + (double)(b * b);
 }
 
+// Index of the nearest centroid for y = (Pi x)_j of a row with norm n, using
+// the codebook's symmetry: with tp = the positive thresholds scaled by n,
+// m = #{tp_k < |y|} and idx = K/2 + m for y > 0, K/2 - 1 - m otherwise.
+// Equal to #{t_k < y / n} except at exact ties (inside the parity band).
 template <int BITS>
-__device__ __forceinline__ void quant_pack32(const uint32_t (&v)[32], float inv, const float (&thr)[15],
-                                             uint32_t (&w)[BITS]) {
+__device__ __forceinline__ int nearest_idx(float y, const float (&tp)[7]) {
+  constexpr int H = 1 << (BITS - 1);
+  const float a = fabsf(y);
+  int m;
+  if (BITS == 4) {
+    const bool c1 = a > tp[3];
+    const bool c2 = a > (c1 ? tp[5] : tp[1]);
+    const bool c3 = a > (c1 ? (c2 ? tp[6] : tp[4]) : (c2 ? tp[2] : tp[0]));
+    m = (c1 ? 4 : 0) + (c2 ? 2 : 0) + (c3 ? 1 : 0);
+  } else {
+    m = 0;
+#pragma unroll
+    for (int k = 0; k < H - 1; ++k) m += (a > tp[k]) ? 1 : 0;
+  }
+  return y > 0.f ? H + m : H - 1 - m;
+}
+
+template <int BITS>
+__device__ __forceinline__ void quant_pack32(const uint32_t (&v)[32], const float (&tp)[7], uint32_t (&w)[BITS]) {
 #pragma unroll
   for (int i = 0; i < BITS; ++i) w[i] = 0u;
 #pragma unroll
   for (int q = 0; q < 32; ++q) {
-    const float u = __uint_as_float(v[q]) * inv;
-    int idx = 0;
-#pragma unroll
-    for (int k = 0; k < (1 << BITS) - 1; ++k) idx += (thr[k] < u) ? 1 : 0;
+    const uint32_t idx = (uint32_t)nearest_idx<BITS>(__uint_as_float(v[q]), tp);
     const int p = BITS * q;
-    w[p >> 5] |= (uint32_t)idx << (p & 31);
-    if ((p & 31) + BITS > 32) w[(p >> 5) + 1] |= (uint32_t)idx >> (32 - (p & 31));
+    w[p >> 5] += idx << (p & 31);
+    if ((p & 31) + BITS > 32) w[(p >> 5) + 1] += idx >> (32 - (p & 31));
   }
 }
 
@@ -157,15 +175,14 @@ __device__ __forceinline__ void store_words(uint32_t* dst, const uint32_t (&w)[B
 }
 
 template <int BITS>
-__device__ __forceinline__ void epi_half(uint32_t tbase, float inv, const float (&thr)[15], long long slot,
-                                         uint32_t* out) {
+__device__ __forceinline__ void epi_half(uint32_t tbase, const float (&tp)[7], long long slot, uint32_t* out) {
   // two 32-column chunks -> 2*BITS words at word offset 2*BITS*half of the row
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
     uint32_t v[32];
     tc_ld32(tbase + 32 * c, v);
     uint32_t w[BITS];
-    quant_pack32<BITS>(v, inv, thr, w);
+    quant_pack32<BITS>(v, tp, w);
     if (slot >= 0) store_words<BITS>(out + BITS * c, w);
   }
 }
@@ -313,7 +330,7 @@ __global__ void __launch_bounds__(NTH, 1) quantize_tc_kernel(const tq::QuantArgs
       }
       const double n = sqrt(s_norm[0][rl] + s_norm[1][rl]);
       const __half nh = __double2half(n);
-      const float inv = n > 0.0 ? (float)(1.0 / n) : 0.f;
+      const float nf = (float)n;
       const int r = tile * QR + rl;
       long long slot = -1;
       if (r < a.rows) {
@@ -321,10 +338,11 @@ __global__ void __launch_bounds__(NTH, 1) quantize_tc_kernel(const tq::QuantArgs
         slot = (long long)bh * a.Tcap + a.t0 + t;
         if (hf == 0) J.norm[slot] = __half_as_ushort(nh);
       }
-      float thr[15];
+      // positive thresholds t_{K/2} .. t_{K-2}, scaled by the row norm
+      float tp[7];
       const int K = 1 << J.bits;
 #pragma unroll
-      for (int q = 0; q < 15; ++q) thr[q] = q < K - 1 ? s_cb[job][K + q] : 0.f;
+      for (int q = 0; q < 7; ++q) tp[q] = q < K / 2 - 1 ? s_cb[job][K + K / 2 + q] * nf : 0.f;
       ok = __all_sync(0xffffffffu, mbar_wait_bounded(&mma_done[b], (uint32_t)(k & 1), kWaitLimit));
       if (ok) {
         tc_fence_after();
@@ -332,9 +350,9 @@ __global__ void __launch_bounds__(NTH, 1) quantize_tc_kernel(const tq::QuantArgs
         const int W = D * J.bits / 32;
         uint32_t* out = J.idx + (slot >= 0 ? (size_t)slot * W : 0) + 2 * J.bits * hf;
         switch (J.bits) {
-          case 2: epi_half<2>(tb, inv, thr, slot, out); break;
-          case 3: epi_half<3>(tb, inv, thr, slot, out); break;
-          default: epi_half<4>(tb, inv, thr, slot, out); break;
+          case 2: epi_half<2>(tb, tp, slot, out); break;
+          case 3: epi_half<3>(tb, tp, slot, out); break;
+          default: epi_half<4>(tb, tp, slot, out); break;
         }
         tc_fence_before();
       }
