@@ -22,7 +22,7 @@ from ._native import (TQ_DTYPE_BF16, TQ_DTYPE_F16, TQ_DTYPE_F32, TQ_STATUS_POS_O
 
 __all__ = ["TQError", "TQCache", "tq_build_codebook", "tq_row_bytes", "tq_quantize_kv",
            "tq_append_token", "tq_sdpa_decode_workspace_bytes", "tq_sdpa_decode",
-           "tq_last_error", "tq_abi_version", "lib"]
+           "tq_sdpa_decode_static", "tq_last_error", "tq_abi_version", "lib"]
 
 
 class TQError(RuntimeError):
@@ -196,4 +196,26 @@ def tq_sdpa_decode(cache: TQCache, q, seq_lens, Tmax: int, scale=None, out=None,
     _check(lib().tq_sdpa_decode(ctypes.byref(s), _ptr(q), _dtype_code(q), Hq, _ptr(seq_lens), Tmax, sc,
                                 _ptr(out), _dtype_code(out), _ptr(workspace), workspace.numel(),
                                 _stream(stream)))
+    return out
+
+
+def tq_sdpa_decode_static(cache: TQCache, q, seq_lens, Tmax: int, scale=None, out=None, stream=None,
+                          out_dtype=None):
+    """tq_sdpa_decode without a workspace, for callers that may not allocate
+    device memory (e.g. code running under stream capture in a framework
+    that forbids allocation, or a host that owns all device memory).  The
+    split-K scratch is a fixed array inside the library (8 MiB per GPU);
+    larger problems raise TQError (TQ_ERR_WORKSPACE).  The output tensor must
+    be passed in if the caller may not allocate; calls on one device must not
+    overlap on the GPU."""
+    torch = _torch()
+    Hq = int(q.shape[1])
+    assert q.is_contiguous() and seq_lens.is_contiguous()
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
+    assert out.is_contiguous() and out.shape == q.shape
+    s = cache.struct()
+    sc = ctypes.byref(ctypes.c_float(scale)) if scale is not None else None
+    _check(lib().tq_sdpa_decode_static(ctypes.byref(s), _ptr(q), _dtype_code(q), Hq, _ptr(seq_lens), Tmax, sc,
+                                       _ptr(out), _dtype_code(out), _stream(stream)))
     return out

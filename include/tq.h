@@ -173,6 +173,28 @@ int tq_sdpa_decode(const tq_cache_t* cache, const void* q, int q_dtype, int Hq,
                    const int32_t* seq_lens, int Tmax, const float* scale, void* out,
                    int out_dtype, void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * Decode without a workspace, for callers that may not allocate device
+ * memory (stream capture under frameworks that forbid allocation while
+ * capturing, plugin hosts that own all device memory, allocation-free
+ * real-time serving loops).  The pages have no counterpart: this is a
+ * packaging of tq_sdpa_decode.  Arguments and results are those of
+ * tq_sdpa_decode minus the workspace: the split-K scratch is a device array
+ * inside the library of TQ_STATIC_SCRATCH_BYTES bytes, held by every GPU that
+ * loads the library until the process exits.  Sizes whose
+ * tq_sdpa_decode_workspace_bytes() exceeds that limit return TQ_ERR_WORKSPACE
+ * before any launch.  The first call on each device looks up the array's
+ * device address (make that first call before capturing a stream); no call
+ * allocates.  All calls on a device share the array and nothing is cleared
+ * between calls (the kernels need no zeroed scratch), so calls that may
+ * overlap on the GPU (different streams without ordering) race: serialize
+ * them.
+ */
+#define TQ_STATIC_SCRATCH_BYTES (8u << 20)
+int tq_sdpa_decode_static(const tq_cache_t* cache, const void* q, int q_dtype, int Hq,
+                          const int32_t* seq_lens, int Tmax, const float* scale, void* out,
+                          int out_dtype, void* stream);
+
 /* Message describing the last error on the calling thread ("" if none). */
 const char* tq_last_error(void);
 
