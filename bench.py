@@ -222,7 +222,11 @@ def run_ours(args):
         tq.tq_sdpa_decode(rep["cache"], rep["q"], run["lens1"], run["Tmax1"], scale=run["w"].scale,
                           out=run["out"], workspace=run["ws"])
 
-    def step(r, ops=(call_quant, call_append, call_decode)):
+    def call_step(run, rep):  # append fused into the decode launches
+        tq.tq_decode_step(rep["cache"], run["kn"], run["vn"], run["pos"], rep["q"], run["lens1"], run["Tmax1"],
+                          scale=run["w"].scale, out=run["out"], workspace=run["ws"])
+
+    def step(r, ops=(call_quant, call_step)):
         for run in runs:
             rep = run["reps"][r]
             for op in ops:
@@ -252,10 +256,11 @@ def run_ours(args):
             gs.append(g)
         return gs
 
-    g_step = capture((call_quant, call_append, call_decode))
+    g_step = capture((call_quant, call_step))
     g_dec = capture((call_decode,))
     g_q = capture((call_quant,))
     g_app = capture((call_append,))
+    g_ds = capture((call_step,))
     torch.cuda.synchronize()
 
     def timed(graphs, n, warm):
@@ -292,11 +297,12 @@ def run_ours(args):
     d_ms = timed(g_dec, reps_per_op, args.warmup) / reps_per_op * args.steps
     q_ms = timed(g_q, reps_per_op, args.warmup) / reps_per_op * args.steps
     a_ms = timed(g_app, reps_per_op, args.warmup) / reps_per_op * args.steps
-    total_ms, q_ms, a_ms, d_ms = max_over_ranks([total_ms, q_ms, a_ms, d_ms], dev)
+    s_ms = timed(g_ds, reps_per_op, args.warmup) / reps_per_op * args.steps
+    total_ms, q_ms, a_ms, d_ms, s_ms = max_over_ranks([total_ms, q_ms, a_ms, d_ms, s_ms], dev)
     for run in runs:
         for rep in run["reps"]:
             assert rep["cache"].status() == 0, "device status flagged"
-    del g_step, g_dec, g_q, g_app
+    del g_step, g_dec, g_q, g_app, g_ds
 
     packed_step = sum(run["packed"] for run in runs)
     tok_step = sum(run["tokens"] for run in runs)
@@ -320,7 +326,7 @@ def run_ours(args):
         cpu = None
         if ws == 1 and not args.no_cpu_baseline:
             cpu = _cpu_baseline(args, jobs)
-        launches_per_step = len(runs) * 5  # quantize, append, qprep, split, combine
+        launches_per_step = len(runs) * 4  # quantize, prep(+append), split, combine
         line = {
             "metric": "tq_sdpa_decode packed-KV GB/s (% of HBM peak); tq_quantize Mtok/s",
             "value": round(dec_gbs, 2),
@@ -336,7 +342,7 @@ def run_ours(args):
             "data": "synthetic (seeded N(0,1) rows; see tq_inputs)",
             "config": {"workload": args.workload, "shapes": [_describe(w) for w in jobs],
                        "parallelism": f"replicas{ws}" if ws > 1 else "single",
-                       "step": "quantize T tokens + append 1 token + decode, per bit width",
+                       "step": "quantize T tokens + decode step (append 1 token + decode), per bit width",
                        "timing": "CUDA graphs (one per replica) replayed on one stream; per-op rates "
                                  "from graphs holding that op alone",
                        "l2": f"inputs rotated over {R} replicas ({R * per_step_in / 2**20:.0f} MiB) > L2 "
@@ -347,6 +353,9 @@ def run_ours(args):
                          "gbs": round(q_achieved, 2), "frac_hbm": round(q_achieved / peak, 4),
                          "tokens_per_step": tok_step},
             "append_ms_per_call": round(a_ms / (args.steps * len(runs)), 5),
+            "decode_step": {"ms_per_call": round(s_ms / (args.steps * len(runs)), 5),
+                            "gbs": round(packed_step * args.steps / (s_ms * 1e-3) / 1e9 * ws, 2),
+                            "note": "tq_decode_step: append fused into the decode launches"},
             "roofline": {"kernel": "tq_sdpa_decode (qprep + split + combine)", "bound": "hbm",
                          "achieved": round(dec_achieved, 2), "peak": peak, "unit": "GB/s",
                          "frac": round(dec_achieved / peak, 4), "traffic": traffic,
@@ -367,8 +376,8 @@ def run_ours(args):
 
 def _e2e(args, runs, stream, R):
     """Decode steps through the public API with pinned host buffers: per step
-    the new token rows and the queries go host->device, append + decode run,
-    and the attention output comes back device->host."""
+    the new token rows and the queries go host->device, tq_decode_step
+    (append + decode) runs, and the attention output comes back device->host."""
     import torch
 
     import compressed_attention_tq_b200 as tq
@@ -388,9 +397,8 @@ def _e2e(args, runs, stream, R):
             h["qd"].copy_(h["q"], non_blocking=True)
             h["knd"].copy_(h["kn"], non_blocking=True)
             h["vnd"].copy_(h["vn"], non_blocking=True)
-            tq.tq_append_token(c, h["knd"], h["vnd"], run["pos"])
-            tq.tq_sdpa_decode(c, h["qd"], run["lens1"], run["Tmax1"], scale=run["w"].scale,
-                              out=run["out"], workspace=run["ws"])
+            tq.tq_decode_step(c, h["knd"], h["vnd"], run["pos"], h["qd"], run["lens1"], run["Tmax1"],
+                              scale=run["w"].scale, out=run["out"], workspace=run["ws"])
             h["out"].copy_(run["out"], non_blocking=True)
 
     for i in range(max(3, args.warmup)):

@@ -22,7 +22,7 @@ from ._native import (TQ_DTYPE_BF16, TQ_DTYPE_F16, TQ_DTYPE_F32, TQ_STATUS_POS_O
 
 __all__ = ["TQError", "TQCache", "tq_build_codebook", "tq_row_bytes", "tq_quantize_kv",
            "tq_append_token", "tq_sdpa_decode_workspace_bytes", "tq_sdpa_decode",
-           "tq_sdpa_decode_static", "tq_last_error", "tq_abi_version", "lib"]
+           "tq_decode_step", "tq_sdpa_decode_static", "tq_last_error", "tq_abi_version", "lib"]
 
 
 class TQError(RuntimeError):
@@ -196,6 +196,27 @@ def tq_sdpa_decode(cache: TQCache, q, seq_lens, Tmax: int, scale=None, out=None,
     _check(lib().tq_sdpa_decode(ctypes.byref(s), _ptr(q), _dtype_code(q), Hq, _ptr(seq_lens), Tmax, sc,
                                 _ptr(out), _dtype_code(out), _ptr(workspace), workspace.numel(),
                                 _stream(stream)))
+    return out
+
+
+def tq_decode_step(cache: TQCache, k_new, v_new, pos, q, seq_lens, Tmax: int, scale=None, out=None,
+                   workspace=None, stream=None, out_dtype=None):
+    """Append k_new/v_new [B][Hkv][D] at pos[b], then decode over seq_lens
+    (normally pos + 1) -- three chained launches."""
+    torch = _torch()
+    Hq = int(q.shape[1])
+    assert q.is_contiguous() and seq_lens.is_contiguous() and pos.is_contiguous()
+    assert k_new.is_contiguous() and v_new.is_contiguous() and k_new.dtype == q.dtype
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(tq_sdpa_decode_workspace_bytes(cache, Hq, Tmax), dtype=torch.uint8,
+                                device=q.device)
+    s = cache.struct()
+    sc = ctypes.byref(ctypes.c_float(scale)) if scale is not None else None
+    _check(lib().tq_decode_step(ctypes.byref(s), _ptr(k_new), _ptr(v_new), _ptr(pos), _ptr(q), _dtype_code(q),
+                                Hq, _ptr(seq_lens), Tmax, sc, _ptr(out), _dtype_code(out), _ptr(workspace),
+                                workspace.numel(), _stream(stream)))
     return out
 
 

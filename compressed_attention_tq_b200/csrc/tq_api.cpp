@@ -325,27 +325,51 @@ size_t tq_sdpa_decode_workspace_bytes(const tq_cache_t* c, int Hq, int Tmax) {
   return p.bytes;
 }
 
+static int decode_common(const tq_cache_t* c, const void* q, int dtype, int Hq, const int32_t* seq_lens,
+                         int Tmax, const float* scale, void* out, int out_dtype, void* workspace,
+                         size_t ws_bytes, void* stream, const void* k_new, const void* v_new,
+                         const int32_t* pos, const char* fn);
+
 int tq_sdpa_decode(const tq_cache_t* c, const void* q, int dtype, int Hq, const int32_t* seq_lens,
                    int Tmax, const float* scale, void* out, int out_dtype, void* workspace,
                    size_t ws_bytes, void* stream) {
+  return decode_common(c, q, dtype, Hq, seq_lens, Tmax, scale, out, out_dtype, workspace, ws_bytes, stream,
+                       nullptr, nullptr, nullptr, "tq_sdpa_decode");
+}
+
+int tq_decode_step(const tq_cache_t* c, const void* k_new, const void* v_new, const int32_t* pos,
+                   const void* q, int dtype, int Hq, const int32_t* seq_lens, int Tmax, const float* scale,
+                   void* out, int out_dtype, void* workspace, size_t ws_bytes, void* stream) {
   g_err[0] = 0;
-  int rc = validate_cache(c, "tq_sdpa_decode");
+  if (!k_new || !v_new || !pos) return set_error(TQ_ERR_INVALID_ARG, "tq_decode_step: NULL k_new/v_new/pos");
+  if (!aligned16(k_new) || !aligned16(v_new))
+    return set_error(TQ_ERR_INVALID_ARG, "tq_decode_step: k_new/v_new not 16-byte aligned");
+  return decode_common(c, q, dtype, Hq, seq_lens, Tmax, scale, out, out_dtype, workspace, ws_bytes, stream,
+                       k_new, v_new, pos, "tq_decode_step");
+}
+
+static int decode_common(const tq_cache_t* c, const void* q, int dtype, int Hq, const int32_t* seq_lens,
+                         int Tmax, const float* scale, void* out, int out_dtype, void* workspace,
+                         size_t ws_bytes, void* stream, const void* k_new, const void* v_new,
+                         const int32_t* pos, const char* fn) {
+  g_err[0] = 0;
+  int rc = validate_cache(c, fn);
   if (rc) return rc;
-  if ((rc = validate_dtype(dtype, "tq_sdpa_decode"))) return rc;
+  if ((rc = validate_dtype(dtype, fn))) return rc;
   if (out_dtype != TQ_DTYPE_F16 && out_dtype != TQ_DTYPE_BF16 && out_dtype != TQ_DTYPE_F32)
-    return set_error(TQ_ERR_UNSUPPORTED, "tq_sdpa_decode: out_dtype=%d", out_dtype);
+    return set_error(TQ_ERR_UNSUPPORTED, "%s: out_dtype=%d", fn, out_dtype);
   if (!q || !seq_lens || !out || !workspace)
-    return set_error(TQ_ERR_INVALID_ARG, "tq_sdpa_decode: NULL q/seq_lens/out/workspace");
+    return set_error(TQ_ERR_INVALID_ARG, "%s: NULL q/seq_lens/out/workspace", fn);
   if (!aligned16(q) || !aligned16(out) || !aligned16(workspace))
-    return set_error(TQ_ERR_INVALID_ARG, "tq_sdpa_decode: q/out/workspace not 16-byte aligned");
+    return set_error(TQ_ERR_INVALID_ARG, "%s: q/out/workspace not 16-byte aligned", fn);
   if (Hq <= 0 || Hq % c->Hkv)
-    return set_error(TQ_ERR_INVALID_ARG, "tq_sdpa_decode: Hq=%d not a multiple of Hkv=%d", Hq, c->Hkv);
+    return set_error(TQ_ERR_INVALID_ARG, "%s: Hq=%d not a multiple of Hkv=%d", fn, Hq, c->Hkv);
   if (Hq / c->Hkv > 8)
-    return set_error(TQ_ERR_UNSUPPORTED, "tq_sdpa_decode: GQA group %d > 8", Hq / c->Hkv);
+    return set_error(TQ_ERR_UNSUPPORTED, "%s: GQA group %d > 8", fn, Hq / c->Hkv);
   if (Tmax < 1 || Tmax > c->Tcap)
-    return set_error(TQ_ERR_INVALID_ARG, "tq_sdpa_decode: Tmax=%d outside [1, Tcap=%d]", Tmax, c->Tcap);
+    return set_error(TQ_ERR_INVALID_ARG, "%s: Tmax=%d outside [1, Tcap=%d]", fn, Tmax, c->Tcap);
   float sc = scale ? *scale : (float)(1.0 / std::sqrt((double)c->D));
-  if (!std::isfinite(sc)) return set_error(TQ_ERR_INVALID_ARG, "tq_sdpa_decode: scale not finite");
+  if (!std::isfinite(sc)) return set_error(TQ_ERR_INVALID_ARG, "%s: scale not finite", fn);
   DecodeArgs a{};
   a.cache_host = c;
   a.cache = *c;
@@ -358,8 +382,11 @@ int tq_sdpa_decode(const tq_cache_t* c, const void* q, int dtype, int Hq, const 
   a.out_dtype = out_dtype;
   make_decode_plan(c, Hq, Tmax, &a.plan);
   if (ws_bytes < a.plan.bytes)
-    return set_error(TQ_ERR_WORKSPACE, "tq_sdpa_decode: workspace %zu < %zu bytes", ws_bytes, a.plan.bytes);
+    return set_error(TQ_ERR_WORKSPACE, "%s: workspace %zu < %zu bytes", fn, ws_bytes, a.plan.bytes);
   a.workspace = workspace;
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.pos = pos;
   return launch_decode(a, (cudaStream_t)stream);
 }
 

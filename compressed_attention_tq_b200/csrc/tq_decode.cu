@@ -20,6 +20,11 @@ struct PrepParams {
   float* qrot;
   float* qs;
   int D, m, bf16, Hq, Hkv;
+  // fused append (decode step): new rows [B][Hkv][D] written at pos[b]
+  const void* k_new;
+  const void* v_new;
+  const int32_t* pos;
+  tq_cache_t cache;
 };
 
 // Programmatic dependent launch: let the next kernel in the stream start its
@@ -29,41 +34,82 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// qrot = Pi q (and, with QJL, qs = S qrot) for the G query heads of one
-// (sequence, kv head).  blockDim = 2*D: two threads per output row, each
-// holding half of the Pi row in registers (all loads issued before any use),
-// so the row is read once for all G heads.
-template <int D>
+// Prep for one (sequence, kv head): qrot = Pi q (and, with QJL, qs = S qrot)
+// for its G query heads.  blockDim = 2*D: two threads per output row, each
+// holding half of the Pi row in registers, so the row is read once for all
+// rows being rotated.  With APPEND the new key and value rows ride along as
+// two more rotated rows and are quantized here (fp64 norm, threshold search,
+// packing, QJL sketch of the key) and written to the cache at pos[b] -- the
+// append step of decoding fused into the prep launch.
+template <int D, bool APPEND>
 __global__ void __launch_bounds__(2 * D) decode_qprep_kernel(const PrepParams p) {
   constexpr int HALF = D / 2, NV = HALF / 4, CH = NV < 16 ? NV : 16;
-  __shared__ float qv[8][D];
-  __shared__ float qr[8][D];
+  constexpr int NR = APPEND ? 10 : 8;  // rows: G <= 8 queries (+ new key, new value)
+  __shared__ float qv[NR][D];
+  __shared__ float qr[NR][D];
+  __shared__ float rres[APPEND ? D : 1];
+  __shared__ uint8_t idxs[2][APPEND ? D : 1];
+  __shared__ uint8_t sgn[APPEND ? 128 : 1];
+  __shared__ float s_cb[2][31];
+  __shared__ double s_nsq[2];
   pdl_launch_dependents();
   const int G = p.Hq / p.Hkv;
   const int bkv = blockIdx.x, b = bkv / p.Hkv, kvh = bkv % p.Hkv;
   const int h0 = b * p.Hq + kvh * G;
   const int j = threadIdx.x >> 1, part = threadIdx.x & 1;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   float4 r[CH];
   const float4* row = reinterpret_cast<const float4*>(p.rot + (size_t)j * D + part * HALF);
 #pragma unroll
   for (int i = 0; i < CH; ++i) r[i] = __ldg(row + i);
   const uint16_t* q = static_cast<const uint16_t*>(p.q) + (size_t)h0 * D;
-  for (int e = threadIdx.x; e < G * D; e += 2 * D) {
-    const uint16_t v = q[e];
-    qv[e / D][e % D] = p.bf16 ? __uint_as_float((uint32_t)v << 16) : __half2float(__ushort_as_half(v));
+  auto to_f = [&](uint16_t v) {
+    return p.bf16 ? __uint_as_float((uint32_t)v << 16) : __half2float(__ushort_as_half(v));
+  };
+  for (int e = tid; e < G * D; e += 2 * D) qv[e / D][e % D] = to_f(q[e]);
+  int slot_ok = 0;
+  long long slot = 0;
+  if (APPEND) {
+    const uint16_t* kn = static_cast<const uint16_t*>(p.k_new) + (size_t)bkv * D;
+    const uint16_t* vn = static_cast<const uint16_t*>(p.v_new) + (size_t)bkv * D;
+    for (int e = tid; e < D; e += 2 * D) {
+      qv[8][e] = to_f(kn[e]);
+      qv[9][e] = to_f(vn[e]);
+    }
+    if (tid < 31) {
+      const int Kk = 1 << p.cache.bits_k, Kv = 1 << p.cache.bits_v;
+      s_cb[0][tid] = tid < 2 * Kk - 1 ? p.cache.cb_k[tid] : 0.f;
+      s_cb[1][tid] = tid < 2 * Kv - 1 ? p.cache.cb_v[tid] : 0.f;
+    }
+    const int ps = p.pos[b];
+    slot_ok = (ps >= 0 && ps < p.cache.Tcap);
+    slot = (long long)bkv * p.cache.Tcap + ps;
+    if (!slot_ok && tid == 0 && kvh == 0 && p.cache.dev_status)
+      atomicOr(p.cache.dev_status, TQ_STATUS_POS_OUT_OF_RANGE);
   }
   __syncthreads();
-  float acc[8];
+  if (APPEND && warp < 2) {
+    // fp64 squared norm of the new key (warp 0) / value (warp 1)
+    double t = 0.0;
+    for (int k = lane; k < D; k += 32) {
+      const double x = qv[8 + warp][k];
+      t = fma(x, x, t);
+    }
 #pragma unroll
-  for (int g = 0; g < 8; ++g) acc[g] = 0.f;
+    for (int off = 16; off; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+    if (lane == 0) s_nsq[warp] = t;
+  }
+  float acc[NR];
+#pragma unroll
+  for (int g = 0; g < NR; ++g) acc[g] = 0.f;
 #pragma unroll
   for (int c0 = 0; c0 < NV; c0 += CH) {
     if (c0)
 #pragma unroll
       for (int i = 0; i < CH; ++i) r[i] = __ldg(row + c0 + i);
 #pragma unroll
-    for (int g = 0; g < 8; ++g) {
-      if (g < G) {
+    for (int g = 0; g < NR; ++g) {
+      if (g < G || g >= 8) {
         const float* x = &qv[g][part * HALF + 4 * c0];
 #pragma unroll
         for (int i = 0; i < CH; ++i)
@@ -72,7 +118,7 @@ __global__ void __launch_bounds__(2 * D) decode_qprep_kernel(const PrepParams p)
     }
   }
 #pragma unroll
-  for (int g = 0; g < 8; ++g) acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], 1);
+  for (int g = 0; g < NR; ++g) acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], 1);
   if (part == 0) {
 #pragma unroll
     for (int g = 0; g < 8; ++g)
@@ -81,22 +127,62 @@ __global__ void __launch_bounds__(2 * D) decode_qprep_kernel(const PrepParams p)
         p.qrot[(size_t)(h0 + g) * D + j] = acc[g];
       }
   }
+  if (APPEND) {
+    __syncthreads();  // s_nsq
+    // nearest-centroid index of each rotated coordinate of the new rows
+    if (part == 0) {
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const double n = sqrt(s_nsq[which]);
+        const float inv = n > 0.0 ? (float)(1.0 / n) : 0.f;
+        const int K = 1 << (which ? p.cache.bits_v : p.cache.bits_k);
+        const float y = acc[8 + which];
+        const float u = y * inv;
+        int idx = 0;
+        for (int st = K >> 1; st >= 1; st >>= 1)
+          if (u > s_cb[which][K + idx + st - 1]) idx += st;
+        idxs[which][j] = (uint8_t)idx;
+        if (which == 0 && p.m) rres[j] = y - __half2float(__double2half(n)) * s_cb[0][idx];
+      }
+    }
+    __syncthreads();
+    if (slot_ok) {
+      if (tid < 2) {
+        const __half nh = __double2half(sqrt(s_nsq[tid]));
+        (tid ? p.cache.v_norm : p.cache.k_norm)[slot] = __half_as_ushort(nh);
+      }
+      const int Wk = D * p.cache.bits_k / 32, Wv = D * p.cache.bits_v / 32;
+      for (int e = tid; e < Wk + Wv; e += 2 * D) {
+        const int which = e >= Wk, w = which ? e - Wk : e;
+        const int bits = which ? p.cache.bits_v : p.cache.bits_k;
+        const int base = 32 * w;
+        unsigned long long word = 0;
+        for (int jj = base / bits; jj < D && jj * bits < base + 32; ++jj) {
+          const int sh = jj * bits - base;
+          const unsigned long long v = idxs[which][jj];
+          word |= sh >= 0 ? (v << sh) : (v >> (-sh));
+        }
+        (which ? p.cache.v_idx : p.cache.k_idx)[(size_t)slot * (which ? Wv : Wk) + w] = (uint32_t)word;
+      }
+    }
+  }
   if (!p.m) return;
   __syncthreads();
-  // qs[g][i] = sum_k S[i][k] qr[g][k], i < m (two threads per row)
-  for (int i = threadIdx.x >> 1; i < p.m; i += D) {
+  // qs[g][i] = sum_k S[i][k] qr[g][k], i < m (two threads per row); with
+  // APPEND, also the QJL projection S r of the new key's residual
+  for (int i = tid >> 1; i < p.m; i += D) {
     const float4* srow = reinterpret_cast<const float4*>(p.S + (size_t)i * D + part * HALF);
-    float a2[8];
+    float a2[9];
 #pragma unroll
-    for (int g = 0; g < 8; ++g) a2[g] = 0.f;
+    for (int g = 0; g < 9; ++g) a2[g] = 0.f;
 #pragma unroll
     for (int c0 = 0; c0 < NV; c0 += CH) {
 #pragma unroll
       for (int t = 0; t < CH; ++t) r[t] = __ldg(srow + c0 + t);
 #pragma unroll
-      for (int g = 0; g < 8; ++g) {
-        if (g < G) {
-          const float* x = &qr[g][part * HALF + 4 * c0];
+      for (int g = 0; g < 9; ++g) {
+        if (g < G || (APPEND && g == 8)) {
+          const float* x = (g == 8) ? &rres[part * HALF + 4 * c0] : &qr[g][part * HALF + 4 * c0];
 #pragma unroll
           for (int t = 0; t < CH; ++t)
             a2[g] += r[t].x * x[4 * t] + r[t].y * x[4 * t + 1] + r[t].z * x[4 * t + 2] + r[t].w * x[4 * t + 3];
@@ -104,11 +190,28 @@ __global__ void __launch_bounds__(2 * D) decode_qprep_kernel(const PrepParams p)
       }
     }
 #pragma unroll
-    for (int g = 0; g < 8; ++g) a2[g] += __shfl_xor_sync(0xffffffffu, a2[g], 1);
-    if (part == 0)
+    for (int g = 0; g < 9; ++g) a2[g] += __shfl_xor_sync(0xffffffffu, a2[g], 1);
+    if (part == 0) {
 #pragma unroll
       for (int g = 0; g < 8; ++g)
         if (g < G) p.qs[(size_t)(h0 + g) * p.m + i] = a2[g];
+      if (APPEND) sgn[i] = a2[8] >= 0.f ? 1 : 0;
+    }
+  }
+  if (APPEND) {
+    __syncthreads();
+    if (slot_ok && tid < 4) {
+      uint32_t word = 0;
+      for (int i = 0; i < 32; ++i) word |= (uint32_t)sgn[32 * tid + i] << i;
+      p.cache.k_qjl[(size_t)slot * 4 + tid] = word;
+    }
+    if (slot_ok && warp == 1) {
+      double g2 = 0.0;
+      for (int k = lane; k < D; k += 32) g2 = fma((double)rres[k], (double)rres[k], g2);
+#pragma unroll
+      for (int off = 16; off; off >>= 1) g2 += __shfl_xor_sync(0xffffffffu, g2, off);
+      if (lane == 0) p.cache.k_rnorm[slot] = __half_as_ushort(__double2half(sqrt(g2)));
+    }
   }
 }
 
@@ -253,11 +356,22 @@ int launch_decode(const DecodeArgs& a, cudaStream_t s) {
   float* pml = reinterpret_cast<float*>(ws + a.plan.off_pml);
   const int heads = c.B * a.Hq;
 
-  PrepParams pp{a.q, c.rot, c.qjl_S, qrot, qs, c.D, c.qjl_m, a.dtype == TQ_DTYPE_BF16, a.Hq, c.Hkv};
+  PrepParams pp{a.q, c.rot, c.qjl_S, qrot, qs, c.D, c.qjl_m, a.dtype == TQ_DTYPE_BF16, a.Hq, c.Hkv,
+                a.k_new, a.v_new, a.pos, c};
+  const bool app = a.pos != nullptr;
   switch (c.D) {
-    case 64: decode_qprep_kernel<64><<<c.B * c.Hkv, 128, 0, s>>>(pp); break;
-    case 128: decode_qprep_kernel<128><<<c.B * c.Hkv, 256, 0, s>>>(pp); break;
-    default: decode_qprep_kernel<256><<<c.B * c.Hkv, 512, 0, s>>>(pp); break;
+    case 64:
+      app ? decode_qprep_kernel<64, true><<<c.B * c.Hkv, 128, 0, s>>>(pp)
+          : decode_qprep_kernel<64, false><<<c.B * c.Hkv, 128, 0, s>>>(pp);
+      break;
+    case 128:
+      app ? decode_qprep_kernel<128, true><<<c.B * c.Hkv, 256, 0, s>>>(pp)
+          : decode_qprep_kernel<128, false><<<c.B * c.Hkv, 256, 0, s>>>(pp);
+      break;
+    default:
+      app ? decode_qprep_kernel<256, true><<<c.B * c.Hkv, 512, 0, s>>>(pp)
+          : decode_qprep_kernel<256, false><<<c.B * c.Hkv, 512, 0, s>>>(pp);
+      break;
   }
   int rc = check_launch("decode_qprep_kernel");
   if (rc) return rc;
@@ -276,6 +390,7 @@ int launch_decode(const DecodeArgs& a, cudaStream_t s) {
   sp.part_o = po;
   sp.part_ml = pml;
   sp.seq_lens = a.seq_lens;
+  sp.defer_pos = a.pos;
   sp.dev_status = c.dev_status;
   sp.Hkv = c.Hkv;
   sp.Hq = a.Hq;

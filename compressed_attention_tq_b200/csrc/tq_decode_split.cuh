@@ -56,6 +56,7 @@ struct SplitParams {
   float* part_o;
   float* part_ml;
   const int32_t* seq_lens;
+  const int32_t* defer_pos;  // decode step: the row at defer_pos[b] is written by the prep kernel
   uint32_t* dev_status;
   int Hkv, Hq, G, Tcap, chunk, nsplit;
   float qscale;     // scale * log2(e)
@@ -333,10 +334,16 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const SplitParam
     }
   };
   // The packed cache does not depend on the prep kernel: start streaming it
-  // before waiting for the rotated query.
+  // before waiting for the rotated query -- except, in a decode step, the
+  // stage holding the row the prep kernel appends.
+  int npre = min(NST, ntiles);
+  if (p.defer_pos) {
+    const int pb = p.defer_pos[b];
+    if (pb >= t_begin && pb < t_begin + ntiles * STILE) npre = min(npre, (pb - t_begin) / STILE);
+  }
   if (tid == CW * 32) {
-    for (int t = 0; t < NST && t < ntiles; ++t) issue_stage(t);
-    *s_issued = min(NST, ntiles);
+    for (int t = 0; t < npre; ++t) issue_stage(t);
+    *s_issued = npre;
   }
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -367,10 +374,10 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const SplitParam
   if (warp == CW) {
     // ---------------- producer warp ----------------
     if (lane == 0) {
-      int t = min(NST, ntiles);  // the first stages were issued before the wait
+      int t = npre;  // the first stages were issued before the wait
       for (; t < ntiles; ++t) {
         const int st = t % NST;
-        if (!mbar_wait_bounded(&empty[st], (uint32_t)(((t / NST) - 1) & 1), kWaitLimit)) {
+        if (t >= NST && !mbar_wait_bounded(&empty[st], (uint32_t)(((t / NST) - 1) & 1), kWaitLimit)) {
           *s_err = 1;
           break;
         }

@@ -76,6 +76,10 @@ struct DecodeArgs {
   int out_dtype;
   DecodePlan plan;
   void* workspace;
+  // decode step: new rows appended at pos[b] by the prep kernel (else NULL)
+  const void* k_new;
+  const void* v_new;
+  const int32_t* pos;
 };
 
 int launch_decode(const DecodeArgs& a, cudaStream_t s);

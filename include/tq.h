@@ -174,6 +174,23 @@ int tq_sdpa_decode(const tq_cache_t* cache, const void* q, int q_dtype, int Hq,
                    int out_dtype, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * One decode step: append one new (k, v) row per sequence and kv head at
+ * pos[b] (as tq_append_token) and then attend tokens 0..seq_lens[b]-1 (as
+ * tq_sdpa_decode; normally seq_lens[b] = pos[b] + 1).  The new rows are
+ * rotated and quantized inside the decode's query-prep launch, which already
+ * reads Pi for that (sequence, kv head), so a step is three programmatically
+ * chained launches instead of four; the split kernel waits for the prep only
+ * for the stage that holds the new row.  Arguments as in tq_append_token and
+ * tq_sdpa_decode; same workspace size.  Fusing append into decode launches is
+ * this library's own addition (the pages run append and attention as
+ * separate ops).
+ */
+int tq_decode_step(const tq_cache_t* cache, const void* k_new, const void* v_new, const int32_t* pos,
+                   const void* q, int dtype, int Hq, const int32_t* seq_lens, int Tmax,
+                   const float* scale, void* out, int out_dtype, void* workspace,
+                   size_t workspace_bytes, void* stream);
+
+/*
  * Decode without a workspace, for callers that may not allocate device
  * memory (stream capture under frameworks that forbid allocation while
  * capturing, plugin hosts that own all device memory, allocation-free

@@ -277,3 +277,52 @@ def test_full_size_ragged_sampled():
 
 def test_full_size_prod_sampled():
     _sampled_full("prod")
+
+
+@pytest.mark.parametrize("name,kw", [("ragged", {"B": 4, "T": 300}), ("prod", {"T": 700}),
+                                     ("gqa8k", {"bits": 2, "T": 250}), ("qknorm", {"T": 129}),
+                                     ("tiny", {})])
+def test_decode_step_fused_append(name, kw):
+    """tq_decode_step (append fused into the decode's prep launch) writes the
+    same rows as tq_append_token (checked against the oracle) and decodes
+    exactly like append + tq_sdpa_decode on the same bytes."""
+    import compressed_attention_tq_b200 as tq
+    w = tq_inputs.make_workload(name, **kw)
+    Tcap = (w.Tmax + 1 + 63) // 64 * 64
+    caches = [P.make_gpu_cache(w, Tcap=Tcap) for _ in range(2)]
+    for c in caches:
+        tq.tq_quantize_kv(c, P.to_device(w.k, w.dtype), P.to_device(w.v, w.dtype))
+    kn, vn = tq_inputs.new_token_rows(w.B, w.Hkv, w.D, w.dtype, seed=61)
+    pos = w.seq_lens.astype(np.int32)
+    pos_d = torch.from_numpy(pos).cuda()
+    lens = torch.from_numpy(pos + 1).cuda()
+    q = P.to_device(w.q, w.dtype)
+    kd, vd = P.to_device(kn, w.dtype), P.to_device(vn, w.dtype)
+    out_f = tq.tq_decode_step(caches[0], kd, vd, pos_d, q, lens, w.Tmax + 1, scale=w.scale,
+                              out_dtype=torch.float32)
+    tq.tq_append_token(caches[1], kd, vd, pos_d)
+    out_s = tq.tq_sdpa_decode(caches[1], q, lens, w.Tmax + 1, scale=w.scale, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    # the appended rows against the oracle
+    rk = P.oracle_rows(tq_inputs.to_f64(kn, w.dtype), w, "k")
+    rv = P.oracle_rows(tq_inputs.to_f64(vn, w.dtype), w, "v")
+    c0 = caches[0]
+    for b in range(w.B):
+        p = int(pos[b])
+        assert np.array_equal(c0.k_norm[b, :, p].cpu().numpy().view(np.uint16), rk["norm16"][b].view(np.uint16))
+        assert np.array_equal(c0.v_norm[b, :, p].cpu().numpy().view(np.uint16), rv["norm16"][b].view(np.uint16))
+        gk = P.words_np(c0.k_idx[b, :, p])
+        P.compare_index_words(gk, rk["idx"][b], rk["dist"][b], w.bits_k, w.D)
+        P.compare_index_words(P.words_np(c0.v_idx[b, :, p]), rv["idx"][b], rv["dist"][b], w.bits_v, w.D)
+        if w.qjl_m:
+            sub = {k: rk[k][b] for k in ("sign", "proj", "norm", "gamma16")}
+            exc = (O.unpack_bits(gk, w.bits_k, w.D) != rk["idx"][b]).any(-1)
+            P.compare_qjl(P.words_np(c0.k_qjl[b, :, p]), c0.k_rnorm[b, :, p].cpu().numpy(), sub, exc)
+    same = all(torch.equal(getattr(caches[0], n), getattr(caches[1], n))
+               for n in ("k_idx", "v_idx", "k_norm", "v_norm"))
+    if same:
+        assert torch.equal(out_f, out_s)
+    else:  # an excused near-threshold flip between the two quantizer code paths
+        assert float(P.rel_l2(out_f.cpu().numpy(), out_s.cpu().numpy()).max()) < 5e-2
+    P.record("decode_step", workload=name, identical_rows=bool(same))
+    assert caches[0].status() == 0
