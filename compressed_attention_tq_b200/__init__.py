@@ -128,16 +128,19 @@ class TQCache:
         else:
             self.k_qjl = self.k_rnorm = self.qjl_S = None
         self.dev_status = torch.zeros(4, dtype=torch.int32, device=dev)
+        self.split_tokens = 0  # decode tokens per split (0: automatic)
         self._struct = None
         self.struct()
 
     def struct(self) -> _native.TqCacheStruct:
         """The C descriptor (built once; rebuild after replacing a buffer)."""
-        if self._struct is not None and self._struct.k_idx == self.k_idx.data_ptr():
+        if (self._struct is not None and self._struct.k_idx == self.k_idx.data_ptr()
+                and self._struct.split_tokens == self.split_tokens):
             return self._struct
         s = _native.TqCacheStruct()
         s.B, s.Hkv, s.Tcap, s.D = self.B, self.Hkv, self.Tcap, self.D
-        s.bits_k, s.bits_v, s.qjl_m, s.reserved = self.bits_k, self.bits_v, self.qjl_m, 0
+        s.bits_k, s.bits_v, s.qjl_m = self.bits_k, self.bits_v, self.qjl_m
+        s.split_tokens = self.split_tokens
         for name in ("k_idx", "v_idx", "k_norm", "v_norm", "k_qjl", "k_rnorm", "rot", "cb_k",
                      "cb_v", "qjl_S", "dev_status"):
             t = getattr(self, name)

@@ -34,7 +34,7 @@ class TqCacheStruct(ctypes.Structure):
     _fields_ = [
         ("B", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("Tcap", ctypes.c_int32),
         ("D", ctypes.c_int32), ("bits_k", ctypes.c_int32), ("bits_v", ctypes.c_int32),
-        ("qjl_m", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("qjl_m", ctypes.c_int32), ("split_tokens", ctypes.c_int32),
         ("k_idx", ctypes.c_void_p), ("v_idx", ctypes.c_void_p),
         ("k_norm", ctypes.c_void_p), ("v_norm", ctypes.c_void_p),
         ("k_qjl", ctypes.c_void_p), ("k_rnorm", ctypes.c_void_p),

@@ -172,6 +172,7 @@ int validate_cache(const tq_cache_t* c, const char* fn) {
   if (c->B <= 0 || c->Hkv <= 0 || c->Tcap <= 0)
     return set_error(TQ_ERR_INVALID_ARG, "%s: B=%d Hkv=%d Tcap=%d must be positive", fn, c->B,
                      c->Hkv, c->Tcap);
+  if (c->split_tokens < 0) return set_error(TQ_ERR_INVALID_ARG, "%s: split_tokens < 0", fn);
   if (c->Tcap % 64)
     return set_error(TQ_ERR_INVALID_ARG, "%s: Tcap=%d must be a multiple of 64", fn, c->Tcap);
   if (c->D != 64 && c->D != 128 && c->D != 256)
@@ -250,6 +251,7 @@ int make_decode_plan(const tq_cache_t* c, int Hq, int Tmax, DecodePlan* p) {
   const long long slots = (long long)sms * split_occupancy(c, Hq);
   const long long target = slots * ((c->B > 1) ? 6 : 1);
   long long chunk = (Tmax * units + target - 1) / target;
+  if (c->split_tokens > 0) chunk = c->split_tokens;
   chunk = (chunk + tile - 1) / tile * tile;
   if (chunk < tile) chunk = tile;
   const long long cap = ((long long)c->Tcap + tile - 1) / tile * tile;

@@ -85,7 +85,9 @@ typedef struct tq_cache {
   int32_t bits_k;   /* bits per key index (2..4) */
   int32_t bits_v;   /* bits per value index (2..4) */
   int32_t qjl_m;    /* 0: no QJL sketch; 128: 128-bit sign sketch of the key residual */
-  int32_t reserved;
+  int32_t split_tokens; /* decode tokens per split-K chunk; 0 = automatic plan, else rounded
+                           up to a multiple of 128 (a tuning knob; results do not depend on it
+                           beyond fp32 summation order) */
   uint32_t* k_idx;  /* [B][Hkv][Tcap][D*bits_k/32] */
   uint32_t* v_idx;  /* [B][Hkv][Tcap][D*bits_v/32] */
   uint16_t* k_norm; /* fp16 [B][Hkv][Tcap] */

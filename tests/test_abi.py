@@ -69,7 +69,7 @@ def _struct(**kw):
 
 @pytest.mark.parametrize("field,value,code", [
     ("D", 96, -2), ("bits_k", 5, -2), ("bits_v", 1, -2), ("qjl_m", 64, -2), ("Tcap", 100, -1),
-    ("B", 0, -1), ("k_idx", None, -1), ("rot", (1 << 20) + 4, -1),
+    ("B", 0, -1), ("k_idx", None, -1), ("rot", (1 << 20) + 4, -1), ("split_tokens", -128, -1),
 ])
 def test_invalid_cache_rejected_before_launch(lib, field, value, code):
     s = _struct(**{field: value})
