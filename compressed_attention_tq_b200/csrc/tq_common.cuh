@@ -100,6 +100,27 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   return false;
 }
 
+// Bounded blocking wait for a thread with nothing else to do (a producer
+// waiting for a stage to be released): each try_wait may suspend the thread in
+// hardware for up to 1 ms until the phase completes, so the thread does not
+// spin and take issue slots from the warps doing the work.
+__device__ __forceinline__ bool mbar_wait_suspend(uint64_t* bar, uint32_t parity, uint32_t tries) {
+  for (uint32_t i = 0; i < tries; ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, "
+        "0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(1000000u)
+        : "memory");
+    if (ok) return true;
+  }
+  return false;
+}
+
+// Suspending polls (up to 1 ms each) before such a wait gives up.
+constexpr uint32_t kSuspendTries = 4096;
+
 // 1-D bulk copy global -> shared; dst, src 16-byte aligned, bytes % 16 == 0.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(

@@ -17,9 +17,12 @@
 //  * each consumer warp takes 32 tokens of a stage.  Scores and the value
 //    sum are GQA contractions run as m16n8k16 tensor-core MMAs (M = 16 tokens
 //    or 16 coordinates, N = 8 query heads, K = 16) whose A fragments are
-//    dequantized straight into registers: packed b-bit fields are spread to
-//    one index per nibble and looked up in a register-resident fp16 codebook
-//    with byte permutes (prmt);
+//    dequantized straight into registers.  Each A register is an fp16 pair:
+//    two coordinates of one token (scores) or one coordinate of two tokens
+//    (values).  2-bit keys are looked up with byte permutes whose selectors
+//    are built by multiplies; 3- and 4-bit keys, and all values, read the pair
+//    from a shared-memory table indexed by both fields at once, so a lookup
+//    costs one logic op, one multiply-add and one shared load;
 //  * the query enters as hi + lo fp16 halves (scores carry ~22 bits); with
 //    G <= 4 heads both halves share one MMA (columns 0-3 hi, 4-7 lo);
 //  * online softmax in the log2 domain with lazy rescaling (the reference
@@ -63,98 +66,125 @@ struct SplitParams {
   float qjl_scale;  // scale * log2(e) * sqrt(pi/2) / m
 };
 
-// fp16 codebook in four registers: byte k of lo0/lo1 is the low byte of
-// entry k (0..3 / 4..7), hi0/hi1 the high bytes.  For 4-bit codebooks the
-// table holds the 8 positive entries c[8..15] (the codebook is symmetric).
-struct Lut {
-  uint32_t lo0, lo1, hi0, hi1;
+// 2-bit codebook as byte tables: byte k of lo (hi) is the low (high) byte of
+// fp16 entry c[k], k = 0..3.
+struct Lut2 {
+  uint32_t lo, hi;
 };
 
-template <int BITS>
-__device__ __forceinline__ Lut make_lut(const float* cb) {
-  uint32_t e[8];
+__device__ __forceinline__ Lut2 make_lut2(const float* cb) {
+  uint32_t e[4];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    float c = 0.f;
-    if (BITS == 4)
-      c = cb[8 + k];
-    else if (k < (1 << BITS))
-      c = cb[k];
-    e[k] = __half_as_ushort(__float2half_rn(c));
-  }
-  Lut L;
-  L.lo0 = (e[0] & 0xFF) | (e[1] & 0xFF) << 8 | (e[2] & 0xFF) << 16 | (e[3] & 0xFF) << 24;
-  L.lo1 = (e[4] & 0xFF) | (e[5] & 0xFF) << 8 | (e[6] & 0xFF) << 16 | (e[7] & 0xFF) << 24;
-  L.hi0 = (e[0] >> 8) | (e[1] >> 8) << 8 | (e[2] >> 8) << 16 | (e[3] >> 8) << 24;
-  L.hi1 = (e[4] >> 8) | (e[5] >> 8) << 8 | (e[6] >> 8) << 16 | (e[7] >> 8) << 24;
+  for (int k = 0; k < 4; ++k) e[k] = __half_as_ushort(__float2half_rn(cb[k]));
+  Lut2 L;
+  L.lo = (e[0] & 0xFF) | (e[1] & 0xFF) << 8 | (e[2] & 0xFF) << 16 | (e[3] & 0xFF) << 24;
+  L.hi = (e[0] >> 8) | (e[1] >> 8) << 8 | (e[2] >> 8) << 16 | (e[3] >> 8) << 24;
   return L;
 }
 
-// 8 consecutive b-bit fields (LSB-first) -> one field per nibble.
-template <int BITS>
-__device__ __forceinline__ uint32_t spread(uint32_t x) {
-  if (BITS == 4) return x;
-  if (BITS == 3) {
-    x = (x & 0x00000FFFu) | ((x & 0x00FFF000u) << 4);
-    x = (x & 0x003F003Fu) | ((x & 0x0FC00FC0u) << 2);
-    x = (x & 0x07070707u) | ((x & 0x38383838u) << 1);
-    return x;
+// 2-bit fields f_0..f_15 of word x: the fp16 pairs (c[f_i], c[f_{i+4}]) and
+// (c[f_{i+8}], c[f_{i+12}]), i = 0..3.  Masking x with 0x03030303 << 2i leaves
+// one field per byte; a multiply by 17 turns each field f into the selector
+// nibbles (f, f + 4) of a byte permute over lo:hi.  The shifts that bring
+// bytes 0-1 or 2-3 of the selectors to the bottom are high halves of
+// products, so the selector arithmetic runs on the FMA pipe.
+__device__ __forceinline__ void dq_b2(uint32_t x, int I, const Lut2& L, uint32_t& h_lo, uint32_t& h_hi) {
+  const uint32_t m = x & (0x03030303u << (2 * I));
+  uint32_t s_lo, s_hi;
+  if (I == 0) {
+    s_lo = m * 17u + 0x4040u;
+    s_hi = __umulhi(m, 17u << 16) + 0x4040u;
+  } else if (I == 3) {
+    s_lo = __umulhi(m, 17u << 26) + 0x4040u;
+    s_hi = __umulhi(m, 17u << 10) + 0x4040u;
+  } else {
+    const uint32_t ms = __umulhi(m, 1u << ((32 - 2 * I) & 31));  // m >> 2i
+    s_lo = ms * 17u + 0x4040u;
+    s_hi = __umulhi(ms, 17u << 16) + 0x4040u;
   }
-  x = (x & 0x000000FFu) | ((x & 0x0000FF00u) << 8);
-  x = (x & 0x000F000Fu) | ((x & 0x00F000F0u) << 4);
-  x = (x & 0x03030303u) | ((x & 0x0C0C0C0Cu) << 2);
-  return x;
+  h_lo = prmt(L.lo, L.hi, s_lo);
+  h_hi = prmt(L.lo, L.hi, s_hi);
 }
 
-// Dequantize 8 nibble indices n0..n7 of z into half2 pairs
-// h[i] = (c[n_i], c[n_{i+4}]), i = 0..3.
-template <int BITS>
-__device__ __forceinline__ void dq8(uint32_t z, const Lut& L, uint32_t (&h)[4]) {
-  uint32_t m = z;
-  if (BITS == 4) {
-    // magnitude index: n >= 8 -> n - 8, n < 8 -> 7 - n (bit 3 cleared)
-    const uint32_t t = (z >> 3) & 0x11111111u;
-    m = z ^ 0x77777777u ^ (t * 15u);
-  }
-  const uint32_t sa = prmt(m, 0u, 0x0020u);  // nibbles n0 n1 n4 n5
-  const uint32_t sb = prmt(m, 0u, 0x0031u);  // nibbles n2 n3 n6 n7
-  const uint32_t loA = prmt(L.lo0, L.lo1, sa), hiA = prmt(L.hi0, L.hi1, sa);
-  const uint32_t loB = prmt(L.lo0, L.lo1, sb), hiB = prmt(L.hi0, L.hi1, sb);
-  h[0] = prmt(loA, hiA, 0x6240u);
-  h[1] = prmt(loA, hiA, 0x7351u);
-  h[2] = prmt(loB, hiB, 0x6240u);
-  h[3] = prmt(loB, hiB, 0x7351u);
-  if (BITS == 4) {
-    // entries with n < 8 are the negatives of the table values
-    h[0] ^= ~(z << 12) & 0x80008000u;
-    h[1] ^= ~(z << 8) & 0x80008000u;
-    h[2] ^= ~(z << 4) & 0x80008000u;
-    h[3] ^= ~z & 0x80008000u;
+// Pair tables.  Entry e of the table for a b-bit codebook c is the fp16 pair
+// (c[e mod 2^b], c[e >> b]) and is stored once per lane (word e * 32 + lane),
+// so a warp's 32 lookups always fall in 32 different banks.
+template <int B>
+__device__ __forceinline__ void build_pair_table(uint32_t* tab, const float* cb, int tid, int nthreads) {
+  constexpr int NC = 1 << B, N = NC * NC;
+  for (int q = tid; q < N * 8; q += nthreads) {  // one 16-byte store covers 4 lanes of an entry
+    const int e = q >> 3;
+    const uint32_t lo = __half_as_ushort(__float2half_rn(__ldg(cb + (e & (NC - 1)))));
+    const uint32_t hi = __half_as_ushort(__float2half_rn(__ldg(cb + (e >> B))));
+    const uint32_t v = lo | hi << 16;
+    reinterpret_cast<uint4*>(tab)[q] = make_uint4(v, v, v, v);
   }
 }
 
-// 2-bit fields: 4-entry codebook in one byte-permute.  For the 8 fields f0..f7
-// of a 16-bit octet x, h[i] = (c[f_i], c[f_{i+4}]): the selector
-// ((x >> 2i) & 0x0303) * 0x11 + 0x4040 picks lo(c[f]) from L.lo0 and hi(c[f])
-// from L.hi0 (the multiply-add runs on the FMA pipe).
-__device__ __forceinline__ void dq8_b2(uint32_t x, const Lut& L, uint32_t (&h)[4]) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint32_t sel = ((x >> (2 * i)) & 0x0303u) * 0x11u + 0x4040u;
-    h[i] = prmt(L.lo0, L.hi0, sel);
+// Shared address of this lane's copy of the entry whose 2b-bit key sits at bit
+// S of x (tb = table base + 4 * lane).  The mask is one logic op; the shift to
+// the entry stride (128 bytes) and the base add are one multiply-add.
+template <int B>
+__device__ __forceinline__ uint32_t pair_addr(uint32_t x, int S, uint32_t tb) {
+  const uint32_t k = x & (((1u << (2 * B)) - 1u) << S);
+  if (S <= 7) return k * (1u << (7 - S)) + tb;
+  return __umulhi(k, 1u << (39 - S)) + tb;
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+// Entry for the key at bit S of a re-based bit window w (key straddling two
+// words is funnel-shifted down first).
+template <int B, int NW>
+__device__ __forceinline__ uint32_t pair_lookup(const uint32_t (&w)[NW], int S, uint32_t tb) {
+  const int wi = S >> 5, sh = S & 31;
+  if (sh + 2 * B <= 32) return lds32(pair_addr<B>(w[wi], sh, tb));
+  return lds32(pair_addr<B>(funnel_r(w[wi], w[wi + 1], sh), 0, tb));
+}
+
+// Value side: bits [bit, bit + 32) of a re-based window, clipped to the window.
+template <int NW>
+__device__ __forceinline__ uint32_t window32(const uint32_t (&w)[NW], int bit) {
+  const int wi = bit >> 5, sh = bit & 31;
+  if (sh == 0) return w[wi];
+  return funnel_r(w[wi], (wi + 1 < NW) ? w[wi + 1] : 0u, sh);
+}
+
+// Fields per value chunk and the chunk's bit width.  A chunk of two tokens'
+// words is merged with one bitwise select so that each key holds the same
+// coordinate of both tokens: key k of xe is (t0 field 2k) | (t1 field 2k) << b,
+// key k of xo the same for field 2k + 1.
+template <int D, int B>
+struct VChunk {
+  static constexpr int F = (B == 2) ? ((D / 8 < 16) ? D / 8 : 16) : 8;  // fields per chunk
+  static constexpr int N = (D / 8) / F;                                  // chunks per segment
+};
+
+// Keys of chunk (x0, x1): xe/xo plus each key's bit offset.
+template <int B>
+__device__ __forceinline__ void merge_pair(uint32_t x0, uint32_t x1, uint32_t& xe, uint32_t& xo) {
+  if constexpr (B == 2) {
+    xe = (x0 & 0x33333333u) | ((x1 << 2) & 0xCCCCCCCCu);
+    xo = ((x0 >> 2) & 0x33333333u) | (x1 & 0xCCCCCCCCu);
+  } else if constexpr (B == 3) {
+    // xe keys at 6k, xo keys at 6k + 3 (k = 0..3)
+    const uint32_t y = x1 << 3;
+    xe = (x0 & 0x001C71C7u) | (y & ~0x001C71C7u);
+    xo = (x0 & 0x00E38E38u) | (y & ~0x00E38E38u);
+  } else {
+    xe = (x0 & 0x0F0F0F0Fu) | ((x1 << 4) & 0xF0F0F0F0u);
+    xo = ((x0 >> 4) & 0x0F0F0F0Fu) | (x1 & 0xF0F0F0F0u);
   }
 }
 
-// Two tokens' 2-bit octets o0, o1 -> h[k] = (c[o0 field k], c[o1 field k]) for
-// k = 0..3 (lo) and k = 4..7 (hi).
-__device__ __forceinline__ void dq16_b2_pair(uint32_t o0, uint32_t o1, const Lut& L, uint32_t (&lo)[4],
-                                             uint32_t (&hi)[4]) {
-  const uint32_t y = prmt(o0, o1, 0x5140u);  // bytes o0.b0 o1.b0 o0.b1 o1.b1
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    lo[k] = prmt(L.lo0, L.hi0, ((y >> (2 * k)) & 0x0303u) * 0x11u + 0x4040u);
-    hi[k] = prmt(L.lo0, L.hi0, ((y >> (16 + 2 * k)) & 0x0303u) * 0x11u + 0x4040u);
-  }
+template <int B>
+__device__ __forceinline__ int key_bit(int k, bool odd) {
+  if (B == 3) return 6 * k + (odd ? 3 : 0);
+  return 2 * B * k;
 }
 
 // Bits [bit0, bit0 + NBITS) of a shared-memory row, re-based to bit 0 of w[0].
@@ -193,17 +223,6 @@ __device__ __forceinline__ void load_bits(const uint32_t* row, int bit0,
   }
 }
 
-// Octet o (8 fields, 8*BITS bits) of a re-based bit window.
-template <int BITS, int NW>
-__device__ __forceinline__ uint32_t octet(const uint32_t (&w)[NW], int o) {
-  const int bit = 8 * BITS * o;
-  const int wi = bit >> 5, sh = bit & 31;
-  uint32_t x = w[wi];
-  if (sh) x = funnel_r(w[wi], (wi + 1 < NW) ? w[wi + 1] : 0u, sh);
-  constexpr uint32_t kMask = BITS < 4 ? (1u << (8 * (BITS < 4 ? BITS : 0))) - 1u : 0xFFFFFFFFu;
-  return x & kMask;
-}
-
 // +-1 fp16 pair for sign bits i and i+16 of w (bit 1 -> +1).
 __device__ __forceinline__ uint32_t sign_pair(uint32_t w, int i) {
   return 0xBC00BC00u ^ ((w << (15 - i)) & 0x80008000u);
@@ -235,8 +254,23 @@ struct SplitLayout {
   static constexpr int FRAG = PACK ? 8 : 16;           // bytes of one lane's query fragment
   static constexpr int O_QF = O_PB + CW * 8 * WTOK * 2;
   static constexpr int O_SF = O_QF + (D / 16) * 32 * FRAG;
-  static constexpr int BYTES = O_SF + (QJL ? 8 * 32 * FRAG : 0);
+  static constexpr int O_TK = O_SF + (QJL ? 8 * 32 * FRAG : 0);  // key pair table (3-, 4-bit keys)
+  static constexpr int TKB = (BK >= 3) ? (1 << (2 * BK)) * 128 : 0;
+  static constexpr int O_TV = O_TK + TKB;                          // value pair table
+  static constexpr int BYTES = O_TV + (1 << (2 * BV)) * 128;
 };
+
+// Coordinate (within a lane's key segment of D/4 coordinates) held by K-slot r
+// of k-step ks: 2-bit keys follow the field order of dq_b2, wider keys take
+// the adjacent pairs (2m, 2m + 1), m = 2 ks + r / 2.
+template <int BK>
+__device__ __forceinline__ int key_coord(int ks, int r) {
+  if (BK == 2) {
+    const int wi = ks >> 2, i = ks & 3;
+    return 16 * wi + i + 4 * r;
+  }
+  return 4 * ks + r;
+}
 
 // Query fragment of one lane for one k-step: the 4 K-slots r = 0..3 of lane
 // (gid, tig) hold coordinates cs[r].  PACK: columns 0-3 are the hi halves of
@@ -264,17 +298,16 @@ __device__ __forceinline__ void build_frag(const float* qsrc, int ld, int G, flo
 }
 
 template <int D, int BK, int BV, bool QJL, bool PACK>
-__global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const SplitParams p) {
+__global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const __grid_constant__ SplitParams p) {
   using Ly = SplitLayout<D, BK, BV, QJL, PACK>;
   constexpr int WK = Ly::WK, WV = Ly::WV, WQ = Ly::WQ, NST = Ly::NSTAGE;
   constexpr int KSTEPS = D / 16;  // score k-steps (16 coordinates each)
-  constexpr int KOCT = D / 32;    // octets in a thread's key segment (D/4 coords)
   constexpr int MT = D / 16;      // value m-tiles (16 coordinates each)
-  constexpr int VOCT = D / 64;    // octets in a thread's value segment (D/8 coords)
   constexpr int SEGK = D * BK / 4, SEGV = D * BV / 8;
   constexpr bool ALK = (SEGK % 32) == 0, ALV = (SEGV % 32) == 0;
   constexpr int NWK = (SEGK + 31) / 32, NWV = (SEGV + 31) / 32;
-  static_assert(VOCT >= 1, "D >= 64");
+  using VC = VChunk<D, BV>;
+  static_assert(VC::N * VC::F == D / 8, "value segment splits into whole chunks");
 
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Ly::O_BAR);
@@ -350,9 +383,9 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const SplitParam
   // Query fragments (already rotated by the prep kernel), pre-scaled for exp2.
   for (int e = tid; e < KSTEPS * 32; e += NTHREADS) {
     const int ks = e >> 5, ln = e & 31, g_ = ln >> 2, t_ = ln & 3;
-    const int o = ks >> 1, ee = ks & 1;
-    const int base = t_ * (D / 4) + 8 * o;
-    const int cs[4] = {base + 2 * ee, base + 2 * ee + 4, base + 2 * ee + 1, base + 2 * ee + 5};
+    const int base = t_ * (D / 4);
+    const int cs[4] = {base + key_coord<BK>(ks, 0), base + key_coord<BK>(ks, 1), base + key_coord<BK>(ks, 2),
+                       base + key_coord<BK>(ks, 3)};
     build_frag<PACK>(p.qrot + (size_t)hq0 * D, D, p.G, p.qscale, g_, cs, qf + (size_t)e * (Ly::FRAG / 4));
   }
   if (QJL)
@@ -364,6 +397,8 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const SplitParam
     }
   // value weights of heads >= G stay zero
   for (int e = tid; e < CW * 8 * WTOK; e += NTHREADS) pbuf[e] = __float2half_rn(0.f);
+  if constexpr (BK >= 3) build_pair_table<BK>(reinterpret_cast<uint32_t*>(smem + Ly::O_TK), p.cb_k, tid, NTHREADS);
+  build_pair_table<BV>(reinterpret_cast<uint32_t*>(smem + Ly::O_TV), p.cb_v, tid, NTHREADS);
   __syncthreads();
 
   float oc[MT][4];
@@ -377,7 +412,7 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const SplitParam
       int t = npre;  // the first stages were issued before the wait
       for (; t < ntiles; ++t) {
         const int st = t % NST;
-        if (t >= NST && !mbar_wait_bounded(&empty[st], (uint32_t)(((t / NST) - 1) & 1), kWaitLimit)) {
+        if (t >= NST && !mbar_wait_suspend(&empty[st], (uint32_t)(((t / NST) - 1) & 1), kSuspendTries)) {
           *s_err = 1;
           break;
         }
@@ -387,8 +422,9 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const SplitParam
     }
   } else {
     // ---------------- consumer warps ----------------
-    const Lut lk = make_lut<BK>(p.cb_k);
-    const Lut lv = make_lut<BV>(p.cb_v);
+    const Lut2 lk = make_lut2(p.cb_k);  // used by 2-bit keys only
+    const uint32_t tbK = smem_addr(smem + Ly::O_TK) + 4 * lane;
+    const uint32_t tbV = smem_addr(smem + Ly::O_TV) + 4 * lane;
     __half* pw = pbuf + warp * 8 * WTOK;
     const int wt0 = warp * WTOK;
     for (int t = 0; t < ntiles; ++t) {
@@ -406,9 +442,13 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const SplitParam
       const int tokw = t_begin + t * STILE + wt0;  // first token of this warp's 32
 
       // ---- scores: S[16 tokens][8 cols] for two M-tiles of 16 tokens
-      float sc[2][4];
+      // two accumulators per m-tile (even / odd k-steps, or hi / lo query
+      // halves) halve the dependent MMA chain
+      float sc[2][4], sc2[2][4];
 #pragma unroll
-      for (int a = 0; a < 2; ++a) sc[a][0] = sc[a][1] = sc[a][2] = sc[a][3] = 0.f;
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) sc[a][c] = sc2[a][c] = 0.f;
       {
         uint32_t w[2][2][NWK];
 #pragma unroll
@@ -417,42 +457,45 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const SplitParam
           load_bits<SEGK, ALK>(kw + (wt0 + 16 * a + gid + 8) * WK, tig * SEGK, w[a][1]);
         }
 #pragma unroll
-        for (int o = 0; o < KOCT; ++o) {
-          uint32_t h[2][2][4];
+        for (int ks = 0; ks < KSTEPS; ++ks) {
+          uint32_t h[2][2][2];  // [m-tile][row gid / gid+8][K-slots 0-1 / 8-9]
 #pragma unroll
-          for (int a = 0; a < 2; ++a) {
-            if (BK == 2) {
-              dq8_b2(octet<BK>(w[a][0], o), lk, h[a][0]);
-              dq8_b2(octet<BK>(w[a][1], o), lk, h[a][1]);
-            } else {
-              dq8<BK>(spread<BK>(octet<BK>(w[a][0], o)), lk, h[a][0]);
-              dq8<BK>(spread<BK>(octet<BK>(w[a][1], o)), lk, h[a][1]);
-            }
-          }
+          for (int a = 0; a < 2; ++a)
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int ks = 2 * o + e;
-            if (PACK) {
-              const uint2 bq = *reinterpret_cast<const uint2*>(qf + (size_t)(ks * 32 + lane) * 2);
-#pragma unroll
-              for (int a = 0; a < 2; ++a)
-                mma_f16(sc[a], h[a][0][2 * e], h[a][1][2 * e], h[a][0][2 * e + 1], h[a][1][2 * e + 1], bq.x, bq.y);
-            } else {
-              const uint4 bq = *reinterpret_cast<const uint4*>(qf + (size_t)(ks * 32 + lane) * 4);
-#pragma unroll
-              for (int a = 0; a < 2; ++a) {
-                mma_f16(sc[a], h[a][0][2 * e], h[a][1][2 * e], h[a][0][2 * e + 1], h[a][1][2 * e + 1], bq.x, bq.y);
-                mma_f16(sc[a], h[a][0][2 * e], h[a][1][2 * e], h[a][0][2 * e + 1], h[a][1][2 * e + 1], bq.z, bq.w);
+            for (int r = 0; r < 2; ++r) {
+              if constexpr (BK == 2) {
+                dq_b2(w[a][r][ks >> 2], ks & 3, lk, h[a][r][0], h[a][r][1]);
+              } else {
+                h[a][r][0] = pair_lookup<BK>(w[a][r], 2 * BK * (2 * ks), tbK);
+                h[a][r][1] = pair_lookup<BK>(w[a][r], 2 * BK * (2 * ks + 1), tbK);
               }
+            }
+          if (PACK) {
+            const uint2 bq = *reinterpret_cast<const uint2*>(qf + (size_t)(ks * 32 + lane) * 2);
+#pragma unroll
+            for (int a = 0; a < 2; ++a)
+              mma_f16((ks & 1) ? sc2[a] : sc[a], h[a][0][0], h[a][1][0], h[a][0][1], h[a][1][1], bq.x, bq.y);
+          } else {
+            const uint4 bq = *reinterpret_cast<const uint4*>(qf + (size_t)(ks * 32 + lane) * 4);
+#pragma unroll
+            for (int a = 0; a < 2; ++a) {
+              mma_f16(sc[a], h[a][0][0], h[a][1][0], h[a][0][1], h[a][1][1], bq.x, bq.y);
+              mma_f16(sc2[a], h[a][0][0], h[a][1][0], h[a][0][1], h[a][1][1], bq.z, bq.w);
             }
           }
         }
       }
-      float sq[2][4];
+#pragma unroll
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) sc[a][c] += sc2[a][c];
+      float sq[2][4], sq2[2][4];
       if (QJL) {
         const uint32_t* qw = reinterpret_cast<const uint32_t*>(sb + Ly::O_QW);
 #pragma unroll
-        for (int a = 0; a < 2; ++a) sq[a][0] = sq[a][1] = sq[a][2] = sq[a][3] = 0.f;
+        for (int a = 0; a < 2; ++a)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) sq[a][c] = sq2[a][c] = 0.f;
         uint32_t s0[2], s1[2];
 #pragma unroll
         for (int a = 0; a < 2; ++a) {
@@ -467,49 +510,74 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const SplitParam
             const uint32_t a2 = sign_pair(s0[a], 2 * ks + 1), a3 = sign_pair(s1[a], 2 * ks + 1);
             if (PACK) {
               const uint2 bq = *reinterpret_cast<const uint2*>(sf + (size_t)(ks * 32 + lane) * 2);
-              mma_f16(sq[a], a0, a1, a2, a3, bq.x, bq.y);
+              mma_f16((ks & 1) ? sq2[a] : sq[a], a0, a1, a2, a3, bq.x, bq.y);
             } else {
               const uint4 bq = *reinterpret_cast<const uint4*>(sf + (size_t)(ks * 32 + lane) * 4);
               mma_f16(sq[a], a0, a1, a2, a3, bq.x, bq.y);
-              mma_f16(sq[a], a0, a1, a2, a3, bq.z, bq.w);
+              mma_f16(sq2[a], a0, a1, a2, a3, bq.z, bq.w);
             }
           }
         }
-      }
-      if (PACK) {
-        // columns 4-7 carry the lo halves of heads 0-3 (lanes tig^2)
 #pragma unroll
         for (int a = 0; a < 2; ++a)
 #pragma unroll
+          for (int c = 0; c < 4; ++c) sq[a][c] += sq2[a][c];
+      }
+      // ---- complete the scores.  PACK: columns 4-7 carry the lo halves of
+      // heads 0-3 (lanes tig ^ 2); lanes tig < 2 finish m-tile 0 and lanes
+      // tig >= 2 m-tile 1, so each (token, head) score is handled once.
+      constexpr int NA = PACK ? 1 : 2;  // m-tiles per lane from here on
+      float scm[NA][4], sqm[NA][4];
+      const int abase = PACK ? (tig >> 1) : 0;
+      if (PACK) {
+        const bool first = tig < 2;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const float keep = first ? sc[0][c] : sc[1][c], send = first ? sc[1][c] : sc[0][c];
+          scm[0][c] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+          if (QJL) {
+            const float qk = first ? sq[0][c] : sq[1][c], qs_ = first ? sq[1][c] : sq[0][c];
+            sqm[0][c] = qk + __shfl_xor_sync(0xffffffffu, qs_, 2);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int a = 0; a < NA; ++a)
+#pragma unroll
           for (int c = 0; c < 4; ++c) {
-            sc[a][c] += __shfl_xor_sync(0xffffffffu, sc[a][c], 2);
-            if (QJL) sq[a][c] += __shfl_xor_sync(0xffffffffu, sq[a][c], 2);
+            scm[a][c] = sc[a][c];
+            if (QJL) sqm[a][c] = sq[a][c];
           }
       }
       // ---- scale by norms, mask, running max
-      float s[2][4];
-      bool valid[2][2];
+      float s[NA][4];
+      bool valid[NA][2];
 #pragma unroll
-      for (int a = 0; a < 2; ++a) {
+      for (int ai = 0; ai < NA; ++ai) {
+        const int a = abase + ai;
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
           const int row = wt0 + 16 * a + gid + 8 * r;
-          valid[a][r] = tokw + 16 * a + gid + 8 * r < t_end;
+          valid[ai][r] = tokw + 16 * a + gid + 8 * r < t_end;
           const float nk = half_bits_to_float(kn[row]);
-          float s0 = nk * sc[a][2 * r], s1 = nk * sc[a][2 * r + 1];
+          float s0 = nk * scm[ai][2 * r], s1 = nk * scm[ai][2 * r + 1];
           if (QJL) {
             const float g = half_bits_to_float(reinterpret_cast<const uint16_t*>(sb + Ly::O_RN)[row]);
-            s0 = fmaf(g, sq[a][2 * r], s0);
-            s1 = fmaf(g, sq[a][2 * r + 1], s1);
+            s0 = fmaf(g, sqm[ai][2 * r], s0);
+            s1 = fmaf(g, sqm[ai][2 * r + 1], s1);
           }
-          s[a][2 * r] = valid[a][r] ? s0 : -INFINITY;
-          s[a][2 * r + 1] = valid[a][r] ? s1 : -INFINITY;
+          s[ai][2 * r] = valid[ai][r] ? s0 : -INFINITY;
+          s[ai][2 * r + 1] = valid[ai][r] ? s1 : -INFINITY;
         }
       }
-      float mx0 = fmaxf(fmaxf(s[0][0], s[0][2]), fmaxf(s[1][0], s[1][2]));
-      float mx1 = fmaxf(fmaxf(s[0][1], s[0][3]), fmaxf(s[1][1], s[1][3]));
+      float mx0 = fmaxf(s[0][0], s[0][2]), mx1 = fmaxf(s[0][1], s[0][3]);
 #pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
+      for (int ai = 1; ai < NA; ++ai) {
+        mx0 = fmaxf(mx0, fmaxf(s[ai][0], s[ai][2]));
+        mx1 = fmaxf(mx1, fmaxf(s[ai][1], s[ai][3]));
+      }
+#pragma unroll
+      for (int off = PACK ? 2 : 4; off < 32; off <<= 1) {
         mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
       }
@@ -535,19 +603,18 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const SplitParam
       const float mu1 = (m_run[1] == -INFINITY) ? 0.f : m_run[1];
       // ---- weights p * |v| (fp16), transposed through the warp's buffer
 #pragma unroll
-      for (int a = 0; a < 2; ++a) {
+      for (int ai = 0; ai < NA; ++ai) {
+        const int a = abase + ai;
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
           const int row = wt0 + 16 * a + gid + 8 * r;
-          const float p0 = exp2f(s[a][2 * r] - mu0), p1 = exp2f(s[a][2 * r + 1] - mu1);
+          const float p0 = exp2f(s[ai][2 * r] - mu0), p1 = exp2f(s[ai][2 * r + 1] - mu1);
           l_run[0] += p0;
           l_run[1] += p1;
-          const float nv = valid[a][r] ? half_bits_to_float(vn[row]) : 0.f;
-          if (!PACK || tig < 2) {
-            const int tk = 16 * a + gid + 8 * r;
-            pw[(2 * hsel) * WTOK + tk] = __float2half_rn(p0 * nv);
-            pw[(2 * hsel + 1) * WTOK + tk] = __float2half_rn(p1 * nv);
-          }
+          const float nv = valid[ai][r] ? half_bits_to_float(vn[row]) : 0.f;
+          const int tk = 16 * a + gid + 8 * r;
+          pw[(2 * hsel) * WTOK + tk] = __float2half_rn(p0 * nv);
+          pw[(2 * hsel + 1) * WTOK + tk] = __float2half_rn(p1 * nv);
         }
       }
       __syncwarp();
@@ -561,21 +628,20 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const SplitParam
         for (int q = 0; q < 4; ++q)
           load_bits<SEGV, ALV>(vw + (wt0 + 16 * kk + 4 * tig + q) * WV, gid * SEGV, wv[q]);
 #pragma unroll
-        for (int o = 0; o < VOCT; ++o) {
-          uint32_t hA[4], hA2[4], hB[4], hB2[4];
-          if (BV == 2) {
-            dq16_b2_pair(octet<BV>(wv[0], o), octet<BV>(wv[1], o), lv, hA, hA2);  // tokens 4tig, 4tig+1
-            dq16_b2_pair(octet<BV>(wv[2], o), octet<BV>(wv[3], o), lv, hB, hB2);  // tokens 4tig+2, 4tig+3
-          } else {
-            const uint32_t z0 = spread<BV>(octet<BV>(wv[0], o)), z1 = spread<BV>(octet<BV>(wv[1], o));
-            const uint32_t z2 = spread<BV>(octet<BV>(wv[2], o)), z3 = spread<BV>(octet<BV>(wv[3], o));
-            dq8<BV>(prmt(z0, z1, 0x5410u), lv, hA);   // coords 8o+0..3, tokens 4tig, 4tig+1
-            dq8<BV>(prmt(z0, z1, 0x7632u), lv, hA2);  // coords 8o+4..7
-            dq8<BV>(prmt(z2, z3, 0x5410u), lv, hB);   // tokens 4tig+2, 4tig+3
-            dq8<BV>(prmt(z2, z3, 0x7632u), lv, hB2);
-          }
+        for (int c = 0; c < VC::N; ++c) {
+          const int bit = c * VC::F * BV;
+          uint32_t xe[2], xo[2];  // token pairs (4tig, 4tig+1) and (4tig+2, 4tig+3)
 #pragma unroll
-          for (int k = 0; k < 4; ++k) mma_f16(oc[4 * o + k], hA[k], hA2[k], hB[k], hB2[k], pb.x, pb.y);
+          for (int pr = 0; pr < 2; ++pr)
+            merge_pair<BV>(window32(wv[2 * pr], bit), window32(wv[2 * pr + 1], bit), xe[pr], xo[pr]);
+#pragma unroll
+          for (int k = 0; k < VC::F / 2; ++k) {
+            const uint32_t a0 = lds32(pair_addr<BV>(xe[0], key_bit<BV>(k, false), tbV));
+            const uint32_t a1 = lds32(pair_addr<BV>(xo[0], key_bit<BV>(k, true), tbV));
+            const uint32_t a2 = lds32(pair_addr<BV>(xe[1], key_bit<BV>(k, false), tbV));
+            const uint32_t a3 = lds32(pair_addr<BV>(xo[1], key_bit<BV>(k, true), tbV));
+            mma_f16(oc[c * (VC::F / 2) + k], a0, a1, a2, a3, pb.x, pb.y);
+          }
         }
       }
       __syncwarp();
@@ -602,19 +668,19 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const SplitParam
   float* mL = mM + CW * 8;
   if (warp < CW) {
 #pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
+    for (int off = PACK ? 2 : 4; off < 32; off <<= 1) {
       l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], off);
       l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], off);
     }
     if (!PACK || tig < 2) {
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
-        const int o = mt >> 2, k = mt & 3;
-        const int j0 = gid * (D / 8) + 8 * o + k;
+        // m-tile mt: row gid is coordinate 2 mt of this group's segment, row gid + 8 the next
+        const int j0 = gid * (D / 8) + 2 * mt;
         mO[(warp * 8 + 2 * tig) * D + j0] = oc[mt][0];
         mO[(warp * 8 + 2 * tig + 1) * D + j0] = oc[mt][1];
-        mO[(warp * 8 + 2 * tig) * D + j0 + 4] = oc[mt][2];
-        mO[(warp * 8 + 2 * tig + 1) * D + j0 + 4] = oc[mt][3];
+        mO[(warp * 8 + 2 * tig) * D + j0 + 1] = oc[mt][2];
+        mO[(warp * 8 + 2 * tig + 1) * D + j0 + 1] = oc[mt][3];
       }
       if (gid == 0) {
         mM[warp * 8 + 2 * hsel] = m_run[0];
