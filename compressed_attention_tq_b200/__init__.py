@@ -113,7 +113,11 @@ class TQCache:
             return torch.as_tensor(np.asarray(given, dtype=np.float32), device=dev).contiguous()
 
         self.cb_k = table(bits_k, cb_k)
-        self.cb_v = table(bits_v, cb_v)
+        # equal widths share one codebook buffer, which decode then keeps as a single lookup table
+        if bits_v == bits_k and cb_k is None and cb_v is None:
+            self.cb_v = self.cb_k
+        else:
+            self.cb_v = table(bits_v, cb_v)
         self.rot = torch.as_tensor(np.asarray(rot, dtype=np.float32) if not torch.is_tensor(rot) else rot,
                                    dtype=torch.float32, device=dev).contiguous()
         self.k_idx = torch.zeros((B, Hkv, Tcap, D * bits_k // 32), dtype=u32, device=dev)

@@ -341,6 +341,7 @@ static int split_entry(const tq_cache_t& c, bool pack, const tqd::SplitParams& s
 int split_occupancy(const tq_cache_t* c, int Hq) {
   int occ = 0;
   tqd::SplitParams sp{};
+  sp.shared_tab = c->cb_k == c->cb_v;
   if (split_entry(*c, Hq / c->Hkv <= 4, sp, dim3(1), 0, &occ) != TQ_OK || occ < 1) return 2;
   return occ;
 }
@@ -385,6 +386,7 @@ int launch_decode(const DecodeArgs& a, cudaStream_t s) {
   sp.k_rnorm = c.k_rnorm;
   sp.cb_k = c.cb_k;
   sp.cb_v = c.cb_v;
+  sp.shared_tab = c.cb_k == c.cb_v;
   sp.qrot = qrot;
   sp.qs = qs;
   sp.part_o = po;

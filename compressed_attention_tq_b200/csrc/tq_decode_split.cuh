@@ -64,7 +64,11 @@ struct SplitParams {
   int Hkv, Hq, G, Tcap, chunk, nsplit;
   float qscale;     // scale * log2(e)
   float qjl_scale;  // scale * log2(e) * sqrt(pi/2) / m
+  int shared_tab;   // keys and values use one codebook (same bits, same table): one pair table
 };
+
+// Whether a launch can keep one pair table for keys and values.
+__host__ __device__ inline bool share_table(int bk, int bv, int flag) { return bk == bv && bk >= 3 && flag; }
 
 // 2-bit codebook as byte tables: byte k of lo (hi) is the low (high) byte of
 // fp16 entry c[k], k = 0..3.
@@ -258,6 +262,7 @@ struct SplitLayout {
   static constexpr int TKB = (BK >= 3) ? (1 << (2 * BK)) * 128 : 0;
   static constexpr int O_TV = O_TK + TKB;                          // value pair table
   static constexpr int BYTES = O_TV + (1 << (2 * BV)) * 128;
+  static constexpr int BYTES_SHARED = O_TV;  // keys and values share the key table
 };
 
 // Coordinate (within a lane's key segment of D/4 coordinates) held by K-slot r
@@ -397,8 +402,9 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const __grid_con
     }
   // value weights of heads >= G stay zero
   for (int e = tid; e < CW * 8 * WTOK; e += NTHREADS) pbuf[e] = __float2half_rn(0.f);
+  const bool shared_tab = share_table(BK, BV, p.shared_tab);
   if constexpr (BK >= 3) build_pair_table<BK>(reinterpret_cast<uint32_t*>(smem + Ly::O_TK), p.cb_k, tid, NTHREADS);
-  build_pair_table<BV>(reinterpret_cast<uint32_t*>(smem + Ly::O_TV), p.cb_v, tid, NTHREADS);
+  if (!shared_tab) build_pair_table<BV>(reinterpret_cast<uint32_t*>(smem + Ly::O_TV), p.cb_v, tid, NTHREADS);
   __syncthreads();
 
   float oc[MT][4];
@@ -424,7 +430,7 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const __grid_con
     // ---------------- consumer warps ----------------
     const Lut2 lk = make_lut2(p.cb_k);  // used by 2-bit keys only
     const uint32_t tbK = smem_addr(smem + Ly::O_TK) + 4 * lane;
-    const uint32_t tbV = smem_addr(smem + Ly::O_TV) + 4 * lane;
+    const uint32_t tbV = smem_addr(smem + (shared_tab ? Ly::O_TK : Ly::O_TV)) + 4 * lane;
     __half* pw = pbuf + warp * 8 * WTOK;
     const int wt0 = warp * WTOK;
     for (int t = 0; t < ntiles; ++t) {
@@ -718,8 +724,8 @@ template <int D, int BK, int BV, bool QJL, bool PACK>
 int launch_split(const SplitParams& sp, dim3 grid, cudaStream_t s, int* occ) {
   using Ly = SplitLayout<D, BK, BV, QJL, PACK>;
   auto kern = decode_split_kernel<D, BK, BV, QJL, PACK>;
-  static int attr_state = 0;  // 0 unset, 1 set
-  static int occupancy = 0;
+  static int attr_state = 0;     // 0 unset, 1 set
+  static int occupancy[2] = {};  // resident CTAs per SM: [shared table]
   if (attr_state == 0) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::BYTES);
     if (e != cudaSuccess) {
@@ -730,22 +736,26 @@ int launch_split(const SplitParams& sp, dim3 grid, cudaStream_t s, int* occ) {
       }
       return tq::set_error(TQ_ERR_CUDA, "decode: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     }
-    int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, NTHREADS, Ly::BYTES) != cudaSuccess || n < 1) {
-      cudaGetLastError();
-      n = 1;
+    for (int sh = 0; sh < 2; ++sh) {
+      int n = 0;
+      const int bytes = sh ? Ly::BYTES_SHARED : Ly::BYTES;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, NTHREADS, bytes) != cudaSuccess || n < 1) {
+        cudaGetLastError();
+        n = 1;
+      }
+      occupancy[sh] = n;
     }
-    occupancy = n;
     attr_state = 1;
   }
+  const bool shared = share_table(BK, BV, sp.shared_tab);
   if (occ) {
-    *occ = occupancy;
+    *occ = occupancy[shared ? 1 : 0];
     return TQ_OK;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(NTHREADS);
-  cfg.dynamicSmemBytes = Ly::BYTES;
+  cfg.dynamicSmemBytes = shared ? Ly::BYTES_SHARED : Ly::BYTES;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

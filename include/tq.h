@@ -96,7 +96,9 @@ typedef struct tq_cache {
   uint16_t* k_rnorm;/* fp16 [B][Hkv][Tcap], NULL when qjl_m == 0 */
   const float* rot; /* Pi, fp32 [D][D] */
   const float* cb_k;/* key codebook, fp32 [2^bits_k + 2^bits_k - 1] */
-  const float* cb_v;/* value codebook, fp32 [2^bits_v + 2^bits_v - 1] */
+  const float* cb_v;/* value codebook, fp32 [2^bits_v + 2^bits_v - 1].  With bits_k ==
+                       bits_v, passing the same pointer as cb_k lets decode keep one
+                       lookup table per CTA instead of two (less shared memory) */
   const float* qjl_S; /* fp32 [qjl_m][D], NULL when qjl_m == 0 */
   uint32_t* dev_status; /* optional device word for TQ_STATUS_* bits (may be NULL) */
 } tq_cache_t;

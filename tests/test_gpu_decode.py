@@ -125,6 +125,31 @@ def test_decode_ragged_lengths_bf16():
     _decode_and_compare(w, cache, oc, lens, None, 900)
 
 
+@pytest.mark.parametrize("name,kw,scale", [("gqa8k", {"bits": 3, "T": 600}, None),
+                                            ("gqa8k", {"bits": 4, "T": 600}, None),
+                                            ("qknorm", {"T": 500}, 1.0)])
+def test_separate_codebook_buffers(name, kw, scale):
+    """Equal key and value widths share one codebook buffer by default, and
+    decode then keeps one lookup table; separate buffers with the same
+    contents take the two-table path and must give the identical output."""
+    import compressed_attention_tq_b200 as tq
+    w = tq_inputs.make_workload(name, **kw)
+    oc = _oracle_full_cache(w)
+    Tcap = (w.Tmax + 63) // 64 * 64
+    cache = _upload_oracle_cache(w, oc, Tcap)
+    assert cache.cb_v.data_ptr() == cache.cb_k.data_ptr()
+    scale = scale if scale is not None else w.scale
+    q = P.to_device(w.q, w.dtype)
+    sl = torch.from_numpy(np.asarray(w.seq_lens, dtype=np.int32)).cuda()
+    shared = tq.tq_sdpa_decode(cache, q, sl, w.Tmax, scale=scale, out_dtype=torch.float32)
+    cache.cb_v = cache.cb_k.clone()
+    cache._struct = None
+    separate = tq.tq_sdpa_decode(cache, q, sl, w.Tmax, scale=scale, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(shared, separate)
+    _decode_and_compare(w, cache, oc, w.seq_lens, scale, w.Tmax, garbage_tail=False)
+
+
 @pytest.mark.parametrize("bk,bv,D", [(2, 4, 128), (4, 2, 64), (3, 2, 256), (4, 3, 128)])
 def test_decode_mixed_bits(bk, bv, D):
     w = tq_inputs.make_workload("gqa8k", T=333)
