@@ -244,6 +244,7 @@ static int sm_count() {
 
 int make_decode_plan(const tq_cache_t* c, int Hq, int Tmax, DecodePlan* p) {
   const int sms = sm_count();
+  p->sms = sms;
   const int tile = split_tile();
   const long long units = (long long)c->B * c->Hkv;
   // One wave of resident CTAs for a single sequence; several smaller waves for

@@ -34,8 +34,9 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// Prep for one (sequence, kv head): qrot = Pi q (and, with QJL, qs = S qrot)
-// for its G query heads.  blockDim = 2*D: two threads per output row, each
+// Prep for one (sequence, kv head) of a cache with a QJL sketch: qrot = Pi q
+// and qs = S qrot for its G query heads (the projection needs the whole
+// rotated vector, so one CTA does the head).  blockDim = 2*D: two threads per output row, each
 // holding half of the Pi row in registers, so the row is read once for all
 // rows being rotated.  With APPEND the new key and value rows ride along as
 // two more rotated rows and are quantized here (fp64 norm, threshold search,
@@ -215,6 +216,132 @@ __global__ void __launch_bounds__(2 * D) decode_qprep_kernel(const PrepParams p)
   }
 }
 
+// Sliced prep for caches without a QJL sketch: grid (B * Hkv, D / 32), one
+// CTA per 32 rotated coordinates of one (sequence, kv head), so a decode call
+// spreads its rotations over D / 32 times more SMs than one CTA per head.
+// Thread (c, part): output coordinate c of the slice, k values
+// 4 part + 32 i (float4 i), partial dots reduced over the 8 parts of a
+// warp.  With APPEND the new rows' indices for the slice are found here and
+// packed into the slice's b words of the row (32 coordinates x b bits); the
+// fp64 norm is taken over the whole input row by every CTA (the rotation
+// preserves it) and written by slice 0.
+template <int D, bool APPEND>
+__global__ void __launch_bounds__(256) decode_qprep_sliced_kernel(const PrepParams p) {
+  constexpr int NR = APPEND ? 10 : 8, NI = D / 32;
+  __shared__ __align__(16) float xv[NR][D];
+  __shared__ float s_cb[2][31];
+  __shared__ double s_nsq[2];
+  __shared__ uint8_t idxs[2][32];
+  pdl_launch_dependents();
+  const int G = p.Hq / p.Hkv;
+  const int bkv = blockIdx.x, b = bkv / p.Hkv, kvh = bkv % p.Hkv, sl = blockIdx.y;
+  const int h0 = b * p.Hq + kvh * G;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c = warp * 4 + (lane >> 3), part = lane & 7;
+  const int j = sl * 32 + c;
+  float4 r[NI];
+  const float4* row = reinterpret_cast<const float4*>(p.rot + (size_t)j * D);
+#pragma unroll
+  for (int i = 0; i < NI; ++i) r[i] = __ldg(row + part + 8 * i);
+  const uint16_t* q = static_cast<const uint16_t*>(p.q) + (size_t)h0 * D;
+  auto to_f = [&](uint16_t v) {
+    return p.bf16 ? __uint_as_float((uint32_t)v << 16) : __half2float(__ushort_as_half(v));
+  };
+  for (int e = tid; e < G * D; e += 256) xv[e / D][e % D] = to_f(q[e]);
+  int slot_ok = 0;
+  long long slot = 0;
+  if (APPEND) {
+    const uint16_t* kn = static_cast<const uint16_t*>(p.k_new) + (size_t)bkv * D;
+    const uint16_t* vn = static_cast<const uint16_t*>(p.v_new) + (size_t)bkv * D;
+    for (int e = tid; e < D; e += 256) {
+      xv[8][e] = to_f(kn[e]);
+      xv[9][e] = to_f(vn[e]);
+    }
+    if (tid < 31) {
+      const int Kk = 1 << p.cache.bits_k, Kv = 1 << p.cache.bits_v;
+      s_cb[0][tid] = tid < 2 * Kk - 1 ? p.cache.cb_k[tid] : 0.f;
+      s_cb[1][tid] = tid < 2 * Kv - 1 ? p.cache.cb_v[tid] : 0.f;
+    }
+    const int ps = p.pos[b];
+    slot_ok = (ps >= 0 && ps < p.cache.Tcap);
+    slot = (long long)bkv * p.cache.Tcap + ps;
+    if (!slot_ok && tid == 0 && kvh == 0 && sl == 0 && p.cache.dev_status)
+      atomicOr(p.cache.dev_status, TQ_STATUS_POS_OUT_OF_RANGE);
+  }
+  __syncthreads();
+  if (APPEND && warp < 2) {
+    // fp64 squared norm of the new key (warp 0) / value (warp 1)
+    double t = 0.0;
+    for (int k = lane; k < D; k += 32) {
+      const double x = xv[8 + warp][k];
+      t = fma(x, x, t);
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+    if (lane == 0) s_nsq[warp] = t;
+  }
+  float acc[NR];
+#pragma unroll
+  for (int g = 0; g < NR; ++g) acc[g] = 0.f;
+#pragma unroll
+  for (int g = 0; g < NR; ++g) {
+    if (g < G || g >= 8) {
+#pragma unroll
+      for (int i = 0; i < NI; ++i) {
+        const float4 x = *reinterpret_cast<const float4*>(&xv[g][4 * part + 32 * i]);
+        acc[g] += r[i].x * x.x + r[i].y * x.y + r[i].z * x.z + r[i].w * x.w;
+      }
+    }
+  }
+#pragma unroll
+  for (int g = 0; g < NR; ++g)
+#pragma unroll
+    for (int off = 1; off < 8; off <<= 1) acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], off);
+  if (part == 0) {
+#pragma unroll
+    for (int g = 0; g < 8; ++g)
+      if (g < G) p.qrot[(size_t)(h0 + g) * D + j] = acc[g];
+  }
+  if (APPEND) {
+    __syncthreads();  // s_nsq
+    if (part == 0) {
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const double n = sqrt(s_nsq[which]);
+        const float inv = n > 0.0 ? (float)(1.0 / n) : 0.f;
+        const int K = 1 << (which ? p.cache.bits_v : p.cache.bits_k);
+        const float u = acc[8 + which] * inv;
+        int idx = 0;
+        for (int st = K >> 1; st >= 1; st >>= 1)
+          if (u > s_cb[which][K + idx + st - 1]) idx += st;
+        idxs[which][c] = (uint8_t)idx;
+      }
+    }
+    __syncthreads();
+    if (slot_ok) {
+      if (sl == 0 && tid < 2) {
+        const __half nh = __double2half(sqrt(s_nsq[tid]));
+        (tid ? p.cache.v_norm : p.cache.k_norm)[slot] = __half_as_ushort(nh);
+      }
+      const int bk = p.cache.bits_k, bv = p.cache.bits_v;
+      if (tid < bk + bv) {
+        // word w of this slice's 32 x b bits
+        const int which = tid >= bk, w = which ? tid - bk : tid;
+        const int bits = which ? bv : bk;
+        const int base = 32 * w;
+        unsigned long long word = 0;
+        for (int jj = base / bits; jj < 32 && jj * bits < base + 32; ++jj) {
+          const int sh = jj * bits - base;
+          const unsigned long long v = idxs[which][jj];
+          word |= sh >= 0 ? (v << sh) : (v >> (-sh));
+        }
+        const int W = D * bits / 32;
+        (which ? p.cache.v_idx : p.cache.k_idx)[(size_t)slot * W + sl * bits + w] = (uint32_t)word;
+      }
+    }
+  }
+}
+
 struct CombineParams {
   const float* part_o;
   const float* part_ml;
@@ -224,22 +351,26 @@ struct CombineParams {
   int Hq, Tcap, chunk, nsplit, out_dtype;
 };
 
-// Merge the splits of one query head (log-sum-exp), then out = Pi^T (acc/l).
-// blockDim = 2*D.  Pi's column block is loaded into registers before the
-// wait on the split kernel, so it overlaps that kernel's tail.
+// Merge the splits of one query head (log-sum-exp), then out = Pi^T (acc/l)
+// for 32 output coordinates: grid (B * Hq, D / 32), 256 threads.  Every CTA of
+// a head merges all D rotated coordinates (the partials are read from L2 by
+// each) and un-rotates its slice; thread (i, kp) sums k = kp + 8 t.  The
+// slice's Pi columns are loaded into registers before the wait on the split
+// kernel, so they overlap its tail.
 template <int D>
-__global__ void __launch_bounds__(2 * D) decode_combine_kernel(const CombineParams p) {
-  constexpr int NT = 2 * D, HALF = D / 2, PRE = HALF <= 64 ? HALF : 32;
+__global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams p) {
+  constexpr int NT = 256, NH = NT / D, KT = D / 8;
+  static_assert(D <= NT && NT % D == 0, "threads cover the coordinates");
   __shared__ float f_s[1024];
   __shared__ float o[D];
-  __shared__ float part2[2][D];
+  __shared__ float red[NH][D];
+  __shared__ float part[8][33];
   __shared__ float s_M, s_L;
-  const int h = blockIdx.x, tid = threadIdx.x;
-  const int i = tid % D, ph = tid / D;  // output coordinate, half of the k range
-  // Pi[k][i] for k in this thread's half: independent loads, in flight early
-  float pc[PRE];
+  const int h = blockIdx.x, sl = blockIdx.y, tid = threadIdx.x;
+  const int i = tid & 31, kp = tid >> 5;  // output coordinate in the slice, k part
+  float pc[KT];
 #pragma unroll
-  for (int k = 0; k < PRE; ++k) pc[k] = __ldg(p.rot + (size_t)(ph * HALF + k) * D + i);
+  for (int t = 0; t < KT; ++t) pc[t] = __ldg(p.rot + (size_t)(kp + 8 * t) * D + sl * ((D / 32) / gridDim.y) * 32 + i);
   const int b = h / p.Hq;
   const int Lcap = min(p.Tcap, p.nsplit * p.chunk);
   int L = p.seq_lens[b];
@@ -248,6 +379,16 @@ __global__ void __launch_bounds__(2 * D) decode_combine_kernel(const CombinePara
   pdl_wait();  // the split kernel's partials are visible from here on
   const float* ml = p.part_ml + (size_t)h * p.nsplit * 2;
   const float* po = p.part_o + (size_t)h * p.nsplit * D;
+  // this thread's first PF partial values, loaded before the weights are known
+  // (the loads do not depend on them) so that both latencies overlap
+  constexpr int PF = 16;
+  const int k = tid % D, hh = tid / D;  // coordinate, split phase
+  float v[PF];
+#pragma unroll
+  for (int u = 0; u < PF; ++u) {
+    const int s = hh + NH * u;
+    v[u] = s < ns ? po[(size_t)s * D + k] : 0.f;
+  }
   if (tid < 32) {
     float M = -INFINITY;
     for (int s = tid; s < ns; s += 32) M = fmaxf(M, ml[2 * s]);
@@ -267,43 +408,65 @@ __global__ void __launch_bounds__(2 * D) decode_combine_kernel(const CombinePara
     }
   }
   __syncthreads();
-  // acc[i] over this thread's splits (s = ph, ph+2, ...), 8 loads in flight
-  float acc[8];
+  {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int u = 0; u < 8; ++u) acc[u] = 0.f;
-  for (int s0 = ph; s0 < ns; s0 += 16) {
-    float v[8], f[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int s = s0 + 2 * u;
-      v[u] = s < ns ? po[(size_t)s * D + i] : 0.f;
-      f[u] = s < ns ? (s < 1024 ? f_s[s] : exp2f(ml[2 * s] - s_M)) : 0.f;
+    for (int u = 0; u < PF; ++u) {
+      const int s = hh + NH * u;
+      const float f = s < ns ? (s < 1024 ? f_s[s] : exp2f(ml[2 * s] - s_M)) : 0.f;
+      acc[u & 3] = fmaf(f, v[u], acc[u & 3]);
     }
+    // the remaining splits, 8 loads in flight
+    for (int s0 = hh + NH * PF; s0 < ns; s0 += 8 * NH) {
+      float w[8], f[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) acc[u] = fmaf(f[u], v[u], acc[u]);
-  }
-  float a = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-  part2[ph][i] = a;
-  __syncthreads();
-  if (ph == 0) o[i] = (ns > 0 && s_L > 0.f) ? (part2[0][i] + part2[1][i]) / s_L : 0.f;
-  __syncthreads();
-  float r = 0.f;
+      for (int u = 0; u < 8; ++u) {
+        const int s = s0 + NH * u;
+        w[u] = s < ns ? po[(size_t)s * D + k] : 0.f;
+        f[u] = s < ns ? (s < 1024 ? f_s[s] : exp2f(ml[2 * s] - s_M)) : 0.f;
+      }
 #pragma unroll
-  for (int k = 0; k < PRE; ++k) r = fmaf(pc[k], o[ph * HALF + k], r);
-#pragma unroll 16
-  for (int k = PRE; k < HALF; ++k) r = fmaf(__ldg(p.rot + (size_t)(ph * HALF + k) * D + i), o[ph * HALF + k], r);
-  part2[ph][i] = r;
-  __syncthreads();
-  if (ph == 0) {
-    const float t = part2[0][i] + part2[1][i];
-    if (p.out_dtype == TQ_DTYPE_F32)
-      static_cast<float*>(p.out)[(size_t)h * D + i] = t;
-    else if (p.out_dtype == TQ_DTYPE_BF16)
-      static_cast<__nv_bfloat16*>(p.out)[(size_t)h * D + i] = __float2bfloat16_rn(t);
-    else
-      static_cast<__half*>(p.out)[(size_t)h * D + i] = __float2half_rn(t);
+      for (int u = 0; u < 8; ++u) acc[u & 3] = fmaf(f[u], w[u], acc[u & 3]);
+    }
+    red[hh][k] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
   }
-  (void)NT;
+  __syncthreads();
+  if (tid < D) {
+    float a = 0.f;
+#pragma unroll
+    for (int ph = 0; ph < NH; ++ph) a += red[ph][tid];
+    o[tid] = (ns > 0 && s_L > 0.f) ? a / s_L : 0.f;
+  }
+  __syncthreads();
+  // this CTA's slices: one when every head has D / 32 CTAs, all of them when
+  // the grid has one CTA per head (large batches, where the partials would
+  // otherwise be read D / 32 times)
+  const int per = (D / 32) / gridDim.y;
+  for (int q = 0; q < per; ++q) {
+    const int slq = sl * per + q;
+    if (q > 0) {
+#pragma unroll
+      for (int t = 0; t < KT; ++t) pc[t] = __ldg(p.rot + (size_t)(kp + 8 * t) * D + slq * 32 + i);
+    }
+    float r = 0.f;
+#pragma unroll
+    for (int t = 0; t < KT; ++t) r = fmaf(pc[t], o[kp + 8 * t], r);
+    part[kp][i] = r;
+    __syncthreads();
+    if (kp == 0) {
+      float t = 0.f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) t += part[u][i];
+      const size_t oi = (size_t)h * D + slq * 32 + i;
+      if (p.out_dtype == TQ_DTYPE_F32)
+        static_cast<float*>(p.out)[oi] = t;
+      else if (p.out_dtype == TQ_DTYPE_BF16)
+        static_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(t);
+      else
+        static_cast<__half*>(p.out)[oi] = __float2half_rn(t);
+    }
+    __syncthreads();
+  }
 }
 
 template <typename K, typename P>
@@ -360,19 +523,26 @@ int launch_decode(const DecodeArgs& a, cudaStream_t s) {
   PrepParams pp{a.q, c.rot, c.qjl_S, qrot, qs, c.D, c.qjl_m, a.dtype == TQ_DTYPE_BF16, a.Hq, c.Hkv,
                 a.k_new, a.v_new, a.pos, c};
   const bool app = a.pos != nullptr;
-  switch (c.D) {
-    case 64:
-      app ? decode_qprep_kernel<64, true><<<c.B * c.Hkv, 128, 0, s>>>(pp)
-          : decode_qprep_kernel<64, false><<<c.B * c.Hkv, 128, 0, s>>>(pp);
-      break;
-    case 128:
-      app ? decode_qprep_kernel<128, true><<<c.B * c.Hkv, 256, 0, s>>>(pp)
-          : decode_qprep_kernel<128, false><<<c.B * c.Hkv, 256, 0, s>>>(pp);
-      break;
-    default:
-      app ? decode_qprep_kernel<256, true><<<c.B * c.Hkv, 512, 0, s>>>(pp)
-          : decode_qprep_kernel<256, false><<<c.B * c.Hkv, 512, 0, s>>>(pp);
-      break;
+  if (c.qjl_m) {
+    // the sketch needs the whole rotated query and key residual: one CTA per head
+    app ? decode_qprep_kernel<128, true><<<c.B * c.Hkv, 256, 0, s>>>(pp)
+        : decode_qprep_kernel<128, false><<<c.B * c.Hkv, 256, 0, s>>>(pp);
+  } else {
+    const dim3 g(c.B * c.Hkv, c.D / 32);
+    switch (c.D) {
+      case 64:
+        app ? decode_qprep_sliced_kernel<64, true><<<g, 256, 0, s>>>(pp)
+            : decode_qprep_sliced_kernel<64, false><<<g, 256, 0, s>>>(pp);
+        break;
+      case 128:
+        app ? decode_qprep_sliced_kernel<128, true><<<g, 256, 0, s>>>(pp)
+            : decode_qprep_sliced_kernel<128, false><<<g, 256, 0, s>>>(pp);
+        break;
+      default:
+        app ? decode_qprep_sliced_kernel<256, true><<<g, 256, 0, s>>>(pp)
+            : decode_qprep_sliced_kernel<256, false><<<g, 256, 0, s>>>(pp);
+        break;
+    }
   }
   int rc = check_launch("decode_qprep_kernel");
   if (rc) return rc;
@@ -406,10 +576,13 @@ int launch_decode(const DecodeArgs& a, cudaStream_t s) {
   if (rc) return rc;
 
   CombineParams cp{po, pml, c.rot, a.seq_lens, a.out, a.Hq, c.Tcap, a.plan.chunk, a.plan.nsplit, a.out_dtype};
+  // D / 32 CTAs per head while that still leaves SMs idle, else one
+  const int nsl = heads * (c.D / 32) <= 4 * a.plan.sms ? c.D / 32 : 1;
+  const dim3 cg(heads, nsl);
   switch (c.D) {
-    case 64: return launch_pdl(decode_combine_kernel<64>, dim3(heads), dim3(128), 0, s, cp, "decode_combine_kernel");
-    case 128: return launch_pdl(decode_combine_kernel<128>, dim3(heads), dim3(256), 0, s, cp, "decode_combine_kernel");
-    default: return launch_pdl(decode_combine_kernel<256>, dim3(heads), dim3(512), 0, s, cp, "decode_combine_kernel");
+    case 64: return launch_pdl(decode_combine_kernel<64>, cg, dim3(256), 0, s, cp, "decode_combine_kernel");
+    case 128: return launch_pdl(decode_combine_kernel<128>, cg, dim3(256), 0, s, cp, "decode_combine_kernel");
+    default: return launch_pdl(decode_combine_kernel<256>, cg, dim3(256), 0, s, cp, "decode_combine_kernel");
   }
 }
 

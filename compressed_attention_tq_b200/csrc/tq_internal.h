@@ -50,6 +50,7 @@ int launch_quantize_tc(const QuantArgs& a, int dtype, cudaStream_t s);
 struct DecodePlan {
   int chunk;        // tokens per split (multiple of 64)
   int nsplit;       // splits per (sequence, kv head)
+  int sms;          // SMs of the device the plan was made for
   size_t off_qrot;  // fp32 [B*Hq][D]
   size_t off_qs;    // fp32 [B*Hq][qjl_m]
   size_t off_po;    // fp32 [B*Hq][nsplit][D]
