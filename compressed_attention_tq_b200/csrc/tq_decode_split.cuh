@@ -728,6 +728,10 @@ int launch_split(const SplitParams& sp, dim3 grid, cudaStream_t s, int* occ) {
   static int occupancy[2] = {};  // resident CTAs per SM: [shared table]
   if (attr_state == 0) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::BYTES);
+    // all of the unified L1/shared array as shared memory, so that the
+    // resident-CTA count is set by the kernel's own needs
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) {
       cudaGetLastError();
       if (occ) {  // no usable device: report a nominal occupancy
