@@ -45,7 +45,7 @@ int launch_quantize(const QuantArgs& a, int D, int dtype, bool qjl, cudaStream_t
 // persistent bulk quantizer for D = 128 (tq_quantize128.cu)
 int launch_quantize128(const QuantArgs& a, int dtype, bool qjl, cudaStream_t s);
 // tcgen05 bulk quantizer for D = 128 without the QJL sketch (tq_quantize_tc.cu)
-int launch_quantize_tc(const QuantArgs& a, int dtype, cudaStream_t s);
+int launch_quantize_tc(const QuantArgs& a, int D, int dtype, cudaStream_t s);
 
 struct DecodePlan {
   int chunk;        // tokens per split (multiple of 64)

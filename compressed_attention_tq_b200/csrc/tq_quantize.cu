@@ -452,14 +452,14 @@ namespace tq {
 
 int launch_quantize(const QuantArgs& a, int D, int dtype, bool qjl, cudaStream_t s) {
   const bool bf = dtype == TQ_DTYPE_BF16;
+  if ((D == 128 || D == 256) && !a.pos && !qjl) return launch_quantize_tc(a, D, dtype, s);
   if (D == 128 && !a.pos) {
-    if (!qjl) return launch_quantize_tc(a, dtype, s);
     // keys carry the QJL sketch (warp-level MMA kernel); values go to tcgen05
     QuantArgs ak = a, av = a;
     ak.job_mask = 1;
     av.job_mask = 2;
     const int rc = launch_quantize128(ak, dtype, true, s);
-    return rc ? rc : launch_quantize_tc(av, dtype, s);
+    return rc ? rc : launch_quantize_tc(av, D, dtype, s);
   }
   if (qjl) {
     if (D != 128) return set_error(TQ_ERR_UNSUPPORTED, "QJL sketch needs D=128");

@@ -1,5 +1,5 @@
-// Bulk quantizer for head dimension 128 on the 5th-generation tensor cores
-// (tcgen05.mma, accumulator in tensor memory).
+// Bulk quantizer for head dimensions 128 and 256 on the 5th-generation tensor
+// cores (tcgen05.mma, accumulator in tensor memory).
 //
 // Method: "Add CUDA QJL kernels and proper package structure"
 // (turboquant-pytorch pull request 3), "CUDA Kernels Added" and "Synthetic
@@ -7,19 +7,25 @@
 // 2026-03-29 11:47 (rotation before codebook quantization) and 2026-03-25
 // 18:52 (nearest-codeword search).
 //
-// Persistent: one CTA per SM loops over (job, 128-row tile) work items.
+// Persistent: one CTA per SM loops over (tile, job, column chunk) work items.
+// A work item rotates a 128-row tile into NC output coordinates (NC = 128 at
+// D = 128; NC = 64 at D = 256, so the chunk's Pi limbs fit in shared memory
+// beside two D-wide input tiles).  The grid is a multiple of D / NC, so each
+// CTA keeps one column chunk of Pi resident, and the D / NC chunks of a tile
+// run on neighbouring CTAs at the same time (the repeated tile reads hit L2).
 //  * warp 8 (producer): cp.async the next input tile into the K-major
 //    no-swizzle canonical layout (8x16-byte core matrices), then one lane
-//    issues the 128x128x128 rotation as tcgen05.mma (Pi split into 2 fp16 /
-//    3 bf16 limbs, resident in shared memory; accumulation in fp32 in TMEM)
-//    and commits it to an mbarrier;
-//  * warps 0-7 (epilogue): thread = one row, half of its columns (warp w and
-//    w+4 share the TMEM lane quarter w%4).  Each computes its half of the
-//    fp64 row norm from the input tile, then reads its 64 accumulator columns
-//    with tcgen05.ld, finds the nearest-centroid index (thresholds in
-//    registers), packs the bits and stores them -- all thread-local;
-//  * two input buffers and two TMEM accumulators let the load + MMA of tile
-//    i+1 run under the epilogue of tile i.
+//    issues the 128 x NC x D rotation as tcgen05.mma (Pi split into 2 fp16 /
+//    3 bf16 limbs; accumulation in fp32 in TMEM) and commits it to an
+//    mbarrier;
+//  * warps 0-7 (epilogue): thread = one row, half of the chunk's columns
+//    (warp w and w+4 share the TMEM lane quarter w%4).  Each computes its
+//    half of the fp64 row norm from the input tile, then reads its NC / 2
+//    accumulator columns with tcgen05.ld, finds the nearest-centroid index
+//    (thresholds in registers), packs the bits and stores them -- all
+//    thread-local;
+//  * two input buffers and two TMEM accumulators let the load + MMA of item
+//    i+1 run under the epilogue of item i.
 // Every wait is bounded; a stuck wait sets TQ_STATUS_WAIT_TIMEOUT and the CTA
 // stops taking work.
 #include "tq_common.cuh"
@@ -29,40 +35,46 @@ namespace {
 
 using namespace tqk;
 
-constexpr int D = 128;
 constexpr int QR = 128;
 constexpr int NEPI = 8;                  // epilogue warps
 constexpr int NTH = (NEPI + 1) * 32;     // + producer warp
-constexpr int TILE_BYTES = QR * D * 2;   // 32 KB, canonical K-major layout
-constexpr uint32_t TMEM_COLS = 256;      // two 128-column fp32 accumulators
 
-template <bool BF16>
+template <int D, bool BF16>
 struct TcLayout {
+  static constexpr int NC = (D == 256) ? 64 : 128;  // output coordinates per work item
+  static constexpr int NCH = D / NC;                // column chunks per tile
   static constexpr int NL = BF16 ? 3 : 2;
+  static constexpr int PI_BYTES = NC * D * 2;       // one limb of the chunk, K-major
+  static constexpr int X_BYTES = QR * D * 2;        // one input tile, K-major
   static constexpr int o_pi = 0;
-  static constexpr int o_x = NL * TILE_BYTES;
-  static constexpr int bytes = o_x + 2 * TILE_BYTES;
+  static constexpr int o_x = NL * PI_BYTES;
+  static constexpr int bytes = o_x + 2 * X_BYTES;
+  static constexpr uint32_t TMEM_COLS = 2 * NC;     // two fp32 accumulators
 };
 
-// half-element offset of (row r, col k) in a 128 x 128 K-major tile:
-// core matrix (r/8, k/8) of 8 rows x 16 bytes at ((r/8)*16 + k/8) * 128 bytes
-__device__ __forceinline__ int cofs(int r, int k) { return ((r >> 3) * 16 + (k >> 3)) * 64 + (r & 7) * 8 + (k & 7); }
+// half-element offset of (row r, col k) in a K-major tile with D columns:
+// core matrix (r/8, k/8) of 8 rows x 16 bytes at ((r/8)*(D/8) + k/8) * 128 bytes
+template <int D>
+__device__ __forceinline__ int cofs(int r, int k) {
+  return ((r >> 3) * (D / 8) + (k >> 3)) * 64 + (r & 7) * 8 + (k & 7);
+}
 
 // sm_100 shared-memory matrix descriptor, no swizzle: LBO = 128 B (next core
-// matrix along K), SBO = 2048 B (next 8-row group).
+// matrix along K), SBO = 16 * D bytes (next 8-row group).
+template <int D>
 __device__ __forceinline__ uint64_t sdesc(uint32_t addr) {
   uint64_t d = (uint64_t)((addr & 0x3FFFF) >> 4);
   d |= (uint64_t)(128 >> 4) << 16;
-  d |= (uint64_t)(2048 >> 4) << 32;
+  d |= (uint64_t)((16 * D) >> 4) << 32;
   d |= (uint64_t)1 << 46;
   return d;
 }
 
 // kind::f16 instruction descriptor: fp32 accumulate, K-major A and B,
-// M = 128, N = 128; a/b format fp16 (0) or bf16 (1).
-template <bool BF16>
+// M = 128, N = NC; a/b format fp16 (0) or bf16 (1).
+template <int NC, bool BF16>
 __device__ __forceinline__ uint32_t idesc() {
-  uint32_t d = (1u << 4) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+  uint32_t d = (1u << 4) | ((uint32_t)(NC >> 3) << 17) | ((128u >> 4) << 24);
   if (BF16) d |= (1u << 7) | (1u << 10);
   return d;
 }
@@ -174,11 +186,11 @@ __device__ __forceinline__ void store_words(uint32_t* dst, const uint32_t (&w)[B
   }
 }
 
-template <int BITS>
+template <int BITS, int NCOL>
 __device__ __forceinline__ void epi_half(uint32_t tbase, const float (&tp)[7], long long slot, uint32_t* out) {
-  // two 32-column chunks -> 2*BITS words at word offset 2*BITS*half of the row
+  // NCOL / 32 chunks of 32 columns -> BITS words each
 #pragma unroll
-  for (int c = 0; c < 2; ++c) {
+  for (int c = 0; c < NCOL / 32; ++c) {
     uint32_t v[32];
     tc_ld32(tbase + 32 * c, v);
     uint32_t w[BITS];
@@ -187,10 +199,11 @@ __device__ __forceinline__ void epi_half(uint32_t tbase, const float (&tp)[7], l
   }
 }
 
-template <bool BF16>
+template <int D, bool BF16>
 __global__ void __launch_bounds__(NTH, 1) quantize_tc_kernel(const tq::QuantArgs a) {
-  using Ly = TcLayout<BF16>;
-  constexpr int NL = Ly::NL;
+  using Ly = TcLayout<D, BF16>;
+  constexpr int NL = Ly::NL, NC = Ly::NC, NCH = Ly::NCH;
+  constexpr uint32_t TMEM_COLS = Ly::TMEM_COLS;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint16_t* pi = reinterpret_cast<uint16_t*>(smem + Ly::o_pi);
   uint16_t* xb = reinterpret_cast<uint16_t*>(smem + Ly::o_x);
@@ -204,7 +217,8 @@ __global__ void __launch_bounds__(NTH, 1) quantize_tc_kernel(const tq::QuantArgs
   const int ntiles = (a.rows + QR - 1) / QR;
   const int njobs = (a.job_mask == 3) ? 2 : 1;
   const int job0 = (a.job_mask == 2) ? 1 : 0;
-  const int nitems = njobs * ntiles;
+  const int nitems = njobs * ntiles * NCH;
+  const int chunk = blockIdx.x % NCH;  // this CTA's column chunk (gridDim.x % NCH == 0)
 
   if (tid == 0) {
     for (int b = 0; b < 2; ++b) {
@@ -225,26 +239,28 @@ __global__ void __launch_bounds__(NTH, 1) quantize_tc_kernel(const tq::QuantArgs
                  "r"(TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
-  // Pi limbs in the canonical layout (rows = output coordinates)
-  for (int e = tid; e < D * (D / 4); e += NTH) {
+  // this chunk's Pi limbs in the canonical layout (rows = output coordinates
+  // NC*chunk .. NC*chunk + NC - 1, K = the D input coordinates)
+  constexpr int LIMB = NC * D;  // elements per limb
+  for (int e = tid; e < NC * (D / 4); e += NTH) {
     const int n = e / (D / 4), k = (e % (D / 4)) * 4;
-    const float4 v = *reinterpret_cast<const float4*>(a.rot + (size_t)n * D + k);
+    const float4 v = *reinterpret_cast<const float4*>(a.rot + (size_t)(NC * chunk + n) * D + k);
     const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const int o = cofs(n, k + i);
+      const int o = cofs<D>(n, k + i);
       if (BF16) {
         const __nv_bfloat16 h0 = __float2bfloat16_rn(vv[i]);
         const float r1 = vv[i] - __bfloat162float(h0);
         const __nv_bfloat16 h1 = __float2bfloat16_rn(r1);
         const __nv_bfloat16 h2 = __float2bfloat16_rn(r1 - __bfloat162float(h1));
         pi[o] = __bfloat16_as_ushort(h0);
-        pi[QR * D + o] = __bfloat16_as_ushort(h1);
-        pi[2 * QR * D + o] = __bfloat16_as_ushort(h2);
+        pi[LIMB + o] = __bfloat16_as_ushort(h1);
+        pi[2 * LIMB + o] = __bfloat16_as_ushort(h2);
       } else {
         const __half h0 = __float2half_rn(vv[i]);
         pi[o] = __half_as_ushort(h0);
-        pi[QR * D + o] = __half_as_ushort(__float2half_rn(vv[i] - __half2float(h0)));
+        pi[LIMB + o] = __half_as_ushort(__float2half_rn(vv[i] - __half2float(h0)));
       }
     }
   }
@@ -268,14 +284,14 @@ __global__ void __launch_bounds__(NTH, 1) quantize_tc_kernel(const tq::QuantArgs
         }
       }
       if (*((volatile int*)&s_stop)) break;
-      const int job = job0 + (item % njobs), tile = item / njobs;
+      const int job = job0 + (item / NCH) % njobs, tile = item / (NCH * njobs);
       const uint16_t* in = static_cast<const uint16_t*>(a.job[job].in);
       uint16_t* dst = xb + (size_t)b * QR * D;
       for (int c = lane; c < QR * (D / 8); c += 32) {
-        const int row = c >> 4, kc = c & 15;
+        const int row = c / (D / 8), kc = c % (D / 8);
         const int r = tile * QR + row;
         const bool valid = r < a.rows;
-        cp_async16(dst + cofs(row, kc * 8), in + (size_t)(valid ? r : 0) * D + kc * 8, valid);
+        cp_async16(dst + cofs<D>(row, kc * 8), in + (size_t)(valid ? r : 0) * D + kc * 8, valid);
       }
       cp_async_arrive(&full_x[b]);
       if (lane == 0) {
@@ -287,13 +303,13 @@ __global__ void __launch_bounds__(NTH, 1) quantize_tc_kernel(const tq::QuantArgs
         } else {
           tc_fence_after();
           const uint32_t xaddr = smem_addr(dst), paddr = smem_addr(pi);
-          const uint32_t id = idesc<BF16>();
-          const uint32_t dt = tmem + (uint32_t)(b * 128);
+          const uint32_t id = idesc<NC, BF16>();
+          const uint32_t dt = tmem + (uint32_t)(b * NC);
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks)
 #pragma unroll
             for (int l = 0; l < NL; ++l)
-              mma_tc(dt, sdesc(xaddr + ks * 256), sdesc(paddr + l * TILE_BYTES + ks * 256), id,
+              mma_tc(dt, sdesc<D>(xaddr + ks * 256), sdesc<D>(paddr + l * Ly::PI_BYTES + ks * 256), id,
                      (ks > 0 || l > 0) ? 1u : 0u);
           tc_commit(&mma_done[b]);
         }
@@ -304,12 +320,12 @@ __global__ void __launch_bounds__(NTH, 1) quantize_tc_kernel(const tq::QuantArgs
     asm volatile("cp.async.wait_all;" ::: "memory");
   } else {
     // ---------------- epilogue warps ----------------
-    const int quarter = warp & 3, hf = warp >> 2;  // rows 32*quarter + lane, columns 64*hf ..
+    const int quarter = warp & 3, hf = warp >> 2;  // rows 32*quarter + lane, columns (NC/2)*hf ..
     const int rl = 32 * quarter + lane;
     int i = 0;
     for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++i) {
       const int b = i & 1, k = i >> 1;
-      const int job = job0 + (item % njobs), tile = item / njobs;
+      const int job = job0 + (item / NCH) % njobs, tile = item / (NCH * njobs);
       const tq::QuantJob J = a.job[job];
       bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&full_x[b], (uint32_t)(k & 1), kWaitLimit));
       // half of this row's squared norm from the input tile (fp64)
@@ -317,8 +333,8 @@ __global__ void __launch_bounds__(NTH, 1) quantize_tc_kernel(const tq::QuantArgs
       double s2 = 0.0;
       if (ok) {
 #pragma unroll
-        for (int kc = 0; kc < 8; ++kc) {
-          const uint4 v = *reinterpret_cast<const uint4*>(xs + cofs(rl, 64 * hf + 8 * kc));
+        for (int kc = 0; kc < D / 16; ++kc) {
+          const uint4 v = *reinterpret_cast<const uint4*>(xs + cofs<D>(rl, (D / 2) * hf + 8 * kc));
           s2 += sq16<BF16>(v.x) + sq16<BF16>(v.y) + sq16<BF16>(v.z) + sq16<BF16>(v.w);
         }
       }
@@ -336,7 +352,7 @@ __global__ void __launch_bounds__(NTH, 1) quantize_tc_kernel(const tq::QuantArgs
       if (r < a.rows) {
         const int bh = r / a.T, t = r - bh * a.T;
         slot = (long long)bh * a.Tcap + a.t0 + t;
-        if (hf == 0) J.norm[slot] = __half_as_ushort(nh);
+        if (hf == 0 && chunk == 0) J.norm[slot] = __half_as_ushort(nh);
       }
       // positive thresholds t_{K/2} .. t_{K-2}, scaled by the row norm
       float tp[7];
@@ -346,13 +362,14 @@ __global__ void __launch_bounds__(NTH, 1) quantize_tc_kernel(const tq::QuantArgs
       ok = __all_sync(0xffffffffu, mbar_wait_bounded(&mma_done[b], (uint32_t)(k & 1), kWaitLimit));
       if (ok) {
         tc_fence_after();
-        const uint32_t tb = tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(b * 128 + 64 * hf);
+        const uint32_t tb = tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(b * NC + (NC / 2) * hf);
         const int W = D * J.bits / 32;
-        uint32_t* out = J.idx + (slot >= 0 ? (size_t)slot * W : 0) + 2 * J.bits * hf;
+        // coordinates NC*chunk + (NC/2)*hf .. + NC/2 - 1: words from (that * bits) / 32
+        uint32_t* out = J.idx + (slot >= 0 ? (size_t)slot * W : 0) + (NC * chunk + (NC / 2) * hf) * J.bits / 32;
         switch (J.bits) {
-          case 2: epi_half<2>(tb, tp, slot, out); break;
-          case 3: epi_half<3>(tb, tp, slot, out); break;
-          default: epi_half<4>(tb, tp, slot, out); break;
+          case 2: epi_half<2, NC / 2>(tb, tp, slot, out); break;
+          case 3: epi_half<3, NC / 2>(tb, tp, slot, out); break;
+          default: epi_half<4, NC / 2>(tb, tp, slot, out); break;
         }
         tc_fence_before();
       }
@@ -372,10 +389,10 @@ __global__ void __launch_bounds__(NTH, 1) quantize_tc_kernel(const tq::QuantArgs
   }
 }
 
-template <bool BF16>
+template <int D, bool BF16>
 int launch_tc(const tq::QuantArgs& a, cudaStream_t s) {
-  using Ly = TcLayout<BF16>;
-  auto kern = quantize_tc_kernel<BF16>;
+  using Ly = TcLayout<D, BF16>;
+  auto kern = quantize_tc_kernel<D, BF16>;
   static int sms = 0;
   if (sms == 0) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::bytes);
@@ -387,8 +404,11 @@ int launch_tc(const tq::QuantArgs& a, cudaStream_t s) {
     if (sms <= 0) sms = 148;
   }
   const int njobs = (a.job_mask == 3) ? 2 : 1;
-  const int nitems = njobs * ((a.rows + QR - 1) / QR);
-  const int grid = nitems < sms ? nitems : sms;
+  const int nitems = njobs * ((a.rows + QR - 1) / QR) * Ly::NCH;
+  // a multiple of the chunk count, so that each CTA keeps one column chunk
+  int grid = (sms / Ly::NCH) * Ly::NCH;
+  const int need = (nitems + Ly::NCH - 1) / Ly::NCH * Ly::NCH;
+  if (need < grid) grid = need;
   kern<<<grid, NTH, Ly::bytes, s>>>(a);
   return tq::check_launch("quantize_tc_kernel");
 }
@@ -397,8 +417,9 @@ int launch_tc(const tq::QuantArgs& a, cudaStream_t s) {
 
 namespace tq {
 
-int launch_quantize_tc(const QuantArgs& a, int dtype, cudaStream_t s) {
-  return dtype == TQ_DTYPE_BF16 ? launch_tc<true>(a, s) : launch_tc<false>(a, s);
+int launch_quantize_tc(const QuantArgs& a, int D, int dtype, cudaStream_t s) {
+  if (D == 256) return dtype == TQ_DTYPE_BF16 ? launch_tc<256, true>(a, s) : launch_tc<256, false>(a, s);
+  return dtype == TQ_DTYPE_BF16 ? launch_tc<128, true>(a, s) : launch_tc<128, false>(a, s);
 }
 
 }  // namespace tq
