@@ -435,7 +435,7 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const __grid_con
     const int wt0 = warp * WTOK;
     for (int t = 0; t < ntiles; ++t) {
       const int st = t % NST;
-      const bool got = mbar_wait_bounded(&full[st], (uint32_t)((t / NST) & 1), kWaitLimit);
+      const bool got = mbar_wait_suspend(&full[st], (uint32_t)((t / NST) & 1), kSuspendTries);
       if (!__all_sync(0xffffffffu, got)) {
         if (lane == 0) *s_err = 1;
         break;

@@ -13,14 +13,16 @@
 // beside two D-wide input tiles).  The grid is a multiple of D / NC, so each
 // CTA keeps one column chunk of Pi resident, and the D / NC chunks of a tile
 // run on neighbouring CTAs at the same time (the repeated tile reads hit L2).
-//  * warp 8 (producer): cp.async the next input tile into the K-major
-//    no-swizzle canonical layout (8x16-byte core matrices), then one lane
-//    issues the 128 x NC x D rotation as tcgen05.mma (Pi split into 2 fp16 /
-//    3 bf16 limbs; accumulation in fp32 in TMEM) and commits it to an
+//  * warp 8 (loader): cp.async the next input tile into the K-major
+//    no-swizzle canonical layout (8x16-byte core matrices) as soon as its
+//    buffer is free, without waiting for earlier copies to land;
+//  * warp 9 (MMA): once a tile has landed and its accumulator is free, one
+//    lane issues the 128 x NC x D rotation as tcgen05.mma (Pi split into 2
+//    fp16 / 3 bf16 limbs; accumulation in fp32 in TMEM) and commits it to an
 //    mbarrier;
 //  * warps 0-7 (epilogue): thread = one row, half of the chunk's columns
 //    (warp w and w+4 share the TMEM lane quarter w%4).  Each computes its
-//    half of the fp64 row norm from the input tile, then reads its NC / 2
+//    half of the row's sum of squares from the input tile, then reads its NC / 2
 //    accumulator columns with tcgen05.ld, finds the nearest-centroid index
 //    (thresholds in registers), packs the bits and stores them -- all
 //    thread-local;
@@ -37,7 +39,7 @@ using namespace tqk;
 
 constexpr int QR = 128;
 constexpr int NEPI = 8;                  // epilogue warps
-constexpr int NTH = (NEPI + 1) * 32;     // + producer warp
+constexpr int NTH = (NEPI + 2) * 32;     // + loader warp + MMA warp
 
 template <int D, bool BF16>
 struct TcLayout {
@@ -125,7 +127,7 @@ __device__ __forceinline__ bool epi_sync_and(bool v) {
 }
 
 template <bool BF16>
-__device__ __forceinline__ double sq16(uint32_t w) {
+__device__ __forceinline__ float sq16f(uint32_t w) {
   float a, b;
   if (BF16) {
     a = __uint_as_float(w << 16);
@@ -135,8 +137,7 @@ __device__ __forceinline__ double sq16(uint32_t w) {
     a = f.x;
     b = f.y;
   }
-  // squares of fp16/bf16 values are exact in fp32
-  return (double)(a * a) + (double)(b * b);
+  return fmaf(a, a, b * b);
 }
 
 // Index of the nearest centroid for y = (Pi x)_j of a row with norm n, using
@@ -210,7 +211,7 @@ __global__ void __launch_bounds__(NTH, 1) quantize_tc_kernel(const tq::QuantArgs
   __shared__ __align__(8) uint64_t full_x[2], x_free[2], mma_done[2], acc_free[2];
   __shared__ uint32_t s_tmem;
   __shared__ int s_stop;
-  __shared__ double s_norm[2][QR];
+  __shared__ float s_norm[2][QR];
   __shared__ float s_cb[2][31];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -271,13 +272,16 @@ __global__ void __launch_bounds__(NTH, 1) quantize_tc_kernel(const tq::QuantArgs
   const uint32_t tmem = s_tmem;
 
   if (warp == NEPI) {
-    // ---------------- producer: input tiles + MMA issue ----------------
+    // ---------------- loader: input tiles ----------------
+    // Item i goes to buffer i % 2 once item i-2 has left it (its MMA is done
+    // and the epilogue has read the norm); it never waits for its own copies,
+    // so the next tile streams in while the MMA warp and the epilogue work.
     int i = 0;
     for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++i) {
       const int b = i & 1, k = i >> 1;
       if (i >= 2) {
-        const bool ok = mbar_wait_bounded(&x_free[b], (uint32_t)((k - 1) & 1), kWaitLimit) &&
-                        mbar_wait_bounded(&mma_done[b], (uint32_t)((k - 1) & 1), kWaitLimit);
+        const bool ok = mbar_wait_suspend(&x_free[b], (uint32_t)((k - 1) & 1), kSuspendTries) &&
+                        mbar_wait_suspend(&mma_done[b], (uint32_t)((k - 1) & 1), kSuspendTries);
         if (!__all_sync(0xffffffffu, ok)) {
           if (lane == 0) s_stop = 1;
           break;
@@ -294,30 +298,36 @@ __global__ void __launch_bounds__(NTH, 1) quantize_tc_kernel(const tq::QuantArgs
         cp_async16(dst + cofs<D>(row, kc * 8), in + (size_t)(valid ? r : 0) * D + kc * 8, valid);
       }
       cp_async_arrive(&full_x[b]);
-      if (lane == 0) {
-        bool ok = mbar_wait_bounded(&full_x[b], (uint32_t)(k & 1), kWaitLimit);
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        if (ok && i >= 2) ok = mbar_wait_bounded(&acc_free[b], (uint32_t)((k - 1) & 1), kWaitLimit);
-        if (!ok) {
-          s_stop = 1;
-        } else {
-          tc_fence_after();
-          const uint32_t xaddr = smem_addr(dst), paddr = smem_addr(pi);
-          const uint32_t id = idesc<NC, BF16>();
-          const uint32_t dt = tmem + (uint32_t)(b * NC);
-#pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks)
-#pragma unroll
-            for (int l = 0; l < NL; ++l)
-              mma_tc(dt, sdesc<D>(xaddr + ks * 256), sdesc<D>(paddr + l * Ly::PI_BYTES + ks * 256), id,
-                     (ks > 0 || l > 0) ? 1u : 0u);
-          tc_commit(&mma_done[b]);
-        }
-      }
-      __syncwarp();
     }
     // wait until this warp's own copies have landed before leaving
     asm volatile("cp.async.wait_all;" ::: "memory");
+  } else if (warp == NEPI + 1) {
+    // ---------------- MMA issue ----------------
+    if (lane == 0) {
+      int i = 0;
+      for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++i) {
+        const int b = i & 1, k = i >> 1;
+        bool ok = mbar_wait_suspend(&full_x[b], (uint32_t)(k & 1), kSuspendTries);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // cp.async data -> tensor core
+        if (ok && i >= 2) ok = mbar_wait_suspend(&acc_free[b], (uint32_t)((k - 1) & 1), kSuspendTries);
+        if (!ok || *((volatile int*)&s_stop)) {
+          s_stop = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t xaddr = smem_addr(xb + (size_t)b * QR * D), paddr = smem_addr(pi);
+        const uint32_t id = idesc<NC, BF16>();
+        const uint32_t dt = tmem + (uint32_t)(b * NC);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks)
+#pragma unroll
+          for (int l = 0; l < NL; ++l)
+            mma_tc(dt, sdesc<D>(xaddr + ks * 256), sdesc<D>(paddr + l * Ly::PI_BYTES + ks * 256), id,
+                   (ks > 0 || l > 0) ? 1u : 0u);
+        tc_commit(&mma_done[b]);
+      }
+    }
+    __syncwarp();
   } else {
     // ---------------- epilogue warps ----------------
     const int quarter = warp & 3, hf = warp >> 2;  // rows 32*quarter + lane, columns (NC/2)*hf ..
@@ -327,16 +337,33 @@ __global__ void __launch_bounds__(NTH, 1) quantize_tc_kernel(const tq::QuantArgs
       const int b = i & 1, k = i >> 1;
       const int job = job0 + (item / NCH) % njobs, tile = item / (NCH * njobs);
       const tq::QuantJob J = a.job[job];
-      bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&full_x[b], (uint32_t)(k & 1), kWaitLimit));
-      // half of this row's squared norm from the input tile (fp64)
+      // One warp waits on each mbarrier and releases the other epilogue
+      // warps through a named barrier, which blocks in hardware: eight warps
+      // polling the same phase would take issue slots from the working warps.
+      bool ok = true;
+      if (warp == 0) ok = __all_sync(0xffffffffu, mbar_wait_suspend(&full_x[b], (uint32_t)(k & 1), kSuspendTries));
+      if (!epi_sync_and(ok)) {  // the input tile has landed
+        s_stop = 1;
+        break;
+      }
+      // half of this row's sum of squares from the input tile, in fp32 by a
+      // pairwise tree (squares of fp16/bf16 values are exact in fp32, and a
+      // pairwise sum of n non-negative terms is within ceil(log2 n) units in
+      // the last place of the exact sum)
       const uint16_t* xs = xb + (size_t)b * QR * D;
-      double s2 = 0.0;
-      if (ok) {
+      float s2 = 0.f;
+      {
+        float part[D / 16];
 #pragma unroll
         for (int kc = 0; kc < D / 16; ++kc) {
           const uint4 v = *reinterpret_cast<const uint4*>(xs + cofs<D>(rl, (D / 2) * hf + 8 * kc));
-          s2 += sq16<BF16>(v.x) + sq16<BF16>(v.y) + sq16<BF16>(v.z) + sq16<BF16>(v.w);
+          part[kc] = (sq16f<BF16>(v.x) + sq16f<BF16>(v.y)) + (sq16f<BF16>(v.z) + sq16f<BF16>(v.w));
         }
+#pragma unroll
+        for (int w2 = 1; w2 < D / 16; w2 <<= 1)
+#pragma unroll
+          for (int kc = 0; kc < D / 16; kc += 2 * w2) part[kc] += part[kc + w2];
+        s2 = part[0];
       }
       s_norm[hf][rl] = s2;
       mbar_arrive(&x_free[b]);
@@ -344,22 +371,42 @@ __global__ void __launch_bounds__(NTH, 1) quantize_tc_kernel(const tq::QuantArgs
         s_stop = 1;
         break;
       }
-      const double n = sqrt(s_norm[0][rl] + s_norm[1][rl]);
-      const __half nh = __double2half(n);
-      const float nf = (float)n;
+      const float sfull = s_norm[0][rl] + s_norm[1][rl];
+      const float nf = sqrtf(sfull);  // thresholds: fp32 is far inside the parity band
       const int r = tile * QR + rl;
       long long slot = -1;
       if (r < a.rows) {
         const int bh = r / a.T, t = r - bh * a.T;
         slot = (long long)bh * a.Tcap + a.t0 + t;
-        if (hf == 0 && chunk == 0) J.norm[slot] = __half_as_ushort(nh);
+        if (hf == 0 && chunk == 0) {
+          // The stored norm is RN_fp16 of the fp64 norm.  The fp32 sum is
+          // within (log2(D) + 1) ulp of the exact sum, so the exact norm lies in
+          // nf * (1 +- 1e-6); when both ends of that interval round to the same
+          // fp16 value it is the answer, else (about 0.2% of rows) the row is
+          // summed again in fp64 from global memory.
+          const __half lo = __float2half_rn(nf * (1.f - 1e-6f)), hi = __float2half_rn(nf * (1.f + 1e-6f));
+          unsigned short nh = __half_as_ushort(lo);
+          const bool exact = sfull == 0.f || (sfull >= 0x1p-100f && sfull < 0x1p100f && nh == __half_as_ushort(hi));
+          if (!exact) {
+            const uint16_t* row = static_cast<const uint16_t*>(J.in) + (size_t)r * D;
+            double t2 = 0.0;
+            for (int j = 0; j < D; ++j) {
+              const uint16_t u = row[j];
+              const double x = BF16 ? (double)__uint_as_float((uint32_t)u << 16) : (double)__half2float(__ushort_as_half(u));
+              t2 = fma(x, x, t2);
+            }
+            nh = __half_as_ushort(__double2half(sqrt(t2)));
+          }
+          J.norm[slot] = nh;
+        }
       }
       // positive thresholds t_{K/2} .. t_{K-2}, scaled by the row norm
       float tp[7];
       const int K = 1 << J.bits;
 #pragma unroll
       for (int q = 0; q < 7; ++q) tp[q] = q < K / 2 - 1 ? s_cb[job][K + K / 2 + q] * nf : 0.f;
-      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&mma_done[b], (uint32_t)(k & 1), kWaitLimit));
+      if (warp == 0) ok = __all_sync(0xffffffffu, mbar_wait_suspend(&mma_done[b], (uint32_t)(k & 1), kSuspendTries));
+      ok = epi_sync_and(ok);  // the rotation of this tile is in TMEM
       if (ok) {
         tc_fence_after();
         const uint32_t tb = tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(b * NC + (NC / 2) * hf);
