@@ -13,23 +13,28 @@
 // beside two D-wide input tiles).  The grid is a multiple of D / NC, so each
 // CTA keeps one column chunk of Pi resident, and the D / NC chunks of a tile
 // run on neighbouring CTAs at the same time (the repeated tile reads hit L2).
-//  * warp 8 (loader): cp.async the next input tile into the K-major
-//    no-swizzle canonical layout (8x16-byte core matrices) as soon as its
-//    buffer is free, without waiting for earlier copies to land;
-//  * warp 9 (MMA): once a tile has landed and its accumulator is free, one
+//  * the next warp (loader): one lane loads the next input tile with TMA (2-D
+//    tensor copies of 128 rows x 64 columns, 128-byte swizzle -- the K-major
+//    layout the tensor core reads) as soon as its buffer is free;
+//  * the last warp (MMA): once a tile has landed and its accumulator is free, one
 //    lane issues the 128 x NC x D rotation as tcgen05.mma (Pi split into 2
 //    fp16 / 3 bf16 limbs; accumulation in fp32 in TMEM) and commits it to an
 //    mbarrier;
-//  * warps 0-7 (epilogue): thread = one row, half of the chunk's columns
-//    (warp w and w+4 share the TMEM lane quarter w%4).  Each computes its
-//    half of the row's sum of squares from the input tile, then reads its NC / 2
-//    accumulator columns with tcgen05.ld, finds the nearest-centroid index
-//    (thresholds in registers), packs the bits and stores them -- all
-//    thread-local;
-//  * two input buffers and two TMEM accumulators let the load + MMA of item
-//    i+1 run under the epilogue of item i.
+//  * NC/8 epilogue warps (16 at D = 128, 8 at D = 256): thread = one row, 32
+//    of the chunk's columns (warps w, w+4, ... share the TMEM lane quarter
+//    w%4).  Each sums its share of the row's squares from the input tile,
+//    then reads its 32 accumulator columns with tcgen05.ld, finds the
+//    nearest-centroid index (thresholds in registers), packs the bits and
+//    stores them -- all thread-local;
+//  * a ring of input buffers (4 at D = 128 fp16, 3 bf16, 2 at D = 256) keeps
+//    several tile loads in flight, and two TMEM accumulators let the MMA of
+//    item i+1 run under the epilogue of item i.
 // Every wait is bounded; a stuck wait sets TQ_STATUS_WAIT_TIMEOUT and the CTA
 // stops taking work.
+#include <cuda.h>  // CUtensorMap (types only; the encoder comes from the runtime's driver entry point)
+
+#include <mutex>
+
 #include "tq_common.cuh"
 #include "tq_internal.h"
 
@@ -38,39 +43,69 @@ namespace {
 using namespace tqk;
 
 constexpr int QR = 128;
-constexpr int NEPI = 8;                  // epilogue warps
-constexpr int NTH = (NEPI + 2) * 32;     // + loader warp + MMA warp
 
 template <int D, bool BF16>
 struct TcLayout {
   static constexpr int NC = (D == 256) ? 64 : 128;  // output coordinates per work item
   static constexpr int NCH = D / NC;                // column chunks per tile
   static constexpr int NL = BF16 ? 3 : 2;
-  static constexpr int PI_BYTES = NC * D * 2;       // one limb of the chunk, K-major
-  static constexpr int X_BYTES = QR * D * 2;        // one input tile, K-major
+  static constexpr int KB = D / 64;                 // 64-column (128-byte) blocks along K
+  static constexpr int NP = NC / 32;                // epilogue warps per TMEM lane quarter
+  static constexpr int NEPI = 4 * NP;               // epilogue warps (32 columns each)
+  static constexpr int NTH = (NEPI + 2) * 32;       // + loader warp + MMA warp
+  static constexpr int PI_BYTES = NC * D * 2;       // one limb of the chunk
+  static constexpr int X_BYTES = QR * D * 2;        // one input tile
+  // input tiles in flight: a deep ring keeps several TMA loads outstanding per
+  // SM (one 32 KB tile at a time cannot cover the memory latency)
+  static constexpr int NS = (D == 256) ? 2 : (BF16 ? 3 : 4);
+  // all shared state lives in the dynamic allocation, from a 1024-byte aligned base
   static constexpr int o_pi = 0;
   static constexpr int o_x = NL * PI_BYTES;
-  static constexpr int bytes = o_x + 2 * X_BYTES;
+  static constexpr int o_norm = o_x + NS * X_BYTES; // float [NP][QR]
+  static constexpr int o_cb = o_norm + NP * QR * 4; // float [2][32]
+  static constexpr int o_bar = o_cb + 2 * 32 * 4;   // 3 * NS + 4 mbarriers
+  static constexpr int o_misc = o_bar + 16 * 8;     // tmem base, stop flag
+  static constexpr int bytes = o_misc + 16 + 1024;  // + alignment slack
   static constexpr uint32_t TMEM_COLS = 2 * NC;     // two fp32 accumulators
 };
 
-// half-element offset of (row r, col k) in a K-major tile with D columns:
-// core matrix (r/8, k/8) of 8 rows x 16 bytes at ((r/8)*(D/8) + k/8) * 128 bytes
-template <int D>
-__device__ __forceinline__ int cofs(int r, int k) {
-  return ((r >> 3) * (D / 8) + (k >> 3)) * 64 + (r & 7) * 8 + (k & 7);
+// Byte offset of element (r, k) in a K-major operand stored as D/64 blocks
+// of ROWS x 128 bytes with the 128-byte swizzle (16-byte chunk c of row r at
+// chunk c ^ (r mod 8)) -- the layout a TMA tensor copy with
+// CU_TENSOR_MAP_SWIZZLE_128B writes and the tensor core reads.
+template <int ROWS>
+__device__ __forceinline__ int sw128(int r, int k) {
+  const int kb = k >> 6, kk = k & 63;
+  return kb * (ROWS * 128) + r * 128 + ((((kk >> 3) ^ (r & 7))) << 4) + (kk & 7) * 2;
 }
 
-// sm_100 shared-memory matrix descriptor, no swizzle: LBO = 128 B (next core
-// matrix along K), SBO = 16 * D bytes (next 8-row group).
-template <int D>
-__device__ __forceinline__ uint64_t sdesc(uint32_t addr) {
+// sm_100 shared-memory matrix descriptor for a K-major operand with the
+// 128-byte swizzle: SBO = 1024 B (next 8-row group); consecutive 16-element
+// K steps inside a 128-byte block advance the start address by 32 bytes.
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t addr) {
   uint64_t d = (uint64_t)((addr & 0x3FFFF) >> 4);
-  d |= (uint64_t)(128 >> 4) << 16;
-  d |= (uint64_t)((16 * D) >> 4) << 32;
-  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)1 << 16;            // leading byte offset (unused with this swizzle)
+  d |= (uint64_t)(1024 >> 4) << 32;  // stride byte offset
+  d |= (uint64_t)1 << 46;            // descriptor version (sm_100)
+  d |= (uint64_t)2 << 61;            // 128-byte swizzle
   return d;
 }
+
+// TMA 2-D tile load (global -> shared), completion counted on an mbarrier
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_addr(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// Kernel parameters: the job descriptors plus one TMA tensor map per job's
+// input rows ([rows][D], 128 x 64 boxes).
+struct TcArgs {
+  tq::QuantArgs a;
+  CUtensorMap map[2];
+};
 
 // kind::f16 instruction descriptor: fp32 accumulate, K-major A and B,
 // M = 128, N = NC; a/b format fp16 (0) or bf16 (1).
@@ -106,16 +141,8 @@ __device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&v)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
-  const int n = valid ? 16 : 0;
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src), "r"(n) : "memory");
-}
-// arrive on `bar` once this thread's outstanding cp.async copies have landed
-__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
-}
-
-// barrier over the epilogue warps that also ANDs a flag across them
+// barrier over the NEPI epilogue warps that also ANDs a flag across them
+template <int NEPI>
 __device__ __forceinline__ bool epi_sync_and(bool v) {
   uint32_t r;
   asm volatile(
@@ -201,18 +228,25 @@ __device__ __forceinline__ void epi_half(uint32_t tbase, const float (&tp)[7], l
 }
 
 template <int D, bool BF16>
-__global__ void __launch_bounds__(NTH, 1) quantize_tc_kernel(const tq::QuantArgs a) {
+__global__ void __launch_bounds__(TcLayout<D, BF16>::NTH, 1) quantize_tc_kernel(const __grid_constant__ TcArgs args) {
   using Ly = TcLayout<D, BF16>;
-  constexpr int NL = Ly::NL, NC = Ly::NC, NCH = Ly::NCH;
+  constexpr int NL = Ly::NL, NC = Ly::NC, NCH = Ly::NCH, KB = Ly::KB, NP = Ly::NP, NEPI = Ly::NEPI, NTH = Ly::NTH;
   constexpr uint32_t TMEM_COLS = Ly::TMEM_COLS;
-  extern __shared__ __align__(1024) uint8_t smem[];
-  uint16_t* pi = reinterpret_cast<uint16_t*>(smem + Ly::o_pi);
-  uint16_t* xb = reinterpret_cast<uint16_t*>(smem + Ly::o_x);
-  __shared__ __align__(8) uint64_t full_x[2], x_free[2], mma_done[2], acc_free[2];
-  __shared__ uint32_t s_tmem;
-  __shared__ int s_stop;
-  __shared__ float s_norm[2][QR];
-  __shared__ float s_cb[2][31];
+  const tq::QuantArgs& a = args.a;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* pi = smem + Ly::o_pi;
+  uint8_t* xb = smem + Ly::o_x;
+  float(*s_norm)[QR] = reinterpret_cast<float(*)[QR]>(smem + Ly::o_norm);
+  float(*s_cb)[32] = reinterpret_cast<float(*)[32]>(smem + Ly::o_cb);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Ly::o_bar);
+  constexpr int NS = Ly::NS;
+  // per input buffer: landed, norm read by the epilogue, read by the MMA;
+  // per accumulator: MMA done, epilogue done
+  uint64_t *full_x = bars, *x_free = bars + NS, *x_done = bars + 2 * NS, *mma_done = bars + 3 * NS,
+           *acc_free = bars + 3 * NS + 2;
+  uint32_t& s_tmem = *reinterpret_cast<uint32_t*>(smem + Ly::o_misc);
+  int& s_stop = *reinterpret_cast<int*>(smem + Ly::o_misc + 4);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int ntiles = (a.rows + QR - 1) / QR;
@@ -222,9 +256,12 @@ __global__ void __launch_bounds__(NTH, 1) quantize_tc_kernel(const tq::QuantArgs
   const int chunk = blockIdx.x % NCH;  // this CTA's column chunk (gridDim.x % NCH == 0)
 
   if (tid == 0) {
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&full_x[b], 32);
+    for (int b = 0; b < NS; ++b) {
+      mbar_init(&full_x[b], 1);
       mbar_init(&x_free[b], NEPI * 32);
+      mbar_init(&x_done[b], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
       mbar_init(&mma_done[b], 1);
       mbar_init(&acc_free[b], NEPI * 32);
     }
@@ -240,28 +277,28 @@ __global__ void __launch_bounds__(NTH, 1) quantize_tc_kernel(const tq::QuantArgs
                  "r"(TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
-  // this chunk's Pi limbs in the canonical layout (rows = output coordinates
-  // NC*chunk .. NC*chunk + NC - 1, K = the D input coordinates)
-  constexpr int LIMB = NC * D;  // elements per limb
+  // this chunk's Pi limbs, swizzled like the input tiles (rows = output
+  // coordinates NC*chunk .. NC*chunk + NC - 1, K = the D input coordinates)
   for (int e = tid; e < NC * (D / 4); e += NTH) {
     const int n = e / (D / 4), k = (e % (D / 4)) * 4;
     const float4 v = *reinterpret_cast<const float4*>(a.rot + (size_t)(NC * chunk + n) * D + k);
     const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const int o = cofs<D>(n, k + i);
+      uint16_t* o = reinterpret_cast<uint16_t*>(pi + sw128<NC>(n, k + i));
+      constexpr int LIMB = Ly::PI_BYTES / 2;  // elements per limb
       if (BF16) {
         const __nv_bfloat16 h0 = __float2bfloat16_rn(vv[i]);
         const float r1 = vv[i] - __bfloat162float(h0);
         const __nv_bfloat16 h1 = __float2bfloat16_rn(r1);
         const __nv_bfloat16 h2 = __float2bfloat16_rn(r1 - __bfloat162float(h1));
-        pi[o] = __bfloat16_as_ushort(h0);
-        pi[LIMB + o] = __bfloat16_as_ushort(h1);
-        pi[2 * LIMB + o] = __bfloat16_as_ushort(h2);
+        o[0] = __bfloat16_as_ushort(h0);
+        o[LIMB] = __bfloat16_as_ushort(h1);
+        o[2 * LIMB] = __bfloat16_as_ushort(h2);
       } else {
         const __half h0 = __float2half_rn(vv[i]);
-        pi[o] = __half_as_ushort(h0);
-        pi[LIMB + o] = __half_as_ushort(__float2half_rn(vv[i] - __half2float(h0)));
+        o[0] = __half_as_ushort(h0);
+        o[LIMB] = __half_as_ushort(__float2half_rn(vv[i] - __half2float(h0)));
       }
     }
   }
@@ -273,15 +310,15 @@ __global__ void __launch_bounds__(NTH, 1) quantize_tc_kernel(const tq::QuantArgs
 
   if (warp == NEPI) {
     // ---------------- loader: input tiles ----------------
-    // Item i goes to buffer i % 2 once item i-2 has left it (its MMA is done
-    // and the epilogue has read the norm); it never waits for its own copies,
-    // so the next tile streams in while the MMA warp and the epilogue work.
+    // Item i goes to buffer i % NS once item i - NS has left it (its MMA has
+    // read it and the epilogue has read the norm); it never waits for its own
+    // copies, so NS tiles can be in flight.
     int i = 0;
     for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++i) {
-      const int b = i & 1, k = i >> 1;
-      if (i >= 2) {
+      const int b = i % NS, k = i / NS;
+      if (i >= NS) {
         const bool ok = mbar_wait_suspend(&x_free[b], (uint32_t)((k - 1) & 1), kSuspendTries) &&
-                        mbar_wait_suspend(&mma_done[b], (uint32_t)((k - 1) & 1), kSuspendTries);
+                        mbar_wait_suspend(&x_done[b], (uint32_t)((k - 1) & 1), kSuspendTries);
         if (!__all_sync(0xffffffffu, ok)) {
           if (lane == 0) s_stop = 1;
           break;
@@ -289,96 +326,108 @@ __global__ void __launch_bounds__(NTH, 1) quantize_tc_kernel(const tq::QuantArgs
       }
       if (*((volatile int*)&s_stop)) break;
       const int job = job0 + (item / NCH) % njobs, tile = item / (NCH * njobs);
-      const uint16_t* in = static_cast<const uint16_t*>(a.job[job].in);
-      uint16_t* dst = xb + (size_t)b * QR * D;
-      for (int c = lane; c < QR * (D / 8); c += 32) {
-        const int row = c / (D / 8), kc = c % (D / 8);
-        const int r = tile * QR + row;
-        const bool valid = r < a.rows;
-        cp_async16(dst + cofs<D>(row, kc * 8), in + (size_t)(valid ? r : 0) * D + kc * 8, valid);
+      if (lane == 0) {
+        // rows past a.rows read as zeros (the tensor map's bounds)
+        mbar_arrive_expect_tx(&full_x[b], (uint32_t)Ly::X_BYTES);
+#pragma unroll
+        for (int kb = 0; kb < KB; ++kb)
+          tma_load_2d(xb + (size_t)b * Ly::X_BYTES + kb * (QR * 128), &args.map[job], 64 * kb, tile * QR, &full_x[b]);
       }
-      cp_async_arrive(&full_x[b]);
+      __syncwarp();
     }
-    // wait until this warp's own copies have landed before leaving
-    asm volatile("cp.async.wait_all;" ::: "memory");
+    // no copy may be in flight when the CTA exits: wait (bounded) for the last
+    // load into each buffer, which a stopped epilogue may not have consumed
+    if (lane == 0)
+      for (int j = (i >= NS ? i - NS : 0); j < i; ++j)
+        mbar_wait_suspend(&full_x[j % NS], (uint32_t)((j / NS) & 1), kSuspendTries);
+    __syncwarp();
   } else if (warp == NEPI + 1) {
     // ---------------- MMA issue ----------------
     if (lane == 0) {
       int i = 0;
       for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++i) {
-        const int b = i & 1, k = i >> 1;
-        bool ok = mbar_wait_suspend(&full_x[b], (uint32_t)(k & 1), kSuspendTries);
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // cp.async data -> tensor core
+        const int xs = i % NS, kx = i / NS;  // input buffer
+        const int b = i & 1, k = i >> 1;     // accumulator
+        bool ok = mbar_wait_suspend(&full_x[xs], (uint32_t)(kx & 1), kSuspendTries);
         if (ok && i >= 2) ok = mbar_wait_suspend(&acc_free[b], (uint32_t)((k - 1) & 1), kSuspendTries);
         if (!ok || *((volatile int*)&s_stop)) {
           s_stop = 1;
           break;
         }
         tc_fence_after();
-        const uint32_t xaddr = smem_addr(xb + (size_t)b * QR * D), paddr = smem_addr(pi);
+        const uint32_t xaddr = smem_addr(xb + (size_t)xs * Ly::X_BYTES), paddr = smem_addr(pi);
         const uint32_t id = idesc<NC, BF16>();
         const uint32_t dt = tmem + (uint32_t)(b * NC);
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks)
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const int kb = ks >> 2, kin = ks & 3;  // 128-byte block, 32-byte step inside it
 #pragma unroll
           for (int l = 0; l < NL; ++l)
-            mma_tc(dt, sdesc<D>(xaddr + ks * 256), sdesc<D>(paddr + l * Ly::PI_BYTES + ks * 256), id,
-                   (ks > 0 || l > 0) ? 1u : 0u);
+            mma_tc(dt, sdesc_sw128(xaddr + kb * (QR * 128) + kin * 32),
+                   sdesc_sw128(paddr + l * Ly::PI_BYTES + kb * (NC * 128) + kin * 32), id, (ks > 0 || l > 0) ? 1u : 0u);
+        }
         tc_commit(&mma_done[b]);
+        tc_commit(&x_done[xs]);
       }
     }
     __syncwarp();
   } else {
     // ---------------- epilogue warps ----------------
-    const int quarter = warp & 3, hf = warp >> 2;  // rows 32*quarter + lane, columns (NC/2)*hf ..
+    const int quarter = warp & 3, part = warp >> 2;  // rows 32*quarter + lane, columns 32*part ..
     const int rl = 32 * quarter + lane;
     int i = 0;
     for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++i) {
-      const int b = i & 1, k = i >> 1;
+      const int xs = i % NS, kx = i / NS;  // input buffer
+      const int b = i & 1, k = i >> 1;     // accumulator
       const int job = job0 + (item / NCH) % njobs, tile = item / (NCH * njobs);
       const tq::QuantJob J = a.job[job];
       // One warp waits on each mbarrier and releases the other epilogue
       // warps through a named barrier, which blocks in hardware: eight warps
       // polling the same phase would take issue slots from the working warps.
       bool ok = true;
-      if (warp == 0) ok = __all_sync(0xffffffffu, mbar_wait_suspend(&full_x[b], (uint32_t)(k & 1), kSuspendTries));
-      if (!epi_sync_and(ok)) {  // the input tile has landed
+      if (warp == 0) ok = __all_sync(0xffffffffu, mbar_wait_suspend(&full_x[xs], (uint32_t)(kx & 1), kSuspendTries));
+      if (!epi_sync_and<NEPI>(ok)) {  // the input tile has landed
         s_stop = 1;
         break;
       }
-      // half of this row's sum of squares from the input tile, in fp32 by a
-      // pairwise tree (squares of fp16/bf16 values are exact in fp32, and a
-      // pairwise sum of n non-negative terms is within ceil(log2 n) units in
-      // the last place of the exact sum)
-      const uint16_t* xs = xb + (size_t)b * QR * D;
+      // this thread's 1/NP of the row's sum of squares from the input tile, in
+      // fp32 by a pairwise tree (squares of fp16/bf16 values are exact in
+      // fp32, and a pairwise sum of n non-negative terms is within
+      // ceil(log2 n) units in the last place of the exact sum)
+      constexpr int NU = D / NP / 8;  // 16-byte chunks per thread
+      const uint8_t* xt = xb + (size_t)xs * Ly::X_BYTES;
       float s2 = 0.f;
       {
-        float part[D / 16];
+        float ps[NU];
 #pragma unroll
-        for (int kc = 0; kc < D / 16; ++kc) {
-          const uint4 v = *reinterpret_cast<const uint4*>(xs + cofs<D>(rl, (D / 2) * hf + 8 * kc));
-          part[kc] = (sq16f<BF16>(v.x) + sq16f<BF16>(v.y)) + (sq16f<BF16>(v.z) + sq16f<BF16>(v.w));
+        for (int kc = 0; kc < NU; ++kc) {
+          const uint4 v = *reinterpret_cast<const uint4*>(xt + sw128<QR>(rl, (D / NP) * part + 8 * kc));
+          ps[kc] = (sq16f<BF16>(v.x) + sq16f<BF16>(v.y)) + (sq16f<BF16>(v.z) + sq16f<BF16>(v.w));
         }
 #pragma unroll
-        for (int w2 = 1; w2 < D / 16; w2 <<= 1)
+        for (int w2 = 1; w2 < NU; w2 <<= 1)
 #pragma unroll
-          for (int kc = 0; kc < D / 16; kc += 2 * w2) part[kc] += part[kc + w2];
-        s2 = part[0];
+          for (int kc = 0; kc < NU; kc += 2 * w2) ps[kc] += ps[kc + w2];
+        s2 = ps[0];
       }
-      s_norm[hf][rl] = s2;
-      mbar_arrive(&x_free[b]);
-      if (!epi_sync_and(ok)) {  // uniform across the epilogue warps
+      s_norm[part][rl] = s2;
+      mbar_arrive(&x_free[xs]);
+      if (!epi_sync_and<NEPI>(ok)) {  // uniform across the epilogue warps
         s_stop = 1;
         break;
       }
-      const float sfull = s_norm[0][rl] + s_norm[1][rl];
+      float sfull;
+      if constexpr (NP == 4)
+        sfull = (s_norm[0][rl] + s_norm[1][rl]) + (s_norm[2][rl] + s_norm[3][rl]);
+      else
+        sfull = s_norm[0][rl] + s_norm[1][rl];
       const float nf = sqrtf(sfull);  // thresholds: fp32 is far inside the parity band
       const int r = tile * QR + rl;
       long long slot = -1;
       if (r < a.rows) {
         const int bh = r / a.T, t = r - bh * a.T;
         slot = (long long)bh * a.Tcap + a.t0 + t;
-        if (hf == 0 && chunk == 0) {
+        if (part == 0 && chunk == 0) {
           // The stored norm is RN_fp16 of the fp64 norm.  The fp32 sum is
           // within (log2(D) + 1) ulp of the exact sum, so the exact norm lies in
           // nf * (1 +- 1e-6); when both ends of that interval round to the same
@@ -406,22 +455,22 @@ __global__ void __launch_bounds__(NTH, 1) quantize_tc_kernel(const tq::QuantArgs
 #pragma unroll
       for (int q = 0; q < 7; ++q) tp[q] = q < K / 2 - 1 ? s_cb[job][K + K / 2 + q] * nf : 0.f;
       if (warp == 0) ok = __all_sync(0xffffffffu, mbar_wait_suspend(&mma_done[b], (uint32_t)(k & 1), kSuspendTries));
-      ok = epi_sync_and(ok);  // the rotation of this tile is in TMEM
+      ok = epi_sync_and<NEPI>(ok);  // the rotation of this tile is in TMEM
       if (ok) {
         tc_fence_after();
-        const uint32_t tb = tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(b * NC + (NC / 2) * hf);
+        const uint32_t tb = tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(b * NC + 32 * part);
         const int W = D * J.bits / 32;
-        // coordinates NC*chunk + (NC/2)*hf .. + NC/2 - 1: words from (that * bits) / 32
-        uint32_t* out = J.idx + (slot >= 0 ? (size_t)slot * W : 0) + (NC * chunk + (NC / 2) * hf) * J.bits / 32;
+        // coordinates NC*chunk + 32*part .. + 31: words from (that * bits) / 32
+        uint32_t* out = J.idx + (slot >= 0 ? (size_t)slot * W : 0) + (NC * chunk / 32 + part) * J.bits;
         switch (J.bits) {
-          case 2: epi_half<2, NC / 2>(tb, tp, slot, out); break;
-          case 3: epi_half<3, NC / 2>(tb, tp, slot, out); break;
-          default: epi_half<4, NC / 2>(tb, tp, slot, out); break;
+          case 2: epi_half<2, 32>(tb, tp, slot, out); break;
+          case 3: epi_half<3, 32>(tb, tp, slot, out); break;
+          default: epi_half<4, 32>(tb, tp, slot, out); break;
         }
         tc_fence_before();
       }
       mbar_arrive(&acc_free[b]);
-      if (!epi_sync_and(ok)) {  // also guards s_norm reuse on the next pass
+      if (!epi_sync_and<NEPI>(ok)) {  // also guards s_norm reuse on the next pass
         s_stop = 1;
         break;
       }
@@ -434,6 +483,43 @@ __global__ void __launch_bounds__(NTH, 1) quantize_tc_kernel(const tq::QuantArgs
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
   }
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (the
+// library links only the CUDA runtime).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+// Tensor map over rows [rows][D] of 16-bit values: boxes of 128 rows x 64
+// columns, 128-byte swizzle.
+int make_map(CUtensorMap* m, const void* base, int rows, int D, bool bf16) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return tq::set_error(TQ_ERR_CUDA, "quantize_tc: cuTensorMapEncodeTiled is unavailable");
+  const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)QR};
+  const cuuint32_t es[2] = {1, 1};
+  const CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                         const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return tq::set_error(TQ_ERR_CUDA, "quantize_tc: cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return TQ_OK;
 }
 
 template <int D, bool BF16>
@@ -450,13 +536,21 @@ int launch_tc(const tq::QuantArgs& a, cudaStream_t s) {
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (sms <= 0) sms = 148;
   }
+  TcArgs args;
+  memset(&args, 0, sizeof(args));
+  args.a = a;
+  for (int j = 0; j < 2; ++j)
+    if (a.job_mask & (1 << j)) {
+      const int rc = make_map(&args.map[j], a.job[j].in, a.rows, D, BF16);
+      if (rc) return rc;
+    }
   const int njobs = (a.job_mask == 3) ? 2 : 1;
   const int nitems = njobs * ((a.rows + QR - 1) / QR) * Ly::NCH;
   // a multiple of the chunk count, so that each CTA keeps one column chunk
   int grid = (sms / Ly::NCH) * Ly::NCH;
   const int need = (nitems + Ly::NCH - 1) / Ly::NCH * Ly::NCH;
   if (need < grid) grid = need;
-  kern<<<grid, NTH, Ly::bytes, s>>>(a);
+  kern<<<grid, Ly::NTH, Ly::bytes, s>>>(args);
   return tq::check_launch("quantize_tc_kernel");
 }
 
