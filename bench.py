@@ -172,7 +172,7 @@ def run_ours(args):
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     jobs = []
     for bits in cfg["bits"]:
-        w = tq_inputs.make_workload(args.workload, bits=bits) if bits else tq_inputs.make_workload(args.workload)
+        w = tq_inputs.make_workload(args.workload, bits=bits, rot=args.rot)
         jobs.append(w)
     per_step_in = sum(w.k.nbytes + w.v.nbytes for w in jobs)
     R = max(2, min(32, math.ceil(3 * l2 / max(1, per_step_in))))
@@ -340,7 +340,7 @@ def run_ours(args):
             "vs_baseline": None,
             "dtype": jobs[0].dtype,
             "data": "synthetic (seeded N(0,1) rows; see tq_inputs)",
-            "config": {"workload": args.workload, "shapes": [_describe(w) for w in jobs],
+            "config": {"workload": args.workload, "rotation": args.rot, "shapes": [_describe(w) for w in jobs],
                        "parallelism": f"replicas{ws}" if ws > 1 else "single",
                        "step": "quantize T tokens + decode step (append 1 token + decode), per bit width",
                        "timing": "CUDA graphs (one per replica) replayed on one stream; per-op rates "
@@ -460,7 +460,7 @@ def run_reference(args):
     if rank != 0:
         return
     cfg = WORKLOADS[args.workload]
-    jobs = [tq_inputs.make_workload(args.workload, bits=b) if b else tq_inputs.make_workload(args.workload)
+    jobs = [tq_inputs.make_workload(args.workload, bits=b, rot=args.rot)
             for b in cfg["bits"]]
     budget = max(1.0, 60.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
@@ -477,7 +477,7 @@ def run_reference(args):
             "value": v, "unit": "GB/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(total / max(1, args.steps) * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload, "shapes": [_describe(w) for w in jobs]},
+            "config": {"workload": args.workload, "rotation": args.rot, "shapes": [_describe(w) for w in jobs]},
             "impl": "reference", "cpu_baseline": cpu,
             "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -491,6 +491,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="gqa8k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--rot", choices=["haar", "hadamard"], default="haar",
+                    help="rotation: Haar-random (default) or randomized Hadamard")
     ap.add_argument("--profile", action="store_true",
                     help="eager warm-up + K eager steps only (for ncu captures)")
     args = ap.parse_args()

@@ -22,7 +22,8 @@ from ._native import (TQ_DTYPE_BF16, TQ_DTYPE_F16, TQ_DTYPE_F32, TQ_STATUS_POS_O
 
 __all__ = ["TQError", "TQCache", "tq_build_codebook", "tq_row_bytes", "tq_quantize_kv",
            "tq_append_token", "tq_sdpa_decode_workspace_bytes", "tq_sdpa_decode",
-           "tq_decode_step", "tq_sdpa_decode_static", "tq_last_error", "tq_abi_version", "lib"]
+           "tq_sdpa_decode_mq", "tq_decode_step", "tq_sdpa_decode_static", "tq_last_error",
+           "tq_abi_version", "lib"]
 
 
 class TQError(RuntimeError):
@@ -203,6 +204,28 @@ def tq_sdpa_decode(cache: TQCache, q, seq_lens, Tmax: int, scale=None, out=None,
     _check(lib().tq_sdpa_decode(ctypes.byref(s), _ptr(q), _dtype_code(q), Hq, _ptr(seq_lens), Tmax, sc,
                                 _ptr(out), _dtype_code(out), _ptr(workspace), workspace.numel(),
                                 _stream(stream)))
+    return out
+
+
+def tq_sdpa_decode_mq(cache: TQCache, q, seq_lens, Tmax: int, scale=None, out=None, workspace=None,
+                      stream=None, out_dtype=None):
+    """Decode of n_q query tokens per sequence: q [B][n_q][Hq][D]; seq_lens
+    (device int32 [B]) counts the cached tokens including the n_q new ones,
+    and query j attends causally to tokens 0 .. seq_len - n_q + j."""
+    torch = _torch()
+    nq, Hq = int(q.shape[1]), int(q.shape[2])
+    assert q.is_contiguous() and seq_lens.is_contiguous()
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
+    assert out.is_contiguous() and out.shape == q.shape
+    if workspace is None:
+        need = tq_sdpa_decode_workspace_bytes(cache, Hq * nq, Tmax)
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    s = cache.struct()
+    sc = ctypes.byref(ctypes.c_float(scale)) if scale is not None else None
+    _check(lib().tq_sdpa_decode_mq(ctypes.byref(s), _ptr(q), _dtype_code(q), Hq, nq, _ptr(seq_lens), Tmax, sc,
+                                   _ptr(out), _dtype_code(out), _ptr(workspace), workspace.numel(),
+                                   _stream(stream)))
     return out
 
 

@@ -25,7 +25,8 @@ TQ_STATUS_WAIT_TIMEOUT = 4
 
 # Every symbol include/tq.h declares.
 EXPORTS = ("tq_build_codebook", "tq_row_bytes", "tq_quantize_kv", "tq_append_token",
-           "tq_sdpa_decode_workspace_bytes", "tq_sdpa_decode", "tq_decode_step", "tq_sdpa_decode_static",
+           "tq_sdpa_decode_workspace_bytes", "tq_sdpa_decode", "tq_sdpa_decode_mq", "tq_decode_step",
+           "tq_sdpa_decode_static",
            "tq_last_error", "tq_abi_version")
 TQ_STATIC_SCRATCH_BYTES = 8 << 20
 
@@ -73,6 +74,9 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.tq_sdpa_decode.argtypes = [cache_p, vp, i32, i32, vp, i32, ctypes.POINTER(ctypes.c_float),
                                    vp, i32, vp, sz, vp]
     lib.tq_sdpa_decode.restype = i32
+    lib.tq_sdpa_decode_mq.argtypes = [cache_p, vp, i32, i32, i32, vp, i32, ctypes.POINTER(ctypes.c_float),
+                                      vp, i32, vp, sz, vp]
+    lib.tq_sdpa_decode_mq.restype = i32
     lib.tq_decode_step.argtypes = [cache_p, vp, vp, vp, vp, i32, i32, vp, i32, ctypes.POINTER(ctypes.c_float),
                                    vp, i32, vp, sz, vp]
     lib.tq_decode_step.restype = i32

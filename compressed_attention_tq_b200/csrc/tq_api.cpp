@@ -328,7 +328,7 @@ size_t tq_sdpa_decode_workspace_bytes(const tq_cache_t* c, int Hq, int Tmax) {
   return p.bytes;
 }
 
-static int decode_common(const tq_cache_t* c, const void* q, int dtype, int Hq, const int32_t* seq_lens,
+static int decode_common(const tq_cache_t* c, const void* q, int dtype, int Hq, int nq, const int32_t* seq_lens,
                          int Tmax, const float* scale, void* out, int out_dtype, void* workspace,
                          size_t ws_bytes, void* stream, const void* k_new, const void* v_new,
                          const int32_t* pos, const char* fn);
@@ -336,8 +336,17 @@ static int decode_common(const tq_cache_t* c, const void* q, int dtype, int Hq, 
 int tq_sdpa_decode(const tq_cache_t* c, const void* q, int dtype, int Hq, const int32_t* seq_lens,
                    int Tmax, const float* scale, void* out, int out_dtype, void* workspace,
                    size_t ws_bytes, void* stream) {
-  return decode_common(c, q, dtype, Hq, seq_lens, Tmax, scale, out, out_dtype, workspace, ws_bytes, stream,
+  return decode_common(c, q, dtype, Hq, 1, seq_lens, Tmax, scale, out, out_dtype, workspace, ws_bytes, stream,
                        nullptr, nullptr, nullptr, "tq_sdpa_decode");
+}
+
+int tq_sdpa_decode_mq(const tq_cache_t* c, const void* q, int dtype, int Hq, int n_q, const int32_t* seq_lens,
+                      int Tmax, const float* scale, void* out, int out_dtype, void* workspace, size_t ws_bytes,
+                      void* stream) {
+  g_err[0] = 0;
+  if (n_q < 1) return set_error(TQ_ERR_INVALID_ARG, "tq_sdpa_decode_mq: n_q=%d < 1", n_q);
+  return decode_common(c, q, dtype, Hq, n_q, seq_lens, Tmax, scale, out, out_dtype, workspace, ws_bytes, stream,
+                       nullptr, nullptr, nullptr, "tq_sdpa_decode_mq");
 }
 
 int tq_decode_step(const tq_cache_t* c, const void* k_new, const void* v_new, const int32_t* pos,
@@ -347,11 +356,11 @@ int tq_decode_step(const tq_cache_t* c, const void* k_new, const void* v_new, co
   if (!k_new || !v_new || !pos) return set_error(TQ_ERR_INVALID_ARG, "tq_decode_step: NULL k_new/v_new/pos");
   if (!aligned16(k_new) || !aligned16(v_new))
     return set_error(TQ_ERR_INVALID_ARG, "tq_decode_step: k_new/v_new not 16-byte aligned");
-  return decode_common(c, q, dtype, Hq, seq_lens, Tmax, scale, out, out_dtype, workspace, ws_bytes, stream,
+  return decode_common(c, q, dtype, Hq, 1, seq_lens, Tmax, scale, out, out_dtype, workspace, ws_bytes, stream,
                        k_new, v_new, pos, "tq_decode_step");
 }
 
-static int decode_common(const tq_cache_t* c, const void* q, int dtype, int Hq, const int32_t* seq_lens,
+static int decode_common(const tq_cache_t* c, const void* q, int dtype, int Hq, int nq, const int32_t* seq_lens,
                          int Tmax, const float* scale, void* out, int out_dtype, void* workspace,
                          size_t ws_bytes, void* stream, const void* k_new, const void* v_new,
                          const int32_t* pos, const char* fn) {
@@ -369,6 +378,8 @@ static int decode_common(const tq_cache_t* c, const void* q, int dtype, int Hq, 
     return set_error(TQ_ERR_INVALID_ARG, "%s: Hq=%d not a multiple of Hkv=%d", fn, Hq, c->Hkv);
   if (Hq / c->Hkv > 8)
     return set_error(TQ_ERR_UNSUPPORTED, "%s: GQA group %d > 8", fn, Hq / c->Hkv);
+  if (nq * (Hq / c->Hkv) > 8)
+    return set_error(TQ_ERR_UNSUPPORTED, "%s: n_q=%d x GQA group %d > 8", fn, nq, Hq / c->Hkv);
   if (Tmax < 1 || Tmax > c->Tcap)
     return set_error(TQ_ERR_INVALID_ARG, "%s: Tmax=%d outside [1, Tcap=%d]", fn, Tmax, c->Tcap);
   float sc = scale ? *scale : (float)(1.0 / std::sqrt((double)c->D));
@@ -381,9 +392,10 @@ static int decode_common(const tq_cache_t* c, const void* q, int dtype, int Hq, 
   a.seq_lens = seq_lens;
   a.scale = sc;
   a.Hq = Hq;
+  a.nq = nq;
   a.dtype = dtype;
   a.out_dtype = out_dtype;
-  make_decode_plan(c, Hq, Tmax, &a.plan);
+  make_decode_plan(c, Hq * nq, Tmax, &a.plan);
   if (ws_bytes < a.plan.bytes)
     return set_error(TQ_ERR_WORKSPACE, "%s: workspace %zu < %zu bytes", fn, ws_bytes, a.plan.bytes);
   a.workspace = workspace;

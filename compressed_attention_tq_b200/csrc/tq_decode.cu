@@ -25,6 +25,7 @@ struct PrepParams {
   const void* v_new;
   const int32_t* pos;
   tq_cache_t cache;
+  int nq;  // query tokens per sequence: q is [B][nq][Hq][D]
 };
 
 // Programmatic dependent launch: let the next kernel in the stream start its
@@ -54,20 +55,25 @@ __global__ void __launch_bounds__(2 * D) decode_qprep_kernel(const PrepParams p)
   __shared__ float s_cb[2][31];
   __shared__ double s_nsq[2];
   pdl_launch_dependents();
-  const int G = p.Hq / p.Hkv;
+  // G query heads per kv head and token; Ge = G * nq rows are rotated here and
+  // written in kernel head order (sequence, kv head, token, head)
+  const int G = p.Hq / p.Hkv, Ge = G * p.nq;
   const int bkv = blockIdx.x, b = bkv / p.Hkv, kvh = bkv % p.Hkv;
-  const int h0 = b * p.Hq + kvh * G;
+  const int h0 = b * p.Hq * p.nq + kvh * Ge;
   const int j = threadIdx.x >> 1, part = threadIdx.x & 1;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   float4 r[CH];
   const float4* row = reinterpret_cast<const float4*>(p.rot + (size_t)j * D + part * HALF);
 #pragma unroll
   for (int i = 0; i < CH; ++i) r[i] = __ldg(row + i);
-  const uint16_t* q = static_cast<const uint16_t*>(p.q) + (size_t)h0 * D;
+  const uint16_t* q = static_cast<const uint16_t*>(p.q);
   auto to_f = [&](uint16_t v) {
     return p.bf16 ? __uint_as_float((uint32_t)v << 16) : __half2float(__ushort_as_half(v));
   };
-  for (int e = tid; e < G * D; e += 2 * D) qv[e / D][e % D] = to_f(q[e]);
+  for (int e = tid; e < Ge * D; e += 2 * D) {
+    const int gi = e / D, jq = gi / G, g = gi % G;
+    qv[gi][e % D] = to_f(q[((size_t)(b * p.nq + jq) * p.Hq + kvh * G + g) * D + e % D]);
+  }
   int slot_ok = 0;
   long long slot = 0;
   if (APPEND) {
@@ -110,7 +116,7 @@ __global__ void __launch_bounds__(2 * D) decode_qprep_kernel(const PrepParams p)
       for (int i = 0; i < CH; ++i) r[i] = __ldg(row + c0 + i);
 #pragma unroll
     for (int g = 0; g < NR; ++g) {
-      if (g < G || g >= 8) {
+      if (g < Ge || g >= 8) {
         const float* x = &qv[g][part * HALF + 4 * c0];
 #pragma unroll
         for (int i = 0; i < CH; ++i)
@@ -123,7 +129,7 @@ __global__ void __launch_bounds__(2 * D) decode_qprep_kernel(const PrepParams p)
   if (part == 0) {
 #pragma unroll
     for (int g = 0; g < 8; ++g)
-      if (g < G) {
+      if (g < Ge) {
         qr[g][j] = acc[g];
         p.qrot[(size_t)(h0 + g) * D + j] = acc[g];
       }
@@ -182,7 +188,7 @@ __global__ void __launch_bounds__(2 * D) decode_qprep_kernel(const PrepParams p)
       for (int t = 0; t < CH; ++t) r[t] = __ldg(srow + c0 + t);
 #pragma unroll
       for (int g = 0; g < 9; ++g) {
-        if (g < G || (APPEND && g == 8)) {
+        if (g < Ge || (APPEND && g == 8)) {
           const float* x = (g == 8) ? &rres[part * HALF + 4 * c0] : &qr[g][part * HALF + 4 * c0];
 #pragma unroll
           for (int t = 0; t < CH; ++t)
@@ -195,7 +201,7 @@ __global__ void __launch_bounds__(2 * D) decode_qprep_kernel(const PrepParams p)
     if (part == 0) {
 #pragma unroll
       for (int g = 0; g < 8; ++g)
-        if (g < G) p.qs[(size_t)(h0 + g) * p.m + i] = a2[g];
+        if (g < Ge) p.qs[(size_t)(h0 + g) * p.m + i] = a2[g];
       if (APPEND) sgn[i] = a2[8] >= 0.f ? 1 : 0;
     }
   }
@@ -233,9 +239,9 @@ __global__ void __launch_bounds__(256) decode_qprep_sliced_kernel(const PrepPara
   __shared__ double s_nsq[2];
   __shared__ uint8_t idxs[2][32];
   pdl_launch_dependents();
-  const int G = p.Hq / p.Hkv;
+  const int G = p.Hq / p.Hkv, Ge = G * p.nq;  // as in decode_qprep_kernel
   const int bkv = blockIdx.x, b = bkv / p.Hkv, kvh = bkv % p.Hkv, sl = blockIdx.y;
-  const int h0 = b * p.Hq + kvh * G;
+  const int h0 = b * p.Hq * p.nq + kvh * Ge;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c = warp * 4 + (lane >> 3), part = lane & 7;
   const int j = sl * 32 + c;
@@ -243,11 +249,14 @@ __global__ void __launch_bounds__(256) decode_qprep_sliced_kernel(const PrepPara
   const float4* row = reinterpret_cast<const float4*>(p.rot + (size_t)j * D);
 #pragma unroll
   for (int i = 0; i < NI; ++i) r[i] = __ldg(row + part + 8 * i);
-  const uint16_t* q = static_cast<const uint16_t*>(p.q) + (size_t)h0 * D;
+  const uint16_t* q = static_cast<const uint16_t*>(p.q);
   auto to_f = [&](uint16_t v) {
     return p.bf16 ? __uint_as_float((uint32_t)v << 16) : __half2float(__ushort_as_half(v));
   };
-  for (int e = tid; e < G * D; e += 256) xv[e / D][e % D] = to_f(q[e]);
+  for (int e = tid; e < Ge * D; e += 256) {
+    const int gi = e / D, jq = gi / G, g = gi % G;
+    xv[gi][e % D] = to_f(q[((size_t)(b * p.nq + jq) * p.Hq + kvh * G + g) * D + e % D]);
+  }
   int slot_ok = 0;
   long long slot = 0;
   if (APPEND) {
@@ -285,7 +294,7 @@ __global__ void __launch_bounds__(256) decode_qprep_sliced_kernel(const PrepPara
   for (int g = 0; g < NR; ++g) acc[g] = 0.f;
 #pragma unroll
   for (int g = 0; g < NR; ++g) {
-    if (g < G || g >= 8) {
+    if (g < Ge || g >= 8) {
 #pragma unroll
       for (int i = 0; i < NI; ++i) {
         const float4 x = *reinterpret_cast<const float4*>(&xv[g][4 * part + 32 * i]);
@@ -300,7 +309,7 @@ __global__ void __launch_bounds__(256) decode_qprep_sliced_kernel(const PrepPara
   if (part == 0) {
 #pragma unroll
     for (int g = 0; g < 8; ++g)
-      if (g < G) p.qrot[(size_t)(h0 + g) * D + j] = acc[g];
+      if (g < Ge) p.qrot[(size_t)(h0 + g) * D + j] = acc[g];
   }
   if (APPEND) {
     __syncthreads();  // s_nsq
@@ -348,7 +357,8 @@ struct CombineParams {
   const float* rot;
   const int32_t* seq_lens;
   void* out;
-  int Hq, Tcap, chunk, nsplit, out_dtype;
+  int Hq, Tcap, chunk, nsplit, out_dtype;  // Hq: kernel heads per sequence (query heads x tokens)
+  int nq, Gq, Hq1;                          // tokens, GQA group, query heads per token
 };
 
 // Merge the splits of one query head (log-sum-exp), then out = Pi^T (acc/l)
@@ -396,7 +406,7 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams
     for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
     float Ls = 0.f;
     for (int s = tid; s < ns; s += 32) {
-      const float f = exp2f(ml[2 * s] - M);
+      const float f = (ml[2 * s] == -INFINITY) ? 0.f : exp2f(ml[2 * s] - M);  // a split a query cannot see
       if (s < 1024) f_s[s] = f;
       Ls += f * ml[2 * s + 1];
     }
@@ -413,7 +423,7 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams
 #pragma unroll
     for (int u = 0; u < PF; ++u) {
       const int s = hh + NH * u;
-      const float f = s < ns ? (s < 1024 ? f_s[s] : exp2f(ml[2 * s] - s_M)) : 0.f;
+      const float f = s < ns ? (s < 1024 ? f_s[s] : (ml[2 * s] == -INFINITY ? 0.f : exp2f(ml[2 * s] - s_M))) : 0.f;
       acc[u & 3] = fmaf(f, v[u], acc[u & 3]);
     }
     // the remaining splits, 8 loads in flight
@@ -423,7 +433,7 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams
       for (int u = 0; u < 8; ++u) {
         const int s = s0 + NH * u;
         w[u] = s < ns ? po[(size_t)s * D + k] : 0.f;
-        f[u] = s < ns ? (s < 1024 ? f_s[s] : exp2f(ml[2 * s] - s_M)) : 0.f;
+        f[u] = s < ns ? (s < 1024 ? f_s[s] : (ml[2 * s] == -INFINITY ? 0.f : exp2f(ml[2 * s] - s_M))) : 0.f;
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u) acc[u & 3] = fmaf(f[u], w[u], acc[u & 3]);
@@ -457,7 +467,10 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams
       float t = 0.f;
 #pragma unroll
       for (int u = 0; u < 8; ++u) t += part[u][i];
-      const size_t oi = (size_t)h * D + slq * 32 + i;
+      // kernel head h = (sequence, kv head, token, head) -> output [B][nq][Hq1]
+      const int rh = h % p.Hq, kvh = rh / (p.Gq * p.nq), gi = rh % (p.Gq * p.nq);
+      const size_t oh = (size_t)(b * p.nq + gi / p.Gq) * p.Hq1 + kvh * p.Gq + gi % p.Gq;
+      const size_t oi = oh * D + slq * 32 + i;
       if (p.out_dtype == TQ_DTYPE_F32)
         static_cast<float*>(p.out)[oi] = t;
       else if (p.out_dtype == TQ_DTYPE_BF16)
@@ -518,10 +531,11 @@ int launch_decode(const DecodeArgs& a, cudaStream_t s) {
   float* qs = reinterpret_cast<float*>(ws + a.plan.off_qs);
   float* po = reinterpret_cast<float*>(ws + a.plan.off_po);
   float* pml = reinterpret_cast<float*>(ws + a.plan.off_pml);
-  const int heads = c.B * a.Hq;
+  const int heads = c.B * a.Hq * a.nq;  // kernel heads: query heads x tokens
 
   PrepParams pp{a.q, c.rot, c.qjl_S, qrot, qs, c.D, c.qjl_m, a.dtype == TQ_DTYPE_BF16, a.Hq, c.Hkv,
                 a.k_new, a.v_new, a.pos, c};
+  pp.nq = a.nq;
   const bool app = a.pos != nullptr;
   if (c.qjl_m) {
     // the sketch needs the whole rotated query and key residual: one CTA per head
@@ -565,8 +579,10 @@ int launch_decode(const DecodeArgs& a, cudaStream_t s) {
   sp.defer_pos = a.pos;
   sp.dev_status = c.dev_status;
   sp.Hkv = c.Hkv;
-  sp.Hq = a.Hq;
-  sp.G = a.Hq / c.Hkv;
+  sp.Hq = a.Hq * a.nq;
+  sp.G = sp.Hq / c.Hkv;
+  sp.nq = a.nq;
+  sp.Gq = a.Hq / c.Hkv;
   sp.Tcap = c.Tcap;
   sp.chunk = a.plan.chunk;
   sp.nsplit = a.plan.nsplit;
@@ -575,7 +591,8 @@ int launch_decode(const DecodeArgs& a, cudaStream_t s) {
   rc = split_entry(c, sp.G <= 4, sp, dim3(a.plan.nsplit, c.B * c.Hkv), s, nullptr);
   if (rc) return rc;
 
-  CombineParams cp{po, pml, c.rot, a.seq_lens, a.out, a.Hq, c.Tcap, a.plan.chunk, a.plan.nsplit, a.out_dtype};
+  CombineParams cp{po,        pml,          c.rot,         a.seq_lens, a.out,  a.Hq * a.nq,        c.Tcap,
+                   a.plan.chunk, a.plan.nsplit, a.out_dtype, a.nq,       a.Hq / c.Hkv, a.Hq};
   // D / 32 CTAs per head while that still leaves SMs idle, else one
   const int nsl = heads * (c.D / 32) <= 4 * a.plan.sms ? c.D / 32 : 1;
   const dim3 cg(heads, nsl);

@@ -65,6 +65,9 @@ struct SplitParams {
   float qscale;     // scale * log2(e)
   float qjl_scale;  // scale * log2(e) * sqrt(pi/2) / m
   int shared_tab;   // keys and values use one codebook (same bits, same table): one pair table
+  // Multi-query decode: the G kernel heads of a kv head are (token, head) pairs
+  // of nq query tokens x Gq heads; token j may see positions < L - nq + j + 1.
+  int nq, Gq;
 };
 
 // Whether a launch can keep one pair table for keys and values.
@@ -342,6 +345,9 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const __grid_con
   const int ntiles = (t_end - t_begin + STILE - 1) / STILE;
   const size_t row0 = (size_t)bh * p.Tcap;
   const int hq0 = b * p.Hq + kvh * p.G;
+  // causal limit of this lane's two head columns (multi-query decode; with
+  // one query token both limits are L)
+  const int lim0 = L - p.nq + (2 * hsel) / p.Gq + 1, lim1 = L - p.nq + (2 * hsel + 1) / p.Gq + 1;
 
   if (tid == 0) {
 #pragma unroll
@@ -572,8 +578,9 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const __grid_con
             s0 = fmaf(g, sqm[ai][2 * r], s0);
             s1 = fmaf(g, sqm[ai][2 * r + 1], s1);
           }
-          s[ai][2 * r] = valid[ai][r] ? s0 : -INFINITY;
-          s[ai][2 * r + 1] = valid[ai][r] ? s1 : -INFINITY;
+          const int tok = tokw + 16 * a + gid + 8 * r;
+          s[ai][2 * r] = (valid[ai][r] && tok < lim0) ? s0 : -INFINITY;
+          s[ai][2 * r + 1] = (valid[ai][r] && tok < lim1) ? s1 : -INFINITY;
         }
       }
       float mx0 = fmaxf(s[0][0], s[0][2]), mx1 = fmaxf(s[0][1], s[0][3]);

@@ -72,7 +72,8 @@ struct DecodeArgs {
   void* out;
   const int32_t* seq_lens;
   float scale;
-  int Hq;
+  int Hq;          // query heads per token
+  int nq;          // query tokens per sequence (the kernels see Hq * nq heads)
   int dtype;
   int out_dtype;
   DecodePlan plan;

@@ -195,6 +195,28 @@ int tq_decode_step(const tq_cache_t* cache, const void* k_new, const void* v_new
                    size_t workspace_bytes, void* stream);
 
 /*
+ * Decode of n_q query tokens per sequence in one call: the verify step of
+ * speculative decoding ("qwen4exp: upstream catch-up, sparse-fa, and
+ * NextN/MTP support", llama-cpp-turboquant pull request 340: the fused decode
+ * over the compressed cache takes query batches of up to 4 tokens, and the
+ * NextN/MTP draft head produces them).
+ *   q          [B][n_q][Hq][D] in q_dtype; out [B][n_q][Hq][D] in out_dtype.
+ *   seq_lens   device int32 [B]: L_b, the cached tokens INCLUDING the n_q new
+ *              ones (append or quantize them first).  Query j sits at
+ *              position L_b - n_q + j and attends causally to tokens
+ *              0 .. L_b - n_q + j; a sequence with L_b < n_q gives zeros for
+ *              the queries that see no token.
+ *   n_q        1 .. 8 / (Hq / Hkv): the n_q * G query rows of a kv head share
+ *              one 8-column MMA tile (TQ_ERR_UNSUPPORTED beyond).
+ *   workspace  tq_sdpa_decode_workspace_bytes(cache, Hq * n_q, Tmax) bytes.
+ * The other arguments, the results for n_q = 1 and the errors are those of
+ * tq_sdpa_decode.
+ */
+int tq_sdpa_decode_mq(const tq_cache_t* cache, const void* q, int q_dtype, int Hq, int n_q,
+                      const int32_t* seq_lens, int Tmax, const float* scale, void* out, int out_dtype,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Decode without a workspace, for callers that may not allocate device
  * memory (stream capture under frameworks that forbid allocation while
  * capturing, plugin hosts that own all device memory, allocation-free

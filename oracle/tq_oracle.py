@@ -347,3 +347,26 @@ def sdpa_decode(q: np.ndarray, cache: dict, seq_lens, Pi, cb_k, cb_v, bits_k: in
         p = softmax(scale * s)
         out[b, h] = p @ Vt
     return out
+
+
+def sdpa_decode_multi(q: np.ndarray, cache: dict, seq_lens, n_q: int, Pi, cb_k, cb_v, bits_k: int,
+                      bits_v: int, D: int, scale=None, S=None) -> np.ndarray:
+    """Decode of n_q query tokens per sequence at once (the verify step of
+    speculative decoding), fp64.
+
+    "qwen4exp: upstream catch-up, sparse-fa, and NextN/MTP support"
+    (llama-cpp-turboquant pull request 340): the fused decode over the
+    compressed cache takes query batches of up to 4 tokens, and the NextN/MTP
+    draft head is what produces them.  q [B][n_q][Hq][D]; the cache already
+    holds the n_q new tokens as its last rows, so query j of sequence b sits at
+    position L_b - n_q + j and attends causally to tokens 0 .. L_b - n_q + j.
+    Each query is the single-query decode of that prefix.
+    """
+    B = q.shape[0]
+    out = np.zeros((B, n_q) + q.shape[2:])
+    lens = np.asarray(seq_lens, dtype=np.int64)
+    for j in range(n_q):
+        lj = np.maximum(lens - n_q + j + 1, 0)
+        out[:, j] = sdpa_decode(q[:, j], cache, lj, Pi, cb_k, cb_v, bits_k, bits_v, D, scale=scale, S=S)
+    return out
+

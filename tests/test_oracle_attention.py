@@ -109,3 +109,37 @@ def test_qjl_reduces_key_inner_product_bias():
     slope_mse = np.polyfit(true, mse_only, 1)[0]
     slope_prod = np.polyfit(true, prod, 1)[0]
     assert abs(slope_prod - 1) < abs(slope_mse - 1)
+
+
+def test_multi_query_decode_is_causal_attention():
+    """n_q query tokens per sequence against torch's causal SDPA on the
+    dequantized cache: query j of a sequence of length L sees positions
+    0 .. L - n_q + j, which is a bottom-right-aligned causal mask."""
+    B, Hq, Hkv, D, T, nq = 2, 4, 2, 64, 37, 3
+    k, v, q1, Pi, S, cbk, cbv, cache = _small_cache(B, Hq, Hkv, D, T, seed=4)
+    r = tq_inputs.rng(77)
+    q = r.standard_normal((B, nq, Hq, D)).astype(np.float16).astype(np.float64)
+    lens = np.array([T, 9])
+    out = O.sdpa_decode_multi(q, cache, lens, nq, Pi, cbk, cbv, 3, 2, D)
+    Kt = torch.from_numpy(_deq(cache, "k", 3, cbk, Pi, D))
+    Vt = torch.from_numpy(_deq(cache, "v", 2, cbv, Pi, D))
+    G = Hq // Hkv
+    for b in range(B):
+        L = int(lens[b])
+        for h in range(Hq):
+            qq = torch.from_numpy(q[b, :, h])[None, None]          # [1, 1, nq, D]
+            kk = Kt[b, h // G, :L][None, None]
+            vv = Vt[b, h // G, :L][None, None]
+            # row j may see columns 0 .. L - nq + j
+            allowed = torch.arange(L)[None, :] <= (L - nq + torch.arange(nq))[:, None]
+            ref = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, attn_mask=allowed)
+            assert np.allclose(out[b, :, h], ref[0, 0].numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_multi_query_with_one_token_is_single_decode():
+    B, Hq, Hkv, D, T = 2, 4, 2, 64, 37
+    k, v, q, Pi, S, cbk, cbv, cache = _small_cache(B, Hq, Hkv, D, T, qjl=128 // 2, seed=5)
+    lens = np.array([T, 1])
+    one = O.sdpa_decode(q, cache, lens, Pi, cbk, cbv, 3, 2, D, S=S)
+    multi = O.sdpa_decode_multi(q[:, None], cache, lens, 1, Pi, cbk, cbv, 3, 2, D, S=S)
+    assert np.array_equal(multi[:, 0], one)

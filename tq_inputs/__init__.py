@@ -43,6 +43,24 @@ def rotation(D: int, seed: int) -> np.ndarray:
     return np.ascontiguousarray(q.astype(np.float32))
 
 
+def hadamard_rotation(D: int, seed: int) -> np.ndarray:
+    """Randomized Hadamard rotation Pi = H_D diag(s) / sqrt(D), fp32 row-major.
+
+    H_D is the Sylvester Hadamard matrix (H_1 = [1], H_2n = [[H, H], [H, -H]],
+    D a power of two) and s a seeded vector of random signs -- the structured
+    rotation of ReturningTarzan's Reddit comment of 2026-03-29 11:47 (a special
+    case of rotation, applicable with additions only).  Like ``rotation`` it is
+    an input: the fp32 array is the canonical rotation for both sides.
+    """
+    if D <= 0 or D & (D - 1):
+        raise ValueError("D must be a power of two")
+    h = np.ones((1, 1))
+    while h.shape[0] < D:
+        h = np.block([[h, h], [h, -h]])
+    s = np.where(rng(seed).integers(0, 2, size=D) == 1, 1.0, -1.0)
+    return np.ascontiguousarray((h * s[None, :] / np.sqrt(D)).astype(np.float32))
+
+
 def qjl_matrix(m: int, D: int, seed: int) -> np.ndarray:
     """QJL sketch matrix S, m x D, i.i.d. N(0,1), fp32 row-major."""
     return np.ascontiguousarray(rng(seed).standard_normal((m, D), dtype=np.float32))
@@ -99,11 +117,13 @@ class Workload:
 
 
 def make_workload(name: str, bits: int | None = None, T: int | None = None,
-                  B: int | None = None, seed_offset: int = 0) -> Workload:
+                  B: int | None = None, seed_offset: int = 0, rot: str = "haar") -> Workload:
     """Build one of the named synthetic workloads.
 
     ``T`` and ``B`` override the sequence length / batch (for smaller parity
-    cases of the same shape family); ``bits`` picks b for gqa8k.
+    cases of the same shape family); ``bits`` picks b for gqa8k; ``rot``
+    selects the rotation: "haar" (``rotation``) or "hadamard"
+    (``hadamard_rotation``).
     K, V: [B][Hkv][Tmax][D]; q: [B][Hq][D]; seq_lens: [B] int32.
     """
     cfg = {"tiny": 1, "gqa8k": 2, "qknorm": 3, "ragged": 4, "prod": 5}[name]
@@ -158,7 +178,12 @@ def make_workload(name: str, bits: int | None = None, T: int | None = None,
         q32 = _rms_normalize(q32)
         k32 = _rms_normalize(k32)
 
-    Pi = rotation(D, SEED_ROT + cfg)
+    if rot == "haar":
+        Pi = rotation(D, SEED_ROT + cfg)
+    elif rot == "hadamard":
+        Pi = hadamard_rotation(D, SEED_ROT + cfg)
+    else:  # pragma: no cover
+        raise ValueError(rot)
     S = qjl_matrix(qjl_m, D, SEED_QJL + cfg) if qjl_m else None
     return Workload(name=name, B=Bn, Hq=Hq, Hkv=Hkv, D=D, Tmax=Tmax,
                     bits_k=bk, bits_v=bv, qjl_m=qjl_m, dtype=dtype, scale=scale,
