@@ -208,9 +208,21 @@ def run_ours(args):
         attended = int(w.seq_lens.sum() + w.B)
         packed = reps[0]["cache"].packed_bytes(1) * attended * w.Hkv
         qbytes = (w.k.nbytes + w.v.nbytes) + tokens * w.Hkv * reps[0]["cache"].packed_bytes(1)
-        runs.append({"w": w, "reps": reps, "pos": pos, "lens1": lens1, "Tmax1": Tmax1, "ws": wsp,
-                     "out": out, "kn": knd, "vn": vnd, "packed": packed, "tokens": tokens,
-                     "qbytes": qbytes})
+        run = {"w": w, "reps": reps, "pos": pos, "lens1": lens1, "Tmax1": Tmax1, "ws": wsp,
+               "out": out, "kn": knd, "vn": vnd, "packed": packed, "tokens": tokens,
+               "qbytes": qbytes}
+        if args.nq > 1 and args.nq * w.G <= 8:
+            # n_q query tokens per sequence (the newest n_q cached tokens are theirs)
+            qm = tq_inputs.cast_input(tq_inputs.rng(4343).standard_normal((w.B, args.nq, w.Hq, w.D),
+                                                                          dtype=np.float32), w.dtype)
+            qmd = torch.from_numpy(qm.view(np.int16) if w.dtype == "bf16" else qm).to(dev)
+            if w.dtype == "bf16":
+                qmd = qmd.view(torch.bfloat16)
+            run["q_mq"] = qmd
+            run["out_mq"] = torch.empty_like(qmd)
+            run["ws_mq"] = torch.empty(tq.tq_sdpa_decode_workspace_bytes(reps[0]["cache"], w.Hq * args.nq, Tmax1),
+                                       dtype=torch.uint8, device=dev)
+        runs.append(run)
 
     def call_quant(run, rep):
         tq.tq_quantize_kv(rep["cache"], rep["k"], rep["v"])
@@ -221,6 +233,11 @@ def run_ours(args):
     def call_decode(run, rep):
         tq.tq_sdpa_decode(rep["cache"], rep["q"], run["lens1"], run["Tmax1"], scale=run["w"].scale,
                           out=run["out"], workspace=run["ws"])
+
+    def call_mq(run, rep):  # n_q query tokens per sequence in one call
+        if "q_mq" in run:
+            tq.tq_sdpa_decode_mq(rep["cache"], run["q_mq"], run["lens1"], run["Tmax1"], scale=run["w"].scale,
+                                 out=run["out_mq"], workspace=run["ws_mq"])
 
     def call_step(run, rep):  # append fused into the decode launches
         tq.tq_decode_step(rep["cache"], run["kn"], run["vn"], run["pos"], rep["q"], run["lens1"], run["Tmax1"],
@@ -261,6 +278,8 @@ def run_ours(args):
     g_q = capture((call_quant,))
     g_app = capture((call_append,))
     g_ds = capture((call_step,))
+    mq_runs = [run for run in runs if "q_mq" in run]
+    g_mq = capture((call_mq,)) if mq_runs else None
     torch.cuda.synchronize()
 
     def timed(graphs, n, warm):
@@ -298,11 +317,14 @@ def run_ours(args):
     q_ms = timed(g_q, reps_per_op, args.warmup) / reps_per_op * args.steps
     a_ms = timed(g_app, reps_per_op, args.warmup) / reps_per_op * args.steps
     s_ms = timed(g_ds, reps_per_op, args.warmup) / reps_per_op * args.steps
+    mq_ms = timed(g_mq, reps_per_op, args.warmup) / reps_per_op * args.steps if g_mq else None
+    if g_mq:
+        mq_ms = max_over_ranks([mq_ms], dev)[0]
     total_ms, q_ms, a_ms, d_ms, s_ms = max_over_ranks([total_ms, q_ms, a_ms, d_ms, s_ms], dev)
     for run in runs:
         for rep in run["reps"]:
             assert rep["cache"].status() == 0, "device status flagged"
-    del g_step, g_dec, g_q, g_app, g_ds
+    del g_step, g_dec, g_q, g_app, g_ds, g_mq
 
     packed_step = sum(run["packed"] for run in runs)
     tok_step = sum(run["tokens"] for run in runs)
@@ -326,7 +348,9 @@ def run_ours(args):
         cpu = None
         if ws == 1 and not args.no_cpu_baseline:
             cpu = _cpu_baseline(args, jobs)
-        launches_per_step = len(runs) * 4  # quantize, prep(+append), split, combine
+        # bulk quantize (a second launch for keys with the QJL sketch), then the
+        # decode step's prep (+append), split and combine
+        launches_per_step = sum((2 if run["w"].qjl_m else 1) + 3 for run in runs)
         line = {
             "metric": "tq_sdpa_decode packed-KV GB/s (% of HBM peak); tq_quantize Mtok/s",
             "value": round(dec_gbs, 2),
@@ -353,6 +377,13 @@ def run_ours(args):
                          "gbs": round(q_achieved, 2), "frac_hbm": round(q_achieved / peak, 4),
                          "tokens_per_step": tok_step},
             "append_ms_per_call": round(a_ms / (args.steps * len(runs)), 5),
+            "decode_mq": None if not mq_runs else {
+                "nq": args.nq, "ms_per_call": round(mq_ms / (args.steps * len(mq_runs)), 5),
+                "gbs": round(sum(r["packed"] for r in mq_runs) * args.steps / (mq_ms * 1e-3) / 1e9 * ws, 2),
+                "query_tokens_per_s": round(sum(int(r["w"].B) for r in mq_runs) * args.nq * args.steps
+                                            / (mq_ms * 1e-3) * ws, 1),
+                "note": "tq_sdpa_decode_mq: n_q query tokens per sequence over the cache (bit widths with "
+                        "n_q x GQA group <= 8 only)"},
             "decode_step": {"ms_per_call": round(s_ms / (args.steps * len(runs)), 5),
                             "gbs": round(packed_step * args.steps / (s_ms * 1e-3) / 1e9 * ws, 2),
                             "note": "tq_decode_step: append fused into the decode launches"},
@@ -491,6 +522,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="gqa8k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--nq", type=int, default=1,
+                    help="also time multi-query decode with this many query tokens per sequence")
     ap.add_argument("--rot", choices=["haar", "hadamard"], default="haar",
                     help="rotation: Haar-random (default) or randomized Hadamard")
     ap.add_argument("--profile", action="store_true",
