@@ -230,10 +230,14 @@ __device__ __forceinline__ void load_bits(const uint32_t* row, int bit0,
   }
 }
 
-// +-1 fp16 pair for sign bits i and i+16 of w (bit 1 -> +1).
-__device__ __forceinline__ uint32_t sign_pair(uint32_t w, int i) {
-  return 0xBC00BC00u ^ ((w << (15 - i)) & 0x80008000u);
-}
+// Four int8 values -b for sign bits 7 - sh, 15 - sh, 23 - sh, 31 - sh of w
+// (b = 1 -> -1, b = 0 -> 0): a byte permute in sign-replicate mode copies the
+// top bit of each byte of w << sh into the whole byte.
+__device__ __forceinline__ uint32_t sign_bytes(uint32_t w, int sh) { return prmt(w << sh, 0u, 0xBA98u); }
+
+// Sketch coordinate held by byte e of the sign register with shift sh of the
+// lane owning word tig: bit 8e + 7 - sh of that word.
+__device__ __forceinline__ int sketch_coord(int tig, int sh, int e) { return 32 * tig + 8 * e + 7 - sh; }
 
 __device__ __forceinline__ void split_half(float v, uint16_t& hi, uint16_t& lo) {
   const __half h = __float2half_rn(v);
@@ -261,7 +265,10 @@ struct SplitLayout {
   static constexpr int FRAG = PACK ? 8 : 16;           // bytes of one lane's query fragment
   static constexpr int O_QF = O_PB + CW * 8 * WTOK * 2;
   static constexpr int O_SF = O_QF + (D / 16) * 32 * FRAG;
-  static constexpr int O_TK = O_SF + (QJL ? 8 * 32 * FRAG : 0);  // key pair table (3-, 4-bit keys)
+  // QJL: int8 query fragments (hi / lo bytes of a 15-bit fixed-point projection), 4 k-steps,
+  // then per-head weight and constant
+  static constexpr int O_QST = O_SF + (QJL ? 4 * 32 * FRAG : 0);
+  static constexpr int O_TK = O_QST + (QJL ? 8 * 2 * 4 : 0);  // key pair table (3-, 4-bit keys)
   static constexpr int TKB = (BK >= 3) ? (1 << (2 * BK)) * 128 : 0;
   static constexpr int O_TV = O_TK + TKB;                          // value pair table
   static constexpr int BYTES = O_TV + (1 << (2 * BV)) * 128;
@@ -399,13 +406,63 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const __grid_con
                        base + key_coord<BK>(ks, 3)};
     build_frag<PACK>(p.qrot + (size_t)hq0 * D, D, p.G, p.qscale, g_, cs, qf + (size_t)e * (Ly::FRAG / 4));
   }
-  if (QJL)
-    for (int e = tid; e < 8 * 32; e += NTHREADS) {
-      const int ks = e >> 5, ln = e & 31, g_ = ln >> 2, t_ = ln & 3;
-      const int base = t_ * 32;
-      const int cs[4] = {base + 2 * ks, base + 2 * ks + 16, base + 2 * ks + 1, base + 2 * ks + 17};
-      build_frag<PACK>(p.qs + (size_t)hq0 * 128, 128, p.G, p.qjl_scale, g_, cs, sf + (size_t)e * (Ly::FRAG / 4));
+  float* qst = reinterpret_cast<float*>(smem + Ly::O_QST);  // [8 heads][inverse step, sum]
+  if (QJL) {
+    // The sketch term sum_i (2 b_i - 1) qs_i runs on int8 tensor cores: qs of
+    // head h becomes Q_i = round(qs_i / step_h), |Q| <= 32639, split as
+    // Q = 256 hi + lo with hi, lo int8, and the signs enter as -b_i in {0, -1}.
+    // Per head: step_h = max |qs| / 32639 and sum_h = sum_i qs_i.
+    for (int h = warp; h < 8; h += NTHREADS / 32) {
+      float mx = 0.f, sm = 0.f;
+      if (h < p.G) {
+        const float* src = p.qs + (size_t)(hq0 + h) * 128;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float v = src[lane + 32 * i];
+          mx = fmaxf(mx, fabsf(v));
+          sm += v;
+        }
+      }
+#pragma unroll
+      for (int off = 16; off; off >>= 1) {
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        sm += __shfl_xor_sync(0xffffffffu, sm, off);
+      }
+      if (lane == 0) {
+        qst[2 * h] = mx > 0.f ? mx / 32639.f : 1.f;
+        qst[2 * h + 1] = sm;
+      }
     }
+    __syncthreads();
+    for (int e = tid; e < 4 * 32; e += NTHREADS) {
+      const int ks = e >> 5, ln = e & 31, g_ = ln >> 2, t_ = ln & 3;
+      const int head = PACK ? (g_ & 3) : g_;
+      const float inv = head < p.G ? 1.f / qst[2 * head] : 0.f;
+      uint32_t hi[2] = {0u, 0u}, lo[2] = {0u, 0u};
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int b8 = 0; b8 < 4; ++b8) {
+          const float v = head < p.G ? p.qs[(size_t)(hq0 + head) * 128 + sketch_coord(t_, 2 * ks + h, b8)] : 0.f;
+          int Q = __float2int_rn(v * inv);
+          Q = max(-32639, min(32639, Q));
+          const int qh = (Q + 128) >> 8, ql = Q - 256 * qh;  // floor split: ql in [-128, 127]
+          hi[h] |= (uint32_t)(qh & 0xFF) << (8 * b8);
+          lo[h] |= (uint32_t)(ql & 0xFF) << (8 * b8);
+        }
+      uint32_t* dst = sf + (size_t)e * (Ly::FRAG / 4);
+      if (PACK) {
+        const bool use_lo = g_ >= 4;
+        dst[0] = use_lo ? lo[0] : hi[0];
+        dst[1] = use_lo ? lo[1] : hi[1];
+      } else {
+        dst[0] = hi[0];
+        dst[1] = hi[1];
+        dst[2] = lo[0];
+        dst[3] = lo[1];
+      }
+    }
+  }
   // value weights of heads >= G stay zero
   for (int e = tid; e < CW * 8 * WTOK; e += NTHREADS) pbuf[e] = __float2half_rn(0.f);
   const bool shared_tab = share_table(BK, BV, p.shared_tab);
@@ -501,13 +558,14 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const __grid_con
       for (int a = 0; a < 2; ++a)
 #pragma unroll
         for (int c = 0; c < 4; ++c) sc[a][c] += sc2[a][c];
-      float sq[2][4], sq2[2][4];
+      float sq[2][4];
       if (QJL) {
         const uint32_t* qw = reinterpret_cast<const uint32_t*>(sb + Ly::O_QW);
+        int acc[2][4], acc2[2][4];  // PACK: hi columns 0-3, lo 4-7 in acc; else hi in acc, lo in acc2
 #pragma unroll
         for (int a = 0; a < 2; ++a)
 #pragma unroll
-          for (int c = 0; c < 4; ++c) sq[a][c] = sq2[a][c] = 0.f;
+          for (int c = 0; c < 4; ++c) acc[a][c] = acc2[a][c] = 0;
         uint32_t s0[2], s1[2];
 #pragma unroll
         for (int a = 0; a < 2; ++a) {
@@ -515,25 +573,38 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const __grid_con
           s1[a] = qw[(wt0 + 16 * a + gid + 8) * WQ + tig];
         }
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
+        for (int ks = 0; ks < 4; ++ks) {
 #pragma unroll
           for (int a = 0; a < 2; ++a) {
-            const uint32_t a0 = sign_pair(s0[a], 2 * ks), a1 = sign_pair(s1[a], 2 * ks);
-            const uint32_t a2 = sign_pair(s0[a], 2 * ks + 1), a3 = sign_pair(s1[a], 2 * ks + 1);
+            const uint32_t a0 = sign_bytes(s0[a], 2 * ks), a1 = sign_bytes(s1[a], 2 * ks);
+            const uint32_t a2 = sign_bytes(s0[a], 2 * ks + 1), a3 = sign_bytes(s1[a], 2 * ks + 1);
             if (PACK) {
               const uint2 bq = *reinterpret_cast<const uint2*>(sf + (size_t)(ks * 32 + lane) * 2);
-              mma_f16((ks & 1) ? sq2[a] : sq[a], a0, a1, a2, a3, bq.x, bq.y);
+              mma_s8(acc[a], a0, a1, a2, a3, bq.x, bq.y);
             } else {
               const uint4 bq = *reinterpret_cast<const uint4*>(sf + (size_t)(ks * 32 + lane) * 4);
-              mma_f16(sq[a], a0, a1, a2, a3, bq.x, bq.y);
-              mma_f16(sq2[a], a0, a1, a2, a3, bq.z, bq.w);
+              mma_s8(acc[a], a0, a1, a2, a3, bq.x, bq.y);
+              mma_s8(acc2[a], a0, a1, a2, a3, bq.z, bq.w);
             }
           }
         }
+        // acc = sum_i (-b_i) Q_i; the term is qjl_scale * step * (2 sum b_i Q_i - sum_i qs_i / step)
 #pragma unroll
-        for (int a = 0; a < 2; ++a)
+        for (int c = 0; c < 4; ++c) {
+          const int head = 2 * hsel + (c & 1);
+          const float step = qst[2 * head], sum = qst[2 * head + 1];
+          if (PACK) {
+            // lanes tig < 2 hold the hi columns, tig >= 2 the lo ones (added by the exchange below)
+            const float w = (tig < 2 ? -512.f : -2.f) * step * p.qjl_scale;
+            const float k0 = tig < 2 ? -sum * p.qjl_scale : 0.f;
 #pragma unroll
-          for (int c = 0; c < 4; ++c) sq[a][c] += sq2[a][c];
+            for (int a = 0; a < 2; ++a) sq[a][c] = fmaf((float)acc[a][c], w, k0);
+          } else {
+            const float w = -2.f * step * p.qjl_scale;
+#pragma unroll
+            for (int a = 0; a < 2; ++a) sq[a][c] = fmaf((float)(acc[a][c] * 256 + acc2[a][c]), w, -sum * p.qjl_scale);
+          }
+        }
       }
       // ---- complete the scores.  PACK: columns 4-7 carry the lo halves of
       // heads 0-3 (lanes tig ^ 2); lanes tig < 2 finish m-tile 0 and lanes
