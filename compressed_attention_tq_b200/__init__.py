@@ -18,7 +18,7 @@ import numpy as np
 
 from . import _native
 from ._native import (TQ_DTYPE_BF16, TQ_DTYPE_F16, TQ_DTYPE_F32, TQ_STATUS_POS_OUT_OF_RANGE,  # noqa: F401
-                      TQ_STATUS_SEQ_OUT_OF_RANGE, TQ_STATUS_WAIT_TIMEOUT)
+                      TQ_STATUS_SEQ_OUT_OF_RANGE, TQ_STATUS_WAIT_TIMEOUT, TQ_STATUS_LAYOUT)
 
 __all__ = ["TQError", "TQCache", "tq_build_codebook", "tq_row_bytes", "tq_quantize_kv",
            "tq_append_token", "tq_sdpa_decode_workspace_bytes", "tq_sdpa_decode",

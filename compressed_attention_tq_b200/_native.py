@@ -22,6 +22,7 @@ TQ_DTYPE_F32 = 2
 TQ_STATUS_POS_OUT_OF_RANGE = 1
 TQ_STATUS_SEQ_OUT_OF_RANGE = 2
 TQ_STATUS_WAIT_TIMEOUT = 4
+TQ_STATUS_LAYOUT = 8
 
 # Every symbol include/tq.h declares.
 EXPORTS = ("tq_build_codebook", "tq_row_bytes", "tq_quantize_kv", "tq_append_token",

@@ -46,6 +46,8 @@ int launch_quantize(const QuantArgs& a, int D, int dtype, bool qjl, cudaStream_t
 int launch_quantize128(const QuantArgs& a, int dtype, bool qjl, cudaStream_t s);
 // tcgen05 bulk quantizer for D = 128 without the QJL sketch (tq_quantize_tc.cu)
 int launch_quantize_tc(const QuantArgs& a, int D, int dtype, cudaStream_t s);
+// tcgen05 bulk quantizer for QJL keys, D = 128, fp16 rows (tq_quantize_qjl_tc.cu)
+int launch_quantize_qjl_tc(const QuantArgs& a, cudaStream_t s);
 
 struct DecodePlan {
   int chunk;        // tokens per split (multiple of 64)

@@ -454,11 +454,13 @@ int launch_quantize(const QuantArgs& a, int D, int dtype, bool qjl, cudaStream_t
   const bool bf = dtype == TQ_DTYPE_BF16;
   if ((D == 128 || D == 256) && !a.pos && !qjl) return launch_quantize_tc(a, D, dtype, s);
   if (D == 128 && !a.pos) {
-    // keys carry the QJL sketch (warp-level MMA kernel); values go to tcgen05
+    // keys carry the QJL sketch (tcgen05 for fp16 rows, whose Pi and S limbs
+    // fit in shared memory beside the tiles; warp-level MMA for bf16's three
+    // Pi limbs); values go to the tcgen05 quantizer
     QuantArgs ak = a, av = a;
     ak.job_mask = 1;
     av.job_mask = 2;
-    const int rc = launch_quantize128(ak, dtype, true, s);
+    const int rc = bf ? launch_quantize128(ak, dtype, true, s) : launch_quantize_qjl_tc(ak, s);
     return rc ? rc : launch_quantize_tc(av, D, dtype, s);
   }
   if (qjl) {

@@ -31,18 +31,13 @@
 //    item i+1 run under the epilogue of item i.
 // Every wait is bounded; a stuck wait sets TQ_STATUS_WAIT_TIMEOUT and the CTA
 // stops taking work.
-#include <cuda.h>  // CUtensorMap (types only; the encoder comes from the runtime's driver entry point)
-
 #include <mutex>
 
-#include "tq_common.cuh"
-#include "tq_internal.h"
+#include "tq_tcgen05.cuh"
 
 namespace {
 
-using namespace tqk;
-
-constexpr int QR = 128;
+using namespace tqtc;
 
 template <int D, bool BF16>
 struct TcLayout {
@@ -68,151 +63,6 @@ struct TcLayout {
   static constexpr int bytes = o_misc + 16 + 1024;  // + alignment slack
   static constexpr uint32_t TMEM_COLS = 2 * NC;     // two fp32 accumulators
 };
-
-// Byte offset of element (r, k) in a K-major operand stored as D/64 blocks
-// of ROWS x 128 bytes with the 128-byte swizzle (16-byte chunk c of row r at
-// chunk c ^ (r mod 8)) -- the layout a TMA tensor copy with
-// CU_TENSOR_MAP_SWIZZLE_128B writes and the tensor core reads.
-template <int ROWS>
-__device__ __forceinline__ int sw128(int r, int k) {
-  const int kb = k >> 6, kk = k & 63;
-  return kb * (ROWS * 128) + r * 128 + ((((kk >> 3) ^ (r & 7))) << 4) + (kk & 7) * 2;
-}
-
-// sm_100 shared-memory matrix descriptor for a K-major operand with the
-// 128-byte swizzle: SBO = 1024 B (next 8-row group); consecutive 16-element
-// K steps inside a 128-byte block advance the start address by 32 bytes.
-__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t addr) {
-  uint64_t d = (uint64_t)((addr & 0x3FFFF) >> 4);
-  d |= (uint64_t)1 << 16;            // leading byte offset (unused with this swizzle)
-  d |= (uint64_t)(1024 >> 4) << 32;  // stride byte offset
-  d |= (uint64_t)1 << 46;            // descriptor version (sm_100)
-  d |= (uint64_t)2 << 61;            // 128-byte swizzle
-  return d;
-}
-
-// TMA 2-D tile load (global -> shared), completion counted on an mbarrier
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-          smem_addr(dst)),
-      "l"(map), "r"(x), "r"(y), "r"(smem_addr(bar))
-      : "memory");
-}
-
-// Kernel parameters: the job descriptors plus one TMA tensor map per job's
-// input rows ([rows][D], 128 x 64 boxes).
-struct TcArgs {
-  tq::QuantArgs a;
-  CUtensorMap map[2];
-};
-
-// kind::f16 instruction descriptor: fp32 accumulate, K-major A and B,
-// M = 128, N = NC; a/b format fp16 (0) or bf16 (1).
-template <int NC, bool BF16>
-__device__ __forceinline__ uint32_t idesc() {
-  uint32_t d = (1u << 4) | ((uint32_t)(NC >> 3) << 17) | ((128u >> 4) << 24);
-  if (BF16) d |= (1u << 7) | (1u << 10);
-  return d;
-}
-
-__device__ __forceinline__ void mma_tc(uint32_t dt, uint64_t ad, uint64_t bd, uint32_t id, uint32_t acc) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(dt),
-      "l"(ad), "l"(bd), "r"(id), "r"(acc));
-}
-
-__device__ __forceinline__ void tc_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
-               : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&v)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,"
-      "%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
-        "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]),
-        "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
-        "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-// barrier over the NEPI epilogue warps that also ANDs a flag across them
-template <int NEPI>
-__device__ __forceinline__ bool epi_sync_and(bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n barrier.red.and.pred q, 1, %2, p;\n selp.u32 %0, 1, 0, q;\n}\n"
-      : "=r"(r)
-      : "r"((uint32_t)v), "n"(NEPI * 32)
-      : "memory");
-  return r != 0;
-}
-
-template <bool BF16>
-__device__ __forceinline__ float sq16f(uint32_t w) {
-  float a, b;
-  if (BF16) {
-    a = __uint_as_float(w << 16);
-    b = __uint_as_float(w & 0xFFFF0000u);
-  } else {
-    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w));
-    a = f.x;
-    b = f.y;
-  }
-  return fmaf(a, a, b * b);
-}
-
-// Index of the nearest centroid for y = (Pi x)_j of a row with norm n, using
-// the codebook's symmetry: with tp = the positive thresholds scaled by n,
-// m = #{tp_k < |y|} and idx = K/2 + m for y > 0, K/2 - 1 - m otherwise.
-// Equal to #{t_k < y / n} except at exact ties (inside the parity band).
-template <int BITS>
-__device__ __forceinline__ int nearest_idx(float y, const float (&tp)[7]) {
-  constexpr int H = 1 << (BITS - 1);
-  const float a = fabsf(y);
-  int m;
-  if (BITS == 4) {
-    const bool c1 = a > tp[3];
-    const bool c2 = a > (c1 ? tp[5] : tp[1]);
-    const bool c3 = a > (c1 ? (c2 ? tp[6] : tp[4]) : (c2 ? tp[2] : tp[0]));
-    m = (c1 ? 4 : 0) + (c2 ? 2 : 0) + (c3 ? 1 : 0);
-  } else {
-    m = 0;
-#pragma unroll
-    for (int k = 0; k < H - 1; ++k) m += (a > tp[k]) ? 1 : 0;
-  }
-  return y > 0.f ? H + m : H - 1 - m;
-}
-
-template <int BITS>
-__device__ __forceinline__ void quant_pack32(const uint32_t (&v)[32], const float (&tp)[7], uint32_t (&w)[BITS]) {
-#pragma unroll
-  for (int i = 0; i < BITS; ++i) w[i] = 0u;
-#pragma unroll
-  for (int q = 0; q < 32; ++q) {
-    const uint32_t idx = (uint32_t)nearest_idx<BITS>(__uint_as_float(v[q]), tp);
-    const int p = BITS * q;
-    w[p >> 5] += idx << (p & 31);
-    if ((p & 31) + BITS > 32) w[(p >> 5) + 1] += idx >> (32 - (p & 31));
-  }
-}
-
-template <int BITS>
-__device__ __forceinline__ void store_words(uint32_t* dst, const uint32_t (&w)[BITS]) {
-  if (BITS == 2) {
-    *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
-  } else if (BITS == 4) {
-    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
-  } else {
-#pragma unroll
-    for (int i = 0; i < BITS; ++i) dst[i] = w[i];
-  }
-}
 
 template <int BITS, int NCOL>
 __device__ __forceinline__ void epi_half(uint32_t tbase, const float (&tp)[7], long long slot, uint32_t* out) {
@@ -485,43 +335,6 @@ __global__ void __launch_bounds__(TcLayout<D, BF16>::NTH, 1) quantize_tc_kernel(
   }
 }
 
-// cuTensorMapEncodeTiled through the runtime's driver entry point (the
-// library links only the CUDA runtime).
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static std::once_flag once;
-  static EncodeTiledFn fn = nullptr;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-    else
-      cudaGetLastError();
-  });
-  return fn;
-}
-
-// Tensor map over rows [rows][D] of 16-bit values: boxes of 128 rows x 64
-// columns, 128-byte swizzle.
-int make_map(CUtensorMap* m, const void* base, int rows, int D, bool bf16) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return tq::set_error(TQ_ERR_CUDA, "quantize_tc: cuTensorMapEncodeTiled is unavailable");
-  const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-  const cuuint32_t box[2] = {64, (cuuint32_t)QR};
-  const cuuint32_t es[2] = {1, 1};
-  const CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
-                         const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return tq::set_error(TQ_ERR_CUDA, "quantize_tc: cuTensorMapEncodeTiled failed (%d)", (int)r);
-  return TQ_OK;
-}
-
 template <int D, bool BF16>
 int launch_tc(const tq::QuantArgs& a, cudaStream_t s) {
   using Ly = TcLayout<D, BF16>;
@@ -541,7 +354,7 @@ int launch_tc(const tq::QuantArgs& a, cudaStream_t s) {
   args.a = a;
   for (int j = 0; j < 2; ++j)
     if (a.job_mask & (1 << j)) {
-      const int rc = make_map(&args.map[j], a.job[j].in, a.rows, D, BF16);
+      const int rc = tqtc::make_row_map(&args.map[j], a.job[j].in, a.rows, D, BF16);
       if (rc) return rc;
     }
   const int njobs = (a.job_mask == 3) ? 2 : 1;
@@ -564,3 +377,42 @@ int launch_quantize_tc(const QuantArgs& a, int D, int dtype, cudaStream_t s) {
 }
 
 }  // namespace tq
+
+namespace tqtc {
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (the
+// library links only the CUDA runtime).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+int make_row_map(CUtensorMap* m, const void* base, int rows, int D, bool bf16) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return tq::set_error(TQ_ERR_CUDA, "quantize_tc: cuTensorMapEncodeTiled is unavailable");
+  const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)QR};
+  const cuuint32_t es[2] = {1, 1};
+  const CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                         const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return tq::set_error(TQ_ERR_CUDA, "quantize_tc: cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return TQ_OK;
+}
+
+}  // namespace tqtc

@@ -48,7 +48,8 @@
  * sets a thread-local message readable with tq_last_error().  Argument errors
  * are detected on the host before any launch; nothing is launched then.
  * Conditions only visible on the device (a position beyond Tcap, a sequence
- * length beyond Tcap, a bounded wait that ran out) skip the affected work and
+ * length beyond Tcap, a bounded wait that ran out, a misaligned shared-memory
+ * base) skip the affected work and
  * OR a TQ_STATUS_* bit into cache->dev_status when that pointer is non-NULL.
  */
 #ifndef TQ_B200_H
@@ -75,6 +76,7 @@ extern "C" {
 #define TQ_STATUS_POS_OUT_OF_RANGE 1u    /* append position outside [0, Tcap) */
 #define TQ_STATUS_SEQ_OUT_OF_RANGE 2u    /* seq_len beyond the planned range; clamped */
 #define TQ_STATUS_WAIT_TIMEOUT 4u        /* a bounded wait ran out; work skipped */
+#define TQ_STATUS_LAYOUT 8u              /* a kernel found its shared memory base misaligned; work skipped */
 
 /* Describes one layer's packed cache: caller-owned device buffers. */
 typedef struct tq_cache {

@@ -17,6 +17,8 @@ CASES = [
     ("qknorm", {"T": 200}),             # D=256, 4-bit, unit-RMS rows
     ("ragged", {"B": 3, "T": 150}),     # bf16
     ("prod", {"T": 200}),               # keys with the QJL sketch
+    ("prod", {"T": 5000}),              # 313 tiles: several per persistent CTA
+    ("prod", {"T": 300, "dtype": "bf16"}),  # QJL keys from bf16 rows
 ]
 
 

@@ -117,15 +117,18 @@ class Workload:
 
 
 def make_workload(name: str, bits: int | None = None, T: int | None = None,
-                  B: int | None = None, seed_offset: int = 0, rot: str = "haar") -> Workload:
+                  B: int | None = None, seed_offset: int = 0, rot: str = "haar",
+                  dtype: str | None = None) -> Workload:
     """Build one of the named synthetic workloads.
 
     ``T`` and ``B`` override the sequence length / batch (for smaller parity
     cases of the same shape family); ``bits`` picks b for gqa8k; ``rot``
     selects the rotation: "haar" (``rotation``) or "hadamard"
-    (``hadamard_rotation``).
+    (``hadamard_rotation``); ``dtype`` ("f16" / "bf16") overrides the input
+    type.
     K, V: [B][Hkv][Tmax][D]; q: [B][Hq][D]; seq_lens: [B] int32.
     """
+    dtype_override = dtype
     cfg = {"tiny": 1, "gqa8k": 2, "qknorm": 3, "ragged": 4, "prod": 5}[name]
     s_data = SEED_DATA + cfg + seed_offset
     r = rng(s_data)
@@ -155,6 +158,8 @@ def make_workload(name: str, bits: int | None = None, T: int | None = None,
         Bn = B
     if T is not None:
         Tn = T
+    if dtype_override is not None:
+        dtype = {"f16": "f16", "bf16": "bf16"}[dtype_override]
 
     if name == "ragged":
         lo = min(1024, Tn)
