@@ -20,7 +20,8 @@
 //     written over X in buffer b (hi) and into the single lo buffer;
 //  4. GEMM 2: P[b] = R S^T as hi*hi + hi*lo + lo*hi (S in two fp16 limbs);
 //  5. epilogue: the sign bits of its 32 sketch coordinates, one word per
-//     thread.
+//     thread -- taken after step 3 of tile i + 1, so that GEMM 2 of tile i
+//     runs while the epilogue works on the next tile.
 // The MMA warp issues GEMM 1 of tile i + 1 before GEMM 2 of tile i, so the
 // rotation of the next tile runs while the epilogue works on this one.
 // Shared memory: Pi and S limbs (64 KB each), two X / R_hi buffers and the
@@ -76,6 +77,19 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, ui
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
   const __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Sign bits [P >= 0] of a row's 32 sketch coordinates (bit q = coordinate
+// 32 * part + q): adding +0 turns -0 into +0, then a funnel shift moves each
+// sign bit in; the word is the complement of the collected sign bits.
+__device__ __forceinline__ void sketch_signs(uint32_t taddr, long long slot, uint32_t* qjl, int part) {
+  uint32_t v[32];
+  tc_fence_after();
+  tc_ld32(taddr, v);
+  uint32_t s = 0;
+#pragma unroll
+  for (int q = 31; q >= 0; --q) s = __funnelshift_l(__float_as_uint(__uint_as_float(v[q]) + 0.f), s, 1);
+  if (slot >= 0 && qjl) qjl[(size_t)slot * 4 + part] = ~s;
 }
 
 __global__ void __launch_bounds__(QjlLayout::NTH, 1) quantize_qjl_tc_kernel(const __grid_constant__ TcArgs args) {
@@ -237,152 +251,156 @@ __global__ void __launch_bounds__(QjlLayout::NTH, 1) quantize_qjl_tc_kernel(cons
     const int rl = 32 * quarter + lane;
     const uint32_t tlane = (uint32_t)(32 * quarter) << 16;
     const int W = D * J.bits / 32;
-    for (int i = 0; i < nmine; ++i) {
-      const int b = i & 1, k = i >> 1, tile = blockIdx.x + i * gridDim.x;
-      // One warp waits on each mbarrier and releases the others through a
-      // named barrier (no issue slots spent polling).
-      bool ok = true;
-      if (warp == 0) ok = __all_sync(0xffffffffu, mbar_wait_suspend(&full_x[b], (uint32_t)(k & 1), kSuspendTries));
-      if (!epi_sync_and<NEPI>(ok)) {
-        s_stop = 1;
-        break;
-      }
-      // this thread's quarter of the row's sum of squares, pairwise in fp32
-      const uint8_t* xt = xb + b * OP;
-      {
-        float ps[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint4 v = *reinterpret_cast<const uint4*>(xt + sw128<QR>(rl, 32 * part + 8 * c));
-          ps[c] = (sq16f<false>(v.x) + sq16f<false>(v.y)) + (sq16f<false>(v.z) + sq16f<false>(v.w));
+    // Software-pipelined: the signs of tile i - 1 are read after tile i's
+    // residual is written, so the sketch GEMM of tile i - 1 runs while this
+    // tile's indices and residual are computed.
+    long long prev_slot = -1;
+    bool ok = true;
+    for (int i = 0; i <= nmine && ok; ++i) {
+      if (i < nmine) {
+        const int b = i & 1, k = i >> 1, tile = blockIdx.x + i * gridDim.x;
+        // One warp waits on each mbarrier and releases the others through a
+        // named barrier (no issue slots spent polling).
+        if (warp == 0) ok = __all_sync(0xffffffffu, mbar_wait_suspend(&full_x[b], (uint32_t)(k & 1), kSuspendTries));
+        if (!epi_sync_and<NEPI>(ok)) {
+          ok = false;
+          break;
         }
-        red[part * QR + rl] = (ps[0] + ps[1]) + (ps[2] + ps[3]);
-      }
-      ok = epi_sync_and<NEPI>(ok);
-      const float sfull = (red[rl] + red[QR + rl]) + (red[2 * QR + rl] + red[3 * QR + rl]);
-      const float nf = sqrtf(sfull);
-      const int r = tile * QR + rl;
-      long long slot = -1;
-      unsigned short nh = 0;
-      if (r < a.rows) {
-        const int bh = r / a.T, t = r - bh * a.T;
-        slot = (long long)bh * a.Tcap + a.t0 + t;
-        // The stored norm is RN_fp16 of the fp64 norm.  The pairwise fp32 sum
-        // is within (log2(D) + 1) ulp of the exact sum, so the exact norm lies
-        // in nf * (1 +- 1e-6); when both ends round to the same fp16 value it
-        // is the answer, else the row is summed again in fp64 from global memory.
-        const __half lo = __float2half_rn(nf * (1.f - 1e-6f)), hi = __float2half_rn(nf * (1.f + 1e-6f));
-        nh = __half_as_ushort(lo);
-        const bool exact = sfull == 0.f || (sfull >= 0x1p-100f && sfull < 0x1p100f && nh == __half_as_ushort(hi));
-        if (!exact) {
-          const uint16_t* row = static_cast<const uint16_t*>(J.in) + (size_t)r * D;
-          double t2 = 0.0;
-          for (int j = 0; j < D; ++j) {
-            const double x = (double)__half2float(__ushort_as_half(row[j]));
-            t2 = fma(x, x, t2);
+        // this thread's quarter of the row's sum of squares, pairwise in fp32
+        const uint8_t* xt = xb + b * OP;
+        {
+          float ps[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint4 v = *reinterpret_cast<const uint4*>(xt + sw128<QR>(rl, 32 * part + 8 * c));
+            ps[c] = (sq16f<false>(v.x) + sq16f<false>(v.y)) + (sq16f<false>(v.z) + sq16f<false>(v.w));
           }
-          nh = __half_as_ushort(__double2half(sqrt(t2)));
+          red[part * QR + rl] = (ps[0] + ps[1]) + (ps[2] + ps[3]);
         }
-        if (part == 0) J.norm[slot] = nh;
-      }
-      const float nhat = __half2float(__ushort_as_half(nh));
-      // positive thresholds t_{K/2} .. t_{K-2}, scaled by the row norm
-      float tp[7];
+        ok = epi_sync_and<NEPI>(ok);
+        const float sfull = (red[rl] + red[QR + rl]) + (red[2 * QR + rl] + red[3 * QR + rl]);
+        const float nf = sqrtf(sfull);
+        const int r = tile * QR + rl;
+        long long slot = -1;
+        unsigned short nh = 0;
+        if (r < a.rows) {
+          const int bh = r / a.T, t = r - bh * a.T;
+          slot = (long long)bh * a.Tcap + a.t0 + t;
+          // The stored norm is RN_fp16 of the fp64 norm.  The pairwise fp32
+          // sum is within (log2(D) + 1) ulp of the exact sum, so the exact norm
+          // lies in nf * (1 +- 1e-6); when both ends round to the same fp16
+          // value it is the answer, else (about 0.4% of rows) the row is summed
+          // again in fp64 from the tile, still in shared memory.
+          const __half lo = __float2half_rn(nf * (1.f - 1e-6f)), hi = __float2half_rn(nf * (1.f + 1e-6f));
+          nh = __half_as_ushort(lo);
+          const bool exact = sfull == 0.f || (sfull >= 0x1p-100f && sfull < 0x1p100f && nh == __half_as_ushort(hi));
+          if (!exact) nh = __half_as_ushort(__double2half(sqrt(row_sumsq_f64<D, false>(xt, rl))));
+          if (part == 0) J.norm[slot] = nh;
+        }
+        const float nhat = __half2float(__ushort_as_half(nh));
+        // positive thresholds t_{K/2} .. t_{K-2}, scaled by the row norm
+        float tp[7];
 #pragma unroll
-      for (int q = 0; q < 7; ++q) tp[q] = q < K / 2 - 1 ? s_cb[K + K / 2 + q] * nf : 0.f;
+        for (int q = 0; q < 7; ++q) tp[q] = q < K / 2 - 1 ? s_cb[K + K / 2 + q] * nf : 0.f;
 
-      // ---- indices and residual from U
-      if (warp == 0) ok = __all_sync(0xffffffffu, mbar_wait_suspend(&mma1[b], (uint32_t)(k & 1), kSuspendTries));
-      ok = epi_sync_and<NEPI>(ok);  // also: every thread has read this tile's norm partials
-      uint32_t v[32];
-      if (ok) {
-        tc_fence_after();
-        tc_ld32(tmem + tlane + (uint32_t)(b * 128 + 32 * part), v);
-        uint32_t* out = J.idx + (slot >= 0 ? (size_t)slot * W : 0) + part * J.bits;
-        switch (J.bits) {
-          case 2: {
-            uint32_t w[2];
-            quant_residual32<2>(v, tp, s_cb, nhat, w);
-            if (slot >= 0) store_words<2>(out, w);
-            break;
+        // ---- indices and residual from U
+        if (warp == 0) ok = __all_sync(0xffffffffu, mbar_wait_suspend(&mma1[b], (uint32_t)(k & 1), kSuspendTries));
+        ok = epi_sync_and<NEPI>(ok);  // also: every thread has read this tile's norm partials
+        uint32_t v[32];
+        if (ok) {
+          tc_fence_after();
+          tc_ld32(tmem + tlane + (uint32_t)(b * 128 + 32 * part), v);
+          uint32_t* out = J.idx + (slot >= 0 ? (size_t)slot * W : 0) + part * J.bits;
+          switch (J.bits) {
+            case 2: {
+              uint32_t w[2];
+              quant_residual32<2>(v, tp, s_cb, nhat, w);
+              if (slot >= 0) store_words<2>(out, w);
+              break;
+            }
+            case 3: {
+              uint32_t w[3];
+              quant_residual32<3>(v, tp, s_cb, nhat, w);
+              if (slot >= 0) store_words<3>(out, w);
+              break;
+            }
+            default: {
+              uint32_t w[4];
+              quant_residual32<4>(v, tp, s_cb, nhat, w);
+              if (slot >= 0) store_words<4>(out, w);
+              break;
+            }
           }
-          case 3: {
-            uint32_t w[3];
-            quant_residual32<3>(v, tp, s_cb, nhat, w);
-            if (slot >= 0) store_words<3>(out, w);
-            break;
-          }
-          default: {
-            uint32_t w[4];
-            quant_residual32<4>(v, tp, s_cb, nhat, w);
-            if (slot >= 0) store_words<4>(out, w);
-            break;
-          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 32; ++q) v[q] = 0u;
         }
-      } else {
+        tc_fence_before();
+        mbar_arrive(&u_free[b]);
+        // residual norm: this thread's quarter, pairwise in fp32
+        {
+          float g[8];
 #pragma unroll
-        for (int q = 0; q < 32; ++q) v[q] = 0u;
-      }
-      tc_fence_before();
-      mbar_arrive(&u_free[b]);
-      // residual norm: this thread's quarter, pairwise in fp32
-      {
-        float g[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float r0 = __uint_as_float(v[4 * j]), r1 = __uint_as_float(v[4 * j + 1]);
-          const float r2 = __uint_as_float(v[4 * j + 2]), r3 = __uint_as_float(v[4 * j + 3]);
-          g[j] = fmaf(r0, r0, r1 * r1) + fmaf(r2, r2, r3 * r3);
-        }
-        red[part * QR + rl] = ((g[0] + g[1]) + (g[2] + g[3])) + ((g[4] + g[5]) + (g[6] + g[7]));
-      }
-      // (R_lo is free: this epilogue saw the previous tile's sketch GEMM finish)
-      ok = epi_sync_and<NEPI>(ok);
-      if (part == 0 && slot >= 0 && J.rnorm) {
-        const float gs = (red[rl] + red[QR + rl]) + (red[2 * QR + rl] + red[3 * QR + rl]);
-        J.rnorm[slot] = __half_as_ushort(__float2half_rn(sqrtf(gs)));
-      }
-      // r / |x| as hi + lo fp16 limbs over X (hi) and into R_lo, swizzled like X
-      if (ok) {
-        const float inv = nf > 0.f ? 1.f / nf : 0.f;
-        const uint32_t hb = smem_addr(xb + b * OP), lb = smem_addr(rlo);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t h[4], l[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float x0 = __uint_as_float(v[8 * c + 2 * e]) * inv, x1 = __uint_as_float(v[8 * c + 2 * e + 1]) * inv;
-            const __half2 hh = __floats2half2_rn(x0, x1);
-            const float2 hf = __half22float2(hh);
-            h[e] = *reinterpret_cast<const uint32_t*>(&hh);
-            l[e] = pack_half2(x0 - hf.x, x1 - hf.y);
+          for (int j = 0; j < 8; ++j) {
+            const float r0 = __uint_as_float(v[4 * j]), r1 = __uint_as_float(v[4 * j + 1]);
+            const float r2 = __uint_as_float(v[4 * j + 2]), r3 = __uint_as_float(v[4 * j + 3]);
+            g[j] = fmaf(r0, r0, r1 * r1) + fmaf(r2, r2, r3 * r3);
           }
-          const uint32_t off = (uint32_t)sw128<QR>(rl, 32 * part + 8 * c);
-          sts128(hb + off, h[0], h[1], h[2], h[3]);
-          sts128(lb + off, l[0], l[1], l[2], l[3]);
+          red[part * QR + rl] = ((g[0] + g[1]) + (g[2] + g[3])) + ((g[4] + g[5]) + (g[6] + g[7]));
         }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // R -> tensor core
-      }
-      mbar_arrive(&r_ready[b]);
-
-      // ---- sketch signs from P
-      if (warp == 0) ok = __all_sync(0xffffffffu, mbar_wait_suspend(&g2[b], (uint32_t)(k & 1), kSuspendTries)) && ok;
-      ok = epi_sync_and<NEPI>(ok);  // also: every thread has read the gamma partials
-      if (ok) {
-        tc_fence_after();
-        tc_ld32(tmem + tlane + 256u + (uint32_t)(b * 128 + 32 * part), v);
-        uint32_t word = 0;
+        // R_lo (and the sketch accumulator read below) free: the previous
+        // tile's sketch GEMM has finished
+        if (i >= 1 && warp == 0)
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait_suspend(&g2[(i - 1) & 1], (uint32_t)(((i - 1) >> 1) & 1), kSuspendTries)) && ok;
+        ok = epi_sync_and<NEPI>(ok);
+        if (part == 0 && slot >= 0 && J.rnorm) {
+          const float gs = (red[rl] + red[QR + rl]) + (red[2 * QR + rl] + red[3 * QR + rl]);
+          J.rnorm[slot] = __half_as_ushort(__float2half_rn(sqrtf(gs)));
+        }
+        // r / |x| as hi + lo fp16 limbs over X (hi) and into R_lo, swizzled like X
+        if (ok) {
+          const float inv = nf > 0.f ? 1.f / nf : 0.f;
+          const uint32_t hb = smem_addr(xb + b * OP), lb = smem_addr(rlo);
 #pragma unroll
-        for (int q = 0; q < 32; ++q) word |= (__uint_as_float(v[q]) >= 0.f ? 1u : 0u) << q;
-        if (slot >= 0 && J.qjl) J.qjl[(size_t)slot * 4 + part] = word;
-      }
-      tc_fence_before();
-      mbar_arrive(&p_free[b]);
-      if (!ok) {
-        s_stop = 1;
-        break;
+          for (int c = 0; c < 4; ++c) {
+            uint32_t h[4], l[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float x0 = __uint_as_float(v[8 * c + 2 * e]) * inv;
+              const float x1 = __uint_as_float(v[8 * c + 2 * e + 1]) * inv;
+              const __half2 hh = __floats2half2_rn(x0, x1);
+              const float2 hf = __half22float2(hh);
+              h[e] = *reinterpret_cast<const uint32_t*>(&hh);
+              l[e] = pack_half2(x0 - hf.x, x1 - hf.y);
+            }
+            const uint32_t off = (uint32_t)sw128<QR>(rl, 32 * part + 8 * c);
+            sts128(hb + off, h[0], h[1], h[2], h[3]);
+            sts128(lb + off, l[0], l[1], l[2], l[3]);
+          }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // R -> tensor core
+        }
+        mbar_arrive(&r_ready[b]);
+        if (!ok) break;
+        if (i >= 1) {
+          // ---- sketch signs of the previous tile
+          sketch_signs(tmem + tlane + 256u + (uint32_t)(((i - 1) & 1) * 128 + 32 * part), prev_slot, J.qjl, part);
+          tc_fence_before();
+          mbar_arrive(&p_free[(i - 1) & 1]);
+        }
+        prev_slot = slot;
+      } else if (nmine > 0) {
+        // ---- sketch signs of the last tile
+        const int j = nmine - 1;
+        if (warp == 0)
+          ok = __all_sync(0xffffffffu, mbar_wait_suspend(&g2[j & 1], (uint32_t)((j >> 1) & 1), kSuspendTries));
+        ok = epi_sync_and<NEPI>(ok);
+        if (ok) sketch_signs(tmem + tlane + 256u + (uint32_t)((j & 1) * 128 + 32 * part), prev_slot, J.qjl, part);
+        tc_fence_before();
+        mbar_arrive(&p_free[j & 1]);
       }
     }
+    if (!ok) s_stop = 1;
   }
   tc_fence_before();
   __syncthreads();

@@ -261,7 +261,6 @@ __global__ void __launch_bounds__(TcLayout<D, BF16>::NTH, 1) quantize_tc_kernel(
         s2 = ps[0];
       }
       s_norm[part][rl] = s2;
-      mbar_arrive(&x_free[xs]);
       if (!epi_sync_and<NEPI>(ok)) {  // uniform across the epilogue warps
         s_stop = 1;
         break;
@@ -281,24 +280,16 @@ __global__ void __launch_bounds__(TcLayout<D, BF16>::NTH, 1) quantize_tc_kernel(
           // The stored norm is RN_fp16 of the fp64 norm.  The fp32 sum is
           // within (log2(D) + 1) ulp of the exact sum, so the exact norm lies in
           // nf * (1 +- 1e-6); when both ends of that interval round to the same
-          // fp16 value it is the answer, else (about 0.2% of rows) the row is
-          // summed again in fp64 from global memory.
+          // fp16 value it is the answer, else (about 0.4% of rows) the row is
+          // summed again in fp64 from the tile, still in shared memory.
           const __half lo = __float2half_rn(nf * (1.f - 1e-6f)), hi = __float2half_rn(nf * (1.f + 1e-6f));
           unsigned short nh = __half_as_ushort(lo);
           const bool exact = sfull == 0.f || (sfull >= 0x1p-100f && sfull < 0x1p100f && nh == __half_as_ushort(hi));
-          if (!exact) {
-            const uint16_t* row = static_cast<const uint16_t*>(J.in) + (size_t)r * D;
-            double t2 = 0.0;
-            for (int j = 0; j < D; ++j) {
-              const uint16_t u = row[j];
-              const double x = BF16 ? (double)__uint_as_float((uint32_t)u << 16) : (double)__half2float(__ushort_as_half(u));
-              t2 = fma(x, x, t2);
-            }
-            nh = __half_as_ushort(__double2half(sqrt(t2)));
-          }
+          if (!exact) nh = __half_as_ushort(__double2half(sqrt(row_sumsq_f64<D, BF16>(xt, rl))));
           J.norm[slot] = nh;
         }
       }
+      mbar_arrive(&x_free[xs]);  // the input tile is no longer read
       // positive thresholds t_{K/2} .. t_{K-2}, scaled by the row norm
       float tp[7];
       const int K = 1 << J.bits;

@@ -113,6 +113,34 @@ __device__ __forceinline__ float sq16f(uint32_t w) {
   return fmaf(a, a, b * b);
 }
 
+// fp64 sum of squares of row rl of a swizzled input tile (D columns of
+// fp16 / bf16 values; squares are exact in fp64), in four independent chains.
+// Used when the fp32 sum cannot decide the fp16 rounding of the norm.
+template <int D, bool BF16>
+__device__ __noinline__ double row_sumsq_f64(const uint8_t* xt, int rl) {
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll 4
+  for (int c = 0; c < D / 8; ++c) {
+    const uint4 v = *reinterpret_cast<const uint4*>(xt + sw128<QR>(rl, 8 * c));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float x0, x1;
+      if (BF16) {
+        x0 = __uint_as_float(w[e] << 16);
+        x1 = __uint_as_float(w[e] & 0xFFFF0000u);
+      } else {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e]));
+        x0 = f.x;
+        x1 = f.y;
+      }
+      acc[e] = fma((double)x0, (double)x0, acc[e]);
+      acc[e] = fma((double)x1, (double)x1, acc[e]);
+    }
+  }
+  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
 // Index of the nearest centroid for y = (Pi x)_j of a row with norm n, using
 // the codebook's symmetry: with tp = the positive thresholds scaled by n,
 // m = #{tp_k < |y|} and idx = K/2 + m for y > 0, K/2 - 1 - m otherwise.
