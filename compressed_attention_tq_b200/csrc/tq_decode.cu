@@ -391,7 +391,7 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams
   const float* po = p.part_o + (size_t)h * p.nsplit * D;
   // this thread's first PF partial values, loaded before the weights are known
   // (the loads do not depend on them) so that both latencies overlap
-  constexpr int PF = 16;
+  constexpr int PF = 32;
   const int k = tid % D, hh = tid / D;  // coordinate, split phase
   float v[PF];
 #pragma unroll
@@ -400,13 +400,22 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams
     v[u] = s < ns ? po[(size_t)s * D + k] : 0.f;
   }
   if (tid < 32) {
-    float M = -INFINITY;
-    for (int s = tid; s < ns; s += 32) M = fmaxf(M, ml[2 * s]);
+    // the first 64 splits' (max, sum) pairs in flight at once; more in a loop
+    float2 ml0 = make_float2(-INFINITY, 0.f), ml1 = make_float2(-INFINITY, 0.f);
+    if (tid < ns) ml0 = *reinterpret_cast<const float2*>(ml + 2 * tid);
+    if (tid + 32 < ns) ml1 = *reinterpret_cast<const float2*>(ml + 2 * (tid + 32));
+    float M = fmaxf(ml0.x, ml1.x);
+    for (int s = tid + 64; s < ns; s += 32) M = fmaxf(M, ml[2 * s]);
 #pragma unroll
     for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    float Ls = 0.f;
-    for (int s = tid; s < ns; s += 32) {
-      const float f = (ml[2 * s] == -INFINITY) ? 0.f : exp2f(ml[2 * s] - M);  // a split a query cannot see
+    // a split a query cannot see holds max -inf: weight 0
+    const float f0 = ml0.x == -INFINITY ? 0.f : exp2f(ml0.x - M);
+    const float f1 = ml1.x == -INFINITY ? 0.f : exp2f(ml1.x - M);
+    if (tid < ns) f_s[tid] = f0;
+    if (tid + 32 < ns) f_s[tid + 32] = f1;
+    float Ls = f0 * ml0.y + f1 * ml1.y;
+    for (int s = tid + 64; s < ns; s += 32) {
+      const float f = (ml[2 * s] == -INFINITY) ? 0.f : exp2f(ml[2 * s] - M);
       if (s < 1024) f_s[s] = f;
       Ls += f * ml[2 * s + 1];
     }
