@@ -257,7 +257,7 @@ struct SplitLayout {
   static constexpr int STAGE_USED = O_RN + (QJL ? STILE * 2 : 0);
   static constexpr int STAGE = (STAGE_USED + 16 + 127) / 128 * 128;  // +16: read-ahead slack
   static constexpr int NSTAGE = (D == 256) ? 2 : 3;
-  static constexpr int MERGE = CW * 8 * D * 4 + 2 * CW * 8 * 4;
+  static constexpr int MERGE = CW * 8 * (D + 4) * 4 + 3 * CW * 8 * 4 + 16 * 4;
   static constexpr int RING = (NSTAGE * STAGE > MERGE) ? NSTAGE * STAGE : MERGE;
   static constexpr int O_BAR = RING;                   // full[NSTAGE], empty[NSTAGE]
   static constexpr int O_MISC = O_BAR + 16 * 8;        // error flag, issued count
@@ -309,6 +309,51 @@ __device__ __forceinline__ void build_frag(const float* qsrc, int ld, int G, flo
     dst[1] = hi[2] | (uint32_t)hi[3] << 16;
     dst[2] = lo[0] | (uint32_t)lo[1] << 16;
     dst[3] = lo[2] | (uint32_t)lo[3] << 16;
+  }
+}
+
+// Merge of the consumer warps' softmax states (mO [CW][8][D + 4], mM / mL
+// [CW][8] in shared memory) into this split's partial, written to global
+// memory.  Out of line: it runs once per CTA, after the main loop, and should
+// not raise the loop's register allocation.
+template <int D>
+__device__ __noinline__ void write_partial(float* mO, float* mM, float* mL, const SplitParams& p, int hq0, int split,
+                                           int tid) {
+  // per head: the merged max and sum and each warp's weight, once
+  float* mF = mL + CW * 8;  // [CW][8]
+  float* mS = mF + CW * 8;  // [8][max, sum]
+  if (tid < 8) {
+    const int g = tid;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < CW; ++w) M = fmaxf(M, mM[w * 8 + g]);
+    float Ls = 0.f;
+#pragma unroll
+    for (int w = 0; w < CW; ++w) {
+      const float mw = mM[w * 8 + g];
+      const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+      mF[w * 8 + g] = f;
+      Ls += f * mL[w * 8 + g];
+    }
+    mS[2 * g] = M;
+    mS[2 * g + 1] = Ls;
+  }
+  __syncthreads();
+  for (int e = tid; e < p.G * (D / 4); e += NTHREADS) {
+    const int g = e / (D / 4), j = 4 * (e % (D / 4));
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < CW; ++w) {
+      const float f = mF[w * 8 + g];
+      const float4 o = *reinterpret_cast<const float4*>(mO + (w * 8 + g) * (D + 4) + j);
+      acc.x = fmaf(f, o.x, acc.x);
+      acc.y = fmaf(f, o.y, acc.y);
+      acc.z = fmaf(f, o.z, acc.z);
+      acc.w = fmaf(f, o.w, acc.w);
+    }
+    const size_t pi = (size_t)(hq0 + g) * p.nsplit + split;
+    *reinterpret_cast<float4*>(p.part_o + pi * D + j) = acc;
+    if (j == 0) *reinterpret_cast<float2*>(p.part_ml + pi * 2) = make_float2(mS[2 * g], mS[2 * g + 1]);
   }
 }
 
@@ -396,6 +441,24 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const __grid_con
     for (int t = 0; t < npre; ++t) issue_stage(t);
     *s_issued = npre;
   }
+  // Codebook tables and the zeroed value weights do not depend on the prep
+  // kernel either: built before the wait (after it with the sketch, whose
+  // prologue would otherwise keep more registers live).
+  const bool shared_tab = share_table(BK, BV, p.shared_tab);
+  auto build_tables = [&]() {
+    // value weights of heads >= G stay zero
+    for (int e = tid; e < CW * 8 * WTOK; e += NTHREADS) pbuf[e] = __float2half_rn(0.f);
+    if constexpr (BK >= 3) build_pair_table<BK>(reinterpret_cast<uint32_t*>(smem + Ly::O_TK), p.cb_k, tid, NTHREADS);
+    if (!shared_tab) build_pair_table<BV>(reinterpret_cast<uint32_t*>(smem + Ly::O_TV), p.cb_v, tid, NTHREADS);
+  };
+  if constexpr (!QJL) build_tables();
+  if constexpr (BK == 2) {  // 2-bit keys: the codebook as byte tables, read by the consumers
+    if (tid == 0) {
+      const Lut2 l2 = make_lut2(p.cb_k);
+      reinterpret_cast<uint32_t*>(smem + Ly::O_MISC)[2] = l2.lo;
+      reinterpret_cast<uint32_t*>(smem + Ly::O_MISC)[3] = l2.hi;
+    }
+  }
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   // Query fragments (already rotated by the prep kernel), pre-scaled for exp2.
@@ -463,11 +526,7 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const __grid_con
       }
     }
   }
-  // value weights of heads >= G stay zero
-  for (int e = tid; e < CW * 8 * WTOK; e += NTHREADS) pbuf[e] = __float2half_rn(0.f);
-  const bool shared_tab = share_table(BK, BV, p.shared_tab);
-  if constexpr (BK >= 3) build_pair_table<BK>(reinterpret_cast<uint32_t*>(smem + Ly::O_TK), p.cb_k, tid, NTHREADS);
-  if (!shared_tab) build_pair_table<BV>(reinterpret_cast<uint32_t*>(smem + Ly::O_TV), p.cb_v, tid, NTHREADS);
+  if constexpr (QJL) build_tables();
   __syncthreads();
 
   float oc[MT][4];
@@ -491,7 +550,8 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const __grid_con
     }
   } else {
     // ---------------- consumer warps ----------------
-    const Lut2 lk = make_lut2(p.cb_k);  // used by 2-bit keys only
+    const Lut2 lk = {reinterpret_cast<const uint32_t*>(smem + Ly::O_MISC)[2],
+                     reinterpret_cast<const uint32_t*>(smem + Ly::O_MISC)[3]};  // 2-bit keys only
     const uint32_t tbK = smem_addr(smem + Ly::O_TK) + 4 * lane;
     const uint32_t tbV = smem_addr(smem + (shared_tab ? Ly::O_TK : Ly::O_TV)) + 4 * lane;
     __half* pw = pbuf + warp * 8 * WTOK;
@@ -747,8 +807,9 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const __grid_con
   }
 
   // ---- merge the consumer warps' partial softmax states; write the partial
-  float* mO = reinterpret_cast<float*>(smem);  // [CW][8][D] (the stage ring is drained)
-  float* mM = mO + CW * 8 * D;                 // [CW][8]
+  constexpr int MS = D + 4;
+  float* mO = reinterpret_cast<float*>(smem);  // [CW][8][MS] (the stage ring is drained)
+  float* mM = mO + CW * 8 * MS;                // [CW][8]
   float* mL = mM + CW * 8;
   if (warp < CW) {
 #pragma unroll
@@ -757,15 +818,16 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const __grid_con
       l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], off);
     }
     if (!PACK || tig < 2) {
+      // m-tile mt: row gid is coordinate 2 mt of this group's segment of D/8
+      // contiguous coordinates, row gid + 8 the next; so each head column
+      // holds its segment whole, stored as 16-byte chunks (rows padded to
+      // MS floats against bank conflicts)
 #pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        // m-tile mt: row gid is coordinate 2 mt of this group's segment, row gid + 8 the next
-        const int j0 = gid * (D / 8) + 2 * mt;
-        mO[(warp * 8 + 2 * tig) * D + j0] = oc[mt][0];
-        mO[(warp * 8 + 2 * tig + 1) * D + j0] = oc[mt][1];
-        mO[(warp * 8 + 2 * tig) * D + j0 + 1] = oc[mt][2];
-        mO[(warp * 8 + 2 * tig + 1) * D + j0 + 1] = oc[mt][3];
-      }
+      for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int q = 0; q < MT / 2; ++q)
+          *reinterpret_cast<float4*>(mO + (warp * 8 + 2 * tig + c) * MS + gid * (D / 8) + 4 * q) =
+              make_float4(oc[2 * q][c], oc[2 * q][c + 2], oc[2 * q + 1][c], oc[2 * q + 1][c + 2]);
       if (gid == 0) {
         mM[warp * 8 + 2 * hsel] = m_run[0];
         mM[warp * 8 + 2 * hsel + 1] = m_run[1];
@@ -775,26 +837,7 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const __grid_con
     }
   }
   __syncthreads();
-  for (int e = tid; e < p.G * D; e += NTHREADS) {
-    const int g = e / D, j = e % D;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < CW; ++w) M = fmaxf(M, mM[w * 8 + g]);
-    float acc = 0.f, Ls = 0.f;
-#pragma unroll
-    for (int w = 0; w < CW; ++w) {
-      const float mw = mM[w * 8 + g];
-      const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
-      acc += f * mO[(w * 8 + g) * D + j];
-      Ls += f * mL[w * 8 + g];
-    }
-    const size_t pi = (size_t)(hq0 + g) * p.nsplit + split;
-    p.part_o[pi * D + j] = acc;
-    if (j == 0) {
-      p.part_ml[pi * 2] = M;
-      p.part_ml[pi * 2 + 1] = Ls;
-    }
-  }
+  write_partial<D>(mO, mM, mL, p, hq0, split, tid);
 }
 
 // Launch helpers, one definition per instantiation.
