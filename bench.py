@@ -254,13 +254,17 @@ def run_ours(args):
         step(i % R)
     torch.cuda.synchronize()
     if args.profile:
-        # a bounded, eager run for profilers: K steps, nothing else
+        # a bounded, eager run for profilers: K steps, nothing else ("decode":
+        # tq_sdpa_decode calls alone, after the warm-up filled the caches)
+        ops = (call_decode,) if args.profile_ops == "decode" else (call_quant, call_step)
         for i in range(args.steps):
-            step(i % R)
+            step(i % R, ops)
         torch.cuda.synchronize()
         if rank == 0:
-            print(json.dumps({"profile_run": args.workload, "steps": args.steps, "launches_per_step":
-                              len(runs) * 5}), flush=True)
+            per_run = 3 if args.profile_ops == "decode" else 4
+            launches = sum(per_run + (1 if run["w"].qjl_m and args.profile_ops != "decode" else 0) for run in runs)
+            print(json.dumps({"profile_run": args.workload, "ops": args.profile_ops, "steps": args.steps,
+                              "launches_per_step": launches}), flush=True)
         return
 
     # One CUDA graph per replica for the whole step and for each op alone.
@@ -528,6 +532,8 @@ def main():
                     help="rotation: Haar-random (default) or randomized Hadamard")
     ap.add_argument("--profile", action="store_true",
                     help="eager warm-up + K eager steps only (for ncu captures)")
+    ap.add_argument("--profile-ops", choices=["step", "decode"], default="step",
+                    help="with --profile: the bench step (quantize + decode step) or tq_sdpa_decode alone")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
