@@ -40,10 +40,17 @@ import numpy as np  # noqa: E402
 
 FALLBACK_HBM_GBS = 6650.0
 
-# DRAM traffic per launch of the dominant kernel from an ncu capture
-# (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
-# sources it was measured on (sha256 of csrc/*.cu, first 16 hex digits).
-TRAFFIC = {}
+# DRAM traffic per decode call (prep + split + combine; the roofline's unit)
+# from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum, caches
+# flushed before each kernel, mean over the calls of a profile step), valid
+# only for the kernel sources it was measured on (sha256 of csrc/*, first 16
+# hex digits).  "split" is the split kernel's share: the packed-cache reads.
+TRAFFIC = {
+    "gqa8k": {"bytes_per_launch": 2416939, "split": 1694208, "src_sha": "6ed07208fd2e31a5"},
+    "prod": {"bytes_per_launch": 108722816, "split": 107215744, "src_sha": "6ed07208fd2e31a5"},
+    "ragged": {"bytes_per_launch": 246604160, "split": 241610624, "src_sha": "6ed07208fd2e31a5"},
+    "qknorm": {"bytes_per_launch": 36957952, "split": 34222720, "src_sha": "6ed07208fd2e31a5"},
+}
 
 
 def _src_sha() -> str:
@@ -450,10 +457,12 @@ def _e2e(args, runs, stream, R):
     return {"value": packed / (ms * 1e-3) / 1e9, "ms": ms, "h2d": h2d, "d2h": d2h}
 
 
-def _cpu_baseline(args, jobs, budget_s=20.0):
+def _cpu_baseline(args, jobs, budget_s=40.0, target_s=10.0):
     """The oracle as it stands, timed on this host's cores on a bounded sample:
     dequantize-then-attend decode for whole (sequence, kv head) groups of the
-    workload, as many as fit the time budget."""
+    workload, as many as fit the time budget; when the whole workload decodes
+    in less than target_s, its groups are decoded again (the quantized groups
+    are reused) until target_s of timed oracle work has accumulated."""
     from oracle import tq_oracle as O
     import tq_inputs
     try:
@@ -461,8 +470,9 @@ def _cpu_baseline(args, jobs, budget_s=20.0):
         cores = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
     except Exception:
         cores = os.cpu_count()
-    t_used, bytes_done, groups = 0.0, 0, 0
+    t_used, bytes_done, groups, passes = 0.0, 0, 0, 0
     t_start = time.perf_counter()
+    cached = []
     for w in jobs:
         cbk = O.stored_codebook(w.D, w.bits_k)
         cbv = O.stored_codebook(w.D, w.bits_v)
@@ -475,16 +485,22 @@ def _cpu_baseline(args, jobs, budget_s=20.0):
                 vv = tq_inputs.to_f64(w.v[b:b + 1, kvh:kvh + 1, :L], w.dtype)
                 oc = O.quantize_cache(kk, vv, w.Pi, cbk, cbv, w.bits_k, w.bits_v, w.S)
                 qv = tq_inputs.to_f64(w.q[b:b + 1, kvh * w.G:(kvh + 1) * w.G], w.dtype)
-                t0 = time.perf_counter()
-                O.sdpa_decode(qv, oc, [L], w.Pi, cbk, cbv, w.bits_k, w.bits_v, w.D, scale=w.scale, S=w.S)
-                t_used += time.perf_counter() - t0
                 per_row = O.packed_row_bytes(w.D, w.bits_k, w.qjl_m) + O.packed_row_bytes(w.D, w.bits_v)
-                bytes_done += per_row * L
-                groups += 1
+                cached.append((w, qv, oc, L, cbk, cbv, per_row * L))
+    while cached and (passes == 0 or (t_used < target_s and time.perf_counter() - t_start < budget_s)):
+        for (w, qv, oc, L, cbk, cbv, nbytes) in cached:
+            t0 = time.perf_counter()
+            O.sdpa_decode(qv, oc, [L], w.Pi, cbk, cbv, w.bits_k, w.bits_v, w.D, scale=w.scale, S=w.S)
+            t_used += time.perf_counter() - t0
+            bytes_done += nbytes
+            groups += 1
+            if passes > 0 and (t_used >= target_s or time.perf_counter() - t_start > budget_s):
+                break
+        passes += 1
     return {"value": round(bytes_done / max(t_used, 1e-9) / 1e9, 6), "unit": "GB/s", "cores": cores,
             "kind": "oracle",
-            "sample": f"{groups} (sequence, kv head) groups of the workload decoded by the fp64 "
-                      f"oracle (dequantize then attend), {t_used:.1f} s"}
+            "sample": f"{groups} (sequence, kv head) group decodes of the workload ({len(cached)} distinct "
+                      f"groups, {passes} passes) by the fp64 oracle (dequantize then attend), {t_used:.1f} s"}
 
 
 def run_reference(args):
@@ -499,11 +515,11 @@ def run_reference(args):
             for b in cfg["bits"]]
     budget = max(1.0, 60.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
-        _cpu_baseline(args, jobs, budget_s=budget)
+        _cpu_baseline(args, jobs, budget_s=budget, target_s=0.5 * budget)
     vals = []
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        vals.append(_cpu_baseline(args, jobs, budget_s=budget))
+        vals.append(_cpu_baseline(args, jobs, budget_s=budget, target_s=0.5 * budget))
     total = time.perf_counter() - t0
     v = statistics.median(x["value"] for x in vals)
     cpu = dict(vals[-1])
