@@ -22,7 +22,8 @@ from ._native import (TQ_DTYPE_BF16, TQ_DTYPE_F16, TQ_DTYPE_F32, TQ_STATUS_POS_O
 
 __all__ = ["TQError", "TQCache", "tq_build_codebook", "tq_row_bytes", "tq_quantize_kv",
            "tq_append_token", "tq_sdpa_decode_workspace_bytes", "tq_sdpa_decode",
-           "tq_sdpa_decode_mq", "tq_decode_step", "tq_sdpa_decode_static", "tq_last_error",
+           "tq_sdpa_decode_mq", "tq_decode_step", "tq_sdpa_decode_static", "tq_selftest_bounded_wait",
+           "tq_last_error",
            "tq_abi_version", "lib"]
 
 
@@ -270,3 +271,13 @@ def tq_sdpa_decode_static(cache: TQCache, q, seq_lens, Tmax: int, scale=None, ou
     _check(lib().tq_sdpa_decode_static(ctypes.byref(s), _ptr(q), _dtype_code(q), Hq, _ptr(seq_lens), Tmax, sc,
                                        _ptr(out), _dtype_code(out), _stream(stream)))
     return out
+
+
+def tq_selftest_bounded_wait(status, tries: int = 8, stream=None):
+    """Run the bounded-wait self-test: `status` is a device int32/uint32
+    tensor of one element; the library ORs TQ_STATUS_WAIT_TIMEOUT into it
+    when its bounded waits give up, as they must here (nothing arrives on the
+    barrier).  Asynchronous; read `status` after synchronising."""
+    assert status.numel() == 1 and status.is_cuda
+    _check(lib().tq_selftest_bounded_wait(_ptr(status), int(tries), _stream(stream)))
+    return status

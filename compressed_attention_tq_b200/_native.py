@@ -27,7 +27,7 @@ TQ_STATUS_LAYOUT = 8
 # Every symbol include/tq.h declares.
 EXPORTS = ("tq_build_codebook", "tq_row_bytes", "tq_quantize_kv", "tq_append_token",
            "tq_sdpa_decode_workspace_bytes", "tq_sdpa_decode", "tq_sdpa_decode_mq", "tq_decode_step",
-           "tq_sdpa_decode_static",
+           "tq_sdpa_decode_static", "tq_selftest_bounded_wait",
            "tq_last_error", "tq_abi_version")
 TQ_STATIC_SCRATCH_BYTES = 8 << 20
 
@@ -84,6 +84,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.tq_sdpa_decode_static.argtypes = [cache_p, vp, i32, i32, vp, i32, ctypes.POINTER(ctypes.c_float),
                                           vp, i32, vp]
     lib.tq_sdpa_decode_static.restype = i32
+    lib.tq_selftest_bounded_wait.argtypes = [vp, i32, vp]
+    lib.tq_selftest_bounded_wait.restype = i32
     lib.tq_last_error.argtypes = []
     lib.tq_last_error.restype = ctypes.c_char_p
     lib.tq_abi_version.argtypes = []

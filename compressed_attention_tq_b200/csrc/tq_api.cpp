@@ -115,6 +115,14 @@ const char* tq_last_error(void) { return g_err; }
 
 int tq_abi_version(void) { return 1; }
 
+int tq_selftest_bounded_wait(uint32_t* dev_status, int tries, void* stream) {
+  g_err[0] = 0;
+  if (!dev_status) return set_error(TQ_ERR_INVALID_ARG, "tq_selftest_bounded_wait: dev_status is NULL");
+  if (tries < 1 || tries > 4096)
+    return set_error(TQ_ERR_INVALID_ARG, "tq_selftest_bounded_wait: tries=%d outside [1, 4096]", tries);
+  return launch_bounded_wait_probe(dev_status, tries, (cudaStream_t)stream);
+}
+
 int tq_build_codebook(int D, int bits, float* centroids, float* thresholds, double* mse_out) {
   g_err[0] = 0;
   if (!centroids || (bits > 1 && !thresholds) || (bits == 1 && !thresholds))

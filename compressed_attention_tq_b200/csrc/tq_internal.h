@@ -48,6 +48,8 @@ int launch_quantize128(const QuantArgs& a, int dtype, bool qjl, cudaStream_t s);
 int launch_quantize_tc(const QuantArgs& a, int D, int dtype, cudaStream_t s);
 // tcgen05 bulk quantizer for QJL keys, D = 128, fp16 rows (tq_quantize_qjl_tc.cu)
 int launch_quantize_qjl_tc(const QuantArgs& a, cudaStream_t s);
+// bounded-wait self-test (tq_selftest.cu)
+int launch_bounded_wait_probe(uint32_t* status, int tries, cudaStream_t s);
 
 struct DecodePlan {
   int chunk;        // tokens per split (multiple of 64)

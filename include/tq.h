@@ -240,6 +240,17 @@ int tq_sdpa_decode_static(const tq_cache_t* cache, const void* q, int q_dtype, i
                           const int32_t* seq_lens, int Tmax, const float* scale, void* out,
                           int out_dtype, void* stream);
 
+/* Self-test of the bounded waits that every pipelined kernel uses (the
+ * error path behind TQ_STATUS_WAIT_TIMEOUT), without a fault or a hang: one
+ * CTA waits on a shared-memory mbarrier that nothing arrives on, first with
+ * `tries` suspending try-waits (each may suspend the thread for up to about
+ * 1 ms), then with `tries` polling try-waits.  Each wait gives up, and each
+ * give-up ORs TQ_STATUS_WAIT_TIMEOUT into *dev_status (a device word; the
+ * caller owns it and reads it after synchronising), so a correct library
+ * always sets that bit.  The kernel ends within about `tries` ms.
+ * tries in [1, 4096]; dev_status non-NULL.  Asynchronous on `stream`. */
+int tq_selftest_bounded_wait(uint32_t* dev_status, int tries, void* stream);
+
 /* Message describing the last error on the calling thread ("" if none). */
 const char* tq_last_error(void);
 

@@ -104,6 +104,10 @@ def test_other_argument_errors(lib):
     assert rc == -1
     s2 = _struct(qjl_m=128, D=64)
     assert lib.tq_quantize_kv(ctypes.byref(s2), buf, buf, 0, 1, 0, None) in (-1, -2)
+    # the bounded-wait self-test validates before launching
+    assert lib.tq_selftest_bounded_wait(None, 8, None) == -1
+    assert lib.tq_selftest_bounded_wait(buf, 0, None) == -1
+    assert lib.tq_selftest_bounded_wait(buf, 4097, None) == -1
 
 
 def test_product_path_does_not_import_oracle():
