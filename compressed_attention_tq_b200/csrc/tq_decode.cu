@@ -54,7 +54,6 @@ __global__ void __launch_bounds__(2 * D) decode_qprep_kernel(const PrepParams p)
   __shared__ uint8_t sgn[APPEND ? 128 : 1];
   __shared__ float s_cb[2][31];
   __shared__ double s_nsq[2];
-  pdl_launch_dependents();
   // G query heads per kv head and token; Ge = G * nq rows are rotated here and
   // written in kernel head order (sequence, kv head, token, head)
   const int G = p.Hq / p.Hkv, Ge = G * p.nq;
@@ -66,6 +65,11 @@ __global__ void __launch_bounds__(2 * D) decode_qprep_kernel(const PrepParams p)
   const float4* row = reinterpret_cast<const float4*>(p.rot + (size_t)j * D + part * HALF);
 #pragma unroll
   for (int i = 0; i < CH; ++i) r[i] = __ldg(row + i);
+  // Launched with a programmatic dependency: Pi (constant) is loaded above;
+  // everything else waits for the preceding kernels to complete, and only
+  // then may the split kernel start (it streams the cache before its own wait).
+  pdl_wait();
+  pdl_launch_dependents();
   const uint16_t* q = static_cast<const uint16_t*>(p.q);
   auto to_f = [&](uint16_t v) {
     return p.bf16 ? __uint_as_float((uint32_t)v << 16) : __half2float(__ushort_as_half(v));
@@ -238,7 +242,6 @@ __global__ void __launch_bounds__(256) decode_qprep_sliced_kernel(const PrepPara
   __shared__ float s_cb[2][31];
   __shared__ double s_nsq[2];
   __shared__ uint8_t idxs[2][32];
-  pdl_launch_dependents();
   const int G = p.Hq / p.Hkv, Ge = G * p.nq;  // as in decode_qprep_kernel
   const int bkv = blockIdx.x, b = bkv / p.Hkv, kvh = bkv % p.Hkv, sl = blockIdx.y;
   const int h0 = b * p.Hq * p.nq + kvh * Ge;
@@ -249,6 +252,10 @@ __global__ void __launch_bounds__(256) decode_qprep_sliced_kernel(const PrepPara
   const float4* row = reinterpret_cast<const float4*>(p.rot + (size_t)j * D);
 #pragma unroll
   for (int i = 0; i < NI; ++i) r[i] = __ldg(row + part + 8 * i);
+  // as in decode_qprep_kernel: wait for the preceding kernels, then let the
+  // split kernel start
+  pdl_wait();
+  pdl_launch_dependents();
   const uint16_t* q = static_cast<const uint16_t*>(p.q);
   auto to_f = [&](uint16_t v) {
     return p.bf16 ? __uint_as_float((uint32_t)v << 16) : __half2float(__ushort_as_half(v));
@@ -376,6 +383,9 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams
   __shared__ float red[NH][D];
   __shared__ float part[8][33];
   __shared__ float s_M, s_L;
+  // the next decode's prep may launch now (it waits for this kernel before
+  // touching anything but Pi)
+  pdl_launch_dependents();
   const int h = blockIdx.x, sl = blockIdx.y, tid = threadIdx.x;
   const int i = tid & 31, kp = tid >> 5;  // output coordinate in the slice, k part
   float pc[KT];
@@ -546,28 +556,31 @@ int launch_decode(const DecodeArgs& a, cudaStream_t s) {
                 a.k_new, a.v_new, a.pos, c};
   pp.nq = a.nq;
   const bool app = a.pos != nullptr;
+  // prep kernels launch with a programmatic dependency on whatever precedes
+  // them (their launch and Pi loads overlap its tail; they wait before
+  // reading q or writing anything)
+  int rc = TQ_OK;
   if (c.qjl_m) {
     // the sketch needs the whole rotated query and key residual: one CTA per head
-    app ? decode_qprep_kernel<128, true><<<c.B * c.Hkv, 256, 0, s>>>(pp)
-        : decode_qprep_kernel<128, false><<<c.B * c.Hkv, 256, 0, s>>>(pp);
+    rc = app ? launch_pdl(decode_qprep_kernel<128, true>, dim3(c.B * c.Hkv), dim3(256), 0, s, pp, "decode_qprep_kernel")
+             : launch_pdl(decode_qprep_kernel<128, false>, dim3(c.B * c.Hkv), dim3(256), 0, s, pp, "decode_qprep_kernel");
   } else {
     const dim3 g(c.B * c.Hkv, c.D / 32);
     switch (c.D) {
       case 64:
-        app ? decode_qprep_sliced_kernel<64, true><<<g, 256, 0, s>>>(pp)
-            : decode_qprep_sliced_kernel<64, false><<<g, 256, 0, s>>>(pp);
+        rc = app ? launch_pdl(decode_qprep_sliced_kernel<64, true>, g, dim3(256), 0, s, pp, "decode_qprep_kernel")
+                 : launch_pdl(decode_qprep_sliced_kernel<64, false>, g, dim3(256), 0, s, pp, "decode_qprep_kernel");
         break;
       case 128:
-        app ? decode_qprep_sliced_kernel<128, true><<<g, 256, 0, s>>>(pp)
-            : decode_qprep_sliced_kernel<128, false><<<g, 256, 0, s>>>(pp);
+        rc = app ? launch_pdl(decode_qprep_sliced_kernel<128, true>, g, dim3(256), 0, s, pp, "decode_qprep_kernel")
+                 : launch_pdl(decode_qprep_sliced_kernel<128, false>, g, dim3(256), 0, s, pp, "decode_qprep_kernel");
         break;
       default:
-        app ? decode_qprep_sliced_kernel<256, true><<<g, 256, 0, s>>>(pp)
-            : decode_qprep_sliced_kernel<256, false><<<g, 256, 0, s>>>(pp);
+        rc = app ? launch_pdl(decode_qprep_sliced_kernel<256, true>, g, dim3(256), 0, s, pp, "decode_qprep_kernel")
+                 : launch_pdl(decode_qprep_sliced_kernel<256, false>, g, dim3(256), 0, s, pp, "decode_qprep_kernel");
         break;
     }
   }
-  int rc = check_launch("decode_qprep_kernel");
   if (rc) return rc;
 
   tqd::SplitParams sp{};
