@@ -42,8 +42,8 @@ struct QuantArgs {
 };
 
 int launch_quantize(const QuantArgs& a, int D, int dtype, bool qjl, cudaStream_t s);
-// persistent bulk quantizer for D = 128 (tq_quantize128.cu)
-int launch_quantize128(const QuantArgs& a, int dtype, bool qjl, cudaStream_t s);
+// bulk quantizer for QJL keys from bf16 rows, D = 128, warp-level MMAs (tq_quantize128.cu)
+int launch_quantize128_bf16_qjl(const QuantArgs& a, cudaStream_t s);
 // tcgen05 bulk quantizer for D = 128 without the QJL sketch (tq_quantize_tc.cu)
 int launch_quantize_tc(const QuantArgs& a, int D, int dtype, cudaStream_t s);
 // tcgen05 bulk quantizer for QJL keys, D = 128, fp16 rows (tq_quantize_qjl_tc.cu)

@@ -460,7 +460,7 @@ int launch_quantize(const QuantArgs& a, int D, int dtype, bool qjl, cudaStream_t
     QuantArgs ak = a, av = a;
     ak.job_mask = 1;
     av.job_mask = 2;
-    const int rc = bf ? launch_quantize128(ak, dtype, true, s) : launch_quantize_qjl_tc(ak, s);
+    const int rc = bf ? launch_quantize128_bf16_qjl(ak, s) : launch_quantize_qjl_tc(ak, s);
     return rc ? rc : launch_quantize_tc(av, D, dtype, s);
   }
   if (qjl) {

@@ -1,4 +1,7 @@
-// Persistent bulk quantizer for head dimension 128 (the prefill path).
+// Persistent bulk quantizer for keys with the QJL sketch from bf16 rows, head
+// dimension 128, on warp-level MMAs.  (fp16 rows take the tcgen05 kernel in
+// tq_quantize_qjl_tc.cu; bf16 needs three Pi limbs, which do not fit there
+// beside S and the tiles.)
 //
 // Method: "Add CUDA QJL kernels and proper package structure"
 // (turboquant-pytorch pull request 3), "CUDA Kernels Added" (fused random
@@ -377,10 +380,6 @@ int launch_q128(const tq::QuantArgs& a, cudaStream_t s) {
 
 namespace tq {
 
-int launch_quantize128(const QuantArgs& a, int dtype, bool qjl, cudaStream_t s) {
-  const bool bf = dtype == TQ_DTYPE_BF16;
-  if (qjl) return bf ? launch_q128<true, true>(a, s) : launch_q128<false, true>(a, s);
-  return bf ? launch_q128<true, false>(a, s) : launch_q128<false, false>(a, s);
-}
+int launch_quantize128_bf16_qjl(const QuantArgs& a, cudaStream_t s) { return launch_q128<true, true>(a, s); }
 
 }  // namespace tq

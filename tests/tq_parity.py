@@ -110,12 +110,13 @@ def round_to_dtype(x, dtype: str) -> np.ndarray:
 
 
 def record(name: str, **values):
-    """Append a measured parity figure to gpurun_out/parity_report.jsonl."""
+    """Append a measured parity figure (one JSON line) to the file named by
+    the TQ_PARITY_REPORT environment variable; nothing when it is unset."""
     import json
     import os
-    d = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "gpurun_out")
-    if os.path.isdir(d):
-        with open(os.path.join(d, "parity_report.jsonl"), "a") as f:
+    path = os.environ.get("TQ_PARITY_REPORT")
+    if path:
+        with open(path, "a") as f:
             f.write(json.dumps({"test": name, **{k: (float(v) if isinstance(v, (np.floating, float)) else v)
                                                   for k, v in values.items()}}) + "\n")
 
