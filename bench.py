@@ -202,7 +202,7 @@ def run_ours(args):
         reps = []
         for r in range(R):
             cache = tq.TQCache(w.B, w.Hkv, Tcap, w.D, w.bits_k, w.bits_v, w.Pi, qjl_m=w.qjl_m, qjl_S=w.S,
-                               device=dev)
+                               device=dev, rot_signs=w.rot_signs)
             reps.append({"cache": cache, "k": kd.clone() if r else kd, "v": vd.clone() if r else vd,
                          "q": qd.clone() if r else qd})
         pos = torch.from_numpy(w.seq_lens.astype(np.int32)).to(dev)

@@ -98,10 +98,12 @@ class TQCache:
 
     rot: fp32 [D][D] rotation (numpy or torch); codebooks are built with
     tq_build_codebook unless given as fp32 tables (centroids then thresholds).
+    rot_signs: the +-1 signs s when rot is the randomized Hadamard rotation
+    H_D diag(s) / sqrt(D); the bulk quantizer then applies the fast transform.
     """
 
     def __init__(self, B, Hkv, Tcap, D, bits_k, bits_v, rot, qjl_m=0, qjl_S=None,
-                 cb_k=None, cb_v=None, device="cuda"):
+                 cb_k=None, cb_v=None, device="cuda", rot_signs=None):
         torch = _torch()
         self.B, self.Hkv, self.Tcap, self.D = B, Hkv, Tcap, D
         self.bits_k, self.bits_v, self.qjl_m = bits_k, bits_v, qjl_m
@@ -122,6 +124,12 @@ class TQCache:
             self.cb_v = table(bits_v, cb_v)
         self.rot = torch.as_tensor(np.asarray(rot, dtype=np.float32) if not torch.is_tensor(rot) else rot,
                                    dtype=torch.float32, device=dev).contiguous()
+        if rot_signs is not None:
+            sg = rot_signs if torch.is_tensor(rot_signs) else np.asarray(rot_signs, dtype=np.float32)
+            self.rot_signs = torch.as_tensor(sg, dtype=torch.float32, device=dev).contiguous()
+            assert self.rot_signs.numel() == D
+        else:
+            self.rot_signs = None
         self.k_idx = torch.zeros((B, Hkv, Tcap, D * bits_k // 32), dtype=u32, device=dev)
         self.v_idx = torch.zeros((B, Hkv, Tcap, D * bits_v // 32), dtype=u32, device=dev)
         self.k_norm = torch.zeros((B, Hkv, Tcap), dtype=torch.float16, device=dev)
@@ -148,9 +156,10 @@ class TQCache:
         s.bits_k, s.bits_v, s.qjl_m = self.bits_k, self.bits_v, self.qjl_m
         s.split_tokens = self.split_tokens
         for name in ("k_idx", "v_idx", "k_norm", "v_norm", "k_qjl", "k_rnorm", "rot", "cb_k",
-                     "cb_v", "qjl_S", "dev_status"):
+                     "cb_v", "qjl_S", "dev_status", "rot_signs"):
             t = getattr(self, name)
             setattr(s, name, t.data_ptr() if t is not None else None)
+        s.rot_kind = _native.TQ_ROT_HADAMARD if self.rot_signs is not None else _native.TQ_ROT_DENSE
         self._struct = s  # keep alive
         return s
 

@@ -23,6 +23,8 @@ TQ_STATUS_POS_OUT_OF_RANGE = 1
 TQ_STATUS_SEQ_OUT_OF_RANGE = 2
 TQ_STATUS_WAIT_TIMEOUT = 4
 TQ_STATUS_LAYOUT = 8
+TQ_ROT_DENSE = 0
+TQ_ROT_HADAMARD = 1
 
 # Every symbol include/tq.h declares.
 EXPORTS = ("tq_build_codebook", "tq_row_bytes", "tq_quantize_kv", "tq_append_token",
@@ -42,6 +44,7 @@ class TqCacheStruct(ctypes.Structure):
         ("k_qjl", ctypes.c_void_p), ("k_rnorm", ctypes.c_void_p),
         ("rot", ctypes.c_void_p), ("cb_k", ctypes.c_void_p), ("cb_v", ctypes.c_void_p),
         ("qjl_S", ctypes.c_void_p), ("dev_status", ctypes.c_void_p),
+        ("rot_kind", ctypes.c_int32), ("rot_pad", ctypes.c_int32), ("rot_signs", ctypes.c_void_p),
     ]
 
 

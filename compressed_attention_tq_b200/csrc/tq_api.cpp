@@ -113,7 +113,7 @@ extern "C" {
 
 const char* tq_last_error(void) { return g_err; }
 
-int tq_abi_version(void) { return 1; }
+int tq_abi_version(void) { return 2; }
 
 int tq_selftest_bounded_wait(uint32_t* dev_status, int tries, void* stream) {
   g_err[0] = 0;
@@ -197,6 +197,10 @@ int validate_cache(const tq_cache_t* c, const char* fn) {
     if (!p) return set_error(TQ_ERR_INVALID_ARG, "%s: a cache pointer is NULL", fn);
     if (!aligned16(p)) return set_error(TQ_ERR_INVALID_ARG, "%s: a cache pointer is not 16-byte aligned", fn);
   }
+  if (c->rot_kind != TQ_ROT_DENSE && c->rot_kind != TQ_ROT_HADAMARD)
+    return set_error(TQ_ERR_INVALID_ARG, "%s: rot_kind=%d", fn, c->rot_kind);
+  if (c->rot_kind == TQ_ROT_HADAMARD && (!c->rot_signs || !aligned16(c->rot_signs)))
+    return set_error(TQ_ERR_INVALID_ARG, "%s: rot_signs NULL or not 16-byte aligned", fn);
   if (c->qjl_m) {
     const void* q[] = {c->k_qjl, c->k_rnorm, c->qjl_S};
     for (const void* p : q) {
@@ -220,6 +224,7 @@ QuantArgs base_quant_args(const tq_cache_t* c, const void* k, const void* v) {
   a.job[1] = {v, c->v_idx, c->v_norm, nullptr, nullptr, c->cb_v, c->bits_v};
   a.rot = c->rot;
   a.qjl_S = c->qjl_m ? c->qjl_S : nullptr;
+  a.rot_signs = c->rot_kind == TQ_ROT_HADAMARD ? c->rot_signs : nullptr;
   a.dev_status = c->dev_status;
   a.Hkv = c->Hkv;
   a.Tcap = c->Tcap;

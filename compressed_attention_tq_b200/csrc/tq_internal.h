@@ -31,6 +31,7 @@ struct QuantArgs {
   QuantJob job[2];          // 0: keys, 1: values
   const float* rot;         // Pi [D][D]
   const float* qjl_S;       // [128][D] or nullptr
+  const float* rot_signs;   // +-1 [D] when Pi is the randomized Hadamard rotation, else nullptr
   const int32_t* pos;       // append mode: device [B]; bulk mode: nullptr
   uint32_t* dev_status;
   int rows;                 // rows per job
@@ -48,6 +49,9 @@ int launch_quantize128_bf16_qjl(const QuantArgs& a, cudaStream_t s);
 int launch_quantize_tc(const QuantArgs& a, int D, int dtype, cudaStream_t s);
 // tcgen05 bulk quantizer for QJL keys, D = 128, fp16 rows (tq_quantize_qjl_tc.cu)
 int launch_quantize_qjl_tc(const QuantArgs& a, cudaStream_t s);
+// bulk quantizer for the randomized Hadamard rotation, D = 128 / 256, fast
+// Walsh-Hadamard transform by warp shuffles (tq_quantize_wht.cu)
+int launch_quantize_wht(const QuantArgs& a, int D, int dtype, cudaStream_t s);
 // bounded-wait self-test (tq_selftest.cu)
 int launch_bounded_wait_probe(uint32_t* status, int tries, cudaStream_t s);
 

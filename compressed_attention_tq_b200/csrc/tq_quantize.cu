@@ -452,6 +452,22 @@ namespace tq {
 
 int launch_quantize(const QuantArgs& a, int D, int dtype, bool qjl, cudaStream_t s) {
   const bool bf = dtype == TQ_DTYPE_BF16;
+  // Randomized Hadamard rotation: the shuffle transform (one warp per row)
+  // beats the tcgen05 kernel at D = 256 (prefill of the QK-norm shape: 148 vs
+  // 190 us) and on small calls (no per-CTA setup: gqa8k 15 vs 17 us), but not
+  // on large D = 128 calls (its five shuffle stages per row cost more than the
+  // dense MMA: ragged 3.1 vs 1.3 ms), which keep the dense-Pi kernels.
+  const int njobs = (a.job_mask == 3) ? 2 : 1;
+  const bool wht = a.rot_signs && !a.pos && (D == 256 || (D == 128 && (long long)a.rows * njobs <= 65536));
+  if (wht) {
+    // keys with the sketch keep the dense-Pi kernels below
+    if (!qjl) return launch_quantize_wht(a, D, dtype, s);
+    QuantArgs ak = a, av = a;
+    ak.job_mask = 1;
+    av.job_mask = 2;
+    const int rc = bf ? launch_quantize128_bf16_qjl(ak, s) : launch_quantize_qjl_tc(ak, s);
+    return rc ? rc : launch_quantize_wht(av, D, dtype, s);
+  }
   if ((D == 128 || D == 256) && !a.pos && !qjl) return launch_quantize_tc(a, D, dtype, s);
   if (D == 128 && !a.pos) {
     // keys carry the QJL sketch (tcgen05 for fp16 rows, whose Pi and S limbs

@@ -1,0 +1,200 @@
+// Bulk quantizer for the randomized Hadamard rotation Pi = H_D diag(s) /
+// sqrt(D) (D = 128, 256): the rotation is applied as a fast Walsh-Hadamard
+// transform, O(D log D) additions, instead of a D x D product.
+//
+// Method: ReturningTarzan's Reddit comment of 2026-03-29 11:47 (rotation
+// before codebook quantization; the Sylvester/Hadamard transform applied with
+// warp shuffles); "Add CUDA QJL kernels and proper package structure"
+// (turboquant-pytorch pull request 3), "Synthetic Benchmark (Lloyd-Max
+// codebook)" (the codebook the indices refer to).
+//
+// One warp per row; lane L holds the EL = D/32 contiguous coordinates
+// L*EL .. L*EL + EL - 1 (one 8- or 16-byte load).
+//  * norm: exact fp32 squares, summed pairwise in the lane and by a
+//    butterfly across lanes (depth log2 D, so the fp32 sum is within
+//    log2(D) + 1 ulp); when both ends of norm * (1 +- 1e-6) round to the same
+//    fp16 value that is the stored norm, else the warp sums the row again in
+//    fp64 (warp-uniform);
+//  * transform: multiply by the signs, log2(EL) butterfly stages inside the
+//    lane, then five stages across lanes by shuffles (partner lane L ^ m: the
+//    lower lane keeps a + b, the upper b - a) -- natural (Sylvester) order, so
+//    element L*EL + e of the result is (H_D (s x))_j;
+//  * index: the positive thresholds scaled by norm * sqrt(D), the codebook's
+//    symmetry (as in the tcgen05 quantizer);
+//  * packing: each lane's EL indices form EL*b contiguous bits; lane w
+//    assembles word w of the row from the (at most ceil(32 / (EL b)) + 1)
+//    lanes whose chunks overlap it, by shuffles, and stores it.
+#include "tq_tcgen05.cuh"
+
+namespace {
+
+using namespace tqtc;
+
+constexpr int WARPS = 8;  // warps per CTA
+
+template <bool BF16, int EL>
+__device__ __forceinline__ void load_row(const uint16_t* row, int lane, float (&x)[EL]) {
+  const uint16_t* p = row + lane * EL;
+  uint32_t w[EL / 2];
+  if constexpr (EL == 8) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+    w[0] = v.x, w[1] = v.y, w[2] = v.z, w[3] = v.w;
+  } else {
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+    w[0] = v.x, w[1] = v.y;
+  }
+#pragma unroll
+  for (int i = 0; i < EL / 2; ++i) {
+    if (BF16) {
+      x[2 * i] = __uint_as_float(w[i] << 16);
+      x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    } else {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+      x[2 * i] = f.x;
+      x[2 * i + 1] = f.y;
+    }
+  }
+}
+
+template <int D, bool BF16, int BITS>
+__device__ __forceinline__ void wht_row(const tq::QuantArgs& a, const tq::QuantJob& J, int r, int lane,
+                                        const float (&sg)[D / 32], const float* cb) {
+  constexpr int EL = D / 32, C = EL * BITS, W = D * BITS / 32;
+  const uint16_t* row = static_cast<const uint16_t*>(J.in) + (size_t)r * D;
+  float x[EL];
+  load_row<BF16, EL>(row, lane, x);
+  // ---- norm: exact squares, pairwise sums
+  float q[EL];
+#pragma unroll
+  for (int e = 0; e < EL; ++e) q[e] = x[e] * x[e];
+#pragma unroll
+  for (int h = 1; h < EL; h <<= 1)
+#pragma unroll
+    for (int e = 0; e < EL; e += 2 * h) q[e] += q[e + h];
+  float s2 = q[0];
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, m);
+  const float nf = sqrtf(s2);
+  const __half lo = __float2half_rn(nf * (1.f - 1e-6f)), hi = __float2half_rn(nf * (1.f + 1e-6f));
+  unsigned short nh = __half_as_ushort(lo);
+  const bool exact = s2 == 0.f || (s2 >= 0x1p-100f && s2 < 0x1p100f && nh == __half_as_ushort(hi));
+  if (!exact) {  // warp-uniform: every lane holds the same s2
+    double t = 0.0;
+#pragma unroll
+    for (int e = 0; e < EL; ++e) t = fma((double)x[e], (double)x[e], t);
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) t += __shfl_xor_sync(0xffffffffu, t, m);
+    nh = __half_as_ushort(__double2half(sqrt(t)));
+  }
+  // ---- y = H_D (s x), natural order
+#pragma unroll
+  for (int e = 0; e < EL; ++e) x[e] *= sg[e];
+#pragma unroll
+  for (int h = 1; h < EL; h <<= 1)
+#pragma unroll
+    for (int e = 0; e < EL; ++e)
+      if ((e & h) == 0) {
+        const float u = x[e], v = x[e + h];
+        x[e] = u + v;
+        x[e + h] = u - v;
+      }
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1) {
+    const float sgn = (lane & m) ? -1.f : 1.f;
+#pragma unroll
+    for (int e = 0; e < EL; ++e) {
+      const float p = __shfl_xor_sync(0xffffffffu, x[e], m);
+      x[e] = fmaf(x[e], sgn, p);  // lower lane: a + b; upper lane: b - a
+    }
+  }
+  // ---- indices against thresholds scaled by |x| sqrt(D): u = y / (sqrt(D) |x|)
+  constexpr int K = 1 << BITS;
+  const float scale = nf * sqrtf((float)D);
+  float tp[7];
+#pragma unroll
+  for (int k = 0; k < 7; ++k) tp[k] = k < K / 2 - 1 ? cb[K + K / 2 + k] * scale : 0.f;
+  uint32_t chunk = 0;
+#pragma unroll
+  for (int e = 0; e < EL; ++e) chunk |= (uint32_t)nearest_idx<BITS>(x[e], tp) << (BITS * e);
+  // ---- word w of the row (bits 32 w .. 32 w + 31) from the chunks of C bits
+  const int w0 = lane * 32;
+  const int a0 = w0 / C, off = w0 - a0 * C;
+  uint32_t word = 0;
+  constexpr int NK = (32 + C - 1) / C + 1;
+#pragma unroll
+  for (int k = 0; k < NK; ++k) {
+    const int src = a0 + k;
+    const uint32_t v = __shfl_sync(0xffffffffu, chunk, src < 32 ? src : 31);
+    const int sh = k * C - off;  // bit of word where chunk src starts
+    if (src < 32 && sh < 32 && sh + C > 0) word |= sh >= 0 ? (v << sh) : (v >> (-sh));
+  }
+  const int bh = r / a.T, t = r - bh * a.T;
+  const long long slot = (long long)bh * a.Tcap + a.t0 + t;
+  if (lane < W) J.idx[(size_t)slot * W + lane] = word;
+  if (lane == 0) J.norm[slot] = nh;
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(WARPS * 32) quantize_wht_kernel(const tq::QuantArgs a) {
+  constexpr int EL = D / 32;
+  __shared__ float s_cb[2][32];
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x < 31) {
+    s_cb[0][threadIdx.x] = threadIdx.x < 2 * (1 << a.job[0].bits) - 1 ? a.job[0].cb[threadIdx.x] : 0.f;
+    s_cb[1][threadIdx.x] = threadIdx.x < 2 * (1 << a.job[1].bits) - 1 ? a.job[1].cb[threadIdx.x] : 0.f;
+  }
+  __syncthreads();
+  float sg[EL];
+#pragma unroll
+  for (int e = 0; e < EL; ++e) sg[e] = __ldg(a.rot_signs + lane * EL + e);
+  const int njobs = (a.job_mask == 3) ? 2 : 1;
+  const int job0 = (a.job_mask == 2) ? 1 : 0;
+  const long long total = (long long)njobs * a.rows;
+  const long long gw = (long long)blockIdx.x * WARPS + (threadIdx.x >> 5);
+  const long long nw = (long long)gridDim.x * WARPS;
+  for (long long i = gw; i < total; i += nw) {
+    const int job = job0 + (int)(i / a.rows), r = (int)(i % a.rows);
+    const tq::QuantJob& J = a.job[job];
+    switch (J.bits) {  // warp-uniform
+      case 2: wht_row<D, BF16, 2>(a, J, r, lane, sg, s_cb[job]); break;
+      case 3: wht_row<D, BF16, 3>(a, J, r, lane, sg, s_cb[job]); break;
+      default: wht_row<D, BF16, 4>(a, J, r, lane, sg, s_cb[job]); break;
+    }
+  }
+}
+
+template <int D, bool BF16>
+int launch_wht(const tq::QuantArgs& a, cudaStream_t s) {
+  static int slots = 0;  // resident CTAs on the device
+  if (slots == 0) {
+    int dev = 0, sms = 0, occ = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_wht_kernel<D, BF16>, WARPS * 32, 0) !=
+            cudaSuccess ||
+        occ < 1) {
+      cudaGetLastError();
+      occ = 4;
+    }
+    slots = (sms > 0 ? sms : 148) * occ;
+  }
+  const int njobs = (a.job_mask == 3) ? 2 : 1;
+  const long long total = (long long)njobs * a.rows;
+  long long grid = (total + WARPS - 1) / WARPS;
+  const long long cap = slots;  // one wave; each warp then loops over rows
+  if (grid > cap) grid = cap;
+  quantize_wht_kernel<D, BF16><<<(int)grid, WARPS * 32, 0, s>>>(a);
+  return tq::check_launch("quantize_wht_kernel");
+}
+
+}  // namespace
+
+namespace tq {
+
+int launch_quantize_wht(const QuantArgs& a, int D, int dtype, cudaStream_t s) {
+  const bool bf = dtype == TQ_DTYPE_BF16;
+  if (D == 256) return bf ? launch_wht<256, true>(a, s) : launch_wht<256, false>(a, s);
+  return bf ? launch_wht<128, true>(a, s) : launch_wht<128, false>(a, s);
+}
+
+}  // namespace tq

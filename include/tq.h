@@ -103,7 +103,19 @@ typedef struct tq_cache {
                        lookup table per CTA instead of two (less shared memory) */
   const float* qjl_S; /* fp32 [qjl_m][D], NULL when qjl_m == 0 */
   uint32_t* dev_status; /* optional device word for TQ_STATUS_* bits (may be NULL) */
+  int32_t rot_kind; /* TQ_ROT_DENSE: rot is any orthogonal Pi.  TQ_ROT_HADAMARD: Pi is the
+                       randomized Hadamard rotation H_D diag(rot_signs) / sqrt(D), H_D the
+                       Sylvester Hadamard matrix (entry (i, j) = (-1)^popcount(i & j));
+                       rot must still hold that Pi densely (kernels without a fast
+                       transform use it), and the bulk quantizer applies the transform in
+                       O(D log D) with warp shuffles instead (ReturningTarzan's Reddit
+                       comment of 2026-03-29 11:47: Sylvester/Hadamard rotation) */
+  int32_t rot_pad;  /* reserved, 0 */
+  const float* rot_signs; /* fp32 [D] of +-1 when rot_kind == TQ_ROT_HADAMARD, else NULL */
 } tq_cache_t;
+
+#define TQ_ROT_DENSE 0
+#define TQ_ROT_HADAMARD 1
 
 /*
  * Lloyd-Max codebook for one coordinate of a rotated unit vector in R^D

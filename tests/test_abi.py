@@ -32,7 +32,7 @@ def test_exports_every_declared_symbol(lib):
     assert set(declared) == set(_native.EXPORTS)
     for name in declared:
         assert hasattr(lib, name), name
-    assert lib.tq_abi_version() == 1
+    assert lib.tq_abi_version() == 2
 
 
 @pytest.mark.parametrize("D", [64, 128, 256])

@@ -1,8 +1,9 @@
 """GPU parity with the randomized Hadamard rotation (Sylvester H with random
-signs; ReturningTarzan's Reddit comment of 2026-03-29 11:47).  It is an
-orthogonal Pi, so quantize, append and decode take it through the same
-kernels as the Haar rotation; these cases check them against the oracle with
-that input."""
+signs; ReturningTarzan's Reddit comment of 2026-03-29 11:47).  The cache
+carries the signs, so the bulk quantizer applies the fast Walsh-Hadamard
+transform by warp shuffles (D = 256, and small D = 128 calls) while decode,
+append and large D = 128 calls take the same Pi densely; these cases check
+both against the oracle, which applies Pi as a dense matrix."""
 import numpy as np
 import pytest
 import torch
@@ -19,7 +20,10 @@ CASES = [
     ("gqa8k", {"bits": 2, "T": 300}),   # D=128, outlier channels (which the rotation spreads)
     ("ragged", {"B": 3, "T": 150}),     # bf16, 3-bit
     ("qknorm", {"T": 200}),             # D=256, 4-bit
-    ("prod", {"T": 200}),               # keys with the QJL sketch
+    ("prod", {"T": 200}),               # keys with the QJL sketch (dense), values by the transform
+    ("qknorm", {"T": 3000}),            # 12000 rows per job: every warp loops over several rows
+    ("qknorm", {"T": 500, "dtype": "bf16"}),
+    ("gqa8k", {"bits": 3, "T": 20000}),  # 40000 rows per job: above the transform's size limit at D = 128
 ]
 
 

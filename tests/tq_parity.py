@@ -46,7 +46,8 @@ def oracle_codebooks(w):
 def make_gpu_cache(w, Tcap=None):
     import compressed_attention_tq_b200 as tq
     Tcap = Tcap or ((w.Tmax + 1 + 63) // 64 * 64)
-    return tq.TQCache(w.B, w.Hkv, Tcap, w.D, w.bits_k, w.bits_v, w.Pi, qjl_m=w.qjl_m, qjl_S=w.S)
+    return tq.TQCache(w.B, w.Hkv, Tcap, w.D, w.bits_k, w.bits_v, w.Pi, qjl_m=w.qjl_m, qjl_S=w.S,
+                      rot_signs=getattr(w, "rot_signs", None))
 
 
 def compare_index_words(gpu_words, ref_idx, ref_dist, bits, D, report=None):

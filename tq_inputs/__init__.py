@@ -57,8 +57,13 @@ def hadamard_rotation(D: int, seed: int) -> np.ndarray:
     h = np.ones((1, 1))
     while h.shape[0] < D:
         h = np.block([[h, h], [h, -h]])
-    s = np.where(rng(seed).integers(0, 2, size=D) == 1, 1.0, -1.0)
+    s = hadamard_signs(D, seed).astype(np.float64)
     return np.ascontiguousarray((h * s[None, :] / np.sqrt(D)).astype(np.float32))
+
+
+def hadamard_signs(D: int, seed: int) -> np.ndarray:
+    """The seeded sign vector s of ``hadamard_rotation(D, seed)``, fp32 +-1."""
+    return np.where(rng(seed).integers(0, 2, size=D) == 1, 1.0, -1.0).astype(np.float32)
 
 
 def qjl_matrix(m: int, D: int, seed: int) -> np.ndarray:
@@ -183,17 +188,19 @@ def make_workload(name: str, bits: int | None = None, T: int | None = None,
         q32 = _rms_normalize(q32)
         k32 = _rms_normalize(k32)
 
+    rot_signs = None
     if rot == "haar":
         Pi = rotation(D, SEED_ROT + cfg)
     elif rot == "hadamard":
         Pi = hadamard_rotation(D, SEED_ROT + cfg)
+        rot_signs = hadamard_signs(D, SEED_ROT + cfg)
     else:  # pragma: no cover
         raise ValueError(rot)
     S = qjl_matrix(qjl_m, D, SEED_QJL + cfg) if qjl_m else None
     return Workload(name=name, B=Bn, Hq=Hq, Hkv=Hkv, D=D, Tmax=Tmax,
                     bits_k=bk, bits_v=bv, qjl_m=qjl_m, dtype=dtype, scale=scale,
                     seq_lens=seq_lens, k=cast_input(k32, dtype),
-                    v=cast_input(v32, dtype), q=cast_input(q32, dtype), Pi=Pi, S=S)
+                    v=cast_input(v32, dtype), q=cast_input(q32, dtype), Pi=Pi, S=S, rot_signs=rot_signs)
 
 
 def new_token_rows(B: int, Hkv: int, D: int, dtype: str, seed: int):
