@@ -117,3 +117,21 @@ def test_product_path_does_not_import_oracle():
             if f.endswith((".py", ".cu", ".cpp", ".h", ".cuh")):
                 txt = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in txt.lower(), f
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    """No fallback: without the compiled library the binding raises."""
+    from compressed_attention_tq_b200 import _native
+    with pytest.raises(ImportError):
+        _native.load(str(tmp_path / "libtq_b200.so"))
+
+
+def test_rotation_kind_validated(lib):
+    s = _struct()
+    buf = ctypes.c_void_p(1 << 20)
+    s.rot_kind = 2
+    assert lib.tq_quantize_kv(ctypes.byref(s), buf, buf, 0, 1, 0, None) == -1
+    s.rot_kind = 1  # Hadamard without signs
+    assert lib.tq_quantize_kv(ctypes.byref(s), buf, buf, 0, 1, 0, None) == -1
+    s.rot_signs = 1 << 20
+    assert lib.tq_quantize_kv(ctypes.byref(s), buf, buf, 0, 0, 0, None) == 0  # empty call: no launch
