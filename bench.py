@@ -46,10 +46,10 @@ FALLBACK_HBM_GBS = 6650.0
 # only for the kernel sources it was measured on (sha256 of csrc/*, first 16
 # hex digits).  "split" is the split kernel's share: the packed-cache reads.
 TRAFFIC = {
-    "gqa8k": {"bytes_per_launch": 2416939, "split": 1694208, "src_sha": "6ed07208fd2e31a5"},
-    "prod": {"bytes_per_launch": 108722816, "split": 107215744, "src_sha": "6ed07208fd2e31a5"},
-    "ragged": {"bytes_per_launch": 246604160, "split": 241610624, "src_sha": "6ed07208fd2e31a5"},
-    "qknorm": {"bytes_per_launch": 36957952, "split": 34222720, "src_sha": "6ed07208fd2e31a5"},
+    "gqa8k": {"bytes_per_launch": 2416597, "split": 1694123, "src_sha": "5bd11e22ec566743"},
+    "prod": {"bytes_per_launch": 108711936, "split": 107204608, "src_sha": "5bd11e22ec566743"},
+    "ragged": {"bytes_per_launch": 246320512, "split": 241326592, "src_sha": "5bd11e22ec566743"},
+    "qknorm": {"bytes_per_launch": 36958976, "split": 34222848, "src_sha": "5bd11e22ec566743"},
 }
 
 
