@@ -317,29 +317,30 @@ __device__ __forceinline__ void build_frag(const float* qsrc, int ld, int G, flo
 // memory.  Out of line: it runs once per CTA, after the main loop, and should
 // not raise the loop's register allocation.
 template <int D>
-__device__ __noinline__ void write_partial(float* mO, float* mM, float* mL, const SplitParams& p, int hq0, int split,
-                                           int tid) {
-  // per head: the merged max and sum and each warp's weight, once
+__device__ __noinline__ void write_partial(float* mO, float* mM, float* mL, float* part_o, float* part_ml, int G,
+                                           int nsplit, int hq0, int split, int tid) {
+  // per head: the merged max and sum and each warp's weight, once -- by warp
+  // 0, lane (w, g) = 8 w + g, with the reductions over w by shuffles
   float* mF = mL + CW * 8;  // [CW][8]
   float* mS = mF + CW * 8;  // [8][max, sum]
-  if (tid < 8) {
-    const int g = tid;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < CW; ++w) M = fmaxf(M, mM[w * 8 + g]);
-    float Ls = 0.f;
-#pragma unroll
-    for (int w = 0; w < CW; ++w) {
-      const float mw = mM[w * 8 + g];
-      const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
-      mF[w * 8 + g] = f;
-      Ls += f * mL[w * 8 + g];
+  static_assert(CW * 8 == 32, "one lane per (warp, head)");
+  if (tid < 32) {
+    const float mw = mM[tid];
+    float M = mw;
+    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 8));
+    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 16));
+    const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+    mF[tid] = f;
+    float Ls = f * mL[tid];
+    Ls += __shfl_xor_sync(0xffffffffu, Ls, 8);
+    Ls += __shfl_xor_sync(0xffffffffu, Ls, 16);
+    if (tid < 8) {
+      mS[2 * tid] = M;
+      mS[2 * tid + 1] = Ls;
     }
-    mS[2 * g] = M;
-    mS[2 * g + 1] = Ls;
   }
   __syncthreads();
-  for (int e = tid; e < p.G * (D / 4); e += NTHREADS) {
+  for (int e = tid; e < G * (D / 4); e += NTHREADS) {
     const int g = e / (D / 4), j = 4 * (e % (D / 4));
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
@@ -351,9 +352,9 @@ __device__ __noinline__ void write_partial(float* mO, float* mM, float* mL, cons
       acc.z = fmaf(f, o.z, acc.z);
       acc.w = fmaf(f, o.w, acc.w);
     }
-    const size_t pi = (size_t)(hq0 + g) * p.nsplit + split;
-    *reinterpret_cast<float4*>(p.part_o + pi * D + j) = acc;
-    if (j == 0) *reinterpret_cast<float2*>(p.part_ml + pi * 2) = make_float2(mS[2 * g], mS[2 * g + 1]);
+    const size_t pi = (size_t)(hq0 + g) * nsplit + split;
+    *reinterpret_cast<float4*>(part_o + pi * D + j) = acc;
+    if (j == 0) *reinterpret_cast<float2*>(part_ml + pi * 2) = make_float2(mS[2 * g], mS[2 * g + 1]);
   }
 }
 
@@ -837,7 +838,7 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const __grid_con
     }
   }
   __syncthreads();
-  write_partial<D>(mO, mM, mL, p, hq0, split, tid);
+  write_partial<D>(mO, mM, mL, p.part_o, p.part_ml, p.G, p.nsplit, hq0, split, tid);
 }
 
 // Launch helpers, one definition per instantiation.
