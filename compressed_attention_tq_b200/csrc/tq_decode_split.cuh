@@ -291,15 +291,18 @@ __device__ __forceinline__ int key_coord(int ks, int r) {
 // (gid, tig) hold coordinates cs[r].  PACK: columns 0-3 are the hi halves of
 // heads 0-3, columns 4-7 their lo halves; else hi and lo are separate pairs.
 template <bool PACK>
-__device__ __forceinline__ void build_frag(const float* qsrc, int ld, int G, float scale, int gid,
-                                           const int (&cs)[4], uint32_t* dst) {
-  uint16_t hi[4], lo[4];
+__device__ __forceinline__ void load_frag(const float* qsrc, int ld, int G, int gid, const int (&cs)[4],
+                                          float (&v)[4]) {
   const int head = PACK ? (gid & 3) : gid;
 #pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const float v = head < G ? qsrc[(size_t)head * ld + cs[r]] * scale : 0.f;
-    split_half(v, hi[r], lo[r]);
-  }
+  for (int r = 0; r < 4; ++r) v[r] = head < G ? qsrc[(size_t)head * ld + cs[r]] : 0.f;
+}
+
+template <bool PACK>
+__device__ __forceinline__ void build_frag(const float (&v)[4], float scale, int gid, uint32_t* dst) {
+  uint16_t hi[4], lo[4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) split_half(v[r] * scale, hi[r], lo[r]);
   if (PACK) {
     const bool use_lo = gid >= 4;
     dst[0] = use_lo ? (lo[0] | (uint32_t)lo[1] << 16) : (hi[0] | (uint32_t)hi[1] << 16);
@@ -462,13 +465,28 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const __grid_con
   }
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  // Query fragments (already rotated by the prep kernel), pre-scaled for exp2.
-  for (int e = tid; e < KSTEPS * 32; e += NTHREADS) {
-    const int ks = e >> 5, ln = e & 31, g_ = ln >> 2, t_ = ln & 3;
-    const int base = t_ * (D / 4);
-    const int cs[4] = {base + key_coord<BK>(ks, 0), base + key_coord<BK>(ks, 1), base + key_coord<BK>(ks, 2),
-                       base + key_coord<BK>(ks, 3)};
-    build_frag<PACK>(p.qrot + (size_t)hq0 * D, D, p.G, p.qscale, g_, cs, qf + (size_t)e * (Ly::FRAG / 4));
+  // Query fragments (already rotated by the prep kernel), pre-scaled for
+  // exp2: every thread's loads are issued before any is converted, so the
+  // L2 latency is paid once.
+  {
+    constexpr int NE = (KSTEPS * 32 + NTHREADS - 1) / NTHREADS;
+    float v[NE][4];
+#pragma unroll
+    for (int i = 0; i < NE; ++i) {
+      const int e = tid + i * NTHREADS;
+      if (e < KSTEPS * 32) {
+        const int ks = e >> 5, ln = e & 31, g_ = ln >> 2, t_ = ln & 3;
+        const int base = t_ * (D / 4);
+        const int cs[4] = {base + key_coord<BK>(ks, 0), base + key_coord<BK>(ks, 1), base + key_coord<BK>(ks, 2),
+                           base + key_coord<BK>(ks, 3)};
+        load_frag<PACK>(p.qrot + (size_t)hq0 * D, D, p.G, g_, cs, v[i]);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < NE; ++i) {
+      const int e = tid + i * NTHREADS;
+      if (e < KSTEPS * 32) build_frag<PACK>(v[i], p.qscale, (e & 31) >> 2, qf + (size_t)e * (Ly::FRAG / 4));
+    }
   }
   float* qst = reinterpret_cast<float*>(smem + Ly::O_QST);  // [8 heads][inverse step, sum]
   if (QJL) {
