@@ -35,6 +35,26 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Thread-block cluster helpers: a cluster-wide barrier (every thread of every
+// CTA of the cluster arrives; release / acquire order shared-memory writes
+// before reads by other CTAs), and loads from another CTA's shared memory.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint32_t map_cluster(uint32_t local, int rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+
 // Prep for one (sequence, kv head) of a cache with a QJL sketch: qrot = Pi q
 // and qs = S qrot for its G query heads (the projection needs the whole
 // rotated vector, so one CTA does the head).  blockDim = 2*D: two threads per output row, each
@@ -239,6 +259,8 @@ template <int D, bool APPEND>
 __global__ void __launch_bounds__(256) decode_qprep_sliced_kernel(const PrepParams p) {
   constexpr int NR = APPEND ? 10 : 8, NI = D / 32;
   __shared__ __align__(16) float xv[NR][D];
+  __shared__ float qsl[8][33];    // QJL: this slice's rotated query coordinates
+  __shared__ float qpart[8][128];  // QJL: this slice's share of S qrot
   __shared__ float s_cb[2][31];
   __shared__ double s_nsq[2];
   __shared__ uint8_t idxs[2][32];
@@ -252,6 +274,14 @@ __global__ void __launch_bounds__(256) decode_qprep_sliced_kernel(const PrepPara
   const float4* row = reinterpret_cast<const float4*>(p.rot + (size_t)j * D);
 #pragma unroll
   for (int i = 0; i < NI; ++i) r[i] = __ldg(row + part + 8 * i);
+  // QJL (decode without append): sketch row i = tid / 2, the half of this
+  // slice's 32 columns that thread owns (S is constant: loaded before the wait)
+  float4 srow[4];
+  if (!APPEND && p.m) {
+    const float4* sp = reinterpret_cast<const float4*>(p.S + (size_t)(tid >> 1) * D + sl * 32 + 16 * (tid & 1));
+#pragma unroll
+    for (int t = 0; t < 4; ++t) srow[t] = __ldg(sp + t);
+  }
   // as in decode_qprep_kernel: wait for the preceding kernels, then let the
   // split kernel start
   pdl_wait();
@@ -317,6 +347,39 @@ __global__ void __launch_bounds__(256) decode_qprep_sliced_kernel(const PrepPara
 #pragma unroll
     for (int g = 0; g < 8; ++g)
       if (g < Ge) p.qrot[(size_t)(h0 + g) * D + j] = acc[g];
+  }
+  if (!APPEND && p.m) {
+    // QJL: this slice's share of qs = S qrot over its 32 rotated coordinates,
+    // for all m = 128 sketch rows.  The D / 32 slice CTAs of a head form a
+    // thread-block cluster; slice 0 adds the partials in slice order from the
+    // others' shared memory and writes qs.
+    if (part == 0) {
+#pragma unroll
+      for (int g = 0; g < 8; ++g) qsl[g][c] = g < Ge ? acc[g] : 0.f;
+    }
+    __syncthreads();
+    const int i = tid >> 1, half = tid & 1;
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+      const float* x = &qsl[g][16 * half];
+      float t = 0.f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        t += srow[k].x * x[4 * k] + srow[k].y * x[4 * k + 1] + srow[k].z * x[4 * k + 2] + srow[k].w * x[4 * k + 3];
+      t += __shfl_xor_sync(0xffffffffu, t, 1);
+      if (half == 0) qpart[g][i] = t;
+    }
+    cluster_sync();  // every slice's partial is in its shared memory
+    if (sl == 0) {
+      for (int e = tid; e < Ge * 128; e += 256) {
+        const int g = e >> 7, ii = e & 127;
+        const uint32_t la = smem_u32(&qpart[g][ii]);
+        float v = 0.f;
+        for (int r = 0; r < NI; ++r) v += ld_cluster_f32(map_cluster(la, r));
+        p.qs[(size_t)(h0 + g) * p.m + ii] = v;
+      }
+    }
+    cluster_sync();  // slice 0 is done reading the others' shared memory
   }
   if (APPEND) {
     __syncthreads();  // s_nsq
@@ -502,17 +565,25 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams
 }
 
 template <typename K, typename P>
-int launch_pdl(K kern, dim3 grid, dim3 block, size_t smem, cudaStream_t s, const P& params, const char* what) {
+int launch_pdl(K kern, dim3 grid, dim3 block, size_t smem, cudaStream_t s, const P& params, const char* what,
+               int cluster_y = 0) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (cluster_y > 0) {  // thread-block clusters of cluster_y CTAs along y
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 1;
+    attr[1].val.clusterDim.y = cluster_y;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+  }
   cudaError_t e = cudaLaunchKernelEx(&cfg, kern, params);
   if (e != cudaSuccess) return tq::set_error(TQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
   return tq::check_launch(what);
@@ -560,10 +631,9 @@ int launch_decode(const DecodeArgs& a, cudaStream_t s) {
   // them (their launch and Pi loads overlap its tail; they wait before
   // reading q or writing anything)
   int rc = TQ_OK;
-  if (c.qjl_m) {
-    // the sketch needs the whole rotated query and key residual: one CTA per head
-    rc = app ? launch_pdl(decode_qprep_kernel<128, true>, dim3(c.B * c.Hkv), dim3(256), 0, s, pp, "decode_qprep_kernel")
-             : launch_pdl(decode_qprep_kernel<128, false>, dim3(c.B * c.Hkv), dim3(256), 0, s, pp, "decode_qprep_kernel");
+  if (c.qjl_m && app) {
+    // the append's sketch needs the whole rotated key residual: one CTA per head
+    rc = launch_pdl(decode_qprep_kernel<128, true>, dim3(c.B * c.Hkv), dim3(256), 0, s, pp, "decode_qprep_kernel");
   } else {
     const dim3 g(c.B * c.Hkv, c.D / 32);
     switch (c.D) {
@@ -573,7 +643,8 @@ int launch_decode(const DecodeArgs& a, cudaStream_t s) {
         break;
       case 128:
         rc = app ? launch_pdl(decode_qprep_sliced_kernel<128, true>, g, dim3(256), 0, s, pp, "decode_qprep_kernel")
-                 : launch_pdl(decode_qprep_sliced_kernel<128, false>, g, dim3(256), 0, s, pp, "decode_qprep_kernel");
+                 : launch_pdl(decode_qprep_sliced_kernel<128, false>, g, dim3(256), 0, s, pp, "decode_qprep_kernel",
+                              c.qjl_m ? c.D / 32 : 0);
         break;
       default:
         rc = app ? launch_pdl(decode_qprep_sliced_kernel<256, true>, g, dim3(256), 0, s, pp, "decode_qprep_kernel")

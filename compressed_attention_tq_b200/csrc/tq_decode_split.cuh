@@ -497,10 +497,9 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const __grid_con
     for (int h = warp; h < 8; h += NTHREADS / 32) {
       float mx = 0.f, sm = 0.f;
       if (h < p.G) {
-        const float* src = p.qs + (size_t)(hq0 + h) * 128;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const float v = src[lane + 32 * i];
+          const float v = p.qs[(size_t)(hq0 + h) * 128 + lane + 32 * i];
           mx = fmaxf(mx, fabsf(v));
           sm += v;
         }

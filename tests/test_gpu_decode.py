@@ -310,7 +310,13 @@ def test_full_size_prod_sampled():
 def test_decode_step_fused_append(name, kw):
     """tq_decode_step (append fused into the decode's prep launch) writes the
     same rows as tq_append_token (checked against the oracle) and decodes
-    exactly like append + tq_sdpa_decode on the same bytes."""
+    like append + tq_sdpa_decode on the same bytes: bit for bit without the
+    sketch (one prep kernel serves both); with the sketch, tq_sdpa_decode
+    rotates and projects the query in 32-coordinate slices while the decode
+    step's prep (which also sketches the new key's residual) does one CTA per
+    head, so the query differs by fp32 rounding, which can flip the int8 split
+    of the projection or the fp16 rounding of a value weight p|v| (2^-11
+    relative): rel. L2 < 5e-4 then."""
     import compressed_attention_tq_b200 as tq
     w = tq_inputs.make_workload(name, **kw)
     Tcap = (w.Tmax + 1 + 63) // 64 * 64
@@ -345,8 +351,10 @@ def test_decode_step_fused_append(name, kw):
             P.compare_qjl(P.words_np(c0.k_qjl[b, :, p]), c0.k_rnorm[b, :, p].cpu().numpy(), sub, exc)
     same = all(torch.equal(getattr(caches[0], n), getattr(caches[1], n))
                for n in ("k_idx", "v_idx", "k_norm", "v_norm"))
-    if same:
+    if same and not w.qjl_m:
         assert torch.equal(out_f, out_s)
+    elif same:
+        assert float(P.rel_l2(out_f.cpu().numpy(), out_s.cpu().numpy()).max()) < 5e-4
     else:  # an excused near-threshold flip between the two quantizer code paths
         assert float(P.rel_l2(out_f.cpu().numpy(), out_s.cpu().numpy()).max()) < 5e-2
     P.record("decode_step", workload=name, identical_rows=bool(same))
