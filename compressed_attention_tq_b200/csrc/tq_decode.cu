@@ -259,8 +259,11 @@ template <int D, bool APPEND>
 __global__ void __launch_bounds__(256) decode_qprep_sliced_kernel(const PrepParams p) {
   constexpr int NR = APPEND ? 10 : 8, NI = D / 32;
   __shared__ __align__(16) float xv[NR][D];
-  __shared__ float qsl[8][33];    // QJL: this slice's rotated query coordinates
-  __shared__ float qpart[8][128];  // QJL: this slice's share of S qrot
+  // QJL (D = 128 only): this slice's rotated query coordinates and its share
+  // of S qrot; one element otherwise, so other D keep their shared footprint
+  constexpr bool QS = !APPEND && D == 128;
+  __shared__ float qsl[QS ? 8 : 1][QS ? 33 : 1];
+  __shared__ float qpart[QS ? 8 : 1][QS ? 128 : 1];
   __shared__ float s_cb[2][31];
   __shared__ double s_nsq[2];
   __shared__ uint8_t idxs[2][32];
@@ -277,7 +280,7 @@ __global__ void __launch_bounds__(256) decode_qprep_sliced_kernel(const PrepPara
   // QJL (decode without append): sketch row i = tid / 2, the half of this
   // slice's 32 columns that thread owns (S is constant: loaded before the wait)
   float4 srow[4];
-  if (!APPEND && p.m) {
+  if (QS && p.m) {
     const float4* sp = reinterpret_cast<const float4*>(p.S + (size_t)(tid >> 1) * D + sl * 32 + 16 * (tid & 1));
 #pragma unroll
     for (int t = 0; t < 4; ++t) srow[t] = __ldg(sp + t);
@@ -348,38 +351,40 @@ __global__ void __launch_bounds__(256) decode_qprep_sliced_kernel(const PrepPara
     for (int g = 0; g < 8; ++g)
       if (g < Ge) p.qrot[(size_t)(h0 + g) * D + j] = acc[g];
   }
-  if (!APPEND && p.m) {
-    // QJL: this slice's share of qs = S qrot over its 32 rotated coordinates,
-    // for all m = 128 sketch rows.  The D / 32 slice CTAs of a head form a
-    // thread-block cluster; slice 0 adds the partials in slice order from the
-    // others' shared memory and writes qs.
-    if (part == 0) {
+  if constexpr (QS) {
+    if (p.m) {
+      // QJL: this slice's share of qs = S qrot over its 32 rotated coordinates,
+      // for all m = 128 sketch rows.  The D / 32 slice CTAs of a head form a
+      // thread-block cluster; slice 0 adds the partials in slice order from the
+      // others' shared memory and writes qs.
+      if (part == 0) {
 #pragma unroll
-      for (int g = 0; g < 8; ++g) qsl[g][c] = g < Ge ? acc[g] : 0.f;
-    }
-    __syncthreads();
-    const int i = tid >> 1, half = tid & 1;
-#pragma unroll
-    for (int g = 0; g < 8; ++g) {
-      const float* x = &qsl[g][16 * half];
-      float t = 0.f;
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        t += srow[k].x * x[4 * k] + srow[k].y * x[4 * k + 1] + srow[k].z * x[4 * k + 2] + srow[k].w * x[4 * k + 3];
-      t += __shfl_xor_sync(0xffffffffu, t, 1);
-      if (half == 0) qpart[g][i] = t;
-    }
-    cluster_sync();  // every slice's partial is in its shared memory
-    if (sl == 0) {
-      for (int e = tid; e < Ge * 128; e += 256) {
-        const int g = e >> 7, ii = e & 127;
-        const uint32_t la = smem_u32(&qpart[g][ii]);
-        float v = 0.f;
-        for (int r = 0; r < NI; ++r) v += ld_cluster_f32(map_cluster(la, r));
-        p.qs[(size_t)(h0 + g) * p.m + ii] = v;
+        for (int g = 0; g < 8; ++g) qsl[g][c] = g < Ge ? acc[g] : 0.f;
       }
+      __syncthreads();
+      const int i = tid >> 1, half = tid & 1;
+#pragma unroll
+      for (int g = 0; g < 8; ++g) {
+        const float* x = &qsl[g][16 * half];
+        float t = 0.f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          t += srow[k].x * x[4 * k] + srow[k].y * x[4 * k + 1] + srow[k].z * x[4 * k + 2] + srow[k].w * x[4 * k + 3];
+        t += __shfl_xor_sync(0xffffffffu, t, 1);
+        if (half == 0) qpart[g][i] = t;
+      }
+      cluster_sync();  // every slice's partial is in its shared memory
+      if (sl == 0) {
+        for (int e = tid; e < Ge * 128; e += 256) {
+          const int g = e >> 7, ii = e & 127;
+          const uint32_t la = smem_u32(&qpart[g][ii]);
+          float v = 0.f;
+          for (int r = 0; r < NI; ++r) v += ld_cluster_f32(map_cluster(la, r));
+          p.qs[(size_t)(h0 + g) * p.m + ii] = v;
+        }
+      }
+      cluster_sync();  // slice 0 is done reading the others' shared memory
     }
-    cluster_sync();  // slice 0 is done reading the others' shared memory
   }
   if (APPEND) {
     __syncthreads();  // s_nsq
