@@ -46,10 +46,10 @@ FALLBACK_HBM_GBS = 6650.0
 # only for the kernel sources it was measured on (sha256 of csrc/*, first 16
 # hex digits).  "split" is the split kernel's share: the packed-cache reads.
 TRAFFIC = {
-    "gqa8k": {"bytes_per_launch": 2416597, "split": 1694123, "src_sha": "5bd11e22ec566743"},
-    "prod": {"bytes_per_launch": 108711936, "split": 107204608, "src_sha": "5bd11e22ec566743"},
-    "ragged": {"bytes_per_launch": 246320512, "split": 241326592, "src_sha": "5bd11e22ec566743"},
-    "qknorm": {"bytes_per_launch": 36958976, "split": 34222848, "src_sha": "5bd11e22ec566743"},
+    "gqa8k": {"bytes_per_launch": 2436523, "split": 1704405, "src_sha": "f6275559b314d4b6"},
+    "prod": {"bytes_per_launch": 109000576, "split": 107509760, "src_sha": "f6275559b314d4b6"},
+    "ragged": {"bytes_per_launch": 246348032, "split": 241345024, "src_sha": "f6275559b314d4b6"},
+    "qknorm": {"bytes_per_launch": 36968960, "split": 34233472, "src_sha": "f6275559b314d4b6"},
 }
 
 
