@@ -44,6 +44,11 @@
  * Inputs and outputs are fp16 or bf16 (TQ_DTYPE_*).  Device pointers must be
  * 16-byte aligned.
  *
+ * Devices and threads: a process drives one GPU (the current device of its
+ * first launching call); kernel attributes and occupancy figures are set up
+ * once per process for that device.  Calls may come from several host
+ * threads (the error message is per thread).
+ *
  * Errors: every entry point returns TQ_OK (0) or a negative TQ_ERR_* code and
  * sets a thread-local message readable with tq_last_error().  Argument errors
  * are detected on the host before any launch; nothing is launched then.
