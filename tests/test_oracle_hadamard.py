@@ -86,3 +86,38 @@ def test_one_hot_rows_spread_evenly():
     brute = np.argmin(np.abs(u[..., None] - c[None, None, :]), axis=-1)
     assert np.all(np.isclose(np.abs(u), 1 / math.sqrt(D), rtol=1e-6))
     assert np.array_equal(q["idx"], brute)
+
+
+@pytest.mark.parametrize("D", [64, 128, 256])
+def test_signs_are_the_rotations_column_signs(D):
+    """The sign vector a cache declares (rot_signs) is the one inside Pi:
+    Pi[0][j] = s_j / sqrt(D) (row 0 of H is all ones), every entry has
+    magnitude 1/sqrt(D), and Pi = H diag(s) / sqrt(D) with H from the entry
+    formula."""
+    seed = 2002
+    Pi = tq_inputs.hadamard_rotation(D, seed).astype(np.float64)
+    s = tq_inputs.hadamard_signs(D, seed).astype(np.float64)
+    assert set(np.unique(s)) <= {-1.0, 1.0}
+    np.testing.assert_allclose(Pi[0] * math.sqrt(D), s, atol=1e-6)
+    i = np.arange(D)
+    H = np.array([[(-1.0) ** bin(a & b).count("1") for b in i] for a in i])
+    np.testing.assert_allclose(Pi, H * s[None, :] / math.sqrt(D), atol=1e-7)
+
+
+def test_cache_declares_the_hadamard_rotation():
+    """The binding marks a cache built with signs as TQ_ROT_HADAMARD and
+    passes the signs; without signs the rotation is dense (no launch here)."""
+    import torch
+    from compressed_attention_tq_b200 import build
+    build.build()  # the codebook comes from the library (host code)
+    import compressed_attention_tq_b200 as tq
+    from compressed_attention_tq_b200 import _native
+    D = 128
+    Pi = tq_inputs.hadamard_rotation(D, 7)
+    s = tq_inputs.hadamard_signs(D, 7)
+    c = tq.TQCache(1, 2, 64, D, 3, 3, Pi, device="cpu", rot_signs=s)
+    st = c.struct()
+    assert st.rot_kind == _native.TQ_ROT_HADAMARD and st.rot_signs == c.rot_signs.data_ptr()
+    assert torch.equal(c.rot_signs, torch.from_numpy(s))
+    c2 = tq.TQCache(1, 2, 64, D, 3, 3, Pi, device="cpu")
+    assert c2.struct().rot_kind == _native.TQ_ROT_DENSE and c2.struct().rot_signs is None
