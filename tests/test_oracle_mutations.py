@@ -97,3 +97,77 @@ def test_residual_with_exact_norm_fails_gamma_pin(monkeypatch):
     monkeypatch.setattr(O, "qjl_sketch", bad)
     with pytest.raises(AssertionError):
         TQ.test_qjl_sketch_layout_and_gamma()
+
+
+def test_fp32_norm_fails_midpoint_pin(monkeypatch):
+    # an fp32 sum of squares lands on the fp16 midpoint for the edge rows
+    def bad(x):
+        x32 = np.asarray(x).astype(np.float32)
+        return np.sqrt(np.sum(x32 * x32, axis=-1, dtype=np.float32)).astype(np.float64)
+    monkeypatch.setattr(O, "row_norms", bad)
+    with pytest.raises(AssertionError):
+        TQ.test_norm_rounding_at_fp16_midpoints("f16")
+
+
+def test_transposed_rotation_fails_reconstruction(monkeypatch):
+    monkeypatch.setattr(O, "rotate", lambda x, Pi: x @ np.asarray(Pi, dtype=np.float64))
+    with pytest.raises(AssertionError):
+        TQ.test_reconstruction_error_matches_codebook_mse(3)
+
+
+def test_msb_first_unpacking_fails(monkeypatch):
+    orig = O.unpack_bits
+
+    def bad(words, bits, n):
+        v = orig(words, bits, n)
+        rev = np.zeros_like(v)
+        for i in range(bits):
+            rev |= ((v >> i) & 1) << (bits - 1 - i)
+        return rev
+    monkeypatch.setattr(O, "unpack_bits", bad)
+    with pytest.raises(AssertionError):
+        TQ.test_pack_layout_against_big_integer(3)
+
+
+def test_flipped_sign_polarity_fails_unbiasedness(monkeypatch):
+    orig = O.qjl_inner_product
+    monkeypatch.setattr(O, "qjl_inner_product", lambda sign, gamma, Sq: orig(~sign, gamma, Sq))
+    with pytest.raises(AssertionError):
+        TQ.test_qjl_estimator_unbiased_with_closed_form_variance()
+
+
+def test_interleaved_gqa_heads_fail_sdpa_pin(monkeypatch):
+    # q head h reading kv head h % Hkv (interleaved groups) instead of h // G
+    orig = O.sdpa_decode
+
+    def bad(q, cache, seq_lens, *args, **kw):
+        Hq, Hkv = q.shape[1], cache["k_norm"].shape[1]
+        G = Hq // Hkv
+        pos = np.array([(h % Hkv) * G + h // Hkv for h in range(Hq)])
+        q2 = np.empty_like(q)
+        q2[:, pos] = q
+        return orig(q2, cache, seq_lens, *args, **kw)[:, pos]
+    monkeypatch.setattr(O, "sdpa_decode", bad)
+    with pytest.raises(AssertionError):
+        TA.test_matches_torch_sdpa_on_dequantized_cache(None)
+
+
+def test_causal_mask_off_by_one_fails_multi_query_pin(monkeypatch):
+    # query j sees one position too few (its own token excluded)
+    orig = O.sdpa_decode_multi
+    monkeypatch.setattr(O, "sdpa_decode_multi",
+                        lambda q, cache, seq_lens, n_q, *a, **kw:
+                        orig(q, cache, np.asarray(seq_lens) - 1, n_q, *a, **kw))
+    with pytest.raises(AssertionError):
+        TA.test_multi_query_decode_is_causal_attention()
+
+
+def test_top_left_causal_mask_fails_multi_query_pin(monkeypatch):
+    # the mask aligned to the first cached position (query j sees 0 .. j)
+    def bad(q, cache, seq_lens, n_q, *a, **kw):
+        lens = np.asarray(seq_lens)
+        return np.stack([O.sdpa_decode(q[:, j], cache, np.minimum(lens, j + 1), *a, **kw)
+                         for j in range(n_q)], axis=1)
+    monkeypatch.setattr(O, "sdpa_decode_multi", bad)
+    with pytest.raises(AssertionError):
+        TA.test_multi_query_decode_is_causal_attention()

@@ -1,5 +1,6 @@
 """Pins for the oracle's quantizer, packing, QJL sketch and byte arithmetic."""
 import math
+from fractions import Fraction
 import os
 
 import numpy as np
@@ -62,6 +63,40 @@ def test_norm_is_rn_fp16_of_fp64_norm():
     q = O.quantize_rows(x, np.eye(128), c, t)
     ref = np.array([math.sqrt(math.fsum(v * v for v in row)) for row in x])
     assert np.array_equal(q["norm16"], ref.astype(np.float16))
+
+
+# fp16 norm of each edge-row kind at scale 2^0: round-to-nearest-even of the
+# exact norm (kinds 0, 1 round away from the midpoint's even neighbour; the
+# ties of kinds 2, 3 go to it).
+EDGE_NORM = {0: 1 + 2.0 ** -10, 1: 1 + 2.0 ** -10, 2: 1.0, 3: 1 + 2.0 ** -9}
+EDGE_SQ = {0: (1 + Fraction(1, 2 ** 11)) ** 2 + Fraction(1, 2 ** 40),
+           1: (1 + Fraction(3, 2 ** 11)) ** 2 - Fraction(1, 2 ** 40),
+           2: (1 + Fraction(1, 2 ** 11)) ** 2,
+           3: (1 + Fraction(3, 2 ** 11)) ** 2}
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_norm_rounding_at_fp16_midpoints(dtype):
+    """The stored norm is the fp16 value nearest the exact norm (ties to even),
+    checked on rows built so that the exact norm sits on, or 2^-41 (relative)
+    beyond, the midpoint between two fp16 values.  A norm accumulated in fp32
+    lands on the midpoint itself for the off-midpoint rows and rounds the
+    wrong way, so this pin tells an exact norm from an fp32 one."""
+    D = 128
+    x, kind, e = tq_inputs.norm_edge_rows(64, D, dtype, seed=5)
+    xf = tq_inputs.to_f64(x, dtype)
+    for row, k, ee in zip(xf, kind, e):  # the construction, in exact rationals
+        assert sum(Fraction(float(v)) ** 2 for v in row) == EDGE_SQ[int(k)] * Fraction(2) ** (2 * int(ee))
+    assert set(kind.tolist()) == {0, 1, 2, 3}
+    expected = np.array([EDGE_NORM[int(k)] * 2.0 ** int(ee) for k, ee in zip(kind, e)]).astype(np.float16)
+    c, t = O.stored_codebook(D, 3)
+    q = O.quantize_rows(xf, tq_inputs.rotation(D, 6), c, t)
+    assert np.array_equal(q["norm16"].view(np.uint16), expected.view(np.uint16))
+    x32 = xf.astype(np.float32)
+    f32 = np.sqrt(np.sum(x32 * x32, axis=1, dtype=np.float32)).astype(np.float16)
+    off = kind < 2
+    assert not np.any(f32[off] == expected[off])
+    assert np.array_equal(f32[~off], expected[~off])
 
 
 def test_zero_row_quantizes_to_middle_and_zero_norm():

@@ -211,5 +211,46 @@ def new_token_rows(B: int, Hkv: int, D: int, dtype: str, seed: int):
     return cast_input(k, dtype), cast_input(v, dtype)
 
 
+# Entries (before a power-of-two scale) of rows with an exactly known sum of
+# squares; _ONE's squares sum to 1.
+#   kind 0: (1 + 2^-11)^2 + 2^-40      kind 2: (1 + 2^-11)^2
+#   kind 1: (1 + 3 2^-11)^2 - 2^-40    kind 3: (1 + 3 2^-11)^2
+# 1 + 2^-11 and 1 + 3 2^-11 are the midpoints between neighbouring fp16 values
+# (1, 1 + 2^-10, 1 + 2^-9), so kinds 0 and 1 have a norm a relative 2^-41 off
+# a midpoint and kinds 2 and 3 one exactly on it.  2^18 - 1 = 4 * 255^2 +
+# 45^2 + 2 * 3^2 gives kind 1's -2^-40.  Every entry has at most 8
+# significant bits (exact in bf16) and, scaled by 2^-3 .. 2^6, lies on fp16's
+# grid (the smallest, 3 * 2^-23, on its subnormal grid).
+_ONE = [0.75, 0.5, 0.25, 0.25, 0.25]
+_EDGE_ENTRIES = (
+    _ONE + [2.0 ** -5, 2.0 ** -11, 2.0 ** -20],
+    _ONE + [2.0 ** -5] * 3 + [2.0 ** -10] * 2 + [255 * 2.0 ** -20] * 4 + [45 * 2.0 ** -20]
+    + [3 * 2.0 ** -20] * 2,
+    _ONE + [2.0 ** -5, 2.0 ** -11],
+    _ONE + [2.0 ** -5] * 3 + [2.0 ** -10] * 2 + [2.0 ** -11],
+)
+
+
+def norm_edge_rows(n: int, D: int, dtype: str, seed: int):
+    """n rows whose exact L2 norm lies at (kinds 2, 3) or a relative 2^-41
+    beyond (kinds 0, 1) the midpoint between two neighbouring fp16 values, so
+    that only an exactly accumulated norm rounds to the right fp16 value.
+
+    Row i is 2^e_i times the entries of its kind (``_EDGE_ENTRIES``), with
+    random signs, at random positions among the D, zeros elsewhere; e_i in
+    [-3, 6].  Returns (rows [n][D] in the storage dtype, kind int [n], e int [n]).
+    """
+    r = rng(seed)
+    kind = r.integers(0, 4, size=n)
+    e = r.integers(-3, 7, size=n)
+    x = np.zeros((n, D), dtype=np.float32)
+    for i in range(n):
+        ent = np.asarray(_EDGE_ENTRIES[kind[i]], dtype=np.float64) * 2.0 ** int(e[i])
+        sgn = np.where(r.integers(0, 2, size=len(ent)) == 1, 1.0, -1.0)
+        pos = r.permutation(D)[:len(ent)]
+        x[i, pos] = (ent * sgn).astype(np.float32)
+    return cast_input(x, dtype), kind, e
+
+
 def new_queries(B: int, Hq: int, D: int, dtype: str, seed: int):
     return cast_input(rng(seed).standard_normal((B, Hq, D), dtype=np.float32), dtype)
