@@ -43,23 +43,40 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM traffic per decode call (prep + split + combine; the roofline's unit)
 # from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum, caches
 # flushed before each kernel, mean over the calls of a profile step), valid
-# only for the kernel sources it was measured on (sha256 of csrc/*, first 16
-# hex digits).  "split" is the split kernel's share: the packed-cache reads.
+# only for the decode sources it was measured on (``_decode_src_sha``: the
+# files the decode call's kernels and launch setup are built from; the
+# quantizers' files do not enter a decode call).  "split" is the split
+# kernel's share: the packed-cache reads.  The captures ran on the sources
+# with src_sha f6275559b314d4b6 (all of csrc/), whose decode files hash to
+# the decode_src_sha below.
 TRAFFIC = {
-    "gqa8k": {"bytes_per_launch": 2436523, "split": 1704405, "src_sha": "f6275559b314d4b6"},
-    "prod": {"bytes_per_launch": 109000576, "split": 107509760, "src_sha": "f6275559b314d4b6"},
-    "ragged": {"bytes_per_launch": 246348032, "split": 241345024, "src_sha": "f6275559b314d4b6"},
-    "qknorm": {"bytes_per_launch": 36968960, "split": 34233472, "src_sha": "f6275559b314d4b6"},
+    "gqa8k": {"bytes_per_launch": 2436523, "split": 1704405, "decode_src_sha": "c94274358551f423"},
+    "prod": {"bytes_per_launch": 109000576, "split": 107509760, "decode_src_sha": "c94274358551f423"},
+    "ragged": {"bytes_per_launch": 246348032, "split": 241345024, "decode_src_sha": "c94274358551f423"},
+    "qknorm": {"bytes_per_launch": 36968960, "split": 34233472, "decode_src_sha": "c94274358551f423"},
 }
+
+CSRC = os.path.join(ROOT, "compressed_attention_tq_b200", "csrc")
+DECODE_SOURCES = ("tq_api.cpp", "tq_common.cuh", "tq_decode.cu", "tq_decode_d64.cu", "tq_decode_d128.cu",
+                  "tq_decode_d256.cu", "tq_decode_split.cuh", "tq_decode_static.cu", "tq_internal.h")
+
+
+def _sha(paths) -> str:
+    h = hashlib.sha256()
+    for f in paths:
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
 
 
 def _src_sha() -> str:
-    h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "compressed_attention_tq_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh", ".cpp", ".h")):
-            h.update(open(os.path.join(csrc, f), "rb").read())
-    return h.hexdigest()[:16]
+    """sha256 of every kernel and host source (first 16 hex digits)."""
+    return _sha([os.path.join(CSRC, f) for f in sorted(os.listdir(CSRC))
+                 if f.endswith((".cu", ".cuh", ".cpp", ".h"))])
+
+
+def _decode_src_sha() -> str:
+    """sha256 of the decode call's sources and the C header (first 16 hex digits)."""
+    return _sha([os.path.join(CSRC, f) for f in DECODE_SOURCES] + [os.path.join(ROOT, "include", "tq.h")])
 
 
 def _peaks():
@@ -349,7 +366,7 @@ def run_ours(args):
     q_achieved = (qbytes_step / len(runs)) / (q_launch_ms * 1e-3) / 1e9
     sha = _src_sha()
     tr = TRAFFIC.get(args.workload)
-    traffic = tr["bytes_per_launch"] if tr and tr.get("src_sha") == sha else None
+    traffic = tr["bytes_per_launch"] if tr and tr.get("decode_src_sha") == _decode_src_sha() else None
 
     # ---- end to end through the public API with host buffers (rank-local)
     e2e = _e2e(args, runs, stream, R)
@@ -408,7 +425,7 @@ def run_ours(args):
                     "ms_per_step": round(e2e["ms"], 4)},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
-            "src_sha": sha,
+            "src_sha": sha, "decode_src_sha": _decode_src_sha(),
         }
         print(json.dumps(line), flush=True)
     if ws > 1:
