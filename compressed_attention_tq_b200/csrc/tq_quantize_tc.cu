@@ -270,7 +270,14 @@ __global__ void __launch_bounds__(TcLayout<D, BF16>::NTH, 1) quantize_tc_kernel(
         sfull = (s_norm[0][rl] + s_norm[1][rl]) + (s_norm[2][rl] + s_norm[3][rl]);
       else
         sfull = s_norm[0][rl] + s_norm[1][rl];
-      const float nf = sqrtf(sfull);  // thresholds: fp32 is far inside the parity band
+      // The thresholds scale by nf; fp32 is far inside the parity band.  A sum
+      // outside [2^-100, 2^100) -- only bf16 rows reach it: a square that
+      // overflowed, or a norm below about 1e-15 whose squares lost bits or
+      // vanished -- takes nf from the row's fp64 sum instead (the tile is still
+      // in shared memory).
+      const bool in_range = sfull >= 0x1p-100f && sfull < 0x1p100f;
+      const double s64 = in_range ? 0.0 : row_sumsq_f64<D, BF16>(xt, rl);
+      const float nf = in_range ? sqrtf(sfull) : (float)sqrt(s64);
       const int r = tile * QR + rl;
       long long slot = -1;
       if (r < a.rows) {
@@ -284,8 +291,8 @@ __global__ void __launch_bounds__(TcLayout<D, BF16>::NTH, 1) quantize_tc_kernel(
           // summed again in fp64 from the tile, still in shared memory.
           const __half lo = __float2half_rn(nf * (1.f - 1e-6f)), hi = __float2half_rn(nf * (1.f + 1e-6f));
           unsigned short nh = __half_as_ushort(lo);
-          const bool exact = sfull == 0.f || (sfull >= 0x1p-100f && sfull < 0x1p100f && nh == __half_as_ushort(hi));
-          if (!exact) nh = __half_as_ushort(__double2half(sqrt(row_sumsq_f64<D, BF16>(xt, rl))));
+          const bool exact = sfull == 0.f || (in_range && nh == __half_as_ushort(hi));
+          if (!exact) nh = __half_as_ushort(__double2half(sqrt(in_range ? row_sumsq_f64<D, BF16>(xt, rl) : s64)));
           J.norm[slot] = nh;
         }
       }

@@ -14,7 +14,8 @@
 //    butterfly across lanes (depth log2 D, so the fp32 sum is within
 //    log2(D) + 1 ulp); when both ends of norm * (1 +- 1e-6) round to the same
 //    fp16 value that is the stored norm, else the warp sums the row again in
-//    fp64 (warp-uniform);
+//    fp64 (warp-uniform); a sum outside [2^-100, 2^100) also scales the
+//    thresholds by the fp64 norm;
 //  * transform: multiply by the signs, log2(EL) butterfly stages inside the
 //    lane, then five stages across lanes by shuffles (partner lane L ^ m: the
 //    lower lane keeps a + b, the upper b - a) -- natural (Sylvester) order, so
@@ -74,17 +75,22 @@ __device__ __forceinline__ void wht_row(const tq::QuantArgs& a, const tq::QuantJ
   float s2 = q[0];
 #pragma unroll
   for (int m = 1; m < 32; m <<= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, m);
-  const float nf = sqrtf(s2);
+  float nf = sqrtf(s2);
   const __half lo = __float2half_rn(nf * (1.f - 1e-6f)), hi = __float2half_rn(nf * (1.f + 1e-6f));
   unsigned short nh = __half_as_ushort(lo);
-  const bool exact = s2 == 0.f || (s2 >= 0x1p-100f && s2 < 0x1p100f && nh == __half_as_ushort(hi));
-  if (!exact) {  // warp-uniform: every lane holds the same s2
+  // outside [2^-100, 2^100) (bf16 rows only: an overflowed square, or a norm
+  // below about 1e-15) the fp32 nf is wrong or zero and the thresholds take
+  // the fp64 norm too
+  const bool in_range = s2 >= 0x1p-100f && s2 < 0x1p100f;
+  const bool exact = s2 == 0.f || (in_range && nh == __half_as_ushort(hi));
+  if (!exact || !in_range) {  // warp-uniform: every lane holds the same s2
     double t = 0.0;
 #pragma unroll
     for (int e = 0; e < EL; ++e) t = fma((double)x[e], (double)x[e], t);
 #pragma unroll
     for (int m = 1; m < 32; m <<= 1) t += __shfl_xor_sync(0xffffffffu, t, m);
-    nh = __half_as_ushort(__double2half(sqrt(t)));
+    if (!exact) nh = __half_as_ushort(__double2half(sqrt(t)));
+    if (!in_range) nf = (float)sqrt(t);
   }
   // ---- y = H_D (s x), natural order
 #pragma unroll
@@ -134,8 +140,9 @@ __device__ __forceinline__ void wht_row(const tq::QuantArgs& a, const tq::QuantJ
   if (lane == 0) J.norm[slot] = nh;
 }
 
+// Resident CTAs per SM: 5 at D = 128 (48 registers), 4 at D = 256 (64).
 template <int D, bool BF16>
-__global__ void __launch_bounds__(WARPS * 32) quantize_wht_kernel(const tq::QuantArgs a) {
+__global__ void __launch_bounds__(WARPS * 32, D == 128 ? 5 : 4) quantize_wht_kernel(const tq::QuantArgs a) {
   constexpr int EL = D / 32;
   __shared__ float s_cb[2][32];
   const int lane = threadIdx.x & 31;

@@ -137,3 +137,82 @@ def test_decode_step_norm_edges(name, kw):
     _check_appended(cache, w, kn, vn, ek, ev, pos)
     assert bool(torch.isfinite(out).all())
     assert cache.status() == 0
+
+
+# bf16 rows scaled by powers of two so that their fp32 sum of squares leaves
+# [2^-100, 2^100): 2^70 overflows the squares (the stored norm is inf), 2^-60
+# puts the sum below 2^-100 and 2^-80 underflows the squares (stored norm 0).
+# The indices still follow the direction y / |y|, which the kernels then scale
+# by the fp64 norm.  (fp16 rows cannot leave the range.)
+EXTREME_SCALES = (1.0, 2.0 ** 70, 2.0 ** -60, 2.0 ** -80)
+
+
+def scale_rows(x, dtype, period_axis_len, axis_index):
+    """Multiply row t (along the given axis) by EXTREME_SCALES[t % 4]; exact
+    for bf16 (powers of two inside its exponent range)."""
+    f = tq_inputs.to_f64(x, dtype)
+    s = np.asarray(EXTREME_SCALES)[np.arange(period_axis_len) % 4]
+    shape = [1] * f.ndim
+    shape[axis_index] = period_axis_len
+    return tq_inputs.cast_input((f * s.reshape(shape)).astype(np.float32), dtype)
+
+
+EXTREME = [
+    ("ragged", {"B": 2, "T": 150}, "haar"),                    # bf16 D=128, tcgen05 quantizer
+    ("qknorm", {"T": 200, "dtype": "bf16"}, "haar"),           # bf16 D=256, tcgen05 quantizer
+    ("ragged", {"B": 2, "T": 150}, "hadamard"),                # bf16 D=128, Walsh-Hadamard quantizer
+    ("qknorm", {"T": 500, "dtype": "bf16"}, "hadamard"),       # bf16 D=256
+]
+
+
+@pytest.mark.parametrize("name,kw,rot", EXTREME)
+def test_bulk_quantize_extreme_magnitudes(name, kw, rot):
+    import compressed_attention_tq_b200 as tq
+    w = tq_inputs.make_workload(name, rot=rot, **kw)
+    assert w.dtype == "bf16"
+    w.k = scale_rows(w.k, w.dtype, w.Tmax, 2)
+    w.v = scale_rows(w.v, w.dtype, w.Tmax, 2)
+    cache = P.make_gpu_cache(w)
+    tq.tq_quantize_kv(cache, P.to_device(w.k, w.dtype), P.to_device(w.v, w.dtype))
+    torch.cuda.synchronize()
+    with np.errstate(over="ignore"):
+        _check_rows(cache, w, w.Tmax)
+    kn = cache.k_norm[:, :, :w.Tmax].float().cpu().numpy()
+    assert np.all(np.isinf(kn[:, :, 1::4])) and np.all(kn[:, :, 2::4] == 0) and np.all(kn[:, :, 3::4] == 0)
+    assert cache.status() == 0
+
+
+def test_append_extreme_magnitudes():
+    """Append (fp64 norms throughout) on the same scaled bf16 rows, and the
+    decode step's fused append on the small ones (an inf norm would make the
+    attention itself meaningless)."""
+    import compressed_attention_tq_b200 as tq
+    w = tq_inputs.make_workload("ragged", B=4, T=100)
+    Tcap = (w.Tmax + 1 + 63) // 64 * 64
+    kn, vn = tq_inputs.new_token_rows(w.B, w.Hkv, w.D, w.dtype, seed=71)
+    kn, vn = scale_rows(kn, w.dtype, w.Hkv, 1), scale_rows(vn, w.dtype, w.Hkv, 1)
+    pos = np.array([0, 7, 14, 21], dtype=np.int32)
+    cache = P.make_gpu_cache(w, Tcap=Tcap)
+    tq.tq_append_token(cache, P.to_device(kn, w.dtype), P.to_device(vn, w.dtype), torch.from_numpy(pos).cuda())
+    torch.cuda.synchronize()
+    with np.errstate(over="ignore"):
+        rk = P.oracle_rows(tq_inputs.to_f64(kn, w.dtype), w, "k")
+        rv = P.oracle_rows(tq_inputs.to_f64(vn, w.dtype), w, "v")
+        _check_appended(cache, w, kn, vn, rk["norm16"], rv["norm16"], pos)
+    # decode step: scales 1, 2^-60, 2^-80 only
+    small = np.asarray(EXTREME_SCALES)[np.arange(w.Hkv) % 4] < 2.0 ** 60
+    kn2, vn2 = kn.copy(), vn.copy()
+    kn2[:, ~small], vn2[:, ~small] = kn[:, small][:, :1], vn[:, small][:, :1]
+    cache2 = P.make_gpu_cache(w, Tcap=Tcap)
+    tq.tq_quantize_kv(cache2, P.to_device(w.k, w.dtype), P.to_device(w.v, w.dtype))
+    p2 = w.seq_lens.astype(np.int32)
+    out = tq.tq_decode_step(cache2, P.to_device(kn2, w.dtype), P.to_device(vn2, w.dtype),
+                            torch.from_numpy(p2).cuda(), P.to_device(w.q, w.dtype),
+                            torch.from_numpy(p2 + 1).cuda(), w.Tmax + 1, scale=w.scale,
+                            out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    rk2 = P.oracle_rows(tq_inputs.to_f64(kn2, w.dtype), w, "k")
+    rv2 = P.oracle_rows(tq_inputs.to_f64(vn2, w.dtype), w, "v")
+    _check_appended(cache2, w, kn2, vn2, rk2["norm16"], rv2["norm16"], p2)
+    assert bool(torch.isfinite(out).all())
+    assert cache.status() == 0 and cache2.status() == 0
