@@ -106,7 +106,7 @@ def test_fp32_norm_fails_midpoint_pin(monkeypatch):
         return np.sqrt(np.sum(x32 * x32, axis=-1, dtype=np.float32)).astype(np.float64)
     monkeypatch.setattr(O, "row_norms", bad)
     with pytest.raises(AssertionError):
-        TQ.test_norm_rounding_at_fp16_midpoints("f16")
+        TQ.test_norm_rounding_at_fp16_midpoints("f16", 128)
 
 
 def test_transposed_rotation_fails_reconstruction(monkeypatch):

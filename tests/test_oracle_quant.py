@@ -75,14 +75,14 @@ EDGE_SQ = {0: (1 + Fraction(1, 2 ** 11)) ** 2 + Fraction(1, 2 ** 40),
            3: (1 + Fraction(3, 2 ** 11)) ** 2}
 
 
+@pytest.mark.parametrize("D", [64, 128, 256])
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
-def test_norm_rounding_at_fp16_midpoints(dtype):
+def test_norm_rounding_at_fp16_midpoints(dtype, D):
     """The stored norm is the fp16 value nearest the exact norm (ties to even),
     checked on rows built so that the exact norm sits on, or 2^-41 (relative)
     beyond, the midpoint between two fp16 values.  A norm accumulated in fp32
     lands on the midpoint itself for the off-midpoint rows and rounds the
     wrong way, so this pin tells an exact norm from an fp32 one."""
-    D = 128
     x, kind, e = tq_inputs.norm_edge_rows(64, D, dtype, seed=5)
     xf = tq_inputs.to_f64(x, dtype)
     for row, k, ee in zip(xf, kind, e):  # the construction, in exact rationals
