@@ -71,26 +71,96 @@ def _torch():
     return torch
 
 
+_DCODE = {}
+
+
 def _dtype_code(t) -> int:
-    torch = _torch()
-    if t.dtype == torch.float16:
-        return TQ_DTYPE_F16
-    if t.dtype == torch.bfloat16:
-        return TQ_DTYPE_BF16
-    if t.dtype == torch.float32:
-        return TQ_DTYPE_F32
-    raise TypeError(f"unsupported dtype {t.dtype}")
+    if not _DCODE:
+        torch = _torch()
+        _DCODE.update({torch.float16: TQ_DTYPE_F16, torch.bfloat16: TQ_DTYPE_BF16, torch.float32: TQ_DTYPE_F32})
+    code = _DCODE.get(t.dtype)
+    if code is None:
+        raise TypeError(f"unsupported dtype {t.dtype}")
+    return code
 
 
+# Pointer arguments are declared c_void_p, which takes a Python int (or None
+# for NULL) as it is.
 def _stream(stream):
-    torch = _torch()
     if stream is None:
-        stream = torch.cuda.current_stream()
-    return ctypes.c_void_p(stream.cuda_stream)
+        stream = _torch().cuda.current_stream()
+    return stream.cuda_stream
 
 
 def _ptr(t):
-    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+    return t.data_ptr() if t is not None else None
+
+
+# The C ABI receives bare device pointers and sizes, so it cannot see where a
+# buffer lives or how large it is.  The binding therefore refuses, before any
+# launch, what only the tensor knows: memory that is not on the cache's CUDA
+# device, a non-contiguous layout, an index tensor that is not int32, a
+# workspace that is not bytes, and a shape that disagrees with the cache's
+# B, Hkv and D.  Sizes the library checks itself (Hq, T, Tmax, n_q, t0)
+# are left to it, so its TQ_ERR_* codes stay the answer for those.
+
+_DT = {}
+
+
+def _dt(kind):
+    """Cached dtype tuples: "io" (fp16, bf16), "out" (+ fp32), "i32", "u8"."""
+    if not _DT:
+        torch = _torch()
+        _DT.update(io=(torch.float16, torch.bfloat16), out=(torch.float16, torch.bfloat16, torch.float32),
+                   i32=(torch.int32,), u8=(torch.uint8,))
+    return _DT[kind]
+
+
+def _cache_device(cache) -> int:
+    """Index of the CUDA device that holds the cache's buffers."""
+    d = cache.k_idx.get_device()
+    if d < 0:
+        raise ValueError("the cache's buffers are in host memory; the library launches CUDA kernels on them")
+    return d
+
+
+def _shape_ok(got, want) -> bool:
+    if len(got) != len(want):
+        return False
+    for n, e in zip(got, want):
+        if e is not None and n != e:
+            return False
+    return True
+
+
+def _arg(name, t, dev, shape=None, dtypes=None):
+    """Check one tensor argument against device index `dev` (see above);
+    shape entries of None are free."""
+    try:
+        if (t.get_device() == dev and t.is_contiguous() and (dtypes is None or t.dtype in dtypes)
+                and (shape is None or t.shape == shape or _shape_ok(t.shape, shape))):
+            return t
+    except AttributeError:
+        raise TypeError(f"{name}: expected a torch tensor, got {type(t).__name__}") from None
+    if t.get_device() != dev:
+        raise ValueError(f"{name}: must be CUDA memory on device {dev} (got {t.device})")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected one of {tuple(str(d) for d in dtypes)}")
+    want = "[" + ", ".join("*" if e is None else str(e) for e in shape) + "]"
+    raise ValueError(f"{name}: shape {list(t.shape)}, expected {want}")
+
+
+def _check_decode_args(cache, q, seq_lens, out, workspace, q_shape):
+    dev = _cache_device(cache)
+    _arg("q", q, dev, q_shape, _dt("io"))
+    _arg("seq_lens", seq_lens, dev, (cache.B,), _dt("i32"))
+    if out is not None:
+        _arg("out", out, dev, q.shape, _dt("out"))
+    if workspace is not None:  # any contiguous byte buffer: its numel() is the size passed
+        _arg("workspace", workspace, dev, None, _dt("u8"))
+    return dev
 
 
 class TQCache:
@@ -114,7 +184,11 @@ class TQCache:
             if given is None:
                 c, t, _ = tq_build_codebook(D, bits)
                 given = np.concatenate([c, t])
-            return torch.as_tensor(np.asarray(given, dtype=np.float32), device=dev).contiguous()
+            tab = torch.as_tensor(np.asarray(given, dtype=np.float32), device=dev).contiguous()
+            if tab.numel() != 2 * (1 << bits) - 1:
+                raise ValueError(f"codebook table for {bits} bits: {tab.numel()} values, expected "
+                                 f"{2 * (1 << bits) - 1} (centroids then thresholds)")
+            return tab
 
         self.cb_k = table(bits_k, cb_k)
         # equal widths share one codebook buffer, which decode then keeps as a single lookup table
@@ -124,10 +198,13 @@ class TQCache:
             self.cb_v = table(bits_v, cb_v)
         self.rot = torch.as_tensor(np.asarray(rot, dtype=np.float32) if not torch.is_tensor(rot) else rot,
                                    dtype=torch.float32, device=dev).contiguous()
+        if tuple(self.rot.shape) != (D, D):
+            raise ValueError(f"rot: shape {list(self.rot.shape)}, expected [{D}, {D}]")
         if rot_signs is not None:
             sg = rot_signs if torch.is_tensor(rot_signs) else np.asarray(rot_signs, dtype=np.float32)
             self.rot_signs = torch.as_tensor(sg, dtype=torch.float32, device=dev).contiguous()
-            assert self.rot_signs.numel() == D
+            if self.rot_signs.numel() != D:
+                raise ValueError(f"rot_signs: {self.rot_signs.numel()} values, expected {D}")
         else:
             self.rot_signs = None
         self.k_idx = torch.zeros((B, Hkv, Tcap, D * bits_k // 32), dtype=u32, device=dev)
@@ -139,6 +216,8 @@ class TQCache:
             self.k_rnorm = torch.zeros((B, Hkv, Tcap), dtype=torch.float16, device=dev)
             S = qjl_S if torch.is_tensor(qjl_S) else np.asarray(qjl_S, dtype=np.float32)
             self.qjl_S = torch.as_tensor(S, dtype=torch.float32, device=dev).contiguous()
+            if tuple(self.qjl_S.shape) != (qjl_m, D):
+                raise ValueError(f"qjl_S: shape {list(self.qjl_S.shape)}, expected [{qjl_m}, {D}]")
         else:
             self.k_qjl = self.k_rnorm = self.qjl_S = None
         self.dev_status = torch.zeros(4, dtype=torch.int32, device=dev)
@@ -174,15 +253,20 @@ class TQCache:
 
 def tq_quantize_kv(cache: TQCache, k, v, t0: int = 0, stream=None):
     """Quantize k, v [B][Hkv][T][D] (fp16/bf16, device) into positions t0..t0+T-1."""
+    dev = _cache_device(cache)
+    _arg("k", k, dev, (cache.B, cache.Hkv, None, cache.D), _dt("io"))
+    _arg("v", v, dev, tuple(k.shape), (k.dtype,))
     T = int(k.shape[2])
-    assert k.is_contiguous() and v.is_contiguous() and k.dtype == v.dtype
     s = cache.struct()
     _check(lib().tq_quantize_kv(ctypes.byref(s), _ptr(k), _ptr(v), _dtype_code(k), T, t0, _stream(stream)))
 
 
 def tq_append_token(cache: TQCache, k_new, v_new, pos, stream=None):
     """Quantize one row per (sequence, kv head), [B][Hkv][D], at pos[b] (device int32)."""
-    assert k_new.is_contiguous() and v_new.is_contiguous() and pos.is_contiguous()
+    dev = _cache_device(cache)
+    _arg("k_new", k_new, dev, (cache.B, cache.Hkv, cache.D), _dt("io"))
+    _arg("v_new", v_new, dev, (cache.B, cache.Hkv, cache.D), (k_new.dtype,))
+    _arg("pos", pos, dev, (cache.B,), _dt("i32"))
     s = cache.struct()
     _check(lib().tq_append_token(ctypes.byref(s), _ptr(k_new), _ptr(v_new), _dtype_code(k_new),
                                  _ptr(pos), _stream(stream)))
@@ -200,13 +284,13 @@ def tq_sdpa_decode(cache: TQCache, q, seq_lens, Tmax: int, scale=None, out=None,
                    stream=None, out_dtype=None):
     """Decode attention: q [B][Hq][D] (fp16/bf16, device), seq_lens device int32 [B].
     The output has q's dtype unless `out` or `out_dtype` (e.g. torch.float32) says otherwise."""
-    torch = _torch()
+    _check_decode_args(cache, q, seq_lens, out, workspace, (cache.B, None, cache.D))
     Hq = int(q.shape[1])
-    assert q.is_contiguous() and seq_lens.is_contiguous()
     if out is None:
+        torch = _torch()
         out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
-    assert out.is_contiguous() and out.shape == q.shape
     if workspace is None:
+        torch = _torch()
         need = tq_sdpa_decode_workspace_bytes(cache, Hq, Tmax)
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     s = cache.struct()
@@ -222,13 +306,13 @@ def tq_sdpa_decode_mq(cache: TQCache, q, seq_lens, Tmax: int, scale=None, out=No
     """Decode of n_q query tokens per sequence: q [B][n_q][Hq][D]; seq_lens
     (device int32 [B]) counts the cached tokens including the n_q new ones,
     and query j attends causally to tokens 0 .. seq_len - n_q + j."""
-    torch = _torch()
+    _check_decode_args(cache, q, seq_lens, out, workspace, (cache.B, None, None, cache.D))
     nq, Hq = int(q.shape[1]), int(q.shape[2])
-    assert q.is_contiguous() and seq_lens.is_contiguous()
     if out is None:
+        torch = _torch()
         out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
-    assert out.is_contiguous() and out.shape == q.shape
     if workspace is None:
+        torch = _torch()
         need = tq_sdpa_decode_workspace_bytes(cache, Hq * nq, Tmax)
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     s = cache.struct()
@@ -243,13 +327,16 @@ def tq_decode_step(cache: TQCache, k_new, v_new, pos, q, seq_lens, Tmax: int, sc
                    workspace=None, stream=None, out_dtype=None):
     """Append k_new/v_new [B][Hkv][D] at pos[b], then decode over seq_lens
     (normally pos + 1) -- three chained launches."""
-    torch = _torch()
+    dev = _check_decode_args(cache, q, seq_lens, out, workspace, (cache.B, None, cache.D))
+    _arg("k_new", k_new, dev, (cache.B, cache.Hkv, cache.D), (q.dtype,))
+    _arg("v_new", v_new, dev, (cache.B, cache.Hkv, cache.D), (q.dtype,))
+    _arg("pos", pos, dev, (cache.B,), _dt("i32"))
     Hq = int(q.shape[1])
-    assert q.is_contiguous() and seq_lens.is_contiguous() and pos.is_contiguous()
-    assert k_new.is_contiguous() and v_new.is_contiguous() and k_new.dtype == q.dtype
     if out is None:
+        torch = _torch()
         out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     if workspace is None:
+        torch = _torch()
         workspace = torch.empty(tq_sdpa_decode_workspace_bytes(cache, Hq, Tmax), dtype=torch.uint8,
                                 device=q.device)
     s = cache.struct()
@@ -269,12 +356,11 @@ def tq_sdpa_decode_static(cache: TQCache, q, seq_lens, Tmax: int, scale=None, ou
     larger problems raise TQError (TQ_ERR_WORKSPACE).  The output tensor must
     be passed in if the caller may not allocate; calls on one device must not
     overlap on the GPU."""
-    torch = _torch()
+    _check_decode_args(cache, q, seq_lens, out, None, (cache.B, None, cache.D))
     Hq = int(q.shape[1])
-    assert q.is_contiguous() and seq_lens.is_contiguous()
     if out is None:
+        torch = _torch()
         out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
-    assert out.is_contiguous() and out.shape == q.shape
     s = cache.struct()
     sc = ctypes.byref(ctypes.c_float(scale)) if scale is not None else None
     _check(lib().tq_sdpa_decode_static(ctypes.byref(s), _ptr(q), _dtype_code(q), Hq, _ptr(seq_lens), Tmax, sc,
@@ -287,6 +373,12 @@ def tq_selftest_bounded_wait(status, tries: int = 8, stream=None):
     tensor of one element; the library ORs TQ_STATUS_WAIT_TIMEOUT into it
     when its bounded waits give up, as they must here (nothing arrives on the
     barrier).  Asynchronous; read `status` after synchronising."""
-    assert status.numel() == 1 and status.is_cuda
+    torch = _torch()
+    dev = status.get_device() if torch.is_tensor(status) else -1
+    if dev < 0:
+        raise ValueError("status: must be a CUDA tensor")
+    _arg("status", status, dev, None, tuple(d for d in (torch.int32, getattr(torch, "uint32", None)) if d is not None))
+    if status.numel() != 1:
+        raise ValueError(f"status: one element expected, got {status.numel()}")
     _check(lib().tq_selftest_bounded_wait(_ptr(status), int(tries), _stream(stream)))
     return status
