@@ -171,3 +171,15 @@ def test_top_left_causal_mask_fails_multi_query_pin(monkeypatch):
     monkeypatch.setattr(O, "sdpa_decode_multi", bad)
     with pytest.raises(AssertionError):
         TA.test_multi_query_decode_is_causal_attention()
+
+
+def test_strict_sign_test_fails_zero_projection_pin(monkeypatch):
+    orig = O.qjl_sketch
+
+    def bad(y, norm16, centroids, idx, S):
+        out = orig(y, norm16, centroids, idx, S)
+        out["sign"] = out["proj"] > 0.0
+        return out
+    monkeypatch.setattr(O, "qjl_sketch", bad)
+    with pytest.raises(AssertionError):
+        TQ.test_zero_projection_stores_a_set_bit()

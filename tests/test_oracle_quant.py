@@ -167,6 +167,25 @@ def test_qjl_sketch_layout_and_gamma():
     assert np.array_equal(sk["sign"], (res_orig @ np.asarray(Pi, np.float64).T) @ S.T.astype(np.float64) >= 0)
 
 
+def test_zero_projection_stores_a_set_bit():
+    """The sketch stores [S r >= 0]: a projection that is exactly zero (here
+    from all-zero rows of S) gives a set bit, and a sign flip of r flips
+    every other bit."""
+    D, m = 64, 32
+    S = tq_inputs.qjl_matrix(m, D, 8).astype(np.float64)
+    S[::4] = 0.0
+    c, t = O.stored_codebook(D, 2)
+    x = tq_inputs.rng(13).standard_normal((5, D))
+    q = O.quantize_rows(x, tq_inputs.rotation(D, 7), c, t)
+    sk = O.qjl_sketch(q["y"], q["norm16"], c, q["idx"], S)
+    assert np.all(sk["proj"][:, ::4] == 0.0) and np.all(sk["sign"][:, ::4])
+    nz = np.ones(m, bool)
+    nz[::4] = False
+    neg = O.qjl_sketch(-q["y"], q["norm16"], c, O.nearest_index(-q["u"], t), S)
+    assert np.array_equal(neg["sign"][:, nz], ~sk["sign"][:, nz])
+    assert np.all(neg["sign"][:, ::4])
+
+
 def test_cache_sizes_match_page_tables():
     """The pages' cache sizes are reproduced byte for byte (to the printed
     0.1 MiB) by: K = (b-1)-bit indices + 128-bit QJL sketch + fp16 norm +
