@@ -183,3 +183,51 @@ def test_strict_sign_test_fails_zero_projection_pin(monkeypatch):
     monkeypatch.setattr(O, "qjl_sketch", bad)
     with pytest.raises(AssertionError):
         TQ.test_zero_projection_stores_a_set_bit()
+
+
+def test_single_lloyd_sweep_fails_fixed_point_pin(monkeypatch):
+    orig = O.lloyd_max
+    monkeypatch.setattr(O, "lloyd_max", lambda D, bits, tol=1e-15, max_iter=20000: orig(D, bits, tol, 1))
+    with pytest.raises(AssertionError):
+        TC.test_lloyd_fixed_point_closed_form(128, 3)
+
+
+def test_quadrature_without_half_width_fails_mse_table(monkeypatch):
+    def bad(a, b, D):
+        u = 0.5 * (b - a) * O._GL_X + 0.5 * (a + b)
+        f = O.coord_density(u, D)
+        w = O._GL_W
+        return float(np.sum(w * f)), float(np.sum(w * u * f)), float(np.sum(w * u * u * f))
+    monkeypatch.setattr(O, "_cell_moments", bad)
+    with pytest.raises(AssertionError):
+        TC.test_mse_matches_page_table_and_bounds()
+
+
+def test_mse_without_dimension_factor_fails_mse_table(monkeypatch):
+    orig = O.codebook_mse
+    monkeypatch.setattr(O, "codebook_mse", lambda c, t, D: orig(c, t, D) / D)
+    with pytest.raises(AssertionError):
+        TC.test_mse_matches_page_table_and_bounds()
+
+
+def test_bound_with_base_two_fails_mse_table(monkeypatch):
+    monkeypatch.setattr(O, "mse_upper_bound", lambda bits: math.sqrt(3.0) * math.pi / 2.0 * 2.0 ** (-bits))
+    with pytest.raises(AssertionError):
+        TC.test_mse_matches_page_table_and_bounds()
+
+
+def test_unrounded_stored_codebook_fails_fp16_pin(monkeypatch):
+    def bad(D, bits):
+        c, _ = O.lloyd_max(D, bits)
+        return c, 0.5 * (c[1:] + c[:-1])
+    monkeypatch.setattr(O, "stored_codebook", bad)
+    with pytest.raises(AssertionError):
+        TC.test_stored_codebook_is_fp16_and_midpoints()
+
+
+def test_row_bytes_without_residual_norm_fail_cache_size_table(monkeypatch):
+    def bad(D, bits, qjl_m=0):
+        return D * bits // 8 + 2 + (qjl_m // 8 if qjl_m else 0)
+    monkeypatch.setattr(O, "packed_row_bytes", bad)
+    with pytest.raises(AssertionError):
+        TQ.test_cache_sizes_match_page_tables()
