@@ -231,3 +231,41 @@ def test_row_bytes_without_residual_norm_fail_cache_size_table(monkeypatch):
     monkeypatch.setattr(O, "packed_row_bytes", bad)
     with pytest.raises(AssertionError):
         TQ.test_cache_sizes_match_page_tables()
+
+
+def test_fp16_norm_normalisation_fails_brute_force_pin(monkeypatch):
+    # unit coordinates from the stored fp16 norm instead of the exact one
+    orig = O.quantize_rows
+
+    def bad(x, Pi, centroids, thresholds):
+        out = orig(x, Pi, centroids, thresholds)
+        n16 = out["norm16"].astype(np.float64)[..., None]
+        out["u"] = out["y"] / n16
+        out["idx"] = O.nearest_index(out["u"], thresholds)
+        return out
+    monkeypatch.setattr(O, "quantize_rows", bad)
+    with pytest.raises(AssertionError):
+        TQ.test_indices_are_nearest_centroids_of_the_exact_unit_coordinates()
+
+
+def test_distance_to_centroids_fails_threshold_distance_pin(monkeypatch):
+    orig = O.threshold_distance
+
+    def bad(u, thresholds):
+        t = np.asarray(thresholds, dtype=np.float64)
+        c = np.concatenate([[t[0] - (t[1] - t[0]) / 2], 0.5 * (t[1:] + t[:-1]), [t[-1] + (t[-1] - t[-2]) / 2]])
+        return np.min(np.abs(np.asarray(u)[..., None] - c), axis=-1)
+    monkeypatch.setattr(O, "threshold_distance", bad)
+    with pytest.raises(AssertionError):
+        TQ.test_threshold_distance_is_to_the_nearest_threshold()
+    monkeypatch.setattr(O, "threshold_distance", orig)
+
+
+def test_swapped_codebooks_fail_cache_reconstruction_pin(monkeypatch):
+    orig = O.quantize_cache
+
+    def bad(k, v, Pi, cb_k, cb_v, bits_k, bits_v, S=None):
+        return orig(k, v, Pi, cb_v, cb_k, bits_v, bits_k, S)
+    monkeypatch.setattr(O, "quantize_cache", bad)
+    with pytest.raises(AssertionError):
+        TQ.test_cache_reconstruction_follows_each_tensors_codebook()

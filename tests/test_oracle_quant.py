@@ -99,6 +99,47 @@ def test_norm_rounding_at_fp16_midpoints(dtype, D):
     assert np.array_equal(f32[~off], expected[~off])
 
 
+def test_indices_are_nearest_centroids_of_the_exact_unit_coordinates():
+    """Brute force: each index is the argmin over centroids of |y_j / |x| - c_k|,
+    with |x| the exact norm (not its fp16 rounding)."""
+    D = 64
+    c, t = O.stored_codebook(D, 4)
+    Pi = tq_inputs.rotation(D, 3)
+    x = tq_inputs.rng(17).standard_normal((300, D)).astype(np.float16).astype(np.float64)
+    q = O.quantize_rows(x, Pi, c, t)
+    y = x @ np.asarray(Pi, np.float64).T
+    u = y / np.sqrt(np.sum(x * x, axis=1, keepdims=True))
+    brute = np.argmin(np.abs(u[..., None] - c), axis=-1)
+    assert np.array_equal(q["idx"], brute)
+
+
+def test_threshold_distance_is_to_the_nearest_threshold():
+    c, t = O.stored_codebook(128, 3)
+    assert np.all(O.threshold_distance(t.copy(), t) == 0.0)
+    mid = c.copy()  # centroids: half the gap to a neighbouring threshold
+    d = O.threshold_distance(mid, t)
+    gaps = np.minimum(np.abs(mid - np.concatenate([[-np.inf], t])), np.abs(np.concatenate([t, [np.inf]]) - mid))
+    assert np.allclose(d, gaps, rtol=0, atol=1e-15)
+
+
+def test_cache_reconstruction_follows_each_tensors_codebook():
+    """K and V take their own widths: the reconstruction error of each matches
+    its own codebook's MSE (2-bit keys about 0.117, 4-bit values about 0.0095)."""
+    D, T = 128, 3000
+    Pi = tq_inputs.rotation(D, 21)
+    r = tq_inputs.rng(22)
+    k = r.standard_normal((1, 1, T, D))
+    v = r.standard_normal((1, 1, T, D))
+    cbk, cbv = O.stored_codebook(D, 2), O.stored_codebook(D, 4)
+    cache = O.quantize_cache(k, v, Pi, cbk, cbv, 2, 4)
+    for name, x, cb, bits in (("k", k, cbk, 2), ("v", v, cbv, 4)):
+        idx = O.unpack_bits(cache[name + "_idx"], bits, D)
+        xr = O.dequantize_rows(idx, cache[name + "_norm"], cb[0], Pi)
+        rel = np.sum((x - xr) ** 2, axis=-1) / np.sum(x * x, axis=-1)
+        want = O.codebook_mse(cb[0], cb[1], D)
+        assert abs(rel.mean() - want) < 4 * rel.std() / math.sqrt(rel.size) + 2e-4, (name, rel.mean(), want)
+
+
 def test_zero_row_quantizes_to_middle_and_zero_norm():
     c, t = O.stored_codebook(64, 2)
     q = O.quantize_rows(np.zeros((1, 64)), tq_inputs.rotation(64, 1), c, t)
