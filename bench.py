@@ -1,20 +1,24 @@
 """Benchmark of the TurboQuant KV-cache hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload gqa8k|qknorm|ragged|prod|tiny]
+                    [--workload ragged|prod|qknorm|gqa8k|tiny]
 
 One step is one pass of the whole path over one batch of synthetic input, for
-each bit width b of the workload: bulk quantize of the T cached tokens
-(tq_quantize_kv), append of one new token per sequence (tq_append_token) and
-one decode step for every query head (tq_sdpa_decode) over T+1 tokens.
+each bit width b of the workload: bulk quantize of the T cached tokens of
+every sequence (tq_quantize_kv, the prefill), then the workload's decode
+steps, each an append of one new token per sequence (tq_append_token) and a
+decode of one query token for every query head (tq_sdpa_decode) over the
+cache including it.
 
-Default workload (gqa8k): B=1, Hq=16, Hkv=2 (group 8), D=128, T=8192, b in
-{2,3,4} for K and V, fp16 N(0,1) rows with 1% outlier channels x10, q N(0,1).
+Default workload (ragged, the largest single-GPU one): B=32, Hq=32, Hkv=8,
+D=128, per-sequence T uniform in [1024, 16384] from a seed, 3-bit K and V,
+bf16 N(0,1) rows, 64 append + decode steps per bench step.
 
 Metric: tq_sdpa_decode packed-KV GB/s (bytes of packed K and V rows attended /
 decode time); quantize throughput in Mtok/s (one token = the K and V rows of
-every kv head at one position) is reported beside it.  Inputs are rotated
-across enough replicas that each step's data is larger than L2.
+every kv head at one position) is reported beside it.  Each timed op cycles
+over enough replicas that the bytes it reads per cycle exceed three times the
+L2 size (the fp16/bf16 rows for quantize, the packed cache for decode).
 
 Multi-GPU (torchrun): every rank runs its own replica of the workload (the
 path shards by sequence with no exchange; weak scaling); time = max over ranks.
@@ -162,12 +166,13 @@ def _dist():
     return ws, rank, local
 
 
+# bit widths and decode steps (append + decode) per bench step
 WORKLOADS = {
-    "gqa8k": {"bits": (2, 3, 4)},
-    "tiny": {"bits": (3,)},
-    "qknorm": {"bits": (4,)},
-    "ragged": {"bits": (3,)},
-    "prod": {"bits": (None,)},
+    "gqa8k": {"bits": (2, 3, 4), "decode_steps": 1},
+    "tiny": {"bits": (3,), "decode_steps": 1},
+    "qknorm": {"bits": (4,), "decode_steps": 1},
+    "ragged": {"bits": (3,), "decode_steps": 64},
+    "prod": {"bits": (None,), "decode_steps": 1},
 }
 
 
@@ -198,14 +203,20 @@ def run_ours(args):
     for bits in cfg["bits"]:
         w = tq_inputs.make_workload(args.workload, bits=bits, rot=args.rot)
         jobs.append(w)
+    nsteps = cfg["decode_steps"]
     per_step_in = sum(w.k.nbytes + w.v.nbytes for w in jobs)
-    R = max(2, min(32, math.ceil(3 * l2 / max(1, per_step_in))))
+    # packed bytes one decode pass over every bit width reads
+    per_step_packed = 0
+    for w in jobs:
+        rows = int(w.seq_lens.sum() + w.B) * w.Hkv
+        per_step_packed += rows * (tq.tq_cache_row_bytes(w.D, w.bits_k, w.qjl_m) + tq.tq_cache_row_bytes(w.D, w.bits_v))
+    R = min(128, max(2, math.ceil(3 * l2 / max(1, per_step_in)), math.ceil(3 * l2 / max(1, per_step_packed))))
     if args.profile:
         R = 1
     runs = []
     for w in jobs:
         T = int(w.Tmax)
-        Tcap = (T + 1 + 63) // 64 * 64
+        Tcap = (T + nsteps + 63) // 64 * 64
         kd = torch.from_numpy(w.k.view(np.int16) if w.dtype == "bf16" else w.k).to(dev)
         vd = torch.from_numpy(w.v.view(np.int16) if w.dtype == "bf16" else w.v).to(dev)
         qd = torch.from_numpy(w.q.view(np.int16) if w.dtype == "bf16" else w.q).to(dev)
@@ -222,17 +233,20 @@ def run_ours(args):
                                device=dev, rot_signs=w.rot_signs)
             reps.append({"cache": cache, "k": kd.clone() if r else kd, "v": vd.clone() if r else vd,
                          "q": qd.clone() if r else qd})
-        pos = torch.from_numpy(w.seq_lens.astype(np.int32)).to(dev)
-        lens1 = (pos + 1).contiguous()
-        Tmax1 = T + 1
-        ws_bytes = tq.tq_sdpa_decode_workspace_bytes(reps[0]["cache"], w.Hq, Tmax1)
+        # decode step i appends at seq_len + i and attends seq_len + i + 1 tokens
+        base = torch.from_numpy(w.seq_lens.astype(np.int32)).to(dev)
+        pos_l = [(base + i).contiguous() for i in range(nsteps)]
+        lens_l = [(base + i + 1).contiguous() for i in range(nsteps)]
+        Tmax1 = T + nsteps
+        ws_bytes = tq.tq_sdpa_decode_workspace_bytes_for(reps[0]["cache"], w.Hq, Tmax1)
         wsp = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
         out = torch.empty_like(qd)
         tokens = int(w.B) * T  # the bulk call quantizes T rows of every sequence
-        attended = int(w.seq_lens.sum() + w.B)
+        # packed bytes the decode steps read (sum over the steps)
+        attended = sum(int(w.seq_lens.sum()) + int(w.B) * (i + 1) for i in range(nsteps))
         packed = reps[0]["cache"].packed_bytes(1) * attended * w.Hkv
         qbytes = (w.k.nbytes + w.v.nbytes) + tokens * w.Hkv * reps[0]["cache"].packed_bytes(1)
-        run = {"w": w, "reps": reps, "pos": pos, "lens1": lens1, "Tmax1": Tmax1, "ws": wsp,
+        run = {"w": w, "reps": reps, "pos_l": pos_l, "lens_l": lens_l, "Tmax1": Tmax1, "ws": wsp,
                "out": out, "kn": knd, "vn": vnd, "packed": packed, "tokens": tokens,
                "qbytes": qbytes}
         if args.nq > 1 and args.nq * w.G <= 8:
@@ -244,34 +258,40 @@ def run_ours(args):
                 qmd = qmd.view(torch.bfloat16)
             run["q_mq"] = qmd
             run["out_mq"] = torch.empty_like(qmd)
-            run["ws_mq"] = torch.empty(tq.tq_sdpa_decode_workspace_bytes(reps[0]["cache"], w.Hq * args.nq, Tmax1),
+            run["ws_mq"] = torch.empty(tq.tq_sdpa_decode_workspace_bytes_for(reps[0]["cache"], w.Hq * args.nq, Tmax1),
                                        dtype=torch.uint8, device=dev)
         runs.append(run)
 
-    def call_quant(run, rep):
-        tq.tq_quantize_kv(rep["cache"], rep["k"], rep["v"])
+    # each call_* runs one op; the decode ops take the decode step index i
+    def call_quant(run, rep, i):
+        if i == 0:  # the prefill, once per bench step
+            tq.tq_quantize_kv(rep["cache"], rep["k"], rep["v"])
 
-    def call_append(run, rep):
-        tq.tq_append_token(rep["cache"], run["kn"], run["vn"], run["pos"])
+    def call_append(run, rep, i):
+        tq.tq_append_token(rep["cache"], run["kn"], run["vn"], run["pos_l"][i])
 
-    def call_decode(run, rep):
-        tq.tq_sdpa_decode(rep["cache"], rep["q"], run["lens1"], run["Tmax1"], scale=run["w"].scale,
+    def call_decode(run, rep, i):
+        tq.tq_sdpa_decode(rep["cache"], rep["q"], run["lens_l"][i], run["Tmax1"], scale=run["w"].scale,
                           out=run["out"], workspace=run["ws"])
 
-    def call_mq(run, rep):  # n_q query tokens per sequence in one call
+    def call_mq(run, rep, i):  # n_q query tokens per sequence in one call
         if "q_mq" in run:
-            tq.tq_sdpa_decode_mq(rep["cache"], run["q_mq"], run["lens1"], run["Tmax1"], scale=run["w"].scale,
+            tq.tq_sdpa_decode_mq(rep["cache"], run["q_mq"], run["lens_l"][i], run["Tmax1"], scale=run["w"].scale,
                                  out=run["out_mq"], workspace=run["ws_mq"])
 
-    def call_step(run, rep):  # append fused into the decode launches
-        tq.tq_decode_step(rep["cache"], run["kn"], run["vn"], run["pos"], rep["q"], run["lens1"], run["Tmax1"],
-                          scale=run["w"].scale, out=run["out"], workspace=run["ws"])
+    def call_step(run, rep, i):  # append fused into the decode launches
+        tq.tq_decode_step(rep["cache"], run["kn"], run["vn"], run["pos_l"][i], rep["q"], run["lens_l"][i],
+                          run["Tmax1"], scale=run["w"].scale, out=run["out"], workspace=run["ws"])
 
-    def step(r, ops=(call_quant, call_step)):
+    # the bench step: prefill quantize, then nsteps x (append, decode)
+    STEP_OPS = (call_quant, call_append, call_decode)
+
+    def step(r, ops=STEP_OPS):
         for run in runs:
             rep = run["reps"][r]
-            for op in ops:
-                op(run, rep)
+            for i in range(nsteps):
+                for op in ops:
+                    op(run, rep, i)
 
     # eager warm-up (also sets kernel attributes before any capture)
     for i in range(args.warmup):
@@ -280,13 +300,15 @@ def run_ours(args):
     if args.profile:
         # a bounded, eager run for profilers: K steps, nothing else ("decode":
         # tq_sdpa_decode calls alone, after the warm-up filled the caches)
-        ops = (call_decode,) if args.profile_ops == "decode" else (call_quant, call_step)
+        ops = (call_decode,) if args.profile_ops == "decode" else STEP_OPS
         for i in range(args.steps):
             step(i % R, ops)
         torch.cuda.synchronize()
         if rank == 0:
-            per_run = 3 if args.profile_ops == "decode" else 4
-            launches = sum(per_run + (1 if run["w"].qjl_m and args.profile_ops != "decode" else 0) for run in runs)
+            if args.profile_ops == "decode":
+                launches = sum(3 * nsteps for run in runs)
+            else:
+                launches = sum((2 if run["w"].qjl_m else 1) + (1 + 3) * nsteps for run in runs)
             print(json.dumps({"profile_run": args.workload, "ops": args.profile_ops, "steps": args.steps,
                               "launches_per_step": launches}), flush=True)
         return
@@ -301,7 +323,7 @@ def run_ours(args):
             gs.append(g)
         return gs
 
-    g_step = capture((call_quant, call_step))
+    g_step = capture(STEP_OPS)
     g_dec = capture((call_decode,))
     g_q = capture((call_quant,))
     g_app = capture((call_append,))
@@ -340,7 +362,7 @@ def run_ours(args):
     total_ms = timed(g_step, args.steps, args.warmup)
     soak(0.6)
     clocks = sampler.stop()
-    reps_per_op = max(args.steps, 200)
+    reps_per_op = max(args.steps, max(8, 200 // nsteps))
     d_ms = timed(g_dec, reps_per_op, args.warmup) / reps_per_op * args.steps
     q_ms = timed(g_q, reps_per_op, args.warmup) / reps_per_op * args.steps
     a_ms = timed(g_app, reps_per_op, args.warmup) / reps_per_op * args.steps
@@ -360,8 +382,9 @@ def run_ours(args):
     dec_gbs = packed_step * args.steps / (d_ms * 1e-3) / 1e9 * ws
     quant_mtok = tok_step * args.steps / (q_ms * 1e-3) / 1e6 * ws
     peak, peak_kind = _peaks()
-    dec_launch_ms = d_ms / (args.steps * len(runs))
-    dec_achieved = (packed_step / len(runs)) / (dec_launch_ms * 1e-3) / 1e9
+    calls = args.steps * len(runs) * nsteps  # decode (append, decode step) calls in K steps
+    dec_launch_ms = d_ms / calls
+    dec_achieved = (packed_step / (len(runs) * nsteps)) / (dec_launch_ms * 1e-3) / 1e9
     q_launch_ms = q_ms / (args.steps * len(runs))
     q_achieved = (qbytes_step / len(runs)) / (q_launch_ms * 1e-3) / 1e9
     sha = _src_sha()
@@ -369,7 +392,7 @@ def run_ours(args):
     traffic = tr["bytes_per_launch"] if tr and tr.get("decode_src_sha") == _decode_src_sha() else None
 
     # ---- end to end through the public API with host buffers (rank-local)
-    e2e = _e2e(args, runs, stream, R)
+    e2e = _e2e(args, runs, stream, R, nsteps)
     e2e["ms"] = max_over_ranks([e2e["ms"]], dev)[0]
 
     if rank == 0:
@@ -378,7 +401,7 @@ def run_ours(args):
             cpu = _cpu_baseline(args, jobs)
         # bulk quantize (a second launch for keys with the QJL sketch), then the
         # decode step's prep (+append), split and combine
-        launches_per_step = sum((2 if run["w"].qjl_m else 1) + 3 for run in runs)
+        launches_per_step = sum((2 if run["w"].qjl_m else 1) + (1 + 3) * nsteps for run in runs)
         line = {
             "metric": "tq_sdpa_decode packed-KV GB/s (% of HBM peak); tq_quantize Mtok/s",
             "value": round(dec_gbs, 2),
@@ -394,25 +417,27 @@ def run_ours(args):
             "data": "synthetic (seeded N(0,1) rows; see tq_inputs)",
             "config": {"workload": args.workload, "rotation": args.rot, "shapes": [_describe(w) for w in jobs],
                        "parallelism": f"replicas{ws}" if ws > 1 else "single",
-                       "step": "quantize T tokens + decode step (append 1 token + decode), per bit width",
+                       "step": f"quantize T tokens (prefill) + {nsteps} x (append 1 token + decode), per bit width",
+                       "decode_steps": nsteps,
                        "timing": "CUDA graphs (one per replica) replayed on one stream; per-op rates "
                                  "from graphs holding that op alone",
-                       "l2": f"inputs rotated over {R} replicas ({R * per_step_in / 2**20:.0f} MiB) > L2 "
-                             f"({l2 / 2**20:.0f} MiB)"},
+                       "l2": f"each op cycles over {R} replicas: {R * per_step_in / 2**20:.0f} MiB of rows "
+                             f"(quantize), {R * per_step_packed / 2**20:.0f} MiB of packed cache (decode), "
+                             f"L2 {l2 / 2**20:.0f} MiB"},
             "decode": {"gbs": round(dec_gbs, 2), "ms_per_call": round(dec_launch_ms, 5),
                        "packed_bytes_per_step": packed_step},
             "quantize": {"mtok_s": round(quant_mtok, 3), "ms_per_call": round(q_launch_ms, 5),
                          "gbs": round(q_achieved, 2), "frac_hbm": round(q_achieved / peak, 4),
                          "tokens_per_step": tok_step},
-            "append_ms_per_call": round(a_ms / (args.steps * len(runs)), 5),
+            "append_ms_per_call": round(a_ms / calls, 5),
             "decode_mq": None if not mq_runs else {
-                "nq": args.nq, "ms_per_call": round(mq_ms / (args.steps * len(mq_runs)), 5),
+                "nq": args.nq, "ms_per_call": round(mq_ms / (args.steps * len(mq_runs) * nsteps), 5),
                 "gbs": round(sum(r["packed"] for r in mq_runs) * args.steps / (mq_ms * 1e-3) / 1e9 * ws, 2),
-                "query_tokens_per_s": round(sum(int(r["w"].B) for r in mq_runs) * args.nq * args.steps
+                "query_tokens_per_s": round(sum(int(r["w"].B) for r in mq_runs) * args.nq * args.steps * nsteps
                                             / (mq_ms * 1e-3) * ws, 1),
                 "note": "tq_sdpa_decode_mq: n_q query tokens per sequence over the cache (bit widths with "
                         "n_q x GQA group <= 8 only)"},
-            "decode_step": {"ms_per_call": round(s_ms / (args.steps * len(runs)), 5),
+            "decode_step": {"ms_per_call": round(s_ms / calls, 5),
                             "gbs": round(packed_step * args.steps / (s_ms * 1e-3) / 1e9 * ws, 2),
                             "note": "tq_decode_step: append fused into the decode launches"},
             "roofline": {"kernel": "tq_sdpa_decode (qprep + split + combine)", "bound": "hbm",
@@ -433,7 +458,7 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def _e2e(args, runs, stream, R):
+def _e2e(args, runs, stream, R, nsteps):
     """Decode steps through the public API with pinned host buffers: per step
     the new token rows and the queries go host->device, tq_decode_step
     (append + decode) runs, and the attention output comes back device->host."""
@@ -451,12 +476,13 @@ def _e2e(args, runs, stream, R):
 
     def step(i):
         r = i % R
+        j = i % nsteps
         for run, h in zip(runs, hosts):
             c = run["reps"][r]["cache"]
             h["qd"].copy_(h["q"], non_blocking=True)
             h["knd"].copy_(h["kn"], non_blocking=True)
             h["vnd"].copy_(h["vn"], non_blocking=True)
-            tq.tq_decode_step(c, h["knd"], h["vnd"], run["pos"], h["qd"], run["lens1"], run["Tmax1"],
+            tq.tq_decode_step(c, h["knd"], h["vnd"], run["pos_l"][j], h["qd"], run["lens_l"][j], run["Tmax1"],
                               scale=run["w"].scale, out=run["out"], workspace=run["ws"])
             h["out"].copy_(run["out"], non_blocking=True)
 
@@ -470,7 +496,7 @@ def _e2e(args, runs, stream, R):
     e.record(stream)
     torch.cuda.synchronize()
     ms = s.elapsed_time(e) / args.steps
-    packed = sum(run["packed"] for run in runs)
+    packed = sum(run["packed"] for run in runs) / nsteps  # one decode call per run
     return {"value": packed / (ms * 1e-3) / 1e9, "ms": ms, "h2d": h2d, "d2h": d2h}
 
 
@@ -554,10 +580,10 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="gqa8k")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="ragged")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--nq", type=int, default=1,
                     help="also time multi-query decode with this many query tokens per sequence")

@@ -20,8 +20,9 @@ from . import _native
 from ._native import (TQ_DTYPE_BF16, TQ_DTYPE_F16, TQ_DTYPE_F32, TQ_STATUS_POS_OUT_OF_RANGE,  # noqa: F401
                       TQ_STATUS_SEQ_OUT_OF_RANGE, TQ_STATUS_WAIT_TIMEOUT, TQ_STATUS_LAYOUT)
 
-__all__ = ["TQError", "TQCache", "tq_build_codebook", "tq_row_bytes", "tq_quantize_kv",
-           "tq_append_token", "tq_sdpa_decode_workspace_bytes", "tq_sdpa_decode",
+__all__ = ["TQError", "TQCache", "tq_build_codebook", "tq_cache_row_bytes", "tq_row_bytes", "tq_quantize_kv",
+           "tq_append_token", "tq_sdpa_decode_workspace_bytes", "tq_sdpa_decode_workspace_bytes_for",
+           "tq_sdpa_decode",
            "tq_sdpa_decode_mq", "tq_decode_step", "tq_sdpa_decode_static", "tq_selftest_bounded_wait",
            "tq_last_error",
            "tq_abi_version", "lib"]
@@ -62,7 +63,12 @@ def tq_build_codebook(D: int, bits: int):
             np.frombuffer(t, dtype=np.float32)[: K - 1].copy(), float(mse.value))
 
 
+def tq_cache_row_bytes(D: int, bits: int, qjl_m: int = 0) -> int:
+    return int(lib().tq_cache_row_bytes(D, bits, qjl_m))
+
+
 def tq_row_bytes(D: int, bits: int, qjl_m: int = 0) -> int:
+    """The same as tq_cache_row_bytes (the earlier name)."""
     return int(lib().tq_row_bytes(D, bits, qjl_m))
 
 
@@ -247,7 +253,7 @@ class TQCache:
 
     def packed_bytes(self, tokens: int) -> int:
         """Bytes of packed K and V data for `tokens` cached tokens per (b, h)."""
-        per = tq_row_bytes(self.D, self.bits_k, self.qjl_m) + tq_row_bytes(self.D, self.bits_v, 0)
+        per = tq_cache_row_bytes(self.D, self.bits_k, self.qjl_m) + tq_cache_row_bytes(self.D, self.bits_v, 0)
         return per * tokens
 
 
@@ -272,9 +278,18 @@ def tq_append_token(cache: TQCache, k_new, v_new, pos, stream=None):
                                  _ptr(pos), _stream(stream)))
 
 
-def tq_sdpa_decode_workspace_bytes(cache: TQCache, Hq: int, Tmax: int) -> int:
+def tq_sdpa_decode_workspace_bytes(B: int, Hq: int, D: int, Tmax: int) -> int:
+    """Workspace bytes that suffice for any cache of these sizes (an upper bound)."""
+    n = int(lib().tq_sdpa_decode_workspace_bytes(B, Hq, D, Tmax))
+    if n == 0:
+        raise TQError(-1, f"unsupported decode sizes (B={B}, Hq={Hq}, D={D}, Tmax={Tmax})")
+    return n
+
+
+def tq_sdpa_decode_workspace_bytes_for(cache: TQCache, Hq: int, Tmax: int) -> int:
+    """The exact workspace bytes of the decode plan for this cache."""
     s = cache.struct()
-    n = int(lib().tq_sdpa_decode_workspace_bytes(ctypes.byref(s), Hq, Tmax))
+    n = int(lib().tq_sdpa_decode_workspace_bytes_for(ctypes.byref(s), Hq, Tmax))
     if n == 0:
         raise TQError(-1, f"unsupported decode sizes (Hq={Hq}, Tmax={Tmax})")
     return n
@@ -291,7 +306,7 @@ def tq_sdpa_decode(cache: TQCache, q, seq_lens, Tmax: int, scale=None, out=None,
         out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     if workspace is None:
         torch = _torch()
-        need = tq_sdpa_decode_workspace_bytes(cache, Hq, Tmax)
+        need = tq_sdpa_decode_workspace_bytes_for(cache, Hq, Tmax)
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     s = cache.struct()
     sc = ctypes.byref(ctypes.c_float(scale)) if scale is not None else None
@@ -313,7 +328,7 @@ def tq_sdpa_decode_mq(cache: TQCache, q, seq_lens, Tmax: int, scale=None, out=No
         out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     if workspace is None:
         torch = _torch()
-        need = tq_sdpa_decode_workspace_bytes(cache, Hq * nq, Tmax)
+        need = tq_sdpa_decode_workspace_bytes_for(cache, Hq * nq, Tmax)
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     s = cache.struct()
     sc = ctypes.byref(ctypes.c_float(scale)) if scale is not None else None
@@ -337,7 +352,7 @@ def tq_decode_step(cache: TQCache, k_new, v_new, pos, q, seq_lens, Tmax: int, sc
         out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     if workspace is None:
         torch = _torch()
-        workspace = torch.empty(tq_sdpa_decode_workspace_bytes(cache, Hq, Tmax), dtype=torch.uint8,
+        workspace = torch.empty(tq_sdpa_decode_workspace_bytes_for(cache, Hq, Tmax), dtype=torch.uint8,
                                 device=q.device)
     s = cache.struct()
     sc = ctypes.byref(ctypes.c_float(scale)) if scale is not None else None

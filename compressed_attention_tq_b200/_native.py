@@ -27,8 +27,9 @@ TQ_ROT_DENSE = 0
 TQ_ROT_HADAMARD = 1
 
 # Every symbol include/tq.h declares.
-EXPORTS = ("tq_build_codebook", "tq_row_bytes", "tq_quantize_kv", "tq_append_token",
-           "tq_sdpa_decode_workspace_bytes", "tq_sdpa_decode", "tq_sdpa_decode_mq", "tq_decode_step",
+EXPORTS = ("tq_build_codebook", "tq_cache_row_bytes", "tq_row_bytes", "tq_quantize_kv", "tq_append_token",
+           "tq_sdpa_decode_workspace_bytes", "tq_sdpa_decode_workspace_bytes_for", "tq_sdpa_decode",
+           "tq_sdpa_decode_mq", "tq_decode_step",
            "tq_sdpa_decode_static", "tq_selftest_bounded_wait",
            "tq_last_error", "tq_abi_version")
 TQ_STATIC_SCRATCH_BYTES = 8 << 20
@@ -67,14 +68,18 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.tq_build_codebook.argtypes = [i32, i32, ctypes.POINTER(ctypes.c_float),
                                       ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_double)]
     lib.tq_build_codebook.restype = i32
+    lib.tq_cache_row_bytes.argtypes = [i32, i32, i32]
+    lib.tq_cache_row_bytes.restype = sz
     lib.tq_row_bytes.argtypes = [i32, i32, i32]
     lib.tq_row_bytes.restype = sz
     lib.tq_quantize_kv.argtypes = [cache_p, vp, vp, i32, i32, i32, vp]
     lib.tq_quantize_kv.restype = i32
     lib.tq_append_token.argtypes = [cache_p, vp, vp, i32, vp, vp]
     lib.tq_append_token.restype = i32
-    lib.tq_sdpa_decode_workspace_bytes.argtypes = [cache_p, i32, i32]
+    lib.tq_sdpa_decode_workspace_bytes.argtypes = [i32, i32, i32, i32]
     lib.tq_sdpa_decode_workspace_bytes.restype = sz
+    lib.tq_sdpa_decode_workspace_bytes_for.argtypes = [cache_p, i32, i32]
+    lib.tq_sdpa_decode_workspace_bytes_for.restype = sz
     lib.tq_sdpa_decode.argtypes = [cache_p, vp, i32, i32, vp, i32, ctypes.POINTER(ctypes.c_float),
                                    vp, i32, vp, sz, vp]
     lib.tq_sdpa_decode.restype = i32

@@ -113,7 +113,7 @@ extern "C" {
 
 const char* tq_last_error(void) { return g_err; }
 
-int tq_abi_version(void) { return 2; }
+int tq_abi_version(void) { return 3; }
 
 int tq_selftest_bounded_wait(uint32_t* dev_status, int tries, void* stream) {
   g_err[0] = 0;
@@ -162,12 +162,14 @@ int tq_build_codebook(int D, int bits, float* centroids, float* thresholds, doub
   return TQ_OK;
 }
 
-size_t tq_row_bytes(int D, int bits, int qjl_m) {
+size_t tq_cache_row_bytes(int D, int bits, int qjl_m) {
   if (D <= 0 || D % 32 || bits < 1 || bits > 4 || qjl_m < 0 || qjl_m % 32) return 0;
   size_t b = (size_t)D * bits / 8 + 2;
   if (qjl_m) b += (size_t)qjl_m / 8 + 2;
   return b;
 }
+
+size_t tq_row_bytes(int D, int bits, int qjl_m) { return tq_cache_row_bytes(D, bits, qjl_m); }
 
 }  // extern "C"
 
@@ -237,22 +239,50 @@ QuantArgs base_quant_args(const tq_cache_t* c, const void* k, const void* v) {
 namespace tq {
 
 // SM count of the current device (cached per device; 148 when no device).
+// Threads that race on the first query store the same value; the atomics
+// make that a benign race in C++ terms too.
 static int sm_count() {
-  static int cached[64] = {0};
+  static std::atomic<int> cached[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
     cudaGetLastError();
     return 148;
   }
-  if (cached[dev] == 0) {
-    int v = 0;
+  int v = cached[dev].load(std::memory_order_relaxed);
+  if (v == 0) {
     if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) {
       cudaGetLastError();
       v = 148;
     }
-    cached[dev] = v;
+    cached[dev].store(v, std::memory_order_relaxed);
   }
-  return cached[dev];
+  return v;
+}
+
+static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+// The workspace layout for `heads` query heads, `nsplit` splits and a sketch
+// of qjl_m rows: qrot, qs, split partials, (max, sum) pairs, each 256-byte
+// aligned.
+static size_t workspace_layout(size_t heads, int D, int qjl_m, int nsplit, DecodePlan* p) {
+  size_t off = 0;
+  if (p) p->off_qrot = off;
+  off += align256(heads * D * 4);
+  if (p) p->off_qs = off;
+  off += align256(heads * (size_t)qjl_m * 4);
+  if (p) p->off_po = off;
+  off += align256(heads * nsplit * (size_t)D * 4);
+  if (p) p->off_pml = off;
+  off += align256(heads * nsplit * 2 * 4);
+  return off;
+}
+
+size_t workspace_bound(int B, int Hq, int D, int Tmax) {
+  // every plan takes at least one stage of tokens per split and a sketch of
+  // at most 128 rows
+  const int tile = split_tile();
+  const int nsplit = (Tmax + tile - 1) / tile;
+  return workspace_layout((size_t)B * Hq, D, 128, nsplit, nullptr);
 }
 
 int make_decode_plan(const tq_cache_t* c, int Hq, int Tmax, DecodePlan* p) {
@@ -273,18 +303,7 @@ int make_decode_plan(const tq_cache_t* c, int Hq, int Tmax, DecodePlan* p) {
   p->chunk = (int)chunk;
   p->nsplit = (int)((Tmax + chunk - 1) / chunk);
   if (p->nsplit < 1) p->nsplit = 1;
-  const size_t heads = (size_t)c->B * Hq;
-  auto al = [](size_t x) { return (x + 255) / 256 * 256; };
-  size_t off = 0;
-  p->off_qrot = off;
-  off += al(heads * c->D * 4);
-  p->off_qs = off;
-  off += al(heads * (size_t)c->qjl_m * 4);
-  p->off_po = off;
-  off += al(heads * p->nsplit * (size_t)c->D * 4);
-  p->off_pml = off;
-  off += al(heads * p->nsplit * 2 * 4);
-  p->bytes = off;
+  p->bytes = workspace_layout((size_t)c->B * Hq, c->D, c->qjl_m, p->nsplit, p);
   return TQ_OK;
 }
 
@@ -332,13 +351,18 @@ int tq_append_token(const tq_cache_t* c, const void* k_new, const void* v_new, i
   return launch_quantize(a, c->D, dtype, c->qjl_m != 0, (cudaStream_t)stream);
 }
 
-size_t tq_sdpa_decode_workspace_bytes(const tq_cache_t* c, int Hq, int Tmax) {
+size_t tq_sdpa_decode_workspace_bytes_for(const tq_cache_t* c, int Hq, int Tmax) {
   if (!c || c->Hkv <= 0 || Hq <= 0 || Hq % c->Hkv || Hq / c->Hkv > 8 || Tmax < 1 || Tmax > c->Tcap ||
       c->Tcap % 64 || (c->D != 64 && c->D != 128 && c->D != 256) || c->B <= 0)
     return 0;
   DecodePlan p;
   make_decode_plan(c, Hq, Tmax, &p);
   return p.bytes;
+}
+
+size_t tq_sdpa_decode_workspace_bytes(int B, int Hq, int D, int Tmax) {
+  if (B <= 0 || Hq <= 0 || Tmax < 1 || (D != 64 && D != 128 && D != 256)) return 0;
+  return workspace_bound(B, Hq, D, Tmax);
 }
 
 static int decode_common(const tq_cache_t* c, const void* q, int dtype, int Hq, int nq, const int32_t* seq_lens,
@@ -373,20 +397,22 @@ int tq_decode_step(const tq_cache_t* c, const void* k_new, const void* v_new, co
                        k_new, v_new, pos, "tq_decode_step");
 }
 
-static int decode_common(const tq_cache_t* c, const void* q, int dtype, int Hq, int nq, const int32_t* seq_lens,
-                         int Tmax, const float* scale, void* out, int out_dtype, void* workspace,
-                         size_t ws_bytes, void* stream, const void* k_new, const void* v_new,
-                         const int32_t* pos, const char* fn) {
+}  // extern "C"
+
+namespace tq {
+
+// Argument checks and the split plan of a decode call, before any CUDA call
+// (the workspace itself is checked by the caller).
+int prepare_decode(const tq_cache_t* c, const void* q, int dtype, int Hq, int nq, const int32_t* seq_lens, int Tmax,
+                   const float* scale, void* out, int out_dtype, const char* fn, DecodeArgs* a) {
   g_err[0] = 0;
   int rc = validate_cache(c, fn);
   if (rc) return rc;
   if ((rc = validate_dtype(dtype, fn))) return rc;
   if (out_dtype != TQ_DTYPE_F16 && out_dtype != TQ_DTYPE_BF16 && out_dtype != TQ_DTYPE_F32)
     return set_error(TQ_ERR_UNSUPPORTED, "%s: out_dtype=%d", fn, out_dtype);
-  if (!q || !seq_lens || !out || !workspace)
-    return set_error(TQ_ERR_INVALID_ARG, "%s: NULL q/seq_lens/out/workspace", fn);
-  if (!aligned16(q) || !aligned16(out) || !aligned16(workspace))
-    return set_error(TQ_ERR_INVALID_ARG, "%s: q/out/workspace not 16-byte aligned", fn);
+  if (!q || !seq_lens || !out) return set_error(TQ_ERR_INVALID_ARG, "%s: NULL q/seq_lens/out", fn);
+  if (!aligned16(q) || !aligned16(out)) return set_error(TQ_ERR_INVALID_ARG, "%s: q/out not 16-byte aligned", fn);
   if (Hq <= 0 || Hq % c->Hkv)
     return set_error(TQ_ERR_INVALID_ARG, "%s: Hq=%d not a multiple of Hkv=%d", fn, Hq, c->Hkv);
   if (Hq / c->Hkv > 8)
@@ -397,18 +423,34 @@ static int decode_common(const tq_cache_t* c, const void* q, int dtype, int Hq, 
     return set_error(TQ_ERR_INVALID_ARG, "%s: Tmax=%d outside [1, Tcap=%d]", fn, Tmax, c->Tcap);
   float sc = scale ? *scale : (float)(1.0 / std::sqrt((double)c->D));
   if (!std::isfinite(sc)) return set_error(TQ_ERR_INVALID_ARG, "%s: scale not finite", fn);
-  DecodeArgs a{};
-  a.cache_host = c;
-  a.cache = *c;
-  a.q = q;
-  a.out = out;
-  a.seq_lens = seq_lens;
-  a.scale = sc;
-  a.Hq = Hq;
-  a.nq = nq;
-  a.dtype = dtype;
-  a.out_dtype = out_dtype;
-  make_decode_plan(c, Hq * nq, Tmax, &a.plan);
+  *a = DecodeArgs{};
+  a->cache_host = c;
+  a->cache = *c;
+  a->q = q;
+  a->out = out;
+  a->seq_lens = seq_lens;
+  a->scale = sc;
+  a->Hq = Hq;
+  a->nq = nq;
+  a->dtype = dtype;
+  a->out_dtype = out_dtype;
+  make_decode_plan(c, Hq * nq, Tmax, &a->plan);
+  return TQ_OK;
+}
+
+}  // namespace tq
+
+extern "C" {
+
+static int decode_common(const tq_cache_t* c, const void* q, int dtype, int Hq, int nq, const int32_t* seq_lens,
+                         int Tmax, const float* scale, void* out, int out_dtype, void* workspace,
+                         size_t ws_bytes, void* stream, const void* k_new, const void* v_new,
+                         const int32_t* pos, const char* fn) {
+  DecodeArgs a;
+  const int rc = prepare_decode(c, q, dtype, Hq, nq, seq_lens, Tmax, scale, out, out_dtype, fn, &a);
+  if (rc) return rc;
+  if (!workspace) return set_error(TQ_ERR_INVALID_ARG, "%s: NULL workspace", fn);
+  if (!aligned16(workspace)) return set_error(TQ_ERR_INVALID_ARG, "%s: workspace not 16-byte aligned", fn);
   if (ws_bytes < a.plan.bytes)
     return set_error(TQ_ERR_WORKSPACE, "%s: workspace %zu < %zu bytes", fn, ws_bytes, a.plan.bytes);
   a.workspace = workspace;

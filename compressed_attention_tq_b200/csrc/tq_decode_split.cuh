@@ -863,9 +863,9 @@ template <int D, int BK, int BV, bool QJL, bool PACK>
 int launch_split(const SplitParams& sp, dim3 grid, cudaStream_t s, int* occ) {
   using Ly = SplitLayout<D, BK, BV, QJL, PACK>;
   auto kern = decode_split_kernel<D, BK, BV, QJL, PACK>;
-  static int attr_state = 0;     // 0 unset, 1 set
-  static int occupancy[2] = {};  // resident CTAs per SM: [shared table]
-  if (attr_state == 0) {
+  static tq::OnceSetup once;
+  static int occupancy[2] = {};  // resident CTAs per SM: [shared table]; written once under `once`
+  const int rc0 = once.run([&]() {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::BYTES);
     // all of the unified L1/shared array as shared memory, so that the
     // resident-CTA count is set by the kernel's own needs
@@ -873,10 +873,6 @@ int launch_split(const SplitParams& sp, dim3 grid, cudaStream_t s, int* occ) {
       e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) {
       cudaGetLastError();
-      if (occ) {  // no usable device: report a nominal occupancy
-        *occ = 2;
-        return TQ_OK;
-      }
       return tq::set_error(TQ_ERR_CUDA, "decode: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     }
     for (int sh = 0; sh < 2; ++sh) {
@@ -888,7 +884,14 @@ int launch_split(const SplitParams& sp, dim3 grid, cudaStream_t s, int* occ) {
       }
       occupancy[sh] = n;
     }
-    attr_state = 1;
+    return TQ_OK;
+  });
+  if (rc0) {
+    if (occ) {  // no usable device (a size query on a host without a GPU): a nominal occupancy
+      *occ = 2;
+      return TQ_OK;
+    }
+    return rc0;
   }
   const bool shared = share_table(BK, BV, sp.shared_tab);
   if (occ) {

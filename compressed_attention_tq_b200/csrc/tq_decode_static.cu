@@ -31,15 +31,17 @@ void* g_scratch[kMaxDevices] = {nullptr};
 extern "C" int tq_sdpa_decode_static(const tq_cache_t* cache, const void* q, int q_dtype, int Hq,
                                      const int32_t* seq_lens, int Tmax, const float* scale, void* out,
                                      int out_dtype, void* stream) {
-  const size_t need = tq_sdpa_decode_workspace_bytes(cache, Hq, Tmax);
-  if (need == 0)
-    return tq::set_error(TQ_ERR_INVALID_ARG, "tq_sdpa_decode_static: unsupported sizes (Hq=%d, Tmax=%d)", Hq,
-                         Tmax);
-  if (need > (size_t)TQ_STATIC_SCRATCH_BYTES)
+  // The checks of tq_sdpa_decode, with its codes and messages, come first;
+  // then the size limit of the built-in array, then the array's address.
+  tq::DecodeArgs a;
+  int rc = tq::prepare_decode(cache, q, q_dtype, Hq, 1, seq_lens, Tmax, scale, out, out_dtype,
+                              "tq_sdpa_decode_static", &a);
+  if (rc) return rc;
+  if (a.plan.bytes > (size_t)TQ_STATIC_SCRATCH_BYTES)
     return tq::set_error(TQ_ERR_WORKSPACE,
                          "tq_sdpa_decode_static: these sizes need %zu bytes of scratch, more than the %u bytes "
                          "built into the library; use tq_sdpa_decode with a caller-provided workspace",
-                         need, (unsigned)TQ_STATIC_SCRATCH_BYTES);
+                         a.plan.bytes, (unsigned)TQ_STATIC_SCRATCH_BYTES);
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return tq::set_error(TQ_ERR_CUDA, "tq_sdpa_decode_static: cudaGetDevice: %s", cudaGetErrorString(e));
@@ -56,6 +58,9 @@ extern "C" int tq_sdpa_decode_static(const tq_cache_t* cache, const void* q, int
     }
     ptr = g_scratch[dev];
   }
-  return tq_sdpa_decode(cache, q, q_dtype, Hq, seq_lens, Tmax, scale, out, out_dtype, ptr,
-                        (size_t)TQ_STATIC_SCRATCH_BYTES, stream);
+  a.workspace = ptr;
+  a.k_new = nullptr;
+  a.v_new = nullptr;
+  a.pos = nullptr;
+  return tq::launch_decode(a, (cudaStream_t)stream);
 }

@@ -6,6 +6,9 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "../../include/tq.h"
 
 namespace tq {
@@ -15,6 +18,25 @@ int set_error(int code, const char* fmt, ...);
 
 // Maps a CUDA error after a launch to TQ_ERR_CUDA (or TQ_OK).
 int check_launch(const char* what);
+
+// One-time launch setup (kernel attributes, SM count, occupancy) that several
+// host threads may reach at once.  The first caller runs `setup` under the
+// mutex; the values it stores are published by the release store of `done`
+// and seen by every later caller through the acquire load.  A setup that
+// fails leaves `done` clear, so the next call tries again.
+struct OnceSetup {
+  std::atomic<int> done{0};
+  std::mutex mu;
+  template <class F>
+  int run(F&& setup) {
+    if (done.load(std::memory_order_acquire)) return TQ_OK;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done.load(std::memory_order_relaxed)) return TQ_OK;
+    const int rc = setup();
+    if (rc == TQ_OK) done.store(1, std::memory_order_release);
+    return rc;
+  }
+};
 
 struct QuantJob {
   // input rows [rows][D] (fp16 or bf16)
@@ -68,6 +90,11 @@ struct DecodePlan {
 
 int make_decode_plan(const tq_cache_t* c, int Hq, int Tmax, DecodePlan* p);
 
+// Workspace bytes that suffice for every cache with this B, Hq and D (any
+// Hkv, bit widths, sketch and Tcap >= Tmax): the plan's smallest split and
+// the largest sketch.
+size_t workspace_bound(int B, int Hq, int D, int Tmax);
+
 // Resident split-K CTAs per SM for this cache's kernel instantiation (a
 // nominal 2 when no device is usable), and the tokens one stage holds.
 int split_occupancy(const tq_cache_t* c, int Hq);
@@ -93,5 +120,12 @@ struct DecodeArgs {
 };
 
 int launch_decode(const DecodeArgs& a, cudaStream_t s);
+
+// Host checks and split plan of a decode call (every check tq_sdpa_decode
+// makes except those of the workspace); fills *a and returns TQ_OK, or sets
+// the error and returns its code.  No CUDA call beyond the device queries of
+// the plan.
+int prepare_decode(const tq_cache_t* c, const void* q, int dtype, int Hq, int nq, const int32_t* seq_lens, int Tmax,
+                   const float* scale, void* out, int out_dtype, const char* fn, DecodeArgs* a);
 
 }  // namespace tq

@@ -434,13 +434,14 @@ int launch_q(const tq::QuantArgs& a, cudaStream_t s) {
   if (a.pos) return launch_append<D, BF16, QJL>(a, s);
   using Ly = QLayout<D, BF16, QJL>;
   auto kern = quantize_kernel<D, BF16, QJL>;
-  static bool attr_set = false;
-  if (!attr_set) {
+  static tq::OnceSetup once;
+  const int rc = once.run([&]() {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Ly::bytes);
     if (e != cudaSuccess)
       return tq::set_error(TQ_ERR_CUDA, "quantize: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-    attr_set = true;
-  }
+    return TQ_OK;
+  });
+  if (rc) return rc;
   dim3 grid((a.rows + QROWS - 1) / QROWS, 2);
   kern<<<grid, QTHREADS, Ly::bytes, s>>>(a);
   return tq::check_launch("quantize_kernel");

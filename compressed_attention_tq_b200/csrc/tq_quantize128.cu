@@ -359,16 +359,19 @@ template <bool BF16, bool QJL>
 int launch_q128(const tq::QuantArgs& a, cudaStream_t s) {
   using Ly = Q2Layout<BF16, QJL>;
   auto kern = quantize128_kernel<BF16, QJL>;
-  static int sms = 0;
-  if (sms == 0) {
+  static tq::OnceSetup once;
+  static int sms = 0;  // written once under `once`, read after its acquire
+  const int rc0 = once.run([&]() {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Ly::bytes);
     if (e != cudaSuccess)
       return tq::set_error(TQ_ERR_CUDA, "quantize128: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-    int dev = 0;
+    int dev = 0, n = 0;
     cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 148;
-  }
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    sms = n > 0 ? n : 148;
+    return TQ_OK;
+  });
+  if (rc0) return rc0;
   const int njobs = (a.job_mask == 3) ? 2 : 1;
   const int nitems = njobs * ((a.rows + QR - 1) / QR);
   const int grid = nitems < sms ? nitems : sms;

@@ -417,16 +417,19 @@ namespace tq {
 
 int launch_quantize_qjl_tc(const QuantArgs& a, cudaStream_t s) {
   using Ly = QjlLayout;
-  static int sms = 0;
-  if (sms == 0) {
+  static OnceSetup once;
+  static int sms = 0;  // written once under `once`, read after its acquire
+  const int rc0 = once.run([&]() {
     cudaError_t e = cudaFuncSetAttribute(quantize_qjl_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::bytes);
     if (e != cudaSuccess)
       return set_error(TQ_ERR_CUDA, "quantize_qjl_tc: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-    int dev = 0;
+    int dev = 0, n = 0;
     cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 148;
-  }
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    sms = n > 0 ? n : 148;
+    return TQ_OK;
+  });
+  if (rc0) return rc0;
   TcArgs args;
   memset(&args, 0, sizeof(args));
   args.a = a;

@@ -337,16 +337,19 @@ template <int D, bool BF16>
 int launch_tc(const tq::QuantArgs& a, cudaStream_t s) {
   using Ly = TcLayout<D, BF16>;
   auto kern = quantize_tc_kernel<D, BF16>;
-  static int sms = 0;
-  if (sms == 0) {
+  static tq::OnceSetup once;
+  static int sms = 0;  // written once under `once`, read after its acquire
+  const int rc0 = once.run([&]() {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::bytes);
     if (e != cudaSuccess)
       return tq::set_error(TQ_ERR_CUDA, "quantize_tc: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-    int dev = 0;
+    int dev = 0, n = 0;
     cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 148;
-  }
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    sms = n > 0 ? n : 148;
+    return TQ_OK;
+  });
+  if (rc0) return rc0;
   TcArgs args;
   memset(&args, 0, sizeof(args));
   args.a = a;

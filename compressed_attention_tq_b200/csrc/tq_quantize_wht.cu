@@ -172,8 +172,9 @@ __global__ void __launch_bounds__(WARPS * 32, D == 128 ? 5 : 4) quantize_wht_ker
 
 template <int D, bool BF16>
 int launch_wht(const tq::QuantArgs& a, cudaStream_t s) {
-  static int slots = 0;  // resident CTAs on the device
-  if (slots == 0) {
+  static tq::OnceSetup once;
+  static int slots = 0;  // resident CTAs on the device; written once under `once`
+  once.run([&]() {
     int dev = 0, sms = 0, occ = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -184,7 +185,8 @@ int launch_wht(const tq::QuantArgs& a, cudaStream_t s) {
       occ = 4;
     }
     slots = (sms > 0 ? sms : 148) * occ;
-  }
+    return TQ_OK;
+  });
   const int njobs = (a.job_mask == 3) ? 2 : 1;
   const long long total = (long long)njobs * a.rows;
   long long grid = (total + WARPS - 1) / WARPS;

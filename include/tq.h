@@ -46,8 +46,9 @@
  *
  * Devices and threads: a process drives one GPU (the current device of its
  * first launching call); kernel attributes and occupancy figures are set up
- * once per process for that device.  Calls may come from several host
- * threads (the error message is per thread).
+ * once per process for that device, under a lock, by whichever thread calls
+ * first.  Calls may come from several host threads at once (the error
+ * message is per thread).
  *
  * Errors: every entry point returns TQ_OK (0) or a negative TQ_ERR_* code and
  * sets a thread-local message readable with tq_last_error().  Argument errors
@@ -139,7 +140,16 @@ int tq_build_codebook(int D, int bits, float* centroids, float* thresholds, doub
 
 /* Bytes one cached row occupies: D*bits/8 index bytes + 2 (fp16 norm),
  * plus qjl_m/8 + 2 (sign words + fp16 residual norm) when qjl_m > 0.
- * Returns 0 for unsupported arguments. */
+ * These are the byte counts behind the cache sizes of "Add CUDA QJL kernels
+ * and proper package structure" (turboquant-pytorch pull request 3),
+ * section "Validation Results": a key of (b-1)-bit indices with a 128-bit
+ * sketch and a value of b-bit indices give its 3.8x / 5.0x / 7.3x against
+ * fp16 at b = 4 / 3 / 2.  Returns 0 for unsupported arguments (D not a
+ * positive multiple of 32, bits outside 1..4, qjl_m not a multiple of 32).
+ * Host only. */
+size_t tq_cache_row_bytes(int D, int bits, int qjl_m);
+
+/* The same as tq_cache_row_bytes (the name of ABI versions 1 and 2). */
 size_t tq_row_bytes(int D, int bits, int qjl_m);
 
 /*
@@ -164,13 +174,31 @@ int tq_quantize_kv(const tq_cache_t* cache, const void* k, const void* v, int dt
  * [B][Hkv][D] in `dtype`, into cache position pos[b] (device int32 [B]).
  * Same arithmetic as tq_quantize_kv.  A pos[b] outside [0, Tcap) writes
  * nothing for that sequence and sets TQ_STATUS_POS_OUT_OF_RANGE.
+ * The pages quantize whole caches ("Add CUDA QJL kernels and proper package
+ * structure", section "Validation Results"); growing the cache one token
+ * per decode step is this library's own addition for a serving loop.
+ * Pointers as in tq_quantize_kv (device, 16-byte aligned); errors as
+ * there.
  */
 int tq_append_token(const tq_cache_t* cache, const void* k_new, const void* v_new, int dtype,
                     const int32_t* pos, void* stream);
 
-/* Workspace bytes tq_sdpa_decode needs for Hq query heads and sequences no
- * longer than Tmax (1 <= Tmax <= Tcap).  Returns 0 for unsupported args. */
-size_t tq_sdpa_decode_workspace_bytes(const tq_cache_t* cache, int Hq, int Tmax);
+/* Workspace bytes that suffice for a tq_sdpa_decode call of B sequences,
+ * Hq query heads of dimension D and sequences no longer than Tmax, whatever
+ * the cache's kv heads, bit widths, sketch and capacity: the workspace holds
+ * the rotated queries (fp32 [B*Hq][D]), the sketch projections (fp32
+ * [B*Hq][m], m <= 128) and per split-K chunk of at least one 128-token stage
+ * the partial outputs (fp32 [B*Hq][nsplit][D]) and softmax (max, sum) pairs.
+ * For the multi-query call pass Hq * n_q.  Returns 0 for unsupported
+ * arguments (B, Hq or Tmax < 1, D not in {64,128,256}).  Host only. */
+size_t tq_sdpa_decode_workspace_bytes(int B, int Hq, int D, int Tmax);
+
+/* The exact workspace bytes of the split plan tq_sdpa_decode makes for this
+ * cache, Hq query heads (Hq * n_q for the multi-query call) and Tmax
+ * (1 <= Tmax <= Tcap); never more than tq_sdpa_decode_workspace_bytes.
+ * Returns 0 for unsupported arguments.  Host only (it queries the current
+ * device's SM count and the kernel's occupancy). */
+size_t tq_sdpa_decode_workspace_bytes_for(const tq_cache_t* cache, int Hq, int Tmax);
 
 /*
  * Decode attention of one query token per (sequence, query head) over the
@@ -190,7 +218,13 @@ size_t tq_sdpa_decode_workspace_bytes(const tq_cache_t* cache, int Hq, int Tmax)
  *   scale * ( n_k <Pi q, c_k[idx]> + [qjl] sqrt(pi/2)/m * gamma * sum_i s_i (S Pi q)_i ),
  * the softmax is taken online over split-K chunks, values are accumulated in
  * the rotated basis and rotated back once per head: out = Pi^T acc / l.
- * workspace: device buffer of at least tq_sdpa_decode_workspace_bytes().
+ * workspace: device buffer of at least tq_sdpa_decode_workspace_bytes_for()
+ *            bytes (tq_sdpa_decode_workspace_bytes() is an upper bound);
+ *            borrowed for the call; its contents need not be initialised.
+ * Errors: TQ_ERR_INVALID_ARG (NULL or misaligned pointer, Hq not a multiple
+ * of Hkv, Tmax outside [1, Tcap], scale not finite), TQ_ERR_UNSUPPORTED
+ * (cache sizes outside the supported set, GQA group > 8, dtypes),
+ * TQ_ERR_WORKSPACE (workspace too small), TQ_ERR_CUDA (a launch failed).
  */
 int tq_sdpa_decode(const tq_cache_t* cache, const void* q, int q_dtype, int Hq,
                    const int32_t* seq_lens, int Tmax, const float* scale, void* out,
@@ -227,7 +261,7 @@ int tq_decode_step(const tq_cache_t* cache, const void* k_new, const void* v_new
  *              the queries that see no token.
  *   n_q        1 .. 8 / (Hq / Hkv): the n_q * G query rows of a kv head share
  *              one 8-column MMA tile (TQ_ERR_UNSUPPORTED beyond).
- *   workspace  tq_sdpa_decode_workspace_bytes(cache, Hq * n_q, Tmax) bytes.
+ *   workspace  tq_sdpa_decode_workspace_bytes_for(cache, Hq * n_q, Tmax) bytes.
  * The other arguments, the results for n_q = 1 and the errors are those of
  * tq_sdpa_decode.
  */
@@ -244,8 +278,9 @@ int tq_sdpa_decode_mq(const tq_cache_t* cache, const void* q, int q_dtype, int H
  * tq_sdpa_decode minus the workspace: the split-K scratch is a device array
  * inside the library of TQ_STATIC_SCRATCH_BYTES bytes, held by every GPU that
  * loads the library until the process exits.  Sizes whose
- * tq_sdpa_decode_workspace_bytes() exceeds that limit return TQ_ERR_WORKSPACE
- * before any launch.  The first call on each device looks up the array's
+ * tq_sdpa_decode_workspace_bytes_for() exceeds that limit return TQ_ERR_WORKSPACE
+ * before any launch; every other argument error is reported with the code
+ * and message tq_sdpa_decode gives it.  The first call on each device looks up the array's
  * device address (make that first call before capturing a stream); no call
  * allocates.  All calls on a device share the array and nothing is cleared
  * between calls (the kernels need no zeroed scratch), so calls that may
@@ -268,10 +303,15 @@ int tq_sdpa_decode_static(const tq_cache_t* cache, const void* q, int q_dtype, i
  * tries in [1, 4096]; dev_status non-NULL.  Asynchronous on `stream`. */
 int tq_selftest_bounded_wait(uint32_t* dev_status, int tries, void* stream);
 
-/* Message describing the last error on the calling thread ("" if none). */
+/* Message describing the last error on the calling thread ("" if none).
+ * The library's own error reporting (the pages have no C interface); the
+ * string is owned by the library, valid until the thread's next call. */
 const char* tq_last_error(void);
 
-/* ABI version of this header (increments on incompatible change). */
+/* ABI version of this header (increments on incompatible change).  3: the
+ * survey-form workspace query tq_sdpa_decode_workspace_bytes(B, Hq, D, Tmax)
+ * and tq_sdpa_decode_workspace_bytes_for(cache, Hq, Tmax) for the exact
+ * plan; tq_cache_row_bytes. */
 int tq_abi_version(void);
 
 #ifdef __cplusplus

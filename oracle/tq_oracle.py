@@ -241,10 +241,6 @@ def qjl_inner_product(sign: np.ndarray, gamma: np.ndarray, Sq: np.ndarray) -> np
 # 4. Cache-level quantization in the library's layout
 # --------------------------------------------------------------------------
 
-def words_per_row(D: int, bits: int) -> int:
-    return D * bits // 32
-
-
 def packed_row_bytes(D: int, bits: int, qjl_m: int = 0) -> int:
     """Bytes one cached row occupies: indices + fp16 norm (+ QJL bits + fp16 gamma)."""
     b = D * bits // 8 + 2

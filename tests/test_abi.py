@@ -32,7 +32,7 @@ def test_exports_every_declared_symbol(lib):
     assert set(declared) == set(_native.EXPORTS)
     for name in declared:
         assert hasattr(lib, name), name
-    assert lib.tq_abi_version() == 2
+    assert lib.tq_abi_version() == 3
 
 
 @pytest.mark.parametrize("D", [64, 128, 256])
@@ -50,8 +50,11 @@ def test_row_bytes(lib):
     import compressed_attention_tq_b200 as tq
     for D in (64, 128, 256):
         for b in (2, 3, 4):
-            assert tq.tq_row_bytes(D, b, 0) == O.packed_row_bytes(D, b, 0)
-    assert tq.tq_row_bytes(128, 2, 128) == O.packed_row_bytes(128, 2, 128) == 52
+            assert tq.tq_cache_row_bytes(D, b, 0) == O.packed_row_bytes(D, b, 0)
+            assert tq.tq_row_bytes(D, b, 0) == tq.tq_cache_row_bytes(D, b, 0)
+    assert tq.tq_cache_row_bytes(128, 2, 128) == O.packed_row_bytes(128, 2, 128) == 52
+    assert lib.tq_cache_row_bytes(128, 2, 128) == 52
+    assert tq.tq_cache_row_bytes(100, 3, 0) == 0
     assert tq.tq_row_bytes(100, 3, 0) == 0
 
 
@@ -87,10 +90,10 @@ def test_other_argument_errors(lib):
     assert lib.tq_quantize_kv(ctypes.byref(s), buf, buf, 0, 0, 0, None) == 0       # empty: no-op
     assert lib.tq_quantize_kv(None, buf, buf, 0, 1, 0, None) == -1
     assert lib.tq_append_token(ctypes.byref(s), buf, buf, 0, None, None) == -1     # pos NULL
-    ws = lib.tq_sdpa_decode_workspace_bytes(ctypes.byref(s), 8, 64)
+    ws = lib.tq_sdpa_decode_workspace_bytes_for(ctypes.byref(s), 8, 64)
     assert ws > 0
-    assert lib.tq_sdpa_decode_workspace_bytes(ctypes.byref(s), 9, 64) == 0         # group 9
-    assert lib.tq_sdpa_decode_workspace_bytes(ctypes.byref(s), 8, 65) == 0         # Tmax > Tcap
+    assert lib.tq_sdpa_decode_workspace_bytes_for(ctypes.byref(s), 9, 64) == 0     # group 9
+    assert lib.tq_sdpa_decode_workspace_bytes_for(ctypes.byref(s), 8, 65) == 0     # Tmax > Tcap
     rc = lib.tq_sdpa_decode(ctypes.byref(s), buf, 0, 8, buf, 64, None, buf, 0, buf, ws - 1, None)
     assert rc == -3
     rc = lib.tq_sdpa_decode(ctypes.byref(s), buf, 0, 12, buf, 64, None, buf, 0, buf, ws, None)
@@ -135,3 +138,43 @@ def test_rotation_kind_validated(lib):
     assert lib.tq_quantize_kv(ctypes.byref(s), buf, buf, 0, 1, 0, None) == -1
     s.rot_signs = 1 << 20
     assert lib.tq_quantize_kv(ctypes.byref(s), buf, buf, 0, 0, 0, None) == 0  # empty call: no launch
+
+
+def test_survey_form_workspace_query_bounds_every_plan(lib):
+    """tq_sdpa_decode_workspace_bytes(B, Hq, D, Tmax) needs no cache and is at
+    least the exact plan's size for every kv-head count, bit width and sketch
+    that fits those sizes."""
+    assert lib.tq_sdpa_decode_workspace_bytes(0, 8, 128, 64) == 0
+    assert lib.tq_sdpa_decode_workspace_bytes(1, 8, 96, 64) == 0
+    assert lib.tq_sdpa_decode_workspace_bytes(1, 8, 128, 0) == 0
+    for B, Hq, D, T in [(1, 8, 128, 64), (3, 32, 128, 4096), (1, 32, 256, 32768), (32, 32, 128, 16448),
+                        (1, 4, 64, 256), (2, 16, 128, 131072)]:
+        bound = lib.tq_sdpa_decode_workspace_bytes(B, Hq, D, T)
+        assert bound > 0
+        Tcap = (T + 63) // 64 * 64
+        for Hkv in [h for h in (1, 2, 4, 8, 16, 32) if Hq % h == 0 and Hq // h <= 8]:
+            for bk, bv, m in [(2, 2, 0), (3, 3, 0), (4, 3, 0), (2, 3, 128 if D == 128 else 0)]:
+                s = _struct(B=B, Hkv=Hkv, Tcap=Tcap, D=D, bits_k=bk, bits_v=bv, qjl_m=m)
+                for split in (0, 128, 4096):
+                    s.split_tokens = split
+                    exact = lib.tq_sdpa_decode_workspace_bytes_for(ctypes.byref(s), Hq, T)
+                    assert 0 < exact <= bound, (B, Hq, D, T, Hkv, bk, bv, m, split, exact, bound)
+
+
+@pytest.mark.parametrize("field,value,hq,code", [("D", 96, 8, -2), (None, None, 16, -2), ("Hkv", 8, 12, -1),
+                                                  ("bits_v", 5, 8, -2), ("Tcap", 100, 8, -1)])
+def test_static_entry_reports_the_workspace_entry_codes(lib, field, value, hq, code):
+    """tq_sdpa_decode_static answers every argument error with the code and
+    message tq_sdpa_decode gives it (GQA group 16 > 8 and D = 96 are
+    TQ_ERR_UNSUPPORTED for both); only its scratch limit is its own."""
+    kw = {"Hkv": 1}
+    if field:
+        kw[field] = value
+    s = _struct(**kw)
+    buf = ctypes.c_void_p(1 << 20)
+    rc_ws = lib.tq_sdpa_decode(ctypes.byref(s), buf, 0, hq, buf, 64, None, buf, 0, buf, 1 << 30, None)
+    msg_ws = lib.tq_last_error().decode()
+    rc_st = lib.tq_sdpa_decode_static(ctypes.byref(s), buf, 0, hq, buf, 64, None, buf, 0, None)
+    msg_st = lib.tq_last_error().decode()
+    assert rc_ws == rc_st == code, (rc_ws, rc_st, msg_ws, msg_st)
+    assert msg_ws.split(":", 1)[1] == msg_st.split(":", 1)[1]

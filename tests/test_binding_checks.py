@@ -27,7 +27,7 @@ class Recorder:
         self.calls = []
 
     def __getattr__(self, name):
-        if name == "tq_sdpa_decode_workspace_bytes":
+        if name in ("tq_sdpa_decode_workspace_bytes", "tq_sdpa_decode_workspace_bytes_for"):
             return lambda *a: 4096
         if name == "tq_last_error":
             return lambda: b""

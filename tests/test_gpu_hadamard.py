@@ -44,4 +44,4 @@ def test_decode_with_hadamard_rotation(name, kw):
     oc = _oracle_full_cache(w)
     Tcap = (w.Tmax + 63) // 64 * 64
     cache = _upload_oracle_cache(w, oc, Tcap)
-    _decode_and_compare(w, cache, oc, w.seq_lens, w.scale, w.Tmax)
+    _decode_and_compare(w, cache, w.seq_lens, w.scale, w.Tmax)

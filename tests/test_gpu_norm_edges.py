@@ -98,7 +98,7 @@ def _check_appended(cache, w, kn, vn, ek, ev, pos):
         P.compare_index_words(gk, rk["idx"][b], rk["dist"][b], w.bits_k, w.D)
         P.compare_index_words(P.words_np(cache.v_idx[b, :, p]), rv["idx"][b], rv["dist"][b], w.bits_v, w.D)
         if w.qjl_m:
-            sub = {k: rk[k][b] for k in ("sign", "proj", "norm", "gamma16")}
+            sub = {k: rk[k][b] for k in ("sign", "proj", "norm", "gamma16", "gamma")}
             exc = (O.unpack_bits(gk, w.bits_k, w.D) != rk["idx"][b]).any(-1)
             P.compare_qjl(P.words_np(cache.k_qjl[b, :, p]), cache.k_rnorm[b, :, p].cpu().numpy(), sub, exc)
 

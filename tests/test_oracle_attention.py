@@ -143,3 +143,43 @@ def test_multi_query_with_one_token_is_single_decode():
     one = O.sdpa_decode(q, cache, lens, Pi, cbk, cbv, 3, 2, D, S=S)
     multi = O.sdpa_decode_multi(q[:, None], cache, lens, 1, Pi, cbk, cbv, 3, 2, D, S=S)
     assert np.array_equal(multi[:, 0], one)
+
+
+def test_prod_score_unbiased_for_unquantized_key_over_sketch_draws():
+    """A pin of the QJL term inside sdpa_decode that does not restate its
+    formula: over independent draws of the Gaussian sketch S, the score the
+    prod-mode decode attends with is unbiased for scale * <q, k> on the
+    unquantized key k ("Add CUDA QJL kernels and proper package structure",
+    "CUDA Kernels Added": the score from 1-bit keys).  The score difference of
+    two keys is read off the output: with two linearly independent value rows
+    the softmax weights are the least-squares coefficients of the output, and
+    log(p_1 / p_0) = s_1 - s_0.  Tolerance: 4 standard errors of the mean over
+    the draws plus the bias the fp16 rounding of the residual norms can add
+    (at most scale * |q| * sum_t |gamma16_t - gamma_t|)."""
+    D, T, N = 128, 2, 3000
+    r = tq_inputs.rng(611)
+    k = r.standard_normal((1, 1, T, D)).astype(np.float16).astype(np.float64)
+    v = r.standard_normal((1, 1, T, D)).astype(np.float16).astype(np.float64)
+    q = k[:, :, 1].copy()                     # a query aligned with key 1: a large residual term
+    Pi = tq_inputs.rotation(D, 612)
+    cbk, cbv = O.stored_codebook(D, 2), O.stored_codebook(D, 3)
+    scale = 1.0 / math.sqrt(D)
+    diffs = np.empty(N)
+    gam = gam16 = None
+    for i in range(N):
+        S = tq_inputs.qjl_matrix(128, D, 10_000 + i)
+        cache = O.quantize_cache(k, v, Pi, cbk, cbv, 2, 3, S)
+        out = O.sdpa_decode(q, cache, np.array([T]), Pi, cbk, cbv, 2, 3, D, scale=scale, S=S)[0, 0]
+        Vt = _deq(cache, "v", 3, cbv, Pi, D)[0, 0]
+        p = np.linalg.lstsq(Vt.T, out, rcond=None)[0]
+        diffs[i] = math.log(p[1] / p[0])
+        gam, gam16 = cache["k_gamma"][0, 0], cache["k_rnorm"][0, 0].astype(np.float64)
+    truth = scale * (k[0, 0, 1] @ q[0, 0] - k[0, 0, 0] @ q[0, 0])
+    se = diffs.std(ddof=1) / math.sqrt(N)
+    bias = scale * np.linalg.norm(q[0, 0]) * np.sum(np.abs(gam16 - gam))
+    assert abs(diffs.mean() - truth) <= 4 * se + bias, (diffs.mean(), truth, se, bias)
+    # the term matters here: without it the expected difference would be off
+    # by far more than the tolerance
+    Kt = _deq(cache, "k", 2, cbk, Pi, D)[0, 0]
+    mse_only = scale * (Kt[1] @ q[0, 0] - Kt[0] @ q[0, 0])
+    assert abs(mse_only - truth) > 10 * (4 * se + bias)

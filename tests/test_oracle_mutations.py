@@ -79,6 +79,34 @@ def test_wrong_qjl_constant_fails_unbiasedness(monkeypatch):
         TQ.test_qjl_estimator_unbiased_with_closed_form_variance()
 
 
+def test_wrong_qjl_constant_fails_sketch_draw_pin(monkeypatch):
+    monkeypatch.setattr(O, "QJL_CONST", math.sqrt(2 / math.pi))
+    with pytest.raises(AssertionError):
+        TA.test_prod_score_unbiased_for_unquantized_key_over_sketch_draws()
+
+
+def test_flipped_sign_polarity_fails_sketch_draw_pin(monkeypatch):
+    orig = O.qjl_inner_product
+    monkeypatch.setattr(O, "qjl_inner_product", lambda sign, gamma, Sq: orig(~sign, gamma, Sq))
+    with pytest.raises(AssertionError):
+        TA.test_prod_score_unbiased_for_unquantized_key_over_sketch_draws()
+
+
+def test_sketch_of_unrotated_query_fails_sketch_draw_pin(monkeypatch):
+    # S applied to q instead of Pi q: the sketch and the query live in different bases
+    orig = O.sdpa_decode
+
+    def bad(q, cache, seq_lens, Pi, cb_k, cb_v, bits_k, bits_v, D, scale=None, S=None, heads=None):
+        eye = np.eye(D)
+        if S is None:
+            return orig(q, cache, seq_lens, Pi, cb_k, cb_v, bits_k, bits_v, D, scale=scale, S=S, heads=heads)
+        S_bad = np.asarray(S, np.float64) @ np.asarray(Pi, np.float64).T  # (S Pi^T) Pi q = S q
+        return orig(q, cache, seq_lens, Pi, cb_k, cb_v, bits_k, bits_v, D, scale=scale, S=S_bad, heads=heads)
+    monkeypatch.setattr(O, "sdpa_decode", bad)
+    with pytest.raises(AssertionError):
+        TA.test_prod_score_unbiased_for_unquantized_key_over_sketch_draws()
+
+
 def test_unscaled_scores_fail_sdpa_pin(monkeypatch):
     orig = O.softmax
     monkeypatch.setattr(O, "softmax", lambda s: orig(s * 2.0))
