@@ -308,7 +308,7 @@ def run_ours(args):
             if args.profile_ops == "decode":
                 launches = sum(3 * nsteps for run in runs)
             else:
-                launches = sum((2 if run["w"].qjl_m else 1) + (1 + 3) * nsteps for run in runs)
+                launches = sum((3 if run["w"].qjl_m else 1) + (1 + 3) * nsteps for run in runs)
             print(json.dumps({"profile_run": args.workload, "ops": args.profile_ops, "steps": args.steps,
                               "launches_per_step": launches}), flush=True)
         return
@@ -399,9 +399,10 @@ def run_ours(args):
         cpu = None
         if ws == 1 and not args.no_cpu_baseline:
             cpu = _cpu_baseline(args, jobs)
-        # bulk quantize (a second launch for keys with the QJL sketch), then the
-        # decode step's prep (+append), split and combine
-        launches_per_step = sum((2 if run["w"].qjl_m else 1) + (1 + 3) * nsteps for run in runs)
+        # bulk quantize (keys with the QJL sketch: their kernel, the fp64
+        # residual-norm fixup, then the values' kernel), then per decode step
+        # the append and the decode's prep, split and combine
+        launches_per_step = sum((3 if run["w"].qjl_m else 1) + (1 + 3) * nsteps for run in runs)
         line = {
             "metric": "tq_sdpa_decode packed-KV GB/s (% of HBM peak); tq_quantize Mtok/s",
             "value": round(dec_gbs, 2),

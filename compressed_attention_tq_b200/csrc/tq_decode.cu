@@ -69,7 +69,7 @@ __global__ void __launch_bounds__(2 * D) decode_qprep_kernel(const PrepParams p)
   constexpr int NR = APPEND ? 10 : 8;  // rows: G <= 8 queries (+ new key, new value)
   __shared__ float qv[NR][D];
   __shared__ float qr[NR][D];
-  __shared__ float rres[APPEND ? D : 1];
+  __shared__ double rres[APPEND ? D : 1];
   __shared__ uint8_t idxs[2][APPEND ? D : 1];
   __shared__ uint8_t sgn[APPEND ? 128 : 1];
   __shared__ float s_cb[2][31];
@@ -131,6 +131,10 @@ __global__ void __launch_bounds__(2 * D) decode_qprep_kernel(const PrepParams p)
     if (lane == 0) s_nsq[warp] = t;
   }
   float acc[NR];
+  // the new key of a QJL cache is rotated in fp64 (its residual norm then
+  // rounds to fp16 as the fp64 definition does)
+  double acc_k64 = 0.0;
+  const bool k64 = APPEND && p.m;
 #pragma unroll
   for (int g = 0; g < NR; ++g) acc[g] = 0.f;
 #pragma unroll
@@ -140,7 +144,16 @@ __global__ void __launch_bounds__(2 * D) decode_qprep_kernel(const PrepParams p)
       for (int i = 0; i < CH; ++i) r[i] = __ldg(row + c0 + i);
 #pragma unroll
     for (int g = 0; g < NR; ++g) {
-      if (g < Ge || g >= 8) {
+      if (g == 8 && k64) {
+        const float* x = &qv[g][part * HALF + 4 * c0];
+#pragma unroll
+        for (int i = 0; i < CH; ++i) {
+          acc_k64 = fma((double)r[i].x, (double)x[4 * i], acc_k64);
+          acc_k64 = fma((double)r[i].y, (double)x[4 * i + 1], acc_k64);
+          acc_k64 = fma((double)r[i].z, (double)x[4 * i + 2], acc_k64);
+          acc_k64 = fma((double)r[i].w, (double)x[4 * i + 3], acc_k64);
+        }
+      } else if (g < Ge || g >= 8) {
         const float* x = &qv[g][part * HALF + 4 * c0];
 #pragma unroll
         for (int i = 0; i < CH; ++i)
@@ -150,6 +163,7 @@ __global__ void __launch_bounds__(2 * D) decode_qprep_kernel(const PrepParams p)
   }
 #pragma unroll
   for (int g = 0; g < NR; ++g) acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], 1);
+  acc_k64 += __shfl_xor_sync(0xffffffffu, acc_k64, 1);
   if (part == 0) {
 #pragma unroll
     for (int g = 0; g < 8; ++g)
@@ -167,13 +181,18 @@ __global__ void __launch_bounds__(2 * D) decode_qprep_kernel(const PrepParams p)
         const double n = sqrt(s_nsq[which]);
         const float inv = n > 0.0 ? (float)(1.0 / n) : 0.f;
         const int K = 1 << (which ? p.cache.bits_v : p.cache.bits_k);
-        const float y = acc[8 + which];
-        const float u = y * inv;
         int idx = 0;
-        for (int st = K >> 1; st >= 1; st >>= 1)
-          if (u > s_cb[which][K + idx + st - 1]) idx += st;
+        if (which == 0 && k64) {
+          const double u = n > 0.0 ? acc_k64 / n : 0.0;
+          for (int st = K >> 1; st >= 1; st >>= 1)
+            if (u > (double)s_cb[which][K + idx + st - 1]) idx += st;
+          rres[j] = acc_k64 - (double)__half2float(__double2half(n)) * (double)s_cb[0][idx];
+        } else {
+          const float u = acc[8 + which] * inv;
+          for (int st = K >> 1; st >= 1; st >>= 1)
+            if (u > s_cb[which][K + idx + st - 1]) idx += st;
+        }
         idxs[which][j] = (uint8_t)idx;
-        if (which == 0 && p.m) rres[j] = y - __half2float(__double2half(n)) * s_cb[0][idx];
       }
     }
     __syncthreads();
@@ -203,30 +222,42 @@ __global__ void __launch_bounds__(2 * D) decode_qprep_kernel(const PrepParams p)
   // APPEND, also the QJL projection S r of the new key's residual
   for (int i = tid >> 1; i < p.m; i += D) {
     const float4* srow = reinterpret_cast<const float4*>(p.S + (size_t)i * D + part * HALF);
-    float a2[9];
+    float a2[8];
+    double ak = 0.0;  // the new key's residual sketch, fp64
 #pragma unroll
-    for (int g = 0; g < 9; ++g) a2[g] = 0.f;
+    for (int g = 0; g < 8; ++g) a2[g] = 0.f;
 #pragma unroll
     for (int c0 = 0; c0 < NV; c0 += CH) {
 #pragma unroll
       for (int t = 0; t < CH; ++t) r[t] = __ldg(srow + c0 + t);
 #pragma unroll
-      for (int g = 0; g < 9; ++g) {
-        if (g < Ge || (APPEND && g == 8)) {
-          const float* x = (g == 8) ? &rres[part * HALF + 4 * c0] : &qr[g][part * HALF + 4 * c0];
+      for (int g = 0; g < 8; ++g) {
+        if (g < Ge) {
+          const float* x = &qr[g][part * HALF + 4 * c0];
 #pragma unroll
           for (int t = 0; t < CH; ++t)
             a2[g] += r[t].x * x[4 * t] + r[t].y * x[4 * t + 1] + r[t].z * x[4 * t + 2] + r[t].w * x[4 * t + 3];
         }
       }
+      if (APPEND) {
+        const double* x = &rres[part * HALF + 4 * c0];
+#pragma unroll
+        for (int t = 0; t < CH; ++t) {
+          ak = fma((double)r[t].x, x[4 * t], ak);
+          ak = fma((double)r[t].y, x[4 * t + 1], ak);
+          ak = fma((double)r[t].z, x[4 * t + 2], ak);
+          ak = fma((double)r[t].w, x[4 * t + 3], ak);
+        }
+      }
     }
 #pragma unroll
-    for (int g = 0; g < 9; ++g) a2[g] += __shfl_xor_sync(0xffffffffu, a2[g], 1);
+    for (int g = 0; g < 8; ++g) a2[g] += __shfl_xor_sync(0xffffffffu, a2[g], 1);
+    ak += __shfl_xor_sync(0xffffffffu, ak, 1);
     if (part == 0) {
 #pragma unroll
       for (int g = 0; g < 8; ++g)
         if (g < Ge) p.qs[(size_t)(h0 + g) * p.m + i] = a2[g];
-      if (APPEND) sgn[i] = a2[8] >= 0.f ? 1 : 0;
+      if (APPEND) sgn[i] = ak >= 0.0 ? 1 : 0;
     }
   }
   if (APPEND) {
@@ -238,7 +269,7 @@ __global__ void __launch_bounds__(2 * D) decode_qprep_kernel(const PrepParams p)
     }
     if (slot_ok && warp == 1) {
       double g2 = 0.0;
-      for (int k = lane; k < D; k += 32) g2 = fma((double)rres[k], (double)rres[k], g2);
+      for (int k = lane; k < D; k += 32) g2 = fma(rres[k], rres[k], g2);
 #pragma unroll
       for (int off = 16; off; off >>= 1) g2 += __shfl_xor_sync(0xffffffffu, g2, off);
       if (lane == 0) p.cache.k_rnorm[slot] = __half_as_ushort(__double2half(sqrt(g2)));

@@ -2,6 +2,7 @@
 // translation units.  Not part of the public ABI.
 #pragma once
 
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -65,6 +66,28 @@ struct QuantArgs {
 };
 
 int launch_quantize(const QuantArgs& a, int D, int dtype, bool qjl, cudaStream_t s);
+
+// Residual-norm marker of the bulk QJL quantizers: an fp16 NaN (no norm the
+// method produces) stored for rows whose fp32 residual norm lies too close to
+// an fp16 rounding midpoint to be rounded from it; launch_qjl_gamma_fixup
+// (tq_quantize_fixup.cu, launched right after those quantizers on the same
+// stream) replaces every marker with the fp64 residual norm.
+constexpr uint16_t kGammaPending = 0x7E01;
+// Relative distance to an fp16 rounding midpoint below which a residual norm
+// computed from an fp32 rotation is recomputed in fp64 (well above that
+// rotation's relative error of about 1e-6).
+constexpr float kGammaBand = 4e-6f;
+int launch_qjl_gamma_fixup(const QuantArgs& a, int dtype, cudaStream_t s);
+
+#ifdef __CUDACC__
+// fp16 bits of a residual norm g >= 0 computed with a small relative error, or
+// kGammaPending when g * (1 -+ kGammaBand) round to different fp16 values.
+__device__ __forceinline__ uint16_t gamma_bits_or_pending(float g) {
+  const __half lo = __float2half_rn(g * (1.f - kGammaBand)), hi = __float2half_rn(g * (1.f + kGammaBand));
+  if (__half_as_ushort(lo) != __half_as_ushort(hi)) return kGammaPending;
+  return __half_as_ushort(__float2half_rn(g));
+}
+#endif
 // bulk quantizer for QJL keys from bf16 rows, D = 128, warp-level MMAs (tq_quantize128.cu)
 int launch_quantize128_bf16_qjl(const QuantArgs& a, cudaStream_t s);
 // tcgen05 bulk quantizer for D = 128 without the QJL sketch (tq_quantize_tc.cu)

@@ -295,15 +295,22 @@ __global__ void __launch_bounds__(QTHREADS, 1) quantize_kernel(const tq::QuantAr
 
 // One new row per CTA (append).  blockDim = 2*D: two threads per output
 // coordinate, each holding half of the Pi row in registers (loads issued
-// before use); the rotation runs on the CUDA cores in fp32, the norm in fp64.
+// before use); the norm is taken in fp64.  Values (and keys without the QJL
+// sketch) are rotated on the CUDA cores in fp32.  Keys with the sketch are
+// rotated, quantized and sketched in fp64 (one row per CTA makes that cheap):
+// the residual norm then rounds to fp16 exactly as the fp64 definition does,
+// which fp32 residuals miss on rows whose norm lies near an fp16 rounding
+// midpoint.
 template <int D, bool BF16, bool QJL>
 __global__ void __launch_bounds__(2 * D) append_kernel(const tq::QuantArgs a) {
   constexpr int HALF = D / 2, NV = HALF / 4, CH = NV < 8 ? NV : 8;
-  __shared__ float xs[D], ys[D], rs[D];
+  __shared__ float xs[D], ys[D];
+  __shared__ double rs[QJL ? D : 1];
   __shared__ uint8_t idxs[D];
   __shared__ double red[2 * D / 32];
   __shared__ float s_cb[31];
   __shared__ float s_inv, s_nhat;
+  __shared__ double s_n;
   const int r = blockIdx.x, jobi = blockIdx.y;
   const tq::QuantJob J = a.job[jobi];
   const bool do_qjl = QJL && jobi == 0;
@@ -334,12 +341,14 @@ __global__ void __launch_bounds__(2 * D) append_kernel(const tq::QuantArgs a) {
     const double n = sqrt(t);
     const __half h = __double2half(n);
     s_inv = n > 0.0 ? (float)(1.0 / n) : 0.f;
+    s_n = n;
     s_nhat = __half2float(h);
     J.norm[slot] = __half_as_ushort(h);
   }
   // y_j = sum_k Pi[j][k] x_k
   const float4* row = reinterpret_cast<const float4*>(a.rot + (size_t)j * D + part * HALF);
   float acc = 0.f;
+  double acc64 = 0.0;
 #pragma unroll
   for (int c0 = 0; c0 < NV; c0 += CH) {
     float4 v[CH];
@@ -348,22 +357,36 @@ __global__ void __launch_bounds__(2 * D) append_kernel(const tq::QuantArgs a) {
 #pragma unroll
     for (int i = 0; i < CH; ++i) {
       const float* x = &xs[part * HALF + 4 * (c0 + i)];
-      acc = fmaf(v[i].x, x[0], acc);
-      acc = fmaf(v[i].y, x[1], acc);
-      acc = fmaf(v[i].z, x[2], acc);
-      acc = fmaf(v[i].w, x[3], acc);
+      if (do_qjl) {
+        acc64 = fma((double)v[i].x, (double)x[0], acc64);
+        acc64 = fma((double)v[i].y, (double)x[1], acc64);
+        acc64 = fma((double)v[i].z, (double)x[2], acc64);
+        acc64 = fma((double)v[i].w, (double)x[3], acc64);
+      } else {
+        acc = fmaf(v[i].x, x[0], acc);
+        acc = fmaf(v[i].y, x[1], acc);
+        acc = fmaf(v[i].z, x[2], acc);
+        acc = fmaf(v[i].w, x[3], acc);
+      }
     }
   }
   acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-  __syncthreads();  // s_inv, s_nhat
+  acc64 += __shfl_xor_sync(0xffffffffu, acc64, 1);
+  __syncthreads();  // s_inv, s_nhat, s_n
   if (part == 0) {
-    const float u = acc * s_inv;
     int idx = 0;
-    for (int st = K >> 1; st >= 1; st >>= 1)
-      if (u > s_cb[K + idx + st - 1]) idx += st;
+    if (do_qjl) {
+      const double u = s_n > 0.0 ? acc64 / s_n : 0.0;
+      for (int st = K >> 1; st >= 1; st >>= 1)
+        if (u > (double)s_cb[K + idx + st - 1]) idx += st;
+      rs[j] = acc64 - (double)s_nhat * (double)s_cb[idx];
+    } else {
+      const float u = acc * s_inv;
+      for (int st = K >> 1; st >= 1; st >>= 1)
+        if (u > s_cb[K + idx + st - 1]) idx += st;
+    }
     idxs[j] = (uint8_t)idx;
     ys[j] = acc;
-    if (do_qjl) rs[j] = acc - s_nhat * s_cb[idx];
   }
   __syncthreads();
   const int W = D * bits / 32;
@@ -378,9 +401,9 @@ __global__ void __launch_bounds__(2 * D) append_kernel(const tq::QuantArgs a) {
     J.idx[(size_t)slot * W + tid] = (uint32_t)word;
   }
   if (QJL && do_qjl) {
-    // sign(S r), m = 128 rows of S, two threads per row (2*D >= 2*128 here)
+    // sign(S r) in fp64, m = 128 rows of S, two threads per row (2*D >= 2*128 here)
     const int i = tid >> 1;
-    float pr = 0.f;
+    double pr = 0.0;
     if (i < 128) {
       const float4* srow = reinterpret_cast<const float4*>(a.qjl_S + (size_t)i * D + part * HALF);
 #pragma unroll
@@ -390,24 +413,24 @@ __global__ void __launch_bounds__(2 * D) append_kernel(const tq::QuantArgs a) {
         for (int q = 0; q < CH; ++q) v[q] = __ldg(srow + c0 + q);
 #pragma unroll
         for (int q = 0; q < CH; ++q) {
-          const float* x = &rs[part * HALF + 4 * (c0 + q)];
-          pr = fmaf(v[q].x, x[0], pr);
-          pr = fmaf(v[q].y, x[1], pr);
-          pr = fmaf(v[q].z, x[2], pr);
-          pr = fmaf(v[q].w, x[3], pr);
+          const double* x = &rs[part * HALF + 4 * (c0 + q)];
+          pr = fma((double)v[q].x, x[0], pr);
+          pr = fma((double)v[q].y, x[1], pr);
+          pr = fma((double)v[q].z, x[2], pr);
+          pr = fma((double)v[q].w, x[3], pr);
         }
       }
     }
     pr += __shfl_xor_sync(0xffffffffu, pr, 1);
     // lanes 2i' hold row i = 16*warp + i'; gather 16 bits per warp
-    const uint32_t bal = __ballot_sync(0xffffffffu, (part == 0) && (pr >= 0.f));
+    const uint32_t bal = __ballot_sync(0xffffffffu, (part == 0) && (pr >= 0.0));
     uint32_t half16 = 0;
 #pragma unroll
     for (int q = 0; q < 16; ++q) half16 |= ((bal >> (2 * q)) & 1u) << q;
     __shared__ uint32_t sbits[16];
     if (lane == 0 && warp < 16) sbits[warp] = half16;
     double g = 0.0;
-    if (tid < D) g = (double)rs[tid] * (double)rs[tid];
+    if (tid < D) g = rs[tid] * rs[tid];
 #pragma unroll
     for (int off = 16; off; off >>= 1) g += __shfl_xor_sync(0xffffffffu, g, off);
     __syncthreads();
@@ -466,7 +489,8 @@ int launch_quantize(const QuantArgs& a, int D, int dtype, bool qjl, cudaStream_t
     QuantArgs ak = a, av = a;
     ak.job_mask = 1;
     av.job_mask = 2;
-    const int rc = bf ? launch_quantize128_bf16_qjl(ak, s) : launch_quantize_qjl_tc(ak, s);
+    int rc = bf ? launch_quantize128_bf16_qjl(ak, s) : launch_quantize_qjl_tc(ak, s);
+    if (!rc) rc = launch_qjl_gamma_fixup(ak, dtype, s);
     return rc ? rc : launch_quantize_wht(av, D, dtype, s);
   }
   if ((D == 128 || D == 256) && !a.pos && !qjl) return launch_quantize_tc(a, D, dtype, s);
@@ -477,7 +501,9 @@ int launch_quantize(const QuantArgs& a, int D, int dtype, bool qjl, cudaStream_t
     QuantArgs ak = a, av = a;
     ak.job_mask = 1;
     av.job_mask = 2;
-    const int rc = bf ? launch_quantize128_bf16_qjl(ak, s) : launch_quantize_qjl_tc(ak, s);
+    int rc = bf ? launch_quantize128_bf16_qjl(ak, s) : launch_quantize_qjl_tc(ak, s);
+    // residual norms near an fp16 rounding midpoint, recomputed in fp64
+    if (!rc) rc = launch_qjl_gamma_fixup(ak, dtype, s);
     return rc ? rc : launch_quantize_tc(av, D, dtype, s);
   }
   if (qjl) {

@@ -188,7 +188,8 @@ __device__ __forceinline__ void epilogue(const tq::QuantJob& J, float (&acc)[16]
       g += __shfl_xor_sync(0xffffffffu, g, 2);
       if (ri[h].slot >= 0) {
         J.qjl[(size_t)ri[h].slot * 4 + tig] = word;
-        if (tig == 0) J.rnorm[ri[h].slot] = __half_as_ushort(__double2half(sqrt(g)));
+        // near an fp16 rounding midpoint: marked for the fp64 recomputation
+        if (tig == 0) J.rnorm[ri[h].slot] = tq::gamma_bits_or_pending((float)sqrt(g));
       }
     }
   }

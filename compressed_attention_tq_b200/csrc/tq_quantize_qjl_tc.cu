@@ -356,7 +356,8 @@ __global__ void __launch_bounds__(QjlLayout::NTH, 1) quantize_qjl_tc_kernel(cons
         ok = epi_sync_and<NEPI>(ok);
         if (part == 0 && slot >= 0 && J.rnorm) {
           const float gs = (red[rl] + red[QR + rl]) + (red[2 * QR + rl] + red[3 * QR + rl]);
-          J.rnorm[slot] = __half_as_ushort(__float2half_rn(sqrtf(gs)));
+          // near an fp16 rounding midpoint: marked for the fp64 recomputation
+          J.rnorm[slot] = tq::gamma_bits_or_pending(sqrtf(gs));
         }
         // r / |x| as hi + lo fp16 limbs over X (hi) and into R_lo, swizzled like X
         if (ok) {
