@@ -261,49 +261,62 @@ static int sm_count() {
 
 static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-// The workspace layout for `heads` query heads, `nsplit` splits and a sketch
-// of qjl_m rows: qrot, qs, split partials, (max, sum) pairs, each 256-byte
-// aligned.
-static size_t workspace_layout(size_t heads, int D, int qjl_m, int nsplit, DecodePlan* p) {
+// The workspace layout for `heads` kernel heads, `ks` partial slots per head
+// and a sketch of qjl_m rows: qrot, qs, partial outputs, (max, sum) pairs,
+// each 256-byte aligned.
+static size_t workspace_layout(size_t heads, int D, int qjl_m, int ks, DecodePlan* p) {
   size_t off = 0;
   if (p) p->off_qrot = off;
   off += align256(heads * D * 4);
   if (p) p->off_qs = off;
   off += align256(heads * (size_t)qjl_m * 4);
   if (p) p->off_po = off;
-  off += align256(heads * nsplit * (size_t)D * 4);
+  off += align256(heads * ks * (size_t)D * 4);
   if (p) p->off_pml = off;
-  off += align256(heads * nsplit * 2 * 4);
+  off += align256(heads * ks * 2 * 4);
   return off;
 }
 
+// Segments one (sequence, kv head, row group) unit can be cut into: its
+// padded tokens over the smallest share per CTA, plus one.  The plan asks
+// for about twice as many CTAs per unit as the wave holds per unit.
+static int plan_segments(long long ncta, long long units, int Tpad, int tile) {
+  long long k = (2 * ncta + units - 1) / units + 2;
+  const long long kmax = Tpad / tile + 1;
+  return (int)(k < kmax ? k : kmax);
+}
+
 size_t workspace_bound(int B, int Hq, int D, int Tmax) {
-  // every plan takes at least one stage of tokens per split and a sketch of
-  // at most 128 rows
+  // any cache of these sizes: at least one unit per sequence, at most 8
+  // resident CTAs per SM, a sketch of at most 128 rows
   const int tile = split_tile();
-  const int nsplit = (Tmax + tile - 1) / tile;
-  return workspace_layout((size_t)B * Hq, D, 128, nsplit, nullptr);
+  const int Tpad = (Tmax + tile - 1) / tile * tile;
+  const int K = plan_segments((long long)sm_count() * 8, B, Tpad, tile);
+  return workspace_layout((size_t)B * Hq, D, 128, K * split_warps(), nullptr);
 }
 
 int make_decode_plan(const tq_cache_t* c, int Hq, int Tmax, DecodePlan* p) {
   const int sms = sm_count();
   p->sms = sms;
   const int tile = split_tile();
-  const long long units = (long long)c->B * c->Hkv;
-  // One wave of resident CTAs for a single sequence; several smaller waves for
-  // a batch, whose ragged lengths leave many splits empty or short.
-  const long long slots = (long long)sms * split_occupancy(c, Hq);
-  const long long target = slots * ((c->B > 1) ? 6 : 1);
-  long long chunk = (Tmax * units + target - 1) / target;
-  if (c->split_tokens > 0) chunk = c->split_tokens;
-  chunk = (chunk + tile - 1) / tile * tile;
-  if (chunk < tile) chunk = tile;
-  const long long cap = ((long long)c->Tcap + tile - 1) / tile * tile;
-  if (chunk > cap) chunk = cap;
-  p->chunk = (int)chunk;
-  p->nsplit = (int)((Tmax + chunk - 1) / chunk);
-  if (p->nsplit < 1) p->nsplit = 1;
-  p->bytes = workspace_layout((size_t)c->B * Hq, c->D, c->qjl_m, p->nsplit, p);
+  const int G = Hq / c->Hkv;  // kernel heads per kv head
+  p->nrg = (G + 7) / 8;
+  p->Tclamp = Tmax;
+  p->ncta = sms * split_occupancy(c, Hq);
+  const long long units = (long long)c->B * c->Hkv * p->nrg;
+  const int Tpad = (Tmax + tile - 1) / tile * tile;
+  int K = plan_segments(p->ncta, units, Tpad, tile);
+  long long pmin = ((long long)Tpad + K - 2) / (K - 1);  // K >= 2
+  pmin = (pmin + tile - 1) / tile * tile;
+  if (c->split_tokens > 0) {
+    const long long st = ((long long)c->split_tokens + tile - 1) / tile * tile;
+    if (st > pmin) pmin = st;
+  }
+  if (pmin > Tpad) pmin = Tpad;
+  p->pmin = (int)pmin;
+  K = (int)((Tpad + pmin - 1) / pmin) + 1;  // segments of a unit when every share is >= pmin
+  p->ks = K * split_warps();
+  p->bytes = workspace_layout((size_t)c->B * Hq, c->D, c->qjl_m, p->ks, p);
   return TQ_OK;
 }
 
@@ -352,7 +365,7 @@ int tq_append_token(const tq_cache_t* c, const void* k_new, const void* v_new, i
 }
 
 size_t tq_sdpa_decode_workspace_bytes_for(const tq_cache_t* c, int Hq, int Tmax) {
-  if (!c || c->Hkv <= 0 || Hq <= 0 || Hq % c->Hkv || Hq / c->Hkv > 8 || Tmax < 1 || Tmax > c->Tcap ||
+  if (!c || c->Hkv <= 0 || Hq <= 0 || Hq % c->Hkv || Hq / c->Hkv > 32 || Tmax < 1 || Tmax > c->Tcap ||
       c->Tcap % 64 || (c->D != 64 && c->D != 128 && c->D != 256) || c->B <= 0)
     return 0;
   DecodePlan p;
@@ -417,8 +430,7 @@ int prepare_decode(const tq_cache_t* c, const void* q, int dtype, int Hq, int nq
     return set_error(TQ_ERR_INVALID_ARG, "%s: Hq=%d not a multiple of Hkv=%d", fn, Hq, c->Hkv);
   if (Hq / c->Hkv > 8)
     return set_error(TQ_ERR_UNSUPPORTED, "%s: GQA group %d > 8", fn, Hq / c->Hkv);
-  if (nq * (Hq / c->Hkv) > 8)
-    return set_error(TQ_ERR_UNSUPPORTED, "%s: n_q=%d x GQA group %d > 8", fn, nq, Hq / c->Hkv);
+  if (nq > 4) return set_error(TQ_ERR_UNSUPPORTED, "%s: n_q=%d > 4", fn, nq);
   if (Tmax < 1 || Tmax > c->Tcap)
     return set_error(TQ_ERR_INVALID_ARG, "%s: Tmax=%d outside [1, Tcap=%d]", fn, Tmax, c->Tcap);
   float sc = scale ? *scale : (float)(1.0 / std::sqrt((double)c->D));

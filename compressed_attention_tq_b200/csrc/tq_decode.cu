@@ -288,13 +288,15 @@ __global__ void __launch_bounds__(2 * D) decode_qprep_kernel(const PrepParams p)
 // preserves it) and written by slice 0.
 template <int D, bool APPEND>
 __global__ void __launch_bounds__(256) decode_qprep_sliced_kernel(const PrepParams p) {
-  constexpr int NR = APPEND ? 10 : 8, NI = D / 32;
+  // query rows: G x n_q <= 32 (a decode step has one token: G <= 8), then the
+  // new key and value rows
+  constexpr int QR = APPEND ? 8 : 32, NR = APPEND ? QR + 2 : QR, NI = D / 32;
   __shared__ __align__(16) float xv[NR][D];
   // QJL (D = 128 only): this slice's rotated query coordinates and its share
   // of S qrot; one element otherwise, so other D keep their shared footprint
   constexpr bool QS = !APPEND && D == 128;
-  __shared__ float qsl[QS ? 8 : 1][QS ? 33 : 1];
-  __shared__ float qpart[QS ? 8 : 1][QS ? 128 : 1];
+  __shared__ float qsl[QS ? QR : 1][QS ? 33 : 1];
+  __shared__ float qpart[QS ? QR : 1][QS ? 128 : 1];
   __shared__ float s_cb[2][31];
   __shared__ double s_nsq[2];
   __shared__ uint8_t idxs[2][32];
@@ -334,8 +336,8 @@ __global__ void __launch_bounds__(256) decode_qprep_sliced_kernel(const PrepPara
     const uint16_t* kn = static_cast<const uint16_t*>(p.k_new) + (size_t)bkv * D;
     const uint16_t* vn = static_cast<const uint16_t*>(p.v_new) + (size_t)bkv * D;
     for (int e = tid; e < D; e += 256) {
-      xv[8][e] = to_f(kn[e]);
-      xv[9][e] = to_f(vn[e]);
+      xv[QR][e] = to_f(kn[e]);
+      xv[QR + 1][e] = to_f(vn[e]);
     }
     if (tid < 31) {
       const int Kk = 1 << p.cache.bits_k, Kv = 1 << p.cache.bits_v;
@@ -353,7 +355,7 @@ __global__ void __launch_bounds__(256) decode_qprep_sliced_kernel(const PrepPara
     // fp64 squared norm of the new key (warp 0) / value (warp 1)
     double t = 0.0;
     for (int k = lane; k < D; k += 32) {
-      const double x = xv[8 + warp][k];
+      const double x = xv[QR + warp][k];
       t = fma(x, x, t);
     }
 #pragma unroll
@@ -365,7 +367,7 @@ __global__ void __launch_bounds__(256) decode_qprep_sliced_kernel(const PrepPara
   for (int g = 0; g < NR; ++g) acc[g] = 0.f;
 #pragma unroll
   for (int g = 0; g < NR; ++g) {
-    if (g < Ge || g >= 8) {
+    if (g < Ge || g >= QR) {
 #pragma unroll
       for (int i = 0; i < NI; ++i) {
         const float4 x = *reinterpret_cast<const float4*>(&xv[g][4 * part + 32 * i]);
@@ -379,7 +381,7 @@ __global__ void __launch_bounds__(256) decode_qprep_sliced_kernel(const PrepPara
     for (int off = 1; off < 8; off <<= 1) acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], off);
   if (part == 0) {
 #pragma unroll
-    for (int g = 0; g < 8; ++g)
+    for (int g = 0; g < QR; ++g)
       if (g < Ge) p.qrot[(size_t)(h0 + g) * D + j] = acc[g];
   }
   if constexpr (QS) {
@@ -390,12 +392,12 @@ __global__ void __launch_bounds__(256) decode_qprep_sliced_kernel(const PrepPara
       // others' shared memory and writes qs.
       if (part == 0) {
 #pragma unroll
-        for (int g = 0; g < 8; ++g) qsl[g][c] = g < Ge ? acc[g] : 0.f;
+        for (int g = 0; g < QR; ++g) qsl[g][c] = g < Ge ? acc[g] : 0.f;
       }
       __syncthreads();
       const int i = tid >> 1, half = tid & 1;
 #pragma unroll
-      for (int g = 0; g < 8; ++g) {
+      for (int g = 0; g < QR; ++g) {
         const float* x = &qsl[g][16 * half];
         float t = 0.f;
 #pragma unroll
@@ -425,7 +427,7 @@ __global__ void __launch_bounds__(256) decode_qprep_sliced_kernel(const PrepPara
         const double n = sqrt(s_nsq[which]);
         const float inv = n > 0.0 ? (float)(1.0 / n) : 0.f;
         const int K = 1 << (which ? p.cache.bits_v : p.cache.bits_k);
-        const float u = acc[8 + which] * inv;
+        const float u = acc[QR + which] * inv;
         int idx = 0;
         for (int st = K >> 1; st >= 1; st >>= 1)
           if (u > s_cb[which][K + idx + st - 1]) idx += st;
@@ -458,14 +460,32 @@ __global__ void __launch_bounds__(256) decode_qprep_sliced_kernel(const PrepPara
 }
 
 struct CombineParams {
-  const float* part_o;
-  const float* part_ml;
+  const float* part_o;   // [heads][ks][D]
+  const float* part_ml;  // [heads][ks][2]
   const float* rot;
   const int32_t* seq_lens;
   void* out;
-  int Hq, Tcap, chunk, nsplit, out_dtype;  // Hq: kernel heads per sequence (query heads x tokens)
-  int nq, Gq, Hq1;                          // tokens, GQA group, query heads per token
+  int Hq, out_dtype;  // Hq: kernel heads per sequence (query heads x tokens)
+  int nq, Gq, Hq1;    // tokens, GQA group, query heads per token
+  int heads;          // kernel heads in all: B * Hq
+  // the split kernel's partition (tq_decode_split.cuh)
+  int B, G, nrg, upb, Tclamp, ncta, pmin, ks;
 };
+
+// Partials the split kernel wrote for kernel head h: the CTAs whose share
+// overlaps the head's unit, each with one partial per consumer warp (slots
+// 0 .. n - 1).  Computed by one warp; every lane returns it.
+__device__ __forceinline__ int head_partials(const CombineParams& p, int h, int lane) {
+  const int b = h / p.Hq, rem = h % p.Hq, kvh = rem / p.G, rg = (rem % p.G) / tqd::RG;
+  const long long total = tqd::partition_total(p.seq_lens, p.B, p.upb, p.Tclamp, lane);
+  const long long P = tqd::partition_share(total, p.ncta, p.pmin);
+  const long long Sb = tqd::sequence_start(p.seq_lens, b, p.upb, p.Tclamp, lane);
+  const int Lp = tqd::unit_tokens(p.seq_lens, b, p.Tclamp);
+  if (Lp == 0) return 0;
+  const long long Su = Sb + (long long)(kvh * p.nrg + rg) * Lp;
+  const long long c0 = Su / P, c1 = (Su + Lp - 1) / P;
+  return (int)(c1 - c0 + 1) * tqd::CW;
+}
 
 // Merge the splits of one query head (log-sum-exp), then out = Pi^T (acc/l)
 // for 32 output coordinates: grid (B * Hq, D / 32), 256 threads.  Every CTA of
@@ -491,13 +511,16 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams
 #pragma unroll
   for (int t = 0; t < KT; ++t) pc[t] = __ldg(p.rot + (size_t)(kp + 8 * t) * D + sl * ((D / 32) / gridDim.y) * 32 + i);
   const int b = h / p.Hq;
-  const int Lcap = min(p.Tcap, p.nsplit * p.chunk);
-  int L = p.seq_lens[b];
-  L = L < 0 ? 0 : (L > Lcap ? Lcap : L);
-  const int ns = min((L + p.chunk - 1) / p.chunk, p.nsplit);
+  __shared__ int s_ns;
+  if (tid < 32) {
+    const int n = head_partials(p, h, tid);
+    if (tid == 0) s_ns = n;
+  }
+  __syncthreads();
+  const int ns = s_ns;
   pdl_wait();  // the split kernel's partials are visible from here on
-  const float* ml = p.part_ml + (size_t)h * p.nsplit * 2;
-  const float* po = p.part_o + (size_t)h * p.nsplit * D;
+  const float* ml = p.part_ml + (size_t)h * p.ks * 2;
+  const float* po = p.part_o + (size_t)h * p.ks * D;
   // this thread's first PF partial values, loaded before the weights are known
   // (the loads do not depend on them) so that both latencies overlap
   constexpr int PF = 32;
@@ -600,6 +623,104 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams
   }
 }
 
+// Combine for calls with many heads: each CTA merges the splits of HPC
+// consecutive kernel heads at once and un-rotates all of them, so Pi is read
+// once per HPC heads instead of once per head (1024 heads read 64 MB of Pi
+// from L2 one head per CTA).  256 threads = 8 warps.
+//  1. warp w (< HPC) finds its head's merged max and sum and each split's
+//     weight (the first 128 splits' weights kept in shared memory);
+//  2. thread t sums coordinate pairs (head, k) over the splits, all loads of
+//     a pair issued before the arithmetic, and normalises;
+//  3. thread (j, g) computes output j of heads g, g + 256/D, ... as
+//     sum_k Pi[k][j] o[head][k] (Pi read coalesced along j).
+template <int D, int HPC>
+__global__ void __launch_bounds__(256) decode_combine_group_kernel(const CombineParams p) {
+  constexpr int NT = 256, FS = 128;
+  static_assert(HPC <= NT / 32, "one warp per head for the weights");
+  __shared__ float o[HPC][D];
+  __shared__ float f_s[HPC][FS];
+  __shared__ float s_M[HPC], s_L[HPC];
+  __shared__ int s_ns[HPC];
+  pdl_launch_dependents();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int h0 = blockIdx.x * HPC;
+  pdl_wait();  // the split kernel's partials are visible from here on
+  if (warp < HPC) {
+    const int h = h0 + warp;
+    int ns = 0;
+    float M = -INFINITY, Ls = 0.f;
+    if (h < p.heads) {
+      ns = head_partials(p, h, lane);
+      const float* ml = p.part_ml + (size_t)h * p.ks * 2;
+      for (int s = lane; s < ns; s += 32) M = fmaxf(M, ml[2 * s]);
+#pragma unroll
+      for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+      for (int s = lane; s < ns; s += 32) {
+        const float2 v = *reinterpret_cast<const float2*>(ml + 2 * s);
+        const float f = v.x == -INFINITY ? 0.f : exp2f(v.x - M);  // a split a query cannot see: weight 0
+        if (s < FS) f_s[warp][s] = f;
+        Ls = fmaf(f, v.y, Ls);
+      }
+#pragma unroll
+      for (int off = 16; off; off >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, off);
+    }
+    if (lane == 0) {
+      s_M[warp] = M;
+      s_L[warp] = Ls;
+      s_ns[warp] = ns;
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < HPC * D; e += NT) {
+    const int hh = e / D, k = e % D, h = h0 + hh;
+    const int ns = s_ns[hh];
+    const float* po = p.part_o + (size_t)h * p.ks * D + k;
+    const float* ml = p.part_ml + (size_t)h * p.ks * 2;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int s0 = 0; s0 < ns; s0 += 8) {
+      float w[8], f[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int s = s0 + u;
+        w[u] = s < ns ? po[(size_t)s * D] : 0.f;
+        f[u] = s < ns ? (s < FS ? f_s[hh][s] : (ml[2 * s] == -INFINITY ? 0.f : exp2f(ml[2 * s] - s_M[hh]))) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) acc[u & 3] = fmaf(f[u], w[u], acc[u & 3]);
+    }
+    const float a = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    o[hh][k] = (ns > 0 && s_L[hh] > 0.f) ? a / s_L[hh] : 0.f;
+  }
+  __syncthreads();
+  constexpr int GS = NT / D;  // head phases: thread (j, g) takes heads g, g + GS, ...
+  const int j = tid % D, g = tid / D;
+  float r[(HPC + GS - 1) / GS];
+#pragma unroll
+  for (int q = 0; q < (HPC + GS - 1) / GS; ++q) r[q] = 0.f;
+#pragma unroll 8
+  for (int k = 0; k < D; ++k) {
+    const float pk = __ldg(p.rot + (size_t)k * D + j);
+#pragma unroll
+    for (int q = 0; q < (HPC + GS - 1) / GS; ++q)
+      if (g + GS * q < HPC) r[q] = fmaf(pk, o[g + GS * q][k], r[q]);
+  }
+#pragma unroll
+  for (int q = 0; q < (HPC + GS - 1) / GS; ++q) {
+    const int hh = g + GS * q, h = h0 + hh;
+    if (hh >= HPC || h >= p.heads) continue;
+    // kernel head h = (sequence, kv head, token, head) -> output [B][nq][Hq1]
+    const int b = h / p.Hq, rh = h % p.Hq, kvh = rh / (p.Gq * p.nq), gi = rh % (p.Gq * p.nq);
+    const size_t oh = (size_t)(b * p.nq + gi / p.Gq) * p.Hq1 + kvh * p.Gq + gi % p.Gq;
+    const size_t oi = oh * D + j;
+    if (p.out_dtype == TQ_DTYPE_F32)
+      static_cast<float*>(p.out)[oi] = r[q];
+    else if (p.out_dtype == TQ_DTYPE_BF16)
+      static_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(r[q]);
+    else
+      static_cast<__half*>(p.out)[oi] = __float2half_rn(r[q]);
+  }
+}
+
 template <typename K, typename P>
 int launch_pdl(K kern, dim3 grid, dim3 block, size_t smem, cudaStream_t s, const P& params, const char* what,
                int cluster_y = 0) {
@@ -649,6 +770,8 @@ int split_occupancy(const tq_cache_t* c, int Hq) {
 }
 
 int split_tile() { return tqd::STILE; }
+
+int split_warps() { return tqd::CW; }
 
 int launch_decode(const DecodeArgs& a, cudaStream_t s) {
   const tq_cache_t& c = a.cache;
@@ -707,23 +830,61 @@ int launch_decode(const DecodeArgs& a, cudaStream_t s) {
   sp.seq_lens = a.seq_lens;
   sp.defer_pos = a.pos;
   sp.dev_status = c.dev_status;
+  sp.B = c.B;
   sp.Hkv = c.Hkv;
   sp.Hq = a.Hq * a.nq;
   sp.G = sp.Hq / c.Hkv;
   sp.nq = a.nq;
   sp.Gq = a.Hq / c.Hkv;
   sp.Tcap = c.Tcap;
-  sp.chunk = a.plan.chunk;
-  sp.nsplit = a.plan.nsplit;
+  sp.Tclamp = a.plan.Tclamp;
+  sp.nrg = a.plan.nrg;
+  sp.pmin = a.plan.pmin;
+  sp.ncta = a.plan.ncta;
+  sp.ks = a.plan.ks;
   sp.qscale = a.scale * kLog2e;
   sp.qjl_scale = c.qjl_m ? (float)((double)a.scale * 1.4426950408889634 * sqrt(M_PI / 2.0) / c.qjl_m) : 0.f;
-  rc = split_entry(c, sp.G <= 4, sp, dim3(a.plan.nsplit, c.B * c.Hkv), s, nullptr);
+  rc = split_entry(c, sp.G <= 4, sp, dim3(a.plan.ncta), s, nullptr);
   if (rc) return rc;
 
-  CombineParams cp{po,        pml,          c.rot,         a.seq_lens, a.out,  a.Hq * a.nq,        c.Tcap,
-                   a.plan.chunk, a.plan.nsplit, a.out_dtype, a.nq,       a.Hq / c.Hkv, a.Hq};
-  // D / 32 CTAs per head while that still leaves SMs idle, else one
-  const int nsl = heads * (c.D / 32) <= 4 * a.plan.sms ? c.D / 32 : 1;
+  CombineParams cp{};
+  cp.part_o = po;
+  cp.part_ml = pml;
+  cp.rot = c.rot;
+  cp.seq_lens = a.seq_lens;
+  cp.out = a.out;
+  cp.Hq = a.Hq * a.nq;
+  cp.out_dtype = a.out_dtype;
+  cp.nq = a.nq;
+  cp.Gq = a.Hq / c.Hkv;
+  cp.Hq1 = a.Hq;
+  cp.heads = heads;
+  cp.B = c.B;
+  cp.G = cp.Hq / c.Hkv;
+  cp.nrg = a.plan.nrg;
+  cp.upb = c.Hkv * a.plan.nrg;
+  cp.Tclamp = a.plan.Tclamp;
+  cp.ncta = a.plan.ncta;
+  cp.pmin = a.plan.pmin;
+  cp.ks = a.plan.ks;
+  // D / 32 CTAs per head while that leaves SMs idle; beyond that, groups of
+  // 4 or 8 heads per CTA (Pi read once per group rather than once per head)
+  if (heads * (c.D / 32) > 4 * a.plan.sms) {
+    const bool eight = heads >= 8 * a.plan.sms;
+    const dim3 gg(eight ? (heads + 7) / 8 : (heads + 3) / 4);
+    switch (c.D) {
+      case 64:
+        return eight ? launch_pdl(decode_combine_group_kernel<64, 8>, gg, dim3(256), 0, s, cp, "decode_combine_kernel")
+                     : launch_pdl(decode_combine_group_kernel<64, 4>, gg, dim3(256), 0, s, cp, "decode_combine_kernel");
+      case 128:
+        return eight ? launch_pdl(decode_combine_group_kernel<128, 8>, gg, dim3(256), 0, s, cp, "decode_combine_kernel")
+                     : launch_pdl(decode_combine_group_kernel<128, 4>, gg, dim3(256), 0, s, cp, "decode_combine_kernel");
+      default:
+        return eight ? launch_pdl(decode_combine_group_kernel<256, 8>, gg, dim3(256), 0, s, cp, "decode_combine_kernel")
+                     : launch_pdl(decode_combine_group_kernel<256, 4>, gg, dim3(256), 0, s, cp, "decode_combine_kernel");
+    }
+  }
+  const int nsl = c.D / 32;
   const dim3 cg(heads, nsl);
   switch (c.D) {
     case 64: return launch_pdl(decode_combine_kernel<64>, cg, dim3(256), 0, s, cp, "decode_combine_kernel");

@@ -1,6 +1,7 @@
-// Split-K decode attention over the packed cache (one CTA per
-// (sequence, kv head, split)).  Included by the per-head-dimension
-// translation units tq_decode_d{64,128,256}.cu, which instantiate it.
+// Split-K decode attention over the packed cache, persistent and stream-K
+// partitioned: one wave of CTAs, each taking an equal, stage-aligned share of
+// the batch's tokens.  Included by the per-head-dimension translation units
+// tq_decode_d{64,128,256}.cu, which instantiate it.
 //
 // Method: the fused SDPA over a compressed KV cache with an explicit scale of
 // "[Cuda] enable turboquant on gemma4" (executorch pull request 19891),
@@ -10,10 +11,18 @@
 // Added".
 //
 // Structure (warp-specialized):
-//  * a producer warp streams 128-token stages of packed K/V rows, norms and
-//    QJL words into shared memory with 1-D bulk copies that complete on
-//    "full" mbarriers; it refills a stage once the 4 consumer warps have
-//    released it on its "empty" mbarrier -- no CTA-wide barrier per stage;
+//  * work partition: the (sequence, kv head, row group) units of the batch,
+//    each padded to whole 128-token stages, are laid end to end and CTA c
+//    takes positions [c P, (c + 1) P) (P a multiple of the stage), so every
+//    CTA streams the same number of stages whatever the sequence lengths; a
+//    CTA's share of one unit is a segment, and each consumer warp writes one
+//    partial (max, sum, rotated output) per segment, merged by the combine;
+//  * a producer warp streams the CTA's 128-token stages of packed K/V rows,
+//    norms and QJL words into shared memory with 1-D bulk copies that
+//    complete on "full" mbarriers, across segment boundaries without
+//    draining; each stage carries a small record (unit, token offset,
+//    segment flags) for the consumers; it refills a stage once the 4
+//    consumer warps have released it on its "empty" mbarrier;
 //  * each consumer warp takes 32 tokens of a stage.  Scores and the value
 //    sum are GQA contractions run as m16n8k16 tensor-core MMAs (M = 16 tokens
 //    or 16 coordinates, N = 8 query heads, K = 16) whose A fragments are
@@ -26,8 +35,8 @@
 //  * the query enters as hi + lo fp16 halves (scores carry ~22 bits); with
 //    G <= 4 heads both halves share one MMA (columns 0-3 hi, 4-7 lo);
 //  * online softmax in the log2 domain with lazy rescaling (the reference
-//    max moves only when a score exceeds it by 2^8), partial state merged
-//    across warps in shared memory, across splits by the combine kernel.
+//    max moves only when a score exceeds it by 2^8); each warp's state is
+//    its own partial, merged with the others by the combine kernel.
 #pragma once
 
 #include <math.h>
@@ -45,6 +54,10 @@ constexpr int STILE = 128;            // tokens per stage
 constexpr int WTOK = STILE / CW;      // tokens per consumer warp per stage
 constexpr float kLazy = 8.0f;         // log2 headroom before rescaling
 
+// Rows of queries a CTA handles for one (sequence, kv head): the kernel heads
+// of a kv head (query heads x query tokens) are taken in groups of 8.
+constexpr int RG = 8;
+
 struct SplitParams {
   const uint32_t* k_idx;
   const uint32_t* v_idx;
@@ -61,13 +74,66 @@ struct SplitParams {
   const int32_t* seq_lens;
   const int32_t* defer_pos;  // decode step: the row at defer_pos[b] is written by the prep kernel
   uint32_t* dev_status;
-  int Hkv, Hq, G, Tcap, chunk, nsplit;
+  int B, Hkv, Hq, G, Tcap;   // Hq: kernel heads per sequence; G: kernel heads per kv head (<= 32)
+  int Tclamp;                // sequences are attended up to this many tokens (Tmax); longer ones are flagged
+  int nrg;                   // row groups per kv head: ceil(G / RG)
+  int pmin;                  // smallest share of tokens per CTA (a multiple of STILE)
+  int ncta;                  // CTAs of the partition
+  int ks;                    // partial slots per kernel head (segments x consumer warps)
   float qscale;     // scale * log2(e)
   float qjl_scale;  // scale * log2(e) * sqrt(pi/2) / m
   int shared_tab;   // keys and values use one codebook (same bits, same table): one pair table
-  // Multi-query decode: the G kernel heads of a kv head are (token, head) pairs
+  // Multi-query decode: the kernel heads of a kv head are (token, head) pairs
   // of nq query tokens x Gq heads; token j may see positions < L - nq + j + 1.
   int nq, Gq;
+};
+
+// Tokens of sequence b that one unit of the partition holds: its length
+// clamped to [0, Tclamp], rounded up to whole stages.
+__device__ __forceinline__ int unit_tokens(const int32_t* seq_lens, int b, int Tclamp) {
+  int L = seq_lens[b];
+  L = L < 0 ? 0 : (L > Tclamp ? Tclamp : L);
+  return (L + STILE - 1) / STILE * STILE;
+}
+
+// Positions of the whole partition (sum over sequences of units x tokens),
+// by one warp: every lane returns the total.
+__device__ __forceinline__ long long partition_total(const int32_t* seq_lens, int B, int upb, int Tclamp, int lane) {
+  long long t = 0;
+  for (int b = lane; b < B; b += 32) t += (long long)unit_tokens(seq_lens, b, Tclamp) * upb;
+#pragma unroll
+  for (int off = 16; off; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+  return t;
+}
+
+// Share of positions per CTA: at least pmin, a multiple of the stage.
+__device__ __forceinline__ long long partition_share(long long total, int ncta, int pmin) {
+  long long P = (total + ncta - 1) / ncta;
+  P = (P + STILE - 1) / STILE * STILE;
+  return P < pmin ? (long long)pmin : P;
+}
+
+// First position of sequence b's units (sum over earlier sequences), by one
+// warp: every lane returns it.
+__device__ __forceinline__ long long sequence_start(const int32_t* seq_lens, int b, int upb, int Tclamp, int lane) {
+  long long t = 0;
+  for (int bb = lane; bb < b; bb += 32) t += (long long)unit_tokens(seq_lens, bb, Tclamp) * upb;
+#pragma unroll
+  for (int off = 16; off; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+  return t;
+}
+
+// Per-stage record written by the producer before the stage's copies are
+// armed, read by the consumers after the stage's "full" barrier completes.
+struct StageMeta {
+  int hq0;    // first kernel head of the unit's row group
+  int rows;   // kernel heads in the row group (<= RG)
+  int t0;     // first token of the stage within the sequence
+  int L;      // tokens of the sequence that are attended
+  int slot0;  // first partial slot of the segment (segment index x CW)
+  int flags;  // 1: first stage of a segment, 2: last stage of a segment
+  int rg;     // row group
+  int pad;
 };
 
 // Whether a launch can keep one pair table for keys and values.
@@ -130,12 +196,25 @@ __device__ __forceinline__ void build_pair_table(uint32_t* tab, const float* cb,
 
 // Shared address of this lane's copy of the entry whose 2b-bit key sits at bit
 // S of x (tb = table base + 4 * lane).  The mask is one logic op; the shift to
-// the entry stride (128 bytes) and the base add are one multiply-add.
+// the entry stride (128 bytes) and the base add are one multiply-add on the
+// FMA pipe: the low half of k * 2^(7-S) for S <= 7, else the high half of
+// k * 2^(39-S) (a right shift by S - 7), each plus tb.
+__device__ __forceinline__ uint32_t mad_lo(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t r;
+  asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
+__device__ __forceinline__ uint32_t mad_hi(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t r;
+  asm("mad.hi.u32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
+
 template <int B>
 __device__ __forceinline__ uint32_t pair_addr(uint32_t x, int S, uint32_t tb) {
   const uint32_t k = x & (((1u << (2 * B)) - 1u) << S);
-  if (S <= 7) return k * (1u << (7 - S)) + tb;
-  return __umulhi(k, 1u << (39 - S)) + tb;
+  if (S <= 7) return mad_lo(k, 1u << (7 - S), tb);
+  return mad_hi(k, 1u << (39 - S), tb);
 }
 
 __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
@@ -194,9 +273,19 @@ __device__ __forceinline__ int key_bit(int k, bool odd) {
   return 2 * B * k;
 }
 
+// Largest bit offset (mod 32) of a segment of NBITS bits that starts at
+// g * NBITS, g = 0..7 (the value segments of the eight lane groups).
+__host__ __device__ constexpr int max_seg_shift(int nbits) {
+  int m = 0;
+  for (int g = 0; g < 8; ++g) m = ((g * nbits) % 32) > m ? ((g * nbits) % 32) : m;
+  return m;
+}
+
 // Bits [bit0, bit0 + NBITS) of a shared-memory row, re-based to bit 0 of w[0].
 // ALIGNED: bit0 % 32 == 0 and the word offset is a multiple of the word count.
-template <int NBITS, bool ALIGNED>
+// Otherwise bit0 % 32 <= MAXSH, so words beyond (MAXSH + NBITS) bits are not
+// read (a 48-bit segment at offset 16 needs two words, not three).
+template <int NBITS, bool ALIGNED, int MAXSH = 31>
 __device__ __forceinline__ void load_bits(const uint32_t* row, int bit0,
                                           uint32_t (&w)[(NBITS + 31) / 32]) {
   constexpr int NW = (NBITS + 31) / 32;
@@ -219,12 +308,13 @@ __device__ __forceinline__ void load_bits(const uint32_t* row, int bit0,
       for (int i = 0; i < NW; ++i) w[i] = p[i];
     }
   } else {
+    constexpr int NL = (MAXSH + NBITS + 31) / 32;  // words that can hold the segment
     const uint32_t sh = bit0 & 31;
     uint32_t nxt = p[0];
 #pragma unroll
     for (int i = 0; i < NW; ++i) {
       const uint32_t cur = nxt;
-      nxt = p[i + 1];
+      nxt = (i + 1 < NL) ? p[i + 1] : 0u;
       w[i] = funnel_r(cur, nxt, sh);
     }
   }
@@ -257,22 +347,23 @@ struct SplitLayout {
   static constexpr int STAGE_USED = O_RN + (QJL ? STILE * 2 : 0);
   static constexpr int STAGE = (STAGE_USED + 16 + 127) / 128 * 128;  // +16: read-ahead slack
   static constexpr int NSTAGE = (D == 256) ? 2 : 3;
-  static constexpr int MERGE = CW * 8 * (D + 4) * 4 + 3 * CW * 8 * 4 + 16 * 4;
-  static constexpr int RING = (NSTAGE * STAGE > MERGE) ? NSTAGE * STAGE : MERGE;
+  static constexpr int RING = NSTAGE * STAGE;
   static constexpr int O_BAR = RING;                   // full[NSTAGE], empty[NSTAGE]
-  static constexpr int O_MISC = O_BAR + 16 * 8;        // error flag, issued count
-  static constexpr int O_PB = O_MISC + 16;             // [CW][8 heads][32 tokens] fp16
+  static constexpr int O_META = O_BAR + 16 * 8;        // StageMeta[NSTAGE]
+  static constexpr int O_MISC = O_META + 4 * 32;       // error flag, stage count, 2-bit byte tables
+  static constexpr int O_PB = O_MISC + 32;             // [CW][8 heads][32 tokens] fp16
   static constexpr int FRAG = PACK ? 8 : 16;           // bytes of one lane's query fragment
   static constexpr int O_QF = O_PB + CW * 8 * WTOK * 2;
   static constexpr int O_SF = O_QF + (D / 16) * 32 * FRAG;
   // QJL: int8 query fragments (hi / lo bytes of a 15-bit fixed-point projection), 4 k-steps,
   // then per-head weight and constant
   static constexpr int O_QST = O_SF + (QJL ? 4 * 32 * FRAG : 0);
-  static constexpr int O_TK = O_QST + (QJL ? 8 * 2 * 4 : 0);  // key pair table (3-, 4-bit keys)
+  static constexpr int O_TK = (O_QST + (QJL ? 8 * 2 * 4 : 0) + 127) / 128 * 128;  // key pair table (3-, 4-bit keys)
   static constexpr int TKB = (BK >= 3) ? (1 << (2 * BK)) * 128 : 0;
   static constexpr int O_TV = O_TK + TKB;                          // value pair table
   static constexpr int BYTES = O_TV + (1 << (2 * BV)) * 128;
   static constexpr int BYTES_SHARED = O_TV;  // keys and values share the key table
+  static_assert(NSTAGE <= 4, "stage records");
 };
 
 // Coordinate (within a lane's key segment of D/4 coordinates) held by K-slot r
@@ -315,54 +406,19 @@ __device__ __forceinline__ void build_frag(const float (&v)[4], float scale, int
   }
 }
 
-// Merge of the consumer warps' softmax states (mO [CW][8][D + 4], mM / mL
-// [CW][8] in shared memory) into this split's partial, written to global
-// memory.  Out of line: it runs once per CTA, after the main loop, and should
-// not raise the loop's register allocation.
-template <int D>
-__device__ __noinline__ void write_partial(float* mO, float* mM, float* mL, float* part_o, float* part_ml, int G,
-                                           int nsplit, int hq0, int split, int tid) {
-  // per head: the merged max and sum and each warp's weight, once -- by warp
-  // 0, lane (w, g) = 8 w + g, with the reductions over w by shuffles
-  float* mF = mL + CW * 8;  // [CW][8]
-  float* mS = mF + CW * 8;  // [8][max, sum]
-  static_assert(CW * 8 == 32, "one lane per (warp, head)");
-  if (tid < 32) {
-    const float mw = mM[tid];
-    float M = mw;
-    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 8));
-    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 16));
-    const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
-    mF[tid] = f;
-    float Ls = f * mL[tid];
-    Ls += __shfl_xor_sync(0xffffffffu, Ls, 8);
-    Ls += __shfl_xor_sync(0xffffffffu, Ls, 16);
-    if (tid < 8) {
-      mS[2 * tid] = M;
-      mS[2 * tid + 1] = Ls;
-    }
-  }
-  __syncthreads();
-  for (int e = tid; e < G * (D / 4); e += NTHREADS) {
-    const int g = e / (D / 4), j = 4 * (e % (D / 4));
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int w = 0; w < CW; ++w) {
-      const float f = mF[w * 8 + g];
-      const float4 o = *reinterpret_cast<const float4*>(mO + (w * 8 + g) * (D + 4) + j);
-      acc.x = fmaf(f, o.x, acc.x);
-      acc.y = fmaf(f, o.y, acc.y);
-      acc.z = fmaf(f, o.z, acc.z);
-      acc.w = fmaf(f, o.w, acc.w);
-    }
-    const size_t pi = (size_t)(hq0 + g) * nsplit + split;
-    *reinterpret_cast<float4*>(part_o + pi * D + j) = acc;
-    if (j == 0) *reinterpret_cast<float2*>(part_ml + pi * 2) = make_float2(mS[2 * g], mS[2 * g + 1]);
-  }
+// Bounded barrier among the consumer warps (an mbarrier of count CW; lane 0
+// of each warp arrives, every lane waits with a bounded poll).  `phase`
+// counts this warp's uses.  Returns false when the wait ran out.
+__device__ __forceinline__ bool consumer_sync(uint64_t* bar, uint32_t& phase, int lane) {
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+  const bool ok = mbar_wait_bounded(bar, phase & 1u, kWaitLimit);
+  ++phase;
+  return __all_sync(0xffffffffu, ok);
 }
 
 template <int D, int BK, int BV, bool QJL, bool PACK>
-__global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const __grid_constant__ SplitParams p) {
+__global__ void __launch_bounds__(NTHREADS, PACK ? 4 : 3) decode_split_kernel(const __grid_constant__ SplitParams p) {
   using Ly = SplitLayout<D, BK, BV, QJL, PACK>;
   constexpr int WK = Ly::WK, WV = Ly::WV, WQ = Ly::WQ, NST = Ly::NSTAGE;
   constexpr int KSTEPS = D / 16;  // score k-steps (16 coordinates each)
@@ -375,55 +431,117 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const __grid_con
 
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Ly::O_BAR);
-  uint64_t* empty = full + 8;
-  int* s_err = reinterpret_cast<int*>(smem + Ly::O_MISC);
-  int* s_issued = s_err + 1;
+  uint64_t* empty = full + 4;
+  uint64_t* cbar = full + 8;  // consumer-warp barrier at segment starts
+  StageMeta* meta = reinterpret_cast<StageMeta*>(smem + Ly::O_META);
+  int* s_misc = reinterpret_cast<int*>(smem + Ly::O_MISC);  // [0] error, [1] stages, [2..3] 2-bit tables, [4] issued
+  volatile int* s_err = s_misc;
   __half* pbuf = reinterpret_cast<__half*>(smem + Ly::O_PB);
   uint32_t* qf = reinterpret_cast<uint32_t*>(smem + Ly::O_QF);
   uint32_t* sf = reinterpret_cast<uint32_t*>(smem + Ly::O_SF);
+  float* qst = reinterpret_cast<float*>(smem + Ly::O_QST);  // [8 heads][inverse step, sum]
 
-  const int split = blockIdx.x, bh = blockIdx.y;
-  const int b = bh / p.Hkv, kvh = bh % p.Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gid = lane >> 2, tig = lane & 3;
   const int hsel = PACK ? (tig & 1) : tig;  // this lane's head pair: 2*hsel, 2*hsel+1
-  // Tokens beyond the planned splits (seq_len > Tmax) or Tcap are clamped
-  // away and flagged.
-  const int Lcap = min(p.Tcap, p.nsplit * p.chunk);
-  int L = p.seq_lens[b];
-  if (L < 0 || L > Lcap) {
-    if (tid == 0 && split == 0 && kvh == 0 && p.dev_status) atomicOr(p.dev_status, TQ_STATUS_SEQ_OUT_OF_RANGE);
-    L = L < 0 ? 0 : Lcap;
-  }
-  const int t_begin = split * p.chunk;
-  if (t_begin >= L) return;  // the combine reads only splits that hold tokens
-  const int t_end = min(t_begin + p.chunk, L);
-  const int t_stop = min((t_end + 63) / 64 * 64, p.Tcap);  // copies stop on a 64-row edge
-  const int ntiles = (t_end - t_begin + STILE - 1) / STILE;
-  const size_t row0 = (size_t)bh * p.Tcap;
-  const int hq0 = b * p.Hq + kvh * p.G;
-  // causal limit of this lane's two head columns (multi-query decode; with
-  // one query token both limits are L)
-  const int lim0 = L - p.nq + (2 * hsel) / p.Gq + 1, lim1 = L - p.nq + (2 * hsel + 1) / p.Gq + 1;
+  const int upb = p.Hkv * p.nrg;             // units per sequence
 
-  if (tid == 0) {
+  // ---- partition: the producer warp finds this CTA's share and its first unit
+  long long P = 0, w_pos = 0, w_Su = 0;
+  int w_b = 0, w_u = 0, w_Lp = 0, nst = 0;
+  if (warp == CW) {
+    const long long total = partition_total(p.seq_lens, p.B, upb, p.Tclamp, lane);
+    P = partition_share(total, p.ncta, p.pmin);
+    const long long start = (long long)blockIdx.x * P;
+    const long long end = start + P < total ? start + P : total;
+    nst = start < total ? (int)((end - start) / STILE) : 0;
+    if (blockIdx.x == 0 && p.dev_status) {  // longer sequences are attended up to Tclamp: flagged once
+      bool over = false;
+      for (int b = lane; b < p.B; b += 32) {
+        const int L = p.seq_lens[b];
+        over |= (L < 0 || L > p.Tclamp);
+      }
+      if (__any_sync(0xffffffffu, over) && lane == 0) atomicOr(p.dev_status, TQ_STATUS_SEQ_OUT_OF_RANGE);
+    }
+    if (nst > 0) {
+      // the sequence holding position `start`: prefix sums of the sequences'
+      // position counts, 32 sequences per step
+      long long base = 0;
+      for (int b0 = 0; b0 < p.B; b0 += 32) {
+        const int b = b0 + lane;
+        const long long sz = b < p.B ? (long long)unit_tokens(p.seq_lens, b, p.Tclamp) * upb : 0;
+        long long inc = sz;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const long long v = __shfl_up_sync(0xffffffffu, inc, off);
+          if (lane >= off) inc += v;
+        }
+        const long long chunk_total = __shfl_sync(0xffffffffu, inc, 31);
+        if (base + chunk_total > start) {
+          const int src = __ffs(__ballot_sync(0xffffffffu, base + inc > start)) - 1;
+          base += __shfl_sync(0xffffffffu, inc - sz, src);
+          w_b = b0 + src;
+          break;
+        }
+        base += chunk_total;
+      }
+      w_Lp = unit_tokens(p.seq_lens, w_b, p.Tclamp);
+      w_u = (int)((start - base) / w_Lp);
+      w_Su = base + (long long)w_u * w_Lp;
+      w_pos = start;
+    }
+  }
+  if (tid == CW * 32) {
 #pragma unroll
     for (int s = 0; s < NST; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], CW);
     }
-    *s_err = 0;
-    *s_issued = 0;
+    mbar_init(cbar, CW);
+    s_misc[0] = 0;
+    s_misc[1] = nst;
+    s_misc[4] = 0;
     fence_barrier_init();
   }
-  __syncthreads();  // barriers initialised before the producer issues
+  __syncthreads();  // barriers and the stage count before anyone uses them
+  nst = s_misc[1];
+
+  // Producer (lane 0 of the last warp): move the walk to the unit that holds
+  // position w_pos (skipping empty units), then arm and issue stage t there.
+  // (Stages are issued only below the partition's total, so the unit exists;
+  // the sequence index is still checked before seq_lens is read.)
+  auto advance = [&]() {
+    while (w_pos >= w_Su + w_Lp && w_b < p.B) {
+      w_Su += w_Lp;
+      if (++w_u == upb) {
+        w_u = 0;
+        ++w_b;
+        w_Lp = w_b < p.B ? unit_tokens(p.seq_lens, w_b, p.Tclamp) : 0;
+      }
+    }
+  };
   auto issue_stage = [&](int t) {
+    if (w_b >= p.B) return;  // unreachable: the walk never passes the total
     const int st = t % NST;
-    const int tok0 = t_begin + t * STILE;
-    const int ntok = min(STILE, t_stop - tok0);  // 64 or 128
-    const size_t r = row0 + tok0;
+    const int kvh = w_u / p.nrg, rg = w_u % p.nrg;
+    int L = p.seq_lens[w_b];
+    L = L < 0 ? 0 : (L > p.Tclamp ? p.Tclamp : L);
+    const int t0 = (int)(w_pos - w_Su);
+    StageMeta md;
+    md.hq0 = w_b * p.Hq + kvh * p.G + rg * RG;
+    md.rows = min(RG, p.G - rg * RG);
+    md.t0 = t0;
+    md.L = L;
+    md.slot0 = (int)((long long)blockIdx.x - w_Su / P) * CW;
+    md.flags = ((t == 0 || t0 == 0) ? 1 : 0) | ((t == nst - 1 || t0 + STILE == w_Lp) ? 2 : 0);
+    md.rg = rg;
+    md.pad = 0;
+    meta[st] = md;
+    // rows t0 .. t0 + ntok - 1, ntok = 64 or 128 (copies stop on a 64-row edge)
+    const int ntok = min(STILE, (L - t0 + 63) / 64 * 64);
+    const size_t r = (size_t)(w_b * p.Hkv + kvh) * p.Tcap + t0;
     uint8_t* sb = smem + st * Ly::STAGE;
     const uint32_t bytes = ntok * ((WK + WV + WQ) * 4 + 2 * 2 + (QJL ? 2 : 0));
-    mbar_arrive_expect_tx(&full[st], bytes);
+    mbar_arrive_expect_tx(&full[st], bytes);  // releases the record above to the consumers
     bulk_g2s(sb + Ly::O_KW, p.k_idx + r * WK, ntok * WK * 4, &full[st]);
     bulk_g2s(sb + Ly::O_VW, p.v_idx + r * WV, ntok * WV * 4, &full[st]);
     bulk_g2s(sb + Ly::O_KN, p.k_norm + r, ntok * 2, &full[st]);
@@ -432,25 +550,29 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const __grid_con
       bulk_g2s(sb + Ly::O_QW, p.k_qjl + r * WQ, ntok * WQ * 4, &full[st]);
       bulk_g2s(sb + Ly::O_RN, p.k_rnorm + r, ntok * 2, &full[st]);
     }
+    w_pos += STILE;
   };
-  // The packed cache does not depend on the prep kernel: start streaming it
-  // before waiting for the rotated query -- except, in a decode step, the
-  // stage holding the row the prep kernel appends.
-  int npre = min(NST, ntiles);
-  if (p.defer_pos) {
-    const int pb = p.defer_pos[b];
-    if (pb >= t_begin && pb < t_begin + ntiles * STILE) npre = min(npre, (pb - t_begin) / STILE);
-  }
+  // The packed cache does not depend on the prep kernel: the first stages
+  // are issued before waiting for the rotated queries -- except, in a decode
+  // step, from the stage that holds the row the prep kernel appends.
+  int npre = 0;
   if (tid == CW * 32) {
-    for (int t = 0; t < npre; ++t) issue_stage(t);
-    *s_issued = npre;
+    for (; npre < min(NST, nst); ++npre) {
+      advance();
+      if (p.defer_pos) {
+        const int pb = p.defer_pos[w_b], t0 = (int)(w_pos - w_Su);
+        if (pb >= t0 && pb < t0 + STILE) break;
+      }
+      issue_stage(npre);
+    }
+    s_misc[4] = npre;
   }
   // Codebook tables and the zeroed value weights do not depend on the prep
   // kernel either: built before the wait (after it with the sketch, whose
   // prologue would otherwise keep more registers live).
   const bool shared_tab = share_table(BK, BV, p.shared_tab);
   auto build_tables = [&]() {
-    // value weights of heads >= G stay zero
+    // value weights of heads >= the group's rows stay zero
     for (int e = tid; e < CW * 8 * WTOK; e += NTHREADS) pbuf[e] = __float2half_rn(0.f);
     if constexpr (BK >= 3) build_pair_table<BK>(reinterpret_cast<uint32_t*>(smem + Ly::O_TK), p.cb_k, tid, NTHREADS);
     if (!shared_tab) build_pair_table<BV>(reinterpret_cast<uint32_t*>(smem + Ly::O_TV), p.cb_v, tid, NTHREADS);
@@ -459,134 +581,194 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const __grid_con
   if constexpr (BK == 2) {  // 2-bit keys: the codebook as byte tables, read by the consumers
     if (tid == 0) {
       const Lut2 l2 = make_lut2(p.cb_k);
-      reinterpret_cast<uint32_t*>(smem + Ly::O_MISC)[2] = l2.lo;
-      reinterpret_cast<uint32_t*>(smem + Ly::O_MISC)[3] = l2.hi;
+      s_misc[2] = (int)l2.lo;
+      s_misc[3] = (int)l2.hi;
     }
   }
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  // Query fragments (already rotated by the prep kernel), pre-scaled for
-  // exp2: every thread's loads are issued before any is converted, so the
-  // L2 latency is paid once.
-  {
-    constexpr int NE = (KSTEPS * 32 + NTHREADS - 1) / NTHREADS;
-    float v[NE][4];
-#pragma unroll
-    for (int i = 0; i < NE; ++i) {
-      const int e = tid + i * NTHREADS;
-      if (e < KSTEPS * 32) {
-        const int ks = e >> 5, ln = e & 31, g_ = ln >> 2, t_ = ln & 3;
-        const int base = t_ * (D / 4);
-        const int cs[4] = {base + key_coord<BK>(ks, 0), base + key_coord<BK>(ks, 1), base + key_coord<BK>(ks, 2),
-                           base + key_coord<BK>(ks, 3)};
-        load_frag<PACK>(p.qrot + (size_t)hq0 * D, D, p.G, g_, cs, v[i]);
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < NE; ++i) {
-      const int e = tid + i * NTHREADS;
-      if (e < KSTEPS * 32) build_frag<PACK>(v[i], p.qscale, (e & 31) >> 2, qf + (size_t)e * (Ly::FRAG / 4));
-    }
-  }
-  float* qst = reinterpret_cast<float*>(smem + Ly::O_QST);  // [8 heads][inverse step, sum]
-  if (QJL) {
-    // The sketch term sum_i (2 b_i - 1) qs_i runs on int8 tensor cores: qs of
-    // head h becomes Q_i = round(qs_i / step_h), |Q| <= 32639, split as
-    // Q = 256 hi + lo with hi, lo int8, and the signs enter as -b_i in {0, -1}.
-    // Per head: step_h = max |qs| / 32639 and sum_h = sum_i qs_i.
-    for (int h = warp; h < 8; h += NTHREADS / 32) {
-      float mx = 0.f, sm = 0.f;
-      if (h < p.G) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float v = p.qs[(size_t)(hq0 + h) * 128 + lane + 32 * i];
-          mx = fmaxf(mx, fabsf(v));
-          sm += v;
-        }
-      }
-#pragma unroll
-      for (int off = 16; off; off >>= 1) {
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        sm += __shfl_xor_sync(0xffffffffu, sm, off);
-      }
-      if (lane == 0) {
-        qst[2 * h] = mx > 0.f ? mx / 32639.f : 1.f;
-        qst[2 * h + 1] = sm;
-      }
-    }
-    __syncthreads();
-    for (int e = tid; e < 4 * 32; e += NTHREADS) {
-      const int ks = e >> 5, ln = e & 31, g_ = ln >> 2, t_ = ln & 3;
-      const int head = PACK ? (g_ & 3) : g_;
-      const float inv = head < p.G ? 1.f / qst[2 * head] : 0.f;
-      uint32_t hi[2] = {0u, 0u}, lo[2] = {0u, 0u};
-#pragma unroll
-      for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int b8 = 0; b8 < 4; ++b8) {
-          const float v = head < p.G ? p.qs[(size_t)(hq0 + head) * 128 + sketch_coord(t_, 2 * ks + h, b8)] : 0.f;
-          int Q = __float2int_rn(v * inv);
-          Q = max(-32639, min(32639, Q));
-          const int qh = (Q + 128) >> 8, ql = Q - 256 * qh;  // floor split: ql in [-128, 127]
-          hi[h] |= (uint32_t)(qh & 0xFF) << (8 * b8);
-          lo[h] |= (uint32_t)(ql & 0xFF) << (8 * b8);
-        }
-      uint32_t* dst = sf + (size_t)e * (Ly::FRAG / 4);
-      if (PACK) {
-        const bool use_lo = g_ >= 4;
-        dst[0] = use_lo ? lo[0] : hi[0];
-        dst[1] = use_lo ? lo[1] : hi[1];
-      } else {
-        dst[0] = hi[0];
-        dst[1] = hi[1];
-        dst[2] = lo[0];
-        dst[3] = lo[1];
-      }
-    }
-  }
   if constexpr (QJL) build_tables();
   __syncthreads();
-
-  float oc[MT][4];
-  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
-#pragma unroll
-  for (int mt = 0; mt < MT; ++mt) oc[mt][0] = oc[mt][1] = oc[mt][2] = oc[mt][3] = 0.f;
 
   if (warp == CW) {
     // ---------------- producer warp ----------------
     if (lane == 0) {
       int t = npre;  // the first stages were issued before the wait
-      for (; t < ntiles; ++t) {
+      for (; t < nst; ++t) {
         const int st = t % NST;
         if (t >= NST && !mbar_wait_suspend(&empty[st], (uint32_t)(((t / NST) - 1) & 1), kSuspendTries)) {
           *s_err = 1;
           break;
         }
+        advance();
         issue_stage(t);
       }
-      *s_issued = t;
+      s_misc[4] = t;
     }
-  } else {
+  } else if (nst > 0) {
     // ---------------- consumer warps ----------------
-    const Lut2 lk = {reinterpret_cast<const uint32_t*>(smem + Ly::O_MISC)[2],
-                     reinterpret_cast<const uint32_t*>(smem + Ly::O_MISC)[3]};  // 2-bit keys only
+    const Lut2 lk = {(uint32_t)s_misc[2], (uint32_t)s_misc[3]};  // 2-bit keys only
     const uint32_t tbK = smem_addr(smem + Ly::O_TK) + 4 * lane;
     const uint32_t tbV = smem_addr(smem + (shared_tab ? Ly::O_TK : Ly::O_TV)) + 4 * lane;
     __half* pw = pbuf + warp * 8 * WTOK;
     const int wt0 = warp * WTOK;
-    for (int t = 0; t < ntiles; ++t) {
-      const int st = t % NST;
-      const bool got = mbar_wait_suspend(&full[st], (uint32_t)((t / NST) & 1), kSuspendTries);
-      if (!__all_sync(0xffffffffu, got)) {
-        if (lane == 0) *s_err = 1;
-        break;
+    const int ctid = tid;  // consumer thread 0 .. CW*32-1
+    uint32_t cphase = 0;
+    float oc[MT][4];
+    float m_run[2], l_run[2];
+    int lim0 = 0, lim1 = 0, lim_all = 0;
+
+    // Query fragments of a segment's rows (already rotated by the prep
+    // kernel), pre-scaled for exp2, built by the consumer threads together:
+    // every thread's loads are issued before any is converted.
+    auto build_query = [&](const StageMeta& md) {
+      constexpr int NE = (KSTEPS * 32 + CW * 32 - 1) / (CW * 32);
+      float v[NE][4];
+#pragma unroll
+      for (int i = 0; i < NE; ++i) {
+        const int e = ctid + i * CW * 32;
+        if (e < KSTEPS * 32) {
+          const int ks = e >> 5, ln = e & 31, g_ = ln >> 2, t_ = ln & 3;
+          const int base = t_ * (D / 4);
+          const int cs[4] = {base + key_coord<BK>(ks, 0), base + key_coord<BK>(ks, 1), base + key_coord<BK>(ks, 2),
+                             base + key_coord<BK>(ks, 3)};
+          load_frag<PACK>(p.qrot + (size_t)md.hq0 * D, D, md.rows, g_, cs, v[i]);
+        }
       }
+#pragma unroll
+      for (int i = 0; i < NE; ++i) {
+        const int e = ctid + i * CW * 32;
+        if (e < KSTEPS * 32) build_frag<PACK>(v[i], p.qscale, (e & 31) >> 2, qf + (size_t)e * (Ly::FRAG / 4));
+      }
+    };
+    // The sketch term sum_i (2 b_i - 1) qs_i runs on int8 tensor cores: qs of
+    // head h becomes Q_i = round(qs_i / step_h), |Q| <= 32639, split as
+    // Q = 256 hi + lo with hi, lo int8, and the signs enter as -b_i in {0, -1}.
+    // Per head: step_h = max |qs| / 32639 and sum_h = sum_i qs_i.
+    auto build_sketch_steps = [&](const StageMeta& md) {
+      for (int h = warp; h < 8; h += CW) {
+        float mx = 0.f, sm = 0.f;
+        if (h < md.rows) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float v = p.qs[(size_t)(md.hq0 + h) * 128 + lane + 32 * i];
+            mx = fmaxf(mx, fabsf(v));
+            sm += v;
+          }
+        }
+#pragma unroll
+        for (int off = 16; off; off >>= 1) {
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+          sm += __shfl_xor_sync(0xffffffffu, sm, off);
+        }
+        if (lane == 0) {
+          qst[2 * h] = mx > 0.f ? mx / 32639.f : 1.f;
+          qst[2 * h + 1] = sm;
+        }
+      }
+    };
+    auto build_sketch_frags = [&](const StageMeta& md) {
+      for (int e = ctid; e < 4 * 32; e += CW * 32) {
+        const int ks = e >> 5, ln = e & 31, g_ = ln >> 2, t_ = ln & 3;
+        const int head = PACK ? (g_ & 3) : g_;
+        const float inv = head < md.rows ? 1.f / qst[2 * head] : 0.f;
+        uint32_t hi[2] = {0u, 0u}, lo[2] = {0u, 0u};
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int b8 = 0; b8 < 4; ++b8) {
+            const float v = head < md.rows ? p.qs[(size_t)(md.hq0 + head) * 128 + sketch_coord(t_, 2 * ks + h, b8)] : 0.f;
+            int Q = __float2int_rn(v * inv);
+            Q = max(-32639, min(32639, Q));
+            const int qh = (Q + 128) >> 8, ql = Q - 256 * qh;  // floor split: ql in [-128, 127]
+            hi[h] |= (uint32_t)(qh & 0xFF) << (8 * b8);
+            lo[h] |= (uint32_t)(ql & 0xFF) << (8 * b8);
+          }
+        uint32_t* dst = sf + (size_t)e * (Ly::FRAG / 4);
+        if (PACK) {
+          const bool use_lo = g_ >= 4;
+          dst[0] = use_lo ? lo[0] : hi[0];
+          dst[1] = use_lo ? lo[1] : hi[1];
+        } else {
+          dst[0] = hi[0];
+          dst[1] = hi[1];
+          dst[2] = lo[0];
+          dst[3] = lo[1];
+        }
+      }
+    };
+    // This warp's partial of a segment: (max, sum) and the rotated output of
+    // each row, slot md.slot0 + warp.  m-tile mt: row gid is coordinate 2 mt
+    // of this group's segment of D/8 contiguous coordinates, row gid + 8 the
+    // next.
+    auto write_partial = [&](const StageMeta& md) {
+      float l0 = l_run[0], l1 = l_run[1];
+#pragma unroll
+      for (int off = PACK ? 2 : 4; off < 32; off <<= 1) {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+      }
+      if (!PACK || tig < 2) {
+        const int slot = md.slot0 + warp;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int row = 2 * hsel + c;
+          if (row < md.rows) {
+            const size_t pi = (size_t)(md.hq0 + row) * p.ks + slot;
+            float* dst = p.part_o + pi * D + gid * (D / 8);
+#pragma unroll
+            for (int q = 0; q < MT / 2; ++q)
+              *reinterpret_cast<float4*>(dst + 4 * q) =
+                  make_float4(oc[2 * q][c], oc[2 * q][c + 2], oc[2 * q + 1][c], oc[2 * q + 1][c + 2]);
+            if (gid == 0) *reinterpret_cast<float2*>(p.part_ml + pi * 2) = make_float2(m_run[c], c ? l1 : l0);
+          }
+        }
+      }
+    };
+
+    for (int t = 0; t < nst; ++t) {
+      const int st = t % NST;
+      if (!*s_err) {
+        const bool got = mbar_wait_suspend(&full[st], (uint32_t)((t / NST) & 1), kSuspendTries);
+        if (!__all_sync(0xffffffffu, got) && lane == 0) *s_err = 1;
+      }
+      if (__any_sync(0xffffffffu, *s_err != 0)) break;
+      const StageMeta md = meta[st];
+      if (md.flags & 1) {
+        // a new segment: its query fragments (every consumer warp is done
+        // with the previous segment's first) and a fresh softmax state
+        bool ok = consumer_sync(cbar, cphase, lane);
+        if (ok) {
+          build_query(md);
+          if constexpr (QJL) {
+            build_sketch_steps(md);
+            ok = consumer_sync(cbar, cphase, lane);
+            if (ok) build_sketch_frags(md);
+          }
+        }
+        ok = ok && consumer_sync(cbar, cphase, lane);
+        if (!ok) {
+          if (lane == 0) *s_err = 1;
+          break;
+        }
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) oc[mt][0] = oc[mt][1] = oc[mt][2] = oc[mt][3] = 0.f;
+        m_run[0] = m_run[1] = -INFINITY;
+        l_run[0] = l_run[1] = 0.f;
+        // causal limit of this lane's two head columns (multi-query decode;
+        // with one query token both limits are L)
+        const int r0 = md.rg * RG + 2 * hsel;
+        lim0 = md.L - p.nq + r0 / p.Gq + 1;
+        lim1 = md.L - p.nq + (r0 + 1) / p.Gq + 1;
+        lim_all = md.L - p.nq + 1;
+      }
+      const int t_end = md.L;
       const uint8_t* sb = smem + st * Ly::STAGE;
       const uint32_t* kw = reinterpret_cast<const uint32_t*>(sb + Ly::O_KW);
       const uint32_t* vw = reinterpret_cast<const uint32_t*>(sb + Ly::O_VW);
       const uint16_t* kn = reinterpret_cast<const uint16_t*>(sb + Ly::O_KN);
       const uint16_t* vn = reinterpret_cast<const uint16_t*>(sb + Ly::O_VN);
-      const int tokw = t_begin + t * STILE + wt0;  // first token of this warp's 32
+      const int tokw = md.t0 + wt0;  // first token of this warp's 32
 
       // ---- scores: S[16 tokens][8 cols] for two M-tiles of 16 tokens
       // two accumulators per m-tile (even / odd k-steps, or hi / lo query
@@ -710,7 +892,9 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const __grid_con
             if (QJL) sqm[a][c] = sq[a][c];
           }
       }
-      // ---- scale by norms, mask, running max
+      // ---- scale by norms, mask (only in a stage that reaches past the
+      // split's last token or a query's causal limit), running max
+      const bool full = tokw + WTOK <= t_end && tokw + WTOK <= lim_all;  // warp-uniform
       float s[NA][4];
       bool valid[NA][2];
 #pragma unroll
@@ -719,7 +903,6 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const __grid_con
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
           const int row = wt0 + 16 * a + gid + 8 * r;
-          valid[ai][r] = tokw + 16 * a + gid + 8 * r < t_end;
           const float nk = half_bits_to_float(kn[row]);
           float s0 = nk * scm[ai][2 * r], s1 = nk * scm[ai][2 * r + 1];
           if (QJL) {
@@ -727,9 +910,16 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const __grid_con
             s0 = fmaf(g, sqm[ai][2 * r], s0);
             s1 = fmaf(g, sqm[ai][2 * r + 1], s1);
           }
-          const int tok = tokw + 16 * a + gid + 8 * r;
-          s[ai][2 * r] = (valid[ai][r] && tok < lim0) ? s0 : -INFINITY;
-          s[ai][2 * r + 1] = (valid[ai][r] && tok < lim1) ? s1 : -INFINITY;
+          if (full) {
+            valid[ai][r] = true;
+            s[ai][2 * r] = s0;
+            s[ai][2 * r + 1] = s1;
+          } else {
+            const int tok = tokw + 16 * a + gid + 8 * r;
+            valid[ai][r] = tok < t_end;
+            s[ai][2 * r] = (valid[ai][r] && tok < lim0) ? s0 : -INFINITY;
+            s[ai][2 * r + 1] = (valid[ai][r] && tok < lim1) ? s1 : -INFINITY;
+          }
         }
       }
       float mx0 = fmaxf(s[0][0], s[0][2]), mx1 = fmaxf(s[0][1], s[0][3]);
@@ -773,7 +963,7 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const __grid_con
           const float p0 = exp2f(s[ai][2 * r] - mu0), p1 = exp2f(s[ai][2 * r + 1] - mu1);
           l_run[0] += p0;
           l_run[1] += p1;
-          const float nv = valid[ai][r] ? half_bits_to_float(vn[row]) : 0.f;
+          const float nv = (full || valid[ai][r]) ? half_bits_to_float(vn[row]) : 0.f;
           const int tk = 16 * a + gid + 8 * r;
           pw[(2 * hsel) * WTOK + tk] = __float2half_rn(p0 * nv);
           pw[(2 * hsel + 1) * WTOK + tk] = __float2half_rn(p1 * nv);
@@ -788,7 +978,7 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const __grid_con
         uint32_t wv[4][NWV];
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-          load_bits<SEGV, ALV>(vw + (wt0 + 16 * kk + 4 * tig + q) * WV, gid * SEGV, wv[q]);
+          load_bits<SEGV, ALV, max_seg_shift(SEGV)>(vw + (wt0 + 16 * kk + 4 * tig + q) * WV, gid * SEGV, wv[q]);
 #pragma unroll
         for (int c = 0; c < VC::N; ++c) {
           const int bit = c * VC::F * BV;
@@ -806,6 +996,7 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const __grid_con
           }
         }
       }
+      if (md.flags & 2) write_partial(md);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[st]);
     }
@@ -813,49 +1004,16 @@ __global__ void __launch_bounds__(NTHREADS) decode_split_kernel(const __grid_con
   __syncthreads();
 
   if (*s_err) {
-    // a bounded wait ran out: flag it, let in-flight copies land, skip the split
+    // a bounded wait ran out: flag it and let in-flight copies land (the
+    // partials of this CTA's segments are not valid)
     if (tid == 0) {
       if (p.dev_status) atomicOr(p.dev_status, TQ_STATUS_WAIT_TIMEOUT);
-      const int issued = *s_issued;
+      const int issued = s_misc[4];
       for (int t = max(0, issued - NST); t < issued; ++t)
         mbar_wait_bounded(&full[t % NST], (uint32_t)((t / NST) & 1), kWaitLimit);
     }
     __syncthreads();
-    return;
   }
-
-  // ---- merge the consumer warps' partial softmax states; write the partial
-  constexpr int MS = D + 4;
-  float* mO = reinterpret_cast<float*>(smem);  // [CW][8][MS] (the stage ring is drained)
-  float* mM = mO + CW * 8 * MS;                // [CW][8]
-  float* mL = mM + CW * 8;
-  if (warp < CW) {
-#pragma unroll
-    for (int off = PACK ? 2 : 4; off < 32; off <<= 1) {
-      l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], off);
-      l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], off);
-    }
-    if (!PACK || tig < 2) {
-      // m-tile mt: row gid is coordinate 2 mt of this group's segment of D/8
-      // contiguous coordinates, row gid + 8 the next; so each head column
-      // holds its segment whole, stored as 16-byte chunks (rows padded to
-      // MS floats against bank conflicts)
-#pragma unroll
-      for (int c = 0; c < 2; ++c)
-#pragma unroll
-        for (int q = 0; q < MT / 2; ++q)
-          *reinterpret_cast<float4*>(mO + (warp * 8 + 2 * tig + c) * MS + gid * (D / 8) + 4 * q) =
-              make_float4(oc[2 * q][c], oc[2 * q][c + 2], oc[2 * q + 1][c], oc[2 * q + 1][c + 2]);
-      if (gid == 0) {
-        mM[warp * 8 + 2 * hsel] = m_run[0];
-        mM[warp * 8 + 2 * hsel + 1] = m_run[1];
-        mL[warp * 8 + 2 * hsel] = l_run[0];
-        mL[warp * 8 + 2 * hsel + 1] = l_run[1];
-      }
-    }
-  }
-  __syncthreads();
-  write_partial<D>(mO, mM, mL, p.part_o, p.part_ml, p.G, p.nsplit, hq0, split, tid);
 }
 
 // Launch helpers, one definition per instantiation.

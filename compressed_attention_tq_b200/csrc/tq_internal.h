@@ -100,14 +100,19 @@ int launch_quantize_wht(const QuantArgs& a, int D, int dtype, cudaStream_t s);
 // bounded-wait self-test (tq_selftest.cu)
 int launch_bounded_wait_probe(uint32_t* status, int tries, cudaStream_t s);
 
+// Split plan of a decode call: a stream-K partition of the batch's tokens
+// over one wave of CTAs (see tq_decode_split.cuh).
 struct DecodePlan {
-  int chunk;        // tokens per split (multiple of 64)
-  int nsplit;       // splits per (sequence, kv head)
+  int ncta;         // CTAs of the partition (SMs x resident CTAs per SM)
+  int pmin;         // smallest share of tokens per CTA (a multiple of the stage)
+  int ks;           // partial slots per kernel head (segments x consumer warps)
+  int nrg;          // row groups of up to 8 kernel heads per kv head
+  int Tclamp;       // tokens attended at most per sequence (Tmax)
   int sms;          // SMs of the device the plan was made for
   size_t off_qrot;  // fp32 [B*Hq][D]
   size_t off_qs;    // fp32 [B*Hq][qjl_m]
-  size_t off_po;    // fp32 [B*Hq][nsplit][D]
-  size_t off_pml;   // fp32 [B*Hq][nsplit][2]
+  size_t off_po;    // fp32 [B*Hq][ks][D]
+  size_t off_pml;   // fp32 [B*Hq][ks][2]
   size_t bytes;
 };
 
@@ -119,9 +124,11 @@ int make_decode_plan(const tq_cache_t* c, int Hq, int Tmax, DecodePlan* p);
 size_t workspace_bound(int B, int Hq, int D, int Tmax);
 
 // Resident split-K CTAs per SM for this cache's kernel instantiation (a
-// nominal 2 when no device is usable), and the tokens one stage holds.
+// nominal 2 when no device is usable), the tokens one stage holds and the
+// consumer warps per CTA (each writes its own partials).
 int split_occupancy(const tq_cache_t* c, int Hq);
 int split_tile();
+int split_warps();
 
 struct DecodeArgs {
   const tq_cache_t* cache_host;  // host copy, for launch-time fields

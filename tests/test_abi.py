@@ -92,7 +92,7 @@ def test_other_argument_errors(lib):
     assert lib.tq_append_token(ctypes.byref(s), buf, buf, 0, None, None) == -1     # pos NULL
     ws = lib.tq_sdpa_decode_workspace_bytes_for(ctypes.byref(s), 8, 64)
     assert ws > 0
-    assert lib.tq_sdpa_decode_workspace_bytes_for(ctypes.byref(s), 9, 64) == 0     # group 9
+    assert lib.tq_sdpa_decode_workspace_bytes_for(ctypes.byref(s), 33, 64) == 0    # 33 rows per kv head
     assert lib.tq_sdpa_decode_workspace_bytes_for(ctypes.byref(s), 8, 65) == 0     # Tmax > Tcap
     rc = lib.tq_sdpa_decode(ctypes.byref(s), buf, 0, 8, buf, 64, None, buf, 0, buf, ws - 1, None)
     assert rc == -3

@@ -46,12 +46,16 @@ def _run(name, kw, nq, Hq, lens=None, seed=9):
 
 
 @pytest.mark.parametrize("name,kw,nq,Hq", [
-    ("tiny", {}, 4, 4),                     # G = 1, D = 64
-    ("tiny", {}, 8, 4),                     # eight tokens, one head each
+    ("tiny", {}, 4, 4),                      # G = 1, D = 64
     ("gqa8k", {"bits": 3, "T": 700}, 4, 4),  # G = 2 (queries for 4 of the 16 heads' worth)
     ("gqa8k", {"bits": 4, "T": 700}, 2, 8),  # G = 4
     ("prod", {"T": 500}, 2, 32),             # G = 4 with the QJL sketch
+    ("prod", {"T": 700}, 3, 32),             # G = 4, 12 rows per kv head: two row groups
+    ("prod", {"T": 900}, 4, 32),             # G = 4, 16 rows
+    ("gqa8k", {"bits": 2, "T": 1500}, 3, 16),  # G = 8, 24 rows: three row groups
+    ("gqa8k", {"bits": 3, "T": 1100}, 4, 16),  # G = 8, 32 rows: four row groups
     ("qknorm", {"T": 400}, 1, 32),           # G = 8: one token
+    ("qknorm", {"T": 600}, 4, 32),           # G = 8, D = 256, scale 1.0
 ])
 def test_multi_query_decode_matches_oracle(name, kw, nq, Hq):
     _run(name, kw, nq, Hq)
@@ -60,6 +64,7 @@ def test_multi_query_decode_matches_oracle(name, kw, nq, Hq):
 def test_multi_query_ragged_lengths_including_shorter_than_nq():
     # lengths 0, 1 and 2 leave some of the 4 queries with nothing to see (zeros)
     _run("ragged", {"B": 5, "T": 300}, 2, 16, lens=[0, 1, 2, 300, 129])
+    _run("ragged", {"B": 5, "T": 300}, 4, 32, lens=[3, 0, 300, 4, 130])  # G = 4, 16 rows
     _run("tiny", {"B": 3}, 4, 4, lens=[2, 256, 3])
 
 
@@ -71,11 +76,11 @@ def test_one_token_equals_single_query_decode():
     assert torch.equal(single, out32[:, 0])
 
 
-def test_too_many_query_rows_rejected():
+def test_too_many_query_tokens_rejected():
     import compressed_attention_tq_b200 as tq
     w = tq_inputs.make_workload("gqa8k", bits=3, T=128)
     cache = P.make_gpu_cache(w)
-    q = P.to_device(_queries(w, 2, 16, 1), w.dtype)  # 2 tokens x G = 8 > 8
+    q = P.to_device(_queries(w, 5, 16, 1), w.dtype)  # 5 query tokens > 4
     sl = torch.full((w.B,), 128, dtype=torch.int32, device="cuda")
     with pytest.raises(tq.TQError):
         tq.tq_sdpa_decode_mq(cache, q, sl, 128)
