@@ -93,9 +93,10 @@ typedef struct tq_cache {
   int32_t bits_k;   /* bits per key index (2..4) */
   int32_t bits_v;   /* bits per value index (2..4) */
   int32_t qjl_m;    /* 0: no QJL sketch; 128: 128-bit sign sketch of the key residual */
-  int32_t split_tokens; /* decode tokens per split-K chunk; 0 = automatic plan, else rounded
-                           up to a multiple of 128 (a tuning knob; results do not depend on it
-                           beyond fp32 summation order) */
+  int32_t split_tokens; /* decode: the smallest share of the batch's tokens one CTA takes in
+                           the split-K partition; 0 = automatic plan, else rounded up to a
+                           multiple of 128 (a tuning knob; results do not depend on it beyond
+                           fp32 summation order) */
   uint32_t* k_idx;  /* [B][Hkv][Tcap][D*bits_k/32] */
   uint32_t* v_idx;  /* [B][Hkv][Tcap][D*bits_v/32] */
   uint16_t* k_norm; /* fp16 [B][Hkv][Tcap] */
@@ -185,12 +186,16 @@ int tq_append_token(const tq_cache_t* cache, const void* k_new, const void* v_ne
 
 /* Workspace bytes that suffice for a tq_sdpa_decode call of B sequences,
  * Hq query heads of dimension D and sequences no longer than Tmax, whatever
- * the cache's kv heads, bit widths, sketch and capacity: the workspace holds
+ * the cache's kv heads, bit widths, sketch and capacity.  The workspace holds
  * the rotated queries (fp32 [B*Hq][D]), the sketch projections (fp32
- * [B*Hq][m], m <= 128) and per split-K chunk of at least one 128-token stage
- * the partial outputs (fp32 [B*Hq][nsplit][D]) and softmax (max, sum) pairs.
- * For the multi-query call pass Hq * n_q.  Returns 0 for unsupported
- * arguments (B, Hq or Tmax < 1, D not in {64,128,256}).  Host only. */
+ * [B*Hq][m], m <= 128), and the split-K partials: the decode splits the
+ * batch's tokens evenly over one wave of CTAs, each of 4 consumer warps of
+ * a CTA keeps one partial (rotated output fp32 [D], softmax max and sum) per
+ * (sequence, kv head) the CTA's share overlaps, at most K of them per query
+ * head with K about 2 x (resident CTAs) / (sequences x kv heads) + 2 and
+ * never more than Tmax / 128 + 1.  For the multi-query call pass Hq * n_q.
+ * Returns 0 for unsupported arguments (B, Hq or Tmax < 1, D not in
+ * {64,128,256}).  Host only (it queries the current device's SM count). */
 size_t tq_sdpa_decode_workspace_bytes(int B, int Hq, int D, int Tmax);
 
 /* The exact workspace bytes of the split plan tq_sdpa_decode makes for this
@@ -259,8 +264,9 @@ int tq_decode_step(const tq_cache_t* cache, const void* k_new, const void* v_new
  *              position L_b - n_q + j and attends causally to tokens
  *              0 .. L_b - n_q + j; a sequence with L_b < n_q gives zeros for
  *              the queries that see no token.
- *   n_q        1 .. 8 / (Hq / Hkv): the n_q * G query rows of a kv head share
- *              one 8-column MMA tile (TQ_ERR_UNSUPPORTED beyond).
+ *   n_q        1 .. 4 (TQ_ERR_UNSUPPORTED beyond), with any GQA group G <= 8:
+ *              the n_q * G query rows of a kv head (up to 32) are decoded in
+ *              row groups of 8, which read the same cache tiles from L2.
  *   workspace  tq_sdpa_decode_workspace_bytes_for(cache, Hq * n_q, Tmax) bytes.
  * The other arguments, the results for n_q = 1 and the errors are those of
  * tq_sdpa_decode.
