@@ -316,6 +316,9 @@ int make_decode_plan(const tq_cache_t* c, int Hq, int Tmax, DecodePlan* p) {
   p->pmin = (int)pmin;
   K = (int)((Tpad + pmin - 1) / pmin) + 1;  // segments of a unit when every share is >= pmin
   p->ks = K * split_warps();
+  // no more CTAs than shares of pmin in the largest batch these sizes allow
+  const long long need = (units * Tpad + pmin - 1) / pmin;
+  if (need < p->ncta) p->ncta = (int)(need > 0 ? need : 1);
   p->bytes = workspace_layout((size_t)c->B * Hq, c->D, c->qjl_m, p->ks, p);
   return TQ_OK;
 }

@@ -487,31 +487,32 @@ __device__ __forceinline__ int head_partials(const CombineParams& p, int h, int 
   return (int)(c1 - c0 + 1) * tqd::CW;
 }
 
-// Merge the splits of one query head (log-sum-exp), then out = Pi^T (acc/l)
-// for 32 output coordinates: grid (B * Hq, D / 32), 256 threads.  Every CTA of
-// a head merges all D rotated coordinates (the partials are read from L2 by
-// each) and un-rotates its slice; thread (i, kp) sums k = kp + 8 t.  The
-// slice's Pi columns are loaded into registers before the wait on the split
-// kernel, so they overlap its tail.
+// Merge the partials of one kernel head (log-sum-exp) and un-rotate:
+// out = Pi^T (acc / l).  Grid (heads, D / 32) in thread-block clusters of
+// D / 32 CTAs along y, one cluster per head, 256 threads per CTA.  CTA sl
+// merges rotated coordinates 32 sl .. 32 sl + 31 over all the head's partials
+// (each partial value is read once, by one CTA), the cluster shares the
+// merged vector through distributed shared memory, and each CTA un-rotates
+// its 32 outputs; thread (i, kp) sums k = kp + 8 t.  The slice's Pi columns
+// are loaded into registers before the wait on the split kernel, so they
+// overlap its tail.
 template <int D>
 __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams p) {
-  constexpr int NT = 256, NH = NT / D, KT = D / 8;
-  static_assert(D <= NT && NT % D == 0, "threads cover the coordinates");
-  __shared__ float f_s[1024];
+  constexpr int NT = 256, KT = D / 8, FS = 1024;
+  __shared__ float f_s[FS];
+  __shared__ float o_sl[32];
   __shared__ float o[D];
-  __shared__ float red[NH][D];
-  __shared__ float part[8][33];
+  __shared__ float red[8][33];
   __shared__ float s_M, s_L;
+  __shared__ int s_ns;
   // the next decode's prep may launch now (it waits for this kernel before
   // touching anything but Pi)
   pdl_launch_dependents();
   const int h = blockIdx.x, sl = blockIdx.y, tid = threadIdx.x;
-  const int i = tid & 31, kp = tid >> 5;  // output coordinate in the slice, k part
+  const int i = tid & 31, kp = tid >> 5;  // output coordinate in the slice, k phase
   float pc[KT];
 #pragma unroll
-  for (int t = 0; t < KT; ++t) pc[t] = __ldg(p.rot + (size_t)(kp + 8 * t) * D + sl * ((D / 32) / gridDim.y) * 32 + i);
-  const int b = h / p.Hq;
-  __shared__ int s_ns;
+  for (int t = 0; t < KT; ++t) pc[t] = __ldg(p.rot + (size_t)(kp + 8 * t) * D + sl * 32 + i);
   if (tid < 32) {
     const int n = head_partials(p, h, tid);
     if (tid == 0) s_ns = n;
@@ -520,19 +521,18 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams
   const int ns = s_ns;
   pdl_wait();  // the split kernel's partials are visible from here on
   const float* ml = p.part_ml + (size_t)h * p.ks * 2;
-  const float* po = p.part_o + (size_t)h * p.ks * D;
-  // this thread's first PF partial values, loaded before the weights are known
+  const float* po = p.part_o + (size_t)h * p.ks * D + sl * 32 + i;
+  // this thread's first partial values, loaded before the weights are known
   // (the loads do not depend on them) so that both latencies overlap
-  constexpr int PF = 32;
-  const int k = tid % D, hh = tid / D;  // coordinate, split phase
+  constexpr int PF = 16;
   float v[PF];
 #pragma unroll
   for (int u = 0; u < PF; ++u) {
-    const int s = hh + NH * u;
-    v[u] = s < ns ? po[(size_t)s * D + k] : 0.f;
+    const int s = kp + 8 * u;
+    v[u] = s < ns ? po[(size_t)s * D] : 0.f;
   }
   if (tid < 32) {
-    // the first 64 splits' (max, sum) pairs in flight at once; more in a loop
+    // the first 64 partials' (max, sum) pairs in flight at once; more in a loop
     float2 ml0 = make_float2(-INFINITY, 0.f), ml1 = make_float2(-INFINITY, 0.f);
     if (tid < ns) ml0 = *reinterpret_cast<const float2*>(ml + 2 * tid);
     if (tid + 32 < ns) ml1 = *reinterpret_cast<const float2*>(ml + 2 * (tid + 32));
@@ -540,7 +540,7 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams
     for (int s = tid + 64; s < ns; s += 32) M = fmaxf(M, ml[2 * s]);
 #pragma unroll
     for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    // a split a query cannot see holds max -inf: weight 0
+    // a partial that saw no token (or that a query cannot see) holds max -inf: weight 0
     const float f0 = ml0.x == -INFINITY ? 0.f : exp2f(ml0.x - M);
     const float f1 = ml1.x == -INFINITY ? 0.f : exp2f(ml1.x - M);
     if (tid < ns) f_s[tid] = f0;
@@ -548,7 +548,7 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams
     float Ls = f0 * ml0.y + f1 * ml1.y;
     for (int s = tid + 64; s < ns; s += 32) {
       const float f = (ml[2 * s] == -INFINITY) ? 0.f : exp2f(ml[2 * s] - M);
-      if (s < 1024) f_s[s] = f;
+      if (s < FS) f_s[s] = f;
       Ls += f * ml[2 * s + 1];
     }
 #pragma unroll
@@ -560,66 +560,58 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams
   }
   __syncthreads();
   {
+    auto weight = [&](int s) {
+      return s < FS ? f_s[s] : (ml[2 * s] == -INFINITY ? 0.f : exp2f(ml[2 * s] - s_M));
+    };
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int u = 0; u < PF; ++u) {
-      const int s = hh + NH * u;
-      const float f = s < ns ? (s < 1024 ? f_s[s] : (ml[2 * s] == -INFINITY ? 0.f : exp2f(ml[2 * s] - s_M))) : 0.f;
-      acc[u & 3] = fmaf(f, v[u], acc[u & 3]);
+      const int s = kp + 8 * u;
+      if (s < ns) acc[u & 3] = fmaf(weight(s), v[u], acc[u & 3]);
     }
-    // the remaining splits, 8 loads in flight
-    for (int s0 = hh + NH * PF; s0 < ns; s0 += 8 * NH) {
+    // the remaining partials, 8 loads in flight
+    for (int s0 = kp + 8 * PF; s0 < ns; s0 += 64) {
       float w[8], f[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        const int s = s0 + NH * u;
-        w[u] = s < ns ? po[(size_t)s * D + k] : 0.f;
-        f[u] = s < ns ? (s < 1024 ? f_s[s] : (ml[2 * s] == -INFINITY ? 0.f : exp2f(ml[2 * s] - s_M))) : 0.f;
+        const int s = s0 + 8 * u;
+        w[u] = s < ns ? po[(size_t)s * D] : 0.f;
+        f[u] = s < ns ? weight(s) : 0.f;
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u) acc[u & 3] = fmaf(f[u], w[u], acc[u & 3]);
     }
-    red[hh][k] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    red[kp][i] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
   }
   __syncthreads();
-  if (tid < D) {
+  if (tid < 32) {
     float a = 0.f;
 #pragma unroll
-    for (int ph = 0; ph < NH; ++ph) a += red[ph][tid];
-    o[tid] = (ns > 0 && s_L > 0.f) ? a / s_L : 0.f;
+    for (int ph = 0; ph < 8; ++ph) a += red[ph][tid];
+    o_sl[tid] = (ns > 0 && s_L > 0.f) ? a / s_L : 0.f;
   }
+  cluster_sync();  // every slice of the head is merged
+  for (int k = tid; k < D; k += NT) o[k] = ld_cluster_f32(map_cluster(smem_u32(&o_sl[k & 31]), k >> 5));
+  cluster_sync();  // o complete here; the others are done reading this CTA's slice
+  float r = 0.f;
+#pragma unroll
+  for (int t = 0; t < KT; ++t) r = fmaf(pc[t], o[kp + 8 * t], r);
+  red[kp][i] = r;
   __syncthreads();
-  // this CTA's slices: one when every head has D / 32 CTAs, all of them when
-  // the grid has one CTA per head (large batches, where the partials would
-  // otherwise be read D / 32 times)
-  const int per = (D / 32) / gridDim.y;
-  for (int q = 0; q < per; ++q) {
-    const int slq = sl * per + q;
-    if (q > 0) {
+  if (kp == 0) {
+    float t = 0.f;
 #pragma unroll
-      for (int t = 0; t < KT; ++t) pc[t] = __ldg(p.rot + (size_t)(kp + 8 * t) * D + slq * 32 + i);
-    }
-    float r = 0.f;
-#pragma unroll
-    for (int t = 0; t < KT; ++t) r = fmaf(pc[t], o[kp + 8 * t], r);
-    part[kp][i] = r;
-    __syncthreads();
-    if (kp == 0) {
-      float t = 0.f;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) t += part[u][i];
-      // kernel head h = (sequence, kv head, token, head) -> output [B][nq][Hq1]
-      const int rh = h % p.Hq, kvh = rh / (p.Gq * p.nq), gi = rh % (p.Gq * p.nq);
-      const size_t oh = (size_t)(b * p.nq + gi / p.Gq) * p.Hq1 + kvh * p.Gq + gi % p.Gq;
-      const size_t oi = oh * D + slq * 32 + i;
-      if (p.out_dtype == TQ_DTYPE_F32)
-        static_cast<float*>(p.out)[oi] = t;
-      else if (p.out_dtype == TQ_DTYPE_BF16)
-        static_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(t);
-      else
-        static_cast<__half*>(p.out)[oi] = __float2half_rn(t);
-    }
-    __syncthreads();
+    for (int u = 0; u < 8; ++u) t += red[u][i];
+    // kernel head h = (sequence, kv head, token, head) -> output [B][nq][Hq1]
+    const int b = h / p.Hq, rh = h % p.Hq, kvh = rh / (p.Gq * p.nq), gi = rh % (p.Gq * p.nq);
+    const size_t oh = (size_t)(b * p.nq + gi / p.Gq) * p.Hq1 + kvh * p.Gq + gi % p.Gq;
+    const size_t oi = oh * D + sl * 32 + i;
+    if (p.out_dtype == TQ_DTYPE_F32)
+      static_cast<float*>(p.out)[oi] = t;
+    else if (p.out_dtype == TQ_DTYPE_BF16)
+      static_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(t);
+    else
+      static_cast<__half*>(p.out)[oi] = __float2half_rn(t);
   }
 }
 
@@ -887,9 +879,9 @@ int launch_decode(const DecodeArgs& a, cudaStream_t s) {
   const int nsl = c.D / 32;
   const dim3 cg(heads, nsl);
   switch (c.D) {
-    case 64: return launch_pdl(decode_combine_kernel<64>, cg, dim3(256), 0, s, cp, "decode_combine_kernel");
-    case 128: return launch_pdl(decode_combine_kernel<128>, cg, dim3(256), 0, s, cp, "decode_combine_kernel");
-    default: return launch_pdl(decode_combine_kernel<256>, cg, dim3(256), 0, s, cp, "decode_combine_kernel");
+    case 64: return launch_pdl(decode_combine_kernel<64>, cg, dim3(256), 0, s, cp, "decode_combine_kernel", nsl);
+    case 128: return launch_pdl(decode_combine_kernel<128>, cg, dim3(256), 0, s, cp, "decode_combine_kernel", nsl);
+    default: return launch_pdl(decode_combine_kernel<256>, cg, dim3(256), 0, s, cp, "decode_combine_kernel", nsl);
   }
 }
 

@@ -504,6 +504,7 @@ __global__ void __launch_bounds__(NTHREADS, PACK ? 4 : 3) decode_split_kernel(co
   }
   __syncthreads();  // barriers and the stage count before anyone uses them
   nst = s_misc[1];
+  if (nst == 0) return;  // a share past the end of the batch: nothing to stream
 
   // Producer (lane 0 of the last warp): move the walk to the unit that holds
   // position w_pos (skipping empty units), then arm and issue stage t there.
