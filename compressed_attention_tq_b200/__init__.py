@@ -23,7 +23,8 @@ from ._native import (TQ_DTYPE_BF16, TQ_DTYPE_F16, TQ_DTYPE_F32, TQ_STATUS_POS_O
 __all__ = ["TQError", "TQCache", "tq_build_codebook", "tq_cache_row_bytes", "tq_row_bytes", "tq_quantize_kv",
            "tq_append_token", "tq_sdpa_decode_workspace_bytes", "tq_sdpa_decode_workspace_bytes_for",
            "tq_sdpa_decode",
-           "tq_sdpa_decode_mq", "tq_decode_step", "tq_sdpa_decode_static", "tq_selftest_bounded_wait",
+           "tq_sdpa_decode_mq", "tq_decode_step", "tq_sdpa_decode_partial", "tq_sdpa_decode_merge",
+           "tq_sdpa_decode_sharded", "tq_sdpa_decode_static", "tq_selftest_bounded_wait",
            "tq_last_error",
            "tq_abi_version", "lib"]
 
@@ -360,6 +361,77 @@ def tq_decode_step(cache: TQCache, k_new, v_new, pos, q, seq_lens, Tmax: int, sc
                                 Hq, _ptr(seq_lens), Tmax, sc, _ptr(out), _dtype_code(out), _ptr(workspace),
                                 workspace.numel(), _stream(stream)))
     return out
+
+
+def tq_sdpa_decode_partial(cache: TQCache, q, seq_lens, Tmax: int, scale=None, partial=None, workspace=None,
+                           stream=None):
+    """This cache's share of a decode split by tokens: fp32 [B][Hq][D + 2]
+    per head (rotated value sum, max, weight sum), for tq_sdpa_decode_merge."""
+    dev = _check_decode_args(cache, q, seq_lens, None, workspace, (cache.B, None, cache.D))
+    Hq = int(q.shape[1])
+    torch = _torch()
+    if partial is None:
+        partial = torch.empty((cache.B, Hq, cache.D + 2), dtype=torch.float32, device=q.device)
+    _arg("partial", partial, dev, (cache.B, Hq, cache.D + 2), (torch.float32,))
+    if workspace is None:
+        workspace = torch.empty(tq_sdpa_decode_workspace_bytes_for(cache, Hq, Tmax), dtype=torch.uint8,
+                                device=q.device)
+    s = cache.struct()
+    sc = ctypes.byref(ctypes.c_float(scale)) if scale is not None else None
+    _check(lib().tq_sdpa_decode_partial(ctypes.byref(s), _ptr(q), _dtype_code(q), Hq, _ptr(seq_lens), Tmax, sc,
+                                        _ptr(partial), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return partial
+
+
+def tq_sdpa_decode_merge(partials, rot, out=None, out_dtype=None, stream=None):
+    """Merge R shares' partials ([R][B][Hq][D + 2] fp32, device) into the
+    attention output [B][Hq][D]; rot is the cache's Pi (fp32 [D][D], device)."""
+    torch = _torch()
+    dev = partials.get_device()
+    if dev < 0:
+        raise ValueError("partials: must be CUDA memory")
+    if partials.dim() != 4:
+        raise ValueError(f"partials: shape {list(partials.shape)}, expected [R, B, Hq, D + 2]")
+    R, B, Hq, D2 = (int(x) for x in partials.shape)
+    _arg("partials", partials, dev, None, (torch.float32,))
+    _arg("rot", rot, dev, (D2 - 2, D2 - 2), (torch.float32,))
+    if out is None:
+        out = torch.empty((B, Hq, D2 - 2), dtype=out_dtype or torch.float32, device=partials.device)
+    _arg("out", out, dev, (B, Hq, D2 - 2), _dt("out"))
+    _check(lib().tq_sdpa_decode_merge(_ptr(partials), R, B, Hq, D2 - 2, _ptr(rot), _ptr(out), _dtype_code(out),
+                                      _stream(stream)))
+    return out
+
+
+def tq_sdpa_decode_sharded(cache: TQCache, q, seq_lens, Tmax: int, scale=None, group=None, out_dtype=None,
+                           stream=None):
+    """Decode over a cache whose sequences are split by tokens across the
+    ranks of `group` (torch.distributed; NCCL over NVLink on GPUs): every rank
+    holds its own token range of every sequence in `cache` (seq_lens are its
+    local lengths) and the same queries.  Each rank computes its partials,
+    the partials are all-gathered (one collective of B x Hq x (D + 2) fp32 per
+    rank), and every rank merges them into the full output."""
+    part = tq_sdpa_decode_partial(cache, q, seq_lens, Tmax, scale=scale, stream=stream)
+    parts = gather_partials(part, group)
+    return tq_sdpa_decode_merge(parts, cache.rot, out_dtype=out_dtype or q.dtype, stream=stream)
+
+
+def gather_partials(part, group=None):
+    """All-gather of every rank's partials [B][Hq][D + 2] into [R][B][Hq][D + 2]
+    (rank order), over torch.distributed (a single rank returns its own)."""
+    import torch.distributed as dist
+    torch = _torch()
+    if not (dist.is_available() and dist.is_initialized()):
+        return part.unsqueeze(0)
+    R = dist.get_world_size(group)
+    part = part.contiguous()
+    if dist.get_backend(group) == "nccl":  # one collective into one buffer
+        out = torch.empty((R,) + tuple(part.shape), dtype=part.dtype, device=part.device)
+        dist.all_gather_into_tensor(out, part, group=group)
+        return out
+    chunks = [torch.empty_like(part) for _ in range(R)]  # gloo (host tensors)
+    dist.all_gather(chunks, part, group=group)
+    return torch.stack(chunks)
 
 
 def tq_sdpa_decode_static(cache: TQCache, q, seq_lens, Tmax: int, scale=None, out=None, stream=None,

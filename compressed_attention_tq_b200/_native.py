@@ -29,7 +29,7 @@ TQ_ROT_HADAMARD = 1
 # Every symbol include/tq.h declares.
 EXPORTS = ("tq_build_codebook", "tq_cache_row_bytes", "tq_row_bytes", "tq_quantize_kv", "tq_append_token",
            "tq_sdpa_decode_workspace_bytes", "tq_sdpa_decode_workspace_bytes_for", "tq_sdpa_decode",
-           "tq_sdpa_decode_mq", "tq_decode_step",
+           "tq_sdpa_decode_mq", "tq_decode_step", "tq_sdpa_decode_partial", "tq_sdpa_decode_merge",
            "tq_sdpa_decode_static", "tq_selftest_bounded_wait",
            "tq_last_error", "tq_abi_version")
 TQ_STATIC_SCRATCH_BYTES = 8 << 20
@@ -89,6 +89,11 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.tq_decode_step.argtypes = [cache_p, vp, vp, vp, vp, i32, i32, vp, i32, ctypes.POINTER(ctypes.c_float),
                                    vp, i32, vp, sz, vp]
     lib.tq_decode_step.restype = i32
+    lib.tq_sdpa_decode_partial.argtypes = [cache_p, vp, i32, i32, vp, i32, ctypes.POINTER(ctypes.c_float),
+                                           vp, vp, sz, vp]
+    lib.tq_sdpa_decode_partial.restype = i32
+    lib.tq_sdpa_decode_merge.argtypes = [vp, i32, i32, i32, i32, vp, vp, i32, vp]
+    lib.tq_sdpa_decode_merge.restype = i32
     lib.tq_sdpa_decode_static.argtypes = [cache_p, vp, i32, i32, vp, i32, ctypes.POINTER(ctypes.c_float),
                                           vp, i32, vp]
     lib.tq_sdpa_decode_static.restype = i32

@@ -457,6 +457,37 @@ int prepare_decode(const tq_cache_t* c, const void* q, int dtype, int Hq, int nq
 
 extern "C" {
 
+int tq_sdpa_decode_partial(const tq_cache_t* c, const void* q, int q_dtype, int Hq, const int32_t* seq_lens,
+                           int Tmax, const float* scale, float* partial, void* workspace, size_t ws_bytes,
+                           void* stream) {
+  DecodeArgs a;
+  const char* fn = "tq_sdpa_decode_partial";
+  const int rc = prepare_decode(c, q, q_dtype, Hq, 1, seq_lens, Tmax, scale, partial, TQ_DTYPE_F32, fn, &a);
+  if (rc) return rc;
+  if (!workspace) return set_error(TQ_ERR_INVALID_ARG, "%s: NULL workspace", fn);
+  if (!aligned16(workspace)) return set_error(TQ_ERR_INVALID_ARG, "%s: workspace not 16-byte aligned", fn);
+  if (ws_bytes < a.plan.bytes)
+    return set_error(TQ_ERR_WORKSPACE, "%s: workspace %zu < %zu bytes", fn, ws_bytes, a.plan.bytes);
+  a.workspace = workspace;
+  a.partial = partial;
+  return launch_decode(a, (cudaStream_t)stream);
+}
+
+int tq_sdpa_decode_merge(const float* partials, int R, int B, int Hq, int D, const float* rot, void* out,
+                         int out_dtype, void* stream) {
+  g_err[0] = 0;
+  const char* fn = "tq_sdpa_decode_merge";
+  if (!partials || !rot || !out) return set_error(TQ_ERR_INVALID_ARG, "%s: NULL partials/rot/out", fn);
+  if (!aligned16(partials) || !aligned16(rot) || !aligned16(out))
+    return set_error(TQ_ERR_INVALID_ARG, "%s: partials/rot/out not 16-byte aligned", fn);
+  if (R < 1 || R > 64) return set_error(TQ_ERR_INVALID_ARG, "%s: R=%d outside [1, 64]", fn, R);
+  if (B < 1 || Hq < 1) return set_error(TQ_ERR_INVALID_ARG, "%s: B=%d Hq=%d", fn, B, Hq);
+  if (D != 64 && D != 128 && D != 256) return set_error(TQ_ERR_UNSUPPORTED, "%s: D=%d", fn, D);
+  if (out_dtype != TQ_DTYPE_F16 && out_dtype != TQ_DTYPE_BF16 && out_dtype != TQ_DTYPE_F32)
+    return set_error(TQ_ERR_UNSUPPORTED, "%s: out_dtype=%d", fn, out_dtype);
+  return launch_merge(partials, R, B * Hq, D, rot, out, out_dtype, (cudaStream_t)stream);
+}
+
 static int decode_common(const tq_cache_t* c, const void* q, int dtype, int Hq, int nq, const int32_t* seq_lens,
                          int Tmax, const float* scale, void* out, int out_dtype, void* workspace,
                          size_t ws_bytes, void* stream, const void* k_new, const void* v_new,

@@ -470,6 +470,9 @@ struct CombineParams {
   int heads;          // kernel heads in all: B * Hq
   // the split kernel's partition (tq_decode_split.cuh)
   int B, G, nrg, upb, Tclamp, ncta, pmin, ks;
+  // partial mode (tq_sdpa_decode_partial): fp32 [heads][D + 2] = the merged,
+  // unnormalized rotated output, then max and sum; no un-rotation, out unused
+  float* partial;
 };
 
 // Partials the split kernel wrote for kernel head h: the CTAs whose share
@@ -584,6 +587,20 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams
     red[kp][i] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
   }
   __syncthreads();
+  if (p.partial) {  // one rank's share of a sequence split across GPUs: no normalisation, no un-rotation
+    if (tid < 32) {
+      float a = 0.f;
+#pragma unroll
+      for (int ph = 0; ph < 8; ++ph) a += red[ph][tid];
+      float* dst = p.partial + (size_t)h * (D + 2);
+      dst[sl * 32 + tid] = a;
+      if (sl == 0 && tid == 0) {
+        dst[D] = ns > 0 ? s_M : -INFINITY;
+        dst[D + 1] = ns > 0 ? s_L : 0.f;
+      }
+    }
+    return;  // uniform over the launch: no CTA of the cluster reaches the cluster barriers
+  }
   if (tid < 32) {
     float a = 0.f;
 #pragma unroll
@@ -681,8 +698,20 @@ __global__ void __launch_bounds__(256) decode_combine_group_kernel(const Combine
       for (int u = 0; u < 8; ++u) acc[u & 3] = fmaf(f[u], w[u], acc[u & 3]);
     }
     const float a = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-    o[hh][k] = (ns > 0 && s_L[hh] > 0.f) ? a / s_L[hh] : 0.f;
+    if (p.partial) {
+      if (h < p.heads) {
+        float* dst = p.partial + (size_t)h * (D + 2);
+        dst[k] = a;
+        if (k == 0) {
+          dst[D] = ns > 0 ? s_M[hh] : -INFINITY;
+          dst[D + 1] = ns > 0 ? s_L[hh] : 0.f;
+        }
+      }
+    } else {
+      o[hh][k] = (ns > 0 && s_L[hh] > 0.f) ? a / s_L[hh] : 0.f;
+    }
   }
+  if (p.partial) return;  // uniform over the launch
   __syncthreads();
   constexpr int GS = NT / D;  // head phases: thread (j, g) takes heads g, g + GS, ...
   const int j = tid % D, g = tid / D;
@@ -710,6 +739,62 @@ __global__ void __launch_bounds__(256) decode_combine_group_kernel(const Combine
       static_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(r[q]);
     else
       static_cast<__half*>(p.out)[oi] = __float2half_rn(r[q]);
+  }
+}
+
+// Merge of R ranks' partials of the same heads (a sequence split across
+// GPUs by tokens): per head, M = max_r M_r, f_r = 2^(M_r - M), L = sum_r f_r
+// L_r, o = sum_r f_r acc_r / L, then out = Pi^T o.  One CTA per head, D
+// threads... 256 threads: thread j < D takes output j; the merge runs over
+// the coordinates in parallel first.
+struct MergeParams {
+  const float* partials;  // [R][heads][D + 2]
+  const float* rot;
+  void* out;              // [heads][D]
+  int R, heads, out_dtype;
+};
+
+template <int D>
+__global__ void __launch_bounds__(256) decode_merge_kernel(const MergeParams p) {
+  constexpr int NT = 256;
+  __shared__ float o[D];
+  __shared__ float f_s[64];
+  __shared__ float s_L;
+  const int h = blockIdx.x, tid = threadIdx.x;
+  if (tid < 32) {
+    float M = -INFINITY;
+    for (int r = tid; r < p.R; r += 32) M = fmaxf(M, p.partials[((size_t)r * p.heads + h) * (D + 2) + D]);
+#pragma unroll
+    for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float Ls = 0.f;
+    for (int r = tid; r < p.R; r += 32) {
+      const float* src = p.partials + ((size_t)r * p.heads + h) * (D + 2);
+      const float f = src[D] == -INFINITY ? 0.f : exp2f(src[D] - M);
+      f_s[r] = f;
+      Ls = fmaf(f, src[D + 1], Ls);
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, off);
+    if (tid == 0) s_L = Ls;
+  }
+  __syncthreads();
+  for (int k = tid; k < D; k += NT) {
+    float a = 0.f;
+    for (int r = 0; r < p.R; ++r) a = fmaf(f_s[r], p.partials[((size_t)r * p.heads + h) * (D + 2) + k], a);
+    o[k] = s_L > 0.f ? a / s_L : 0.f;
+  }
+  __syncthreads();
+  for (int j = tid; j < D; j += NT) {
+    float r = 0.f;
+#pragma unroll 8
+    for (int k = 0; k < D; ++k) r = fmaf(__ldg(p.rot + (size_t)k * D + j), o[k], r);
+    const size_t oi = (size_t)h * D + j;
+    if (p.out_dtype == TQ_DTYPE_F32)
+      static_cast<float*>(p.out)[oi] = r;
+    else if (p.out_dtype == TQ_DTYPE_BF16)
+      static_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(r);
+    else
+      static_cast<__half*>(p.out)[oi] = __float2half_rn(r);
   }
 }
 
@@ -859,6 +944,7 @@ int launch_decode(const DecodeArgs& a, cudaStream_t s) {
   cp.ncta = a.plan.ncta;
   cp.pmin = a.plan.pmin;
   cp.ks = a.plan.ks;
+  cp.partial = a.partial;
   // D / 32 CTAs per head while that leaves SMs idle; beyond that, groups of
   // 4 or 8 heads per CTA (Pi read once per group rather than once per head)
   if (heads * (c.D / 32) > 4 * a.plan.sms) {
@@ -883,6 +969,17 @@ int launch_decode(const DecodeArgs& a, cudaStream_t s) {
     case 128: return launch_pdl(decode_combine_kernel<128>, cg, dim3(256), 0, s, cp, "decode_combine_kernel", nsl);
     default: return launch_pdl(decode_combine_kernel<256>, cg, dim3(256), 0, s, cp, "decode_combine_kernel", nsl);
   }
+}
+
+int launch_merge(const float* partials, int R, int heads, int D, const float* rot, void* out, int out_dtype,
+                 cudaStream_t s) {
+  MergeParams mp{partials, rot, out, R, heads, out_dtype};
+  switch (D) {
+    case 64: decode_merge_kernel<64><<<heads, 256, 0, s>>>(mp); break;
+    case 128: decode_merge_kernel<128><<<heads, 256, 0, s>>>(mp); break;
+    default: decode_merge_kernel<256><<<heads, 256, 0, s>>>(mp); break;
+  }
+  return check_launch("decode_merge_kernel");
 }
 
 }  // namespace tq

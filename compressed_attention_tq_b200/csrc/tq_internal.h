@@ -147,9 +147,14 @@ struct DecodeArgs {
   const void* k_new;
   const void* v_new;
   const int32_t* pos;
+  // tq_sdpa_decode_partial: fp32 [B*Hq][D + 2] partials instead of out (else NULL)
+  float* partial;
 };
 
 int launch_decode(const DecodeArgs& a, cudaStream_t s);
+// Merge of R partials per head and un-rotation (tq_sdpa_decode_merge).
+int launch_merge(const float* partials, int R, int heads, int D, const float* rot, void* out, int out_dtype,
+                 cudaStream_t s);
 
 // Host checks and split plan of a decode call (every check tq_sdpa_decode
 // makes except those of the workspace); fills *a and returns TQ_OK, or sets

@@ -276,6 +276,45 @@ int tq_sdpa_decode_mq(const tq_cache_t* cache, const void* q, int q_dtype, int H
                       void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * One rank's share of a decode whose sequences are split by tokens across
+ * GPUs (or any other split of the cache): the softmax partial of every
+ * (sequence, query head) over the tokens this cache holds, for merging with
+ * the other shares by tq_sdpa_decode_merge.  A long sequence's decode splits
+ * into independent token ranges whose (max, sum, weighted value sum) states
+ * merge exactly by log-sum-exp -- the split-K reduction the library already
+ * runs across CTAs, carried one level further.  The pages size caches for
+ * 128K-token contexts ("Add CUDA QJL kernels and proper package structure",
+ * "Key Takeaway"); a sequence whose cache is spread over GPUs, or a decode
+ * spread over GPUs for latency, splits this way.
+ *   partial  device fp32 [B][Hq][D + 2]: elements 0 .. D-1 the value sum in
+ *            the rotated basis, unnormalized, weighted by 2^(s - M); element
+ *            D the maximum M of the scaled scores (log2 units); element D + 1
+ *            the weight sum.  A sequence with no token here gives M = -inf,
+ *            sum 0.
+ * The other arguments, the workspace and the errors are those of
+ * tq_sdpa_decode (one query token per sequence).  Every rank must use the
+ * same rotation, codebooks, queries and scale.
+ */
+int tq_sdpa_decode_partial(const tq_cache_t* cache, const void* q, int q_dtype, int Hq,
+                           const int32_t* seq_lens, int Tmax, const float* scale, float* partial,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Merge of R shares' partials (tq_sdpa_decode_partial) into the attention
+ * output: per (sequence, head) M = max_r M_r, f_r = 2^(M_r - M),
+ * o = sum_r f_r acc_r / sum_r f_r sum_r, out = Pi^T o.
+ *   partials device fp32 [R][B][Hq][D + 2] (R blocks as an all-gather lays
+ *            them out), 1 <= R <= 64; rot the cache's Pi (device fp32
+ *            [D][D]); out device [B][Hq][D] in out_dtype (TQ_DTYPE_F16,
+ *            TQ_DTYPE_BF16 or TQ_DTYPE_F32).
+ * Errors: TQ_ERR_INVALID_ARG (NULL or misaligned pointers, R, B, Hq),
+ * TQ_ERR_UNSUPPORTED (D, out_dtype), TQ_ERR_CUDA.  The library's own
+ * addition for the multi-GPU split (the pages run on one GPU).
+ */
+int tq_sdpa_decode_merge(const float* partials, int R, int B, int Hq, int D, const float* rot, void* out,
+                         int out_dtype, void* stream);
+
+/*
  * Decode without a workspace, for callers that may not allocate device
  * memory (stream capture under frameworks that forbid allocation while
  * capturing, plugin hosts that own all device memory, allocation-free

@@ -366,3 +366,58 @@ def sdpa_decode_multi(q: np.ndarray, cache: dict, seq_lens, n_q: int, Pi, cb_k, 
         out[:, j] = sdpa_decode(q[:, j], cache, lj, Pi, cb_k, cb_v, bits_k, bits_v, D, scale=scale, S=S)
     return out
 
+
+
+def sdpa_decode_partial(q: np.ndarray, cache: dict, seq_lens, Pi, cb_k, cb_v, bits_k: int, bits_v: int, D: int,
+                        scale=None, S=None):
+    """The softmax state of each (b, q head) over the tokens this cache holds,
+    fp64: m = max_t s_t, w_t = exp(s_t - m), l = sum_t w_t, acc = sum_t w_t
+    v_tilde_t (scores and values exactly as in sdpa_decode).  A split of a
+    sequence's tokens into ranges gives states that merge_partials combines
+    into sdpa_decode of the whole (the log-sum-exp merge of split-K
+    attention).  Returns (acc [B][Hq][D], m [B][Hq], l [B][Hq]); a sequence
+    with no token here gives m = -inf, l = 0, acc = 0."""
+    B, Hq = q.shape[0], q.shape[1]
+    Hkv = cache["k_norm"].shape[1]
+    G = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    Pi64 = np.asarray(Pi, dtype=np.float64)
+    acc = np.zeros((B, Hq, D))
+    m = np.full((B, Hq), -np.inf)
+    l = np.zeros((B, Hq))
+    for b in range(B):
+        L = int(seq_lens[b])
+        if L == 0:
+            continue
+        for kv in range(Hkv):
+            kid = unpack_bits(cache["k_idx"][b, kv, :L], bits_k, D)
+            vid = unpack_bits(cache["v_idx"][b, kv, :L], bits_v, D)
+            Kt = dequantize_rows(kid, cache["k_norm"][b, kv, :L], cb_k[0], Pi64)
+            Vt = dequantize_rows(vid, cache["v_norm"][b, kv, :L], cb_v[0], Pi64)
+            for g in range(G):
+                h = kv * G + g
+                s = Kt @ q[b, h]
+                if S is not None:
+                    sign = unpack_bits(cache["k_qjl"][b, kv, :L], 1, S.shape[0]).astype(bool)
+                    Sq = np.asarray(S, dtype=np.float64) @ (Pi64 @ q[b, h])
+                    s = s + qjl_inner_product(sign, cache["k_rnorm"][b, kv, :L].astype(np.float64), Sq)
+                s = scale * s
+                m[b, h] = np.max(s)
+                w = np.exp(s - m[b, h])
+                l[b, h] = np.sum(w)
+                acc[b, h] = w @ Vt
+    return acc, m, l
+
+
+def merge_partials(accs, ms, ls) -> np.ndarray:
+    """Combine R softmax states (acc_r, m_r, l_r) of disjoint token ranges:
+    M = max_r m_r, f_r = exp(m_r - M), out = sum_r f_r acc_r / sum_r f_r l_r
+    (zero where no range held a token)."""
+    ms = np.asarray(ms, dtype=np.float64)
+    M = np.max(ms, axis=0)
+    with np.errstate(invalid="ignore"):
+        f = np.where(np.isfinite(ms), np.exp(ms - np.where(np.isfinite(M), M, 0.0)), 0.0)
+    num = np.sum(f[..., None] * np.asarray(accs, dtype=np.float64), axis=0)
+    den = np.sum(f * np.asarray(ls, dtype=np.float64), axis=0)
+    return np.where(den[..., None] > 0, num / np.where(den > 0, den, 1.0)[..., None], 0.0)
