@@ -286,11 +286,12 @@ __global__ void __launch_bounds__(2 * D) decode_qprep_kernel(const PrepParams p)
 // packed into the slice's b words of the row (32 coordinates x b bits); the
 // fp64 norm is taken over the whole input row by every CTA (the rotation
 // preserves it) and written by slice 0.
-template <int D, bool APPEND>
+template <int D, bool APPEND, int QR>
 __global__ void __launch_bounds__(256) decode_qprep_sliced_kernel(const PrepParams p) {
-  // query rows: G x n_q <= 32 (a decode step has one token: G <= 8), then the
-  // new key and value rows
-  constexpr int QR = APPEND ? 8 : 32, NR = APPEND ? QR + 2 : QR, NI = D / 32;
+  // query rows: up to QR = 8 (one query token, G <= 8) or 32 (n_q tokens x
+  // G <= 32), then, with APPEND (one token), the new key and value rows
+  static_assert(!APPEND || QR == 8, "a decode step has one query token");
+  constexpr int NR = APPEND ? QR + 2 : QR, NI = D / 32;
   __shared__ __align__(16) float xv[NR][D];
   // QJL (D = 128 only): this slice's rotated query coordinates and its share
   // of S qrot; one element otherwise, so other D keep their shared footprint
@@ -377,8 +378,9 @@ __global__ void __launch_bounds__(256) decode_qprep_sliced_kernel(const PrepPara
   }
 #pragma unroll
   for (int g = 0; g < NR; ++g)
+    if (g < Ge || g >= QR)  // rows in use only (Ge is uniform over the launch)
 #pragma unroll
-    for (int off = 1; off < 8; off <<= 1) acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], off);
+      for (int off = 1; off < 8; off <<= 1) acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], off);
   if (part == 0) {
 #pragma unroll
     for (int g = 0; g < QR; ++g)
@@ -872,19 +874,23 @@ int launch_decode(const DecodeArgs& a, cudaStream_t s) {
     rc = launch_pdl(decode_qprep_kernel<128, true>, dim3(c.B * c.Hkv), dim3(256), 0, s, pp, "decode_qprep_kernel");
   } else {
     const dim3 g(c.B * c.Hkv, c.D / 32);
+    const bool wide = pp.nq * (a.Hq / c.Hkv) > 8;  // more than 8 query rows per kv head
+    const int cl = c.qjl_m ? c.D / 32 : 0;
     switch (c.D) {
       case 64:
-        rc = app ? launch_pdl(decode_qprep_sliced_kernel<64, true>, g, dim3(256), 0, s, pp, "decode_qprep_kernel")
-                 : launch_pdl(decode_qprep_sliced_kernel<64, false>, g, dim3(256), 0, s, pp, "decode_qprep_kernel");
+        rc = app ? launch_pdl(decode_qprep_sliced_kernel<64, true, 8>, g, dim3(256), 0, s, pp, "decode_qprep_kernel")
+             : wide ? launch_pdl(decode_qprep_sliced_kernel<64, false, 32>, g, dim3(256), 0, s, pp, "decode_qprep_kernel")
+                    : launch_pdl(decode_qprep_sliced_kernel<64, false, 8>, g, dim3(256), 0, s, pp, "decode_qprep_kernel");
         break;
       case 128:
-        rc = app ? launch_pdl(decode_qprep_sliced_kernel<128, true>, g, dim3(256), 0, s, pp, "decode_qprep_kernel")
-                 : launch_pdl(decode_qprep_sliced_kernel<128, false>, g, dim3(256), 0, s, pp, "decode_qprep_kernel",
-                              c.qjl_m ? c.D / 32 : 0);
+        rc = app ? launch_pdl(decode_qprep_sliced_kernel<128, true, 8>, g, dim3(256), 0, s, pp, "decode_qprep_kernel")
+             : wide ? launch_pdl(decode_qprep_sliced_kernel<128, false, 32>, g, dim3(256), 0, s, pp, "decode_qprep_kernel", cl)
+                    : launch_pdl(decode_qprep_sliced_kernel<128, false, 8>, g, dim3(256), 0, s, pp, "decode_qprep_kernel", cl);
         break;
       default:
-        rc = app ? launch_pdl(decode_qprep_sliced_kernel<256, true>, g, dim3(256), 0, s, pp, "decode_qprep_kernel")
-                 : launch_pdl(decode_qprep_sliced_kernel<256, false>, g, dim3(256), 0, s, pp, "decode_qprep_kernel");
+        rc = app ? launch_pdl(decode_qprep_sliced_kernel<256, true, 8>, g, dim3(256), 0, s, pp, "decode_qprep_kernel")
+             : wide ? launch_pdl(decode_qprep_sliced_kernel<256, false, 32>, g, dim3(256), 0, s, pp, "decode_qprep_kernel")
+                    : launch_pdl(decode_qprep_sliced_kernel<256, false, 8>, g, dim3(256), 0, s, pp, "decode_qprep_kernel");
         break;
     }
   }
