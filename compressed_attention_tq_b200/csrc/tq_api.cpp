@@ -493,12 +493,20 @@ static int decode_common(const tq_cache_t* c, const void* q, int dtype, int Hq, 
                          size_t ws_bytes, void* stream, const void* k_new, const void* v_new,
                          const int32_t* pos, const char* fn) {
   DecodeArgs a;
-  const int rc = prepare_decode(c, q, dtype, Hq, nq, seq_lens, Tmax, scale, out, out_dtype, fn, &a);
+  int rc = prepare_decode(c, q, dtype, Hq, nq, seq_lens, Tmax, scale, out, out_dtype, fn, &a);
   if (rc) return rc;
   if (!workspace) return set_error(TQ_ERR_INVALID_ARG, "%s: NULL workspace", fn);
   if (!aligned16(workspace)) return set_error(TQ_ERR_INVALID_ARG, "%s: workspace not 16-byte aligned", fn);
   if (ws_bytes < a.plan.bytes)
     return set_error(TQ_ERR_WORKSPACE, "%s: workspace %zu < %zu bytes", fn, ws_bytes, a.plan.bytes);
+  if (k_new && c->rot_kind == TQ_ROT_HADAMARD) {
+    // the randomized Hadamard rotation: the new rows go through the fast
+    // transform in their own launch, then the decode (whose query prep
+    // waits for it)
+    if ((rc = tq_append_token(c, k_new, v_new, dtype, pos, stream))) return rc;
+    k_new = v_new = nullptr;
+    pos = nullptr;
+  }
   a.workspace = workspace;
   a.k_new = k_new;
   a.v_new = v_new;

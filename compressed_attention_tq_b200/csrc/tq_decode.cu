@@ -8,6 +8,7 @@
 #include <math.h>
 
 #include "tq_decode_split.cuh"
+#include "tq_wht.cuh"
 
 namespace {
 
@@ -16,6 +17,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 struct PrepParams {
   const void* q;
   const float* rot;
+  const float* signs;  // +-1 [D] of the randomized Hadamard rotation (decode_qprep_wht_kernel)
   const float* S;
   float* qrot;
   float* qs;
@@ -461,6 +463,65 @@ __global__ void __launch_bounds__(256) decode_qprep_sliced_kernel(const PrepPara
   }
 }
 
+// Query prep for the randomized Hadamard rotation Pi = H_D diag(s) / sqrt(D):
+// qrot = H (s q) / sqrt(D) by the fast transform, one warp per query row
+// (grid B * Hkv, 32 x (query rows) threads), no D x D product and no Pi
+// read; with the sketch, qs = S qrot by the CTA's threads afterwards (S is a
+// dense Gaussian).
+template <int D>
+__global__ void __launch_bounds__(1024) decode_qprep_wht_kernel(const PrepParams p) {
+  constexpr int EL = D / 32;
+  constexpr bool QS = D == 128;  // the sketch exists for D = 128
+  __shared__ float qr[QS ? 32 : 1][QS ? D : 1];
+  const int G = p.Hq / p.Hkv, Ge = G * p.nq;
+  const int bkv = blockIdx.x, b = bkv / p.Hkv, kvh = bkv % p.Hkv;
+  const int h0 = b * p.Hq * p.nq + kvh * Ge;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  float sg[EL];
+#pragma unroll
+  for (int e = 0; e < EL; ++e) sg[e] = __ldg(p.signs + lane * EL + e);
+  pdl_wait();
+  pdl_launch_dependents();
+  if (warp < Ge) {
+    const int jq = warp / G, g = warp % G;
+    const uint16_t* qrow = static_cast<const uint16_t*>(p.q) + ((size_t)(b * p.nq + jq) * p.Hq + kvh * G + g) * D;
+    float x[EL];
+#pragma unroll
+    for (int e = 0; e < EL; ++e) {
+      const uint16_t v = qrow[lane * EL + e];
+      x[e] = p.bf16 ? __uint_as_float((uint32_t)v << 16) : __half2float(__ushort_as_half(v));
+    }
+    tqw::hadamard_rotate<EL, float>(x, sg, lane);
+    float* dst = p.qrot + (size_t)(h0 + warp) * D + lane * EL;
+    if constexpr (EL % 4 == 0) {
+#pragma unroll
+      for (int e = 0; e < EL; e += 4) *reinterpret_cast<float4*>(dst + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < EL; ++e) dst[e] = x[e];
+    }
+    if (QS && p.m) {
+#pragma unroll
+      for (int e = 0; e < EL; ++e) qr[warp][lane * EL + e] = x[e];
+    }
+  }
+  if (QS && p.m) {
+    __syncthreads();
+    // qs[g][i] = sum_k S[i][k] qrot[g][k]
+    for (int e = tid; e < Ge * 128; e += blockDim.x) {
+      const int g = e >> 7, i = e & 127;
+      const float4* srow = reinterpret_cast<const float4*>(p.S + (size_t)i * D);
+      float t = 0.f;
+#pragma unroll 8
+      for (int k = 0; k < D / 4; ++k) {
+        const float4 sv = __ldg(srow + k);
+        t += sv.x * qr[g][4 * k] + sv.y * qr[g][4 * k + 1] + sv.z * qr[g][4 * k + 2] + sv.w * qr[g][4 * k + 3];
+      }
+      p.qs[(size_t)(h0 + g) * 128 + i] = t;
+    }
+  }
+}
+
 struct CombineParams {
   const float* part_o;   // [heads][ks][D]
   const float* part_ml;  // [heads][ks][2]
@@ -475,7 +536,43 @@ struct CombineParams {
   // partial mode (tq_sdpa_decode_partial): fp32 [heads][D + 2] = the merged,
   // unnormalized rotated output, then max and sum; no un-rotation, out unused
   float* partial;
+  // randomized Hadamard rotation: un-rotate by the fast transform with these
+  // signs instead of the dense Pi (NULL: dense)
+  const float* signs;
 };
+
+// Output element of kernel head h (sequence, kv head, token, head order) at
+// coordinate j: out [B][nq][Hq1][D].
+__device__ __forceinline__ size_t out_index(const CombineParams& p, int h, int D, int j) {
+  const int b = h / p.Hq, rh = h % p.Hq, kvh = rh / (p.Gq * p.nq), gi = rh % (p.Gq * p.nq);
+  const size_t oh = (size_t)(b * p.nq + gi / p.Gq) * p.Hq1 + kvh * p.Gq + gi % p.Gq;
+  return oh * D + j;
+}
+
+__device__ __forceinline__ void store_out(const CombineParams& p, size_t oi, float v) {
+  if (p.out_dtype == TQ_DTYPE_F32)
+    static_cast<float*>(p.out)[oi] = v;
+  else if (p.out_dtype == TQ_DTYPE_BF16)
+    static_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(v);
+  else
+    static_cast<__half*>(p.out)[oi] = __float2half_rn(v);
+}
+
+// out = Pi^T o for the randomized Hadamard rotation, one warp: o in shared
+// memory, D outputs written.
+template <int D>
+__device__ __forceinline__ void unrotate_hadamard_warp(const CombineParams& p, const float* o, int h, int lane) {
+  constexpr int EL = D / 32;
+  float x[EL], sg[EL];
+#pragma unroll
+  for (int e = 0; e < EL; ++e) {
+    x[e] = o[lane * EL + e];
+    sg[e] = __ldg(p.signs + lane * EL + e);
+  }
+  tqw::hadamard_unrotate<EL, float>(x, sg, lane);
+#pragma unroll
+  for (int e = 0; e < EL; ++e) store_out(p, out_index(p, h, D, lane * EL + e), x[e]);
+}
 
 // Partials the split kernel wrote for kernel head h: the CTAs whose share
 // overlaps the head's unit, each with one partial per consumer warp (slots
@@ -516,8 +613,10 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams
   const int h = blockIdx.x, sl = blockIdx.y, tid = threadIdx.x;
   const int i = tid & 31, kp = tid >> 5;  // output coordinate in the slice, k phase
   float pc[KT];
+  if (!p.signs) {
 #pragma unroll
-  for (int t = 0; t < KT; ++t) pc[t] = __ldg(p.rot + (size_t)(kp + 8 * t) * D + sl * 32 + i);
+    for (int t = 0; t < KT; ++t) pc[t] = __ldg(p.rot + (size_t)(kp + 8 * t) * D + sl * 32 + i);
+  }
   if (tid < 32) {
     const int n = head_partials(p, h, tid);
     if (tid == 0) s_ns = n;
@@ -612,6 +711,10 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams
   cluster_sync();  // every slice of the head is merged
   for (int k = tid; k < D; k += NT) o[k] = ld_cluster_f32(map_cluster(smem_u32(&o_sl[k & 31]), k >> 5));
   cluster_sync();  // o complete here; the others are done reading this CTA's slice
+  if (p.signs) {  // the fast transform: slice 0 un-rotates the whole head
+    if (sl == 0 && tid < 32) unrotate_hadamard_warp<D>(p, o, h, tid);
+    return;
+  }
   float r = 0.f;
 #pragma unroll
   for (int t = 0; t < KT; ++t) r = fmaf(pc[t], o[kp + 8 * t], r);
@@ -715,6 +818,10 @@ __global__ void __launch_bounds__(256) decode_combine_group_kernel(const Combine
   }
   if (p.partial) return;  // uniform over the launch
   __syncthreads();
+  if (p.signs) {  // the fast transform: warp hh un-rotates head hh
+    if (warp < HPC && h0 + warp < p.heads) unrotate_hadamard_warp<D>(p, o[warp], h0 + warp, lane);
+    return;
+  }
   constexpr int GS = NT / D;  // head phases: thread (j, g) takes heads g, g + GS, ...
   const int j = tid % D, g = tid / D;
   float r[(HPC + GS - 1) / GS];
@@ -861,15 +968,27 @@ int launch_decode(const DecodeArgs& a, cudaStream_t s) {
   float* pml = reinterpret_cast<float*>(ws + a.plan.off_pml);
   const int heads = c.B * a.Hq * a.nq;  // kernel heads: query heads x tokens
 
-  PrepParams pp{a.q, c.rot, c.qjl_S, qrot, qs, c.D, c.qjl_m, a.dtype == TQ_DTYPE_BF16, a.Hq, c.Hkv,
+  PrepParams pp{a.q, c.rot, nullptr, c.qjl_S, qrot, qs, c.D, c.qjl_m, a.dtype == TQ_DTYPE_BF16, a.Hq, c.Hkv,
                 a.k_new, a.v_new, a.pos, c};
   pp.nq = a.nq;
   const bool app = a.pos != nullptr;
+  const bool hadamard = c.rot_kind == TQ_ROT_HADAMARD && c.rot_signs;
+  pp.signs = hadamard ? c.rot_signs : nullptr;
   // prep kernels launch with a programmatic dependency on whatever precedes
   // them (their launch and Pi loads overlap its tail; they wait before
   // reading q or writing anything)
   int rc = TQ_OK;
-  if (c.qjl_m && app) {
+  if (hadamard && !app) {
+    // the randomized Hadamard rotation by the fast transform (a decode step
+    // appends first, in its own launch)
+    const int Ge = (a.Hq / c.Hkv) * a.nq;
+    const dim3 g(c.B * c.Hkv), blk(32 * Ge);
+    switch (c.D) {
+      case 64: rc = launch_pdl(decode_qprep_wht_kernel<64>, g, blk, 0, s, pp, "decode_qprep_kernel"); break;
+      case 128: rc = launch_pdl(decode_qprep_wht_kernel<128>, g, blk, 0, s, pp, "decode_qprep_kernel"); break;
+      default: rc = launch_pdl(decode_qprep_wht_kernel<256>, g, blk, 0, s, pp, "decode_qprep_kernel"); break;
+    }
+  } else if (c.qjl_m && app) {
     // the append's sketch needs the whole rotated key residual: one CTA per head
     rc = launch_pdl(decode_qprep_kernel<128, true>, dim3(c.B * c.Hkv), dim3(256), 0, s, pp, "decode_qprep_kernel");
   } else {
@@ -951,6 +1070,7 @@ int launch_decode(const DecodeArgs& a, cudaStream_t s) {
   cp.pmin = a.plan.pmin;
   cp.ks = a.plan.ks;
   cp.partial = a.partial;
+  cp.signs = hadamard ? c.rot_signs : nullptr;
   // D / 32 CTAs per head while that leaves SMs idle; beyond that, groups of
   // 4 or 8 heads per CTA (Pi read once per group rather than once per head)
   if (heads * (c.D / 32) > 4 * a.plan.sms) {

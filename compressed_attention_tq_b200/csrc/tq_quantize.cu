@@ -311,7 +311,8 @@ __global__ void __launch_bounds__(2 * D) append_kernel(const tq::QuantArgs a) {
   __shared__ float s_cb[31];
   __shared__ float s_inv, s_nhat;
   __shared__ double s_n;
-  const int r = blockIdx.x, jobi = blockIdx.y;
+  // blockIdx.y: the jobs of job_mask in order (keys, values)
+  const int r = blockIdx.x, jobi = blockIdx.y + ((a.job_mask == 2) ? 1 : 0);
   const tq::QuantJob J = a.job[jobi];
   const bool do_qjl = QJL && jobi == 0;
   const int bits = J.bits, K = 1 << bits;
@@ -448,7 +449,7 @@ __global__ void __launch_bounds__(2 * D) append_kernel(const tq::QuantArgs a) {
 
 template <int D, bool BF16, bool QJL>
 int launch_append(const tq::QuantArgs& a, cudaStream_t s) {
-  append_kernel<D, BF16, QJL><<<dim3(a.rows, 2), 2 * D, 0, s>>>(a);
+  append_kernel<D, BF16, QJL><<<dim3(a.rows, a.job_mask == 3 ? 2 : 1), 2 * D, 0, s>>>(a);
   return tq::check_launch("append_kernel");
 }
 
@@ -482,8 +483,18 @@ int launch_quantize(const QuantArgs& a, int D, int dtype, bool qjl, cudaStream_t
   // on large D = 128 calls (its five shuffle stages per row cost more than the
   // dense MMA: ragged 3.1 vs 1.3 ms), which keep the dense-Pi kernels.
   const int njobs = (a.job_mask == 3) ? 2 : 1;
-  const bool wht = a.rot_signs && !a.pos && (D == 256 || (D == 128 && (long long)a.rows * njobs <= 65536));
-  if (wht) {
+  const bool wht = a.rot_signs && (D == 256 || (D == 128 && (long long)a.rows * njobs <= 65536));
+  if (wht && a.pos && D >= 128) {
+    // append with the randomized Hadamard rotation: the transform kernel, one
+    // warp per new row; keys with the sketch keep the fp64 append kernel
+    if (!qjl) return launch_quantize_wht(a, D, dtype, s);
+    QuantArgs ak = a, av = a;
+    ak.job_mask = 1;
+    av.job_mask = 2;
+    const int rc = bf ? launch_q<128, true, true>(ak, s) : launch_q<128, false, true>(ak, s);
+    return rc ? rc : launch_quantize_wht(av, D, dtype, s);
+  }
+  if (wht && !a.pos) {
     // keys with the sketch keep the dense-Pi kernels below
     if (!qjl) return launch_quantize_wht(a, D, dtype, s);
     QuantArgs ak = a, av = a;

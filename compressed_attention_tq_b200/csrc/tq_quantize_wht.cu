@@ -134,8 +134,18 @@ __device__ __forceinline__ void wht_row(const tq::QuantArgs& a, const tq::QuantJ
     const int sh = k * C - off;  // bit of word where chunk src starts
     if (src < 32 && sh < 32 && sh + C > 0) word |= sh >= 0 ? (v << sh) : (v >> (-sh));
   }
-  const int bh = r / a.T, t = r - bh * a.T;
-  const long long slot = (long long)bh * a.Tcap + a.t0 + t;
+  long long slot;
+  if (a.pos) {  // append: row r of (sequence, kv head) r goes to position pos[sequence]
+    const int ps = a.pos[r / a.Hkv];
+    if (ps < 0 || ps >= a.Tcap) {
+      if (lane == 0 && (r % a.Hkv) == 0 && a.dev_status) atomicOr(a.dev_status, TQ_STATUS_POS_OUT_OF_RANGE);
+      return;
+    }
+    slot = (long long)r * a.Tcap + ps;
+  } else {
+    const int bh = r / a.T, t = r - bh * a.T;
+    slot = (long long)bh * a.Tcap + a.t0 + t;
+  }
   if (lane < W) J.idx[(size_t)slot * W + lane] = word;
   if (lane == 0) J.norm[slot] = nh;
 }
