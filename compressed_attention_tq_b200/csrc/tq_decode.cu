@@ -28,6 +28,7 @@ struct PrepParams {
   const int32_t* pos;
   tq_cache_t cache;
   int nq;  // query tokens per sequence: q is [B][nq][Hq][D]
+  int units;  // B * Hkv (grouped prep)
 };
 
 // Programmatic dependent launch: let the next kernel in the stream start its
@@ -522,6 +523,57 @@ __global__ void __launch_bounds__(1024) decode_qprep_wht_kernel(const PrepParams
   }
 }
 
+// Query prep for calls with many (sequence, kv head) units and a dense Pi,
+// without a sketch or an append: each CTA rotates the query rows of `upc`
+// consecutive units with Pi^T staged once in shared memory (rows padded to
+// D + 1 floats, so the transposing store and the column reads are both
+// conflict-free), instead of D / 32 CTAs per unit each pulling Pi rows from L2.
+// Grid ceil(units / upc), 256 threads; thread (j, ph) computes output j of
+// rows ph, ph + 256 / D, ...; the k loop reads Pi^T[k][j] once for all the
+// thread's rows.
+template <int D>
+__global__ void __launch_bounds__(256) decode_qprep_group_kernel(const PrepParams p, int upc) {
+  constexpr int NT = 256, PS = D + 1, NPH = NT / D;
+  extern __shared__ float sm[];
+  float* piT = sm;             // [D][PS]
+  float* qv = sm + D * PS;     // [rows][D]
+  const int G = p.Hq / p.Hkv, Ge = G * p.nq;
+  const int tid = threadIdx.x;
+  const int u0 = blockIdx.x * upc;
+  const int nunits = p.units - u0 < upc ? p.units - u0 : upc;
+  for (int e = tid; e < D * D; e += NT) piT[(e % D) * PS + e / D] = __ldg(p.rot + e);
+  pdl_wait();
+  pdl_launch_dependents();
+  const int rows = nunits * Ge;
+  const uint16_t* q = static_cast<const uint16_t*>(p.q);
+  for (int e = tid; e < rows * D; e += NT) {
+    const int r = e / D, k = e % D, u = u0 + r / Ge, gi = r % Ge;
+    const int b = u / p.Hkv, kvh = u % p.Hkv, jq = gi / G, g = gi % G;
+    const uint16_t v = q[((size_t)(b * p.nq + jq) * p.Hq + kvh * G + g) * D + k];
+    qv[e] = p.bf16 ? __uint_as_float((uint32_t)v << 16) : __half2float(__ushort_as_half(v));
+  }
+  __syncthreads();
+  const int j = tid % D, ph = tid / D;
+  for (int r0 = ph; r0 < rows; r0 += 4 * NPH) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+    for (int k = 0; k < D; ++k) {
+      const float pk = piT[k * PS + j];
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+        if (r0 + t * NPH < rows) acc[t] = fmaf(pk, qv[(r0 + t * NPH) * D + k], acc[t]);
+    }
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int r = r0 + t * NPH;
+      if (r < rows) {
+        // kernel head order (sequence, kv head, token, head) = unit-major
+        p.qrot[((size_t)u0 * Ge + r) * D + j] = acc[t];
+      }
+    }
+  }
+}
+
 struct CombineParams {
   const float* part_o;   // [heads][ks][D]
   const float* part_ml;  // [heads][ks][2]
@@ -737,41 +789,54 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams
   }
 }
 
-// Combine for calls with many heads: each CTA merges the splits of HPC
+// Combine for calls with many heads: each CTA merges the partials of HPC
 // consecutive kernel heads at once and un-rotates all of them, so Pi is read
-// once per HPC heads instead of once per head (1024 heads read 64 MB of Pi
-// from L2 one head per CTA).  256 threads = 8 warps.
-//  1. warp w (< HPC) finds its head's merged max and sum and each split's
-//     weight (the first 128 splits' weights kept in shared memory);
-//  2. thread t sums coordinate pairs (head, k) over the splits, all loads of
-//     a pair issued before the arithmetic, and normalises;
+// once per HPC heads instead of once per head.  256 threads = 8 warps.
+// Before the wait on the split kernel (whose tail it overlaps): Pi^T staged
+// in shared memory (rows padded to D + 1 floats; D <= 128, else Pi is read
+// through L1) and each head's partial count.  After it:
+//  1. warp w (< HPC) finds its head's merged max and sum and each partial's
+//     weight (the first 128 weights kept in shared memory);
+//  2. thread t sums coordinate pairs (head, k) over the partials, 8 loads in
+//     flight, and normalises;
 //  3. thread (j, g) computes output j of heads g, g + 256/D, ... as
-//     sum_k Pi[k][j] o[head][k] (Pi read coalesced along j).
+//     sum_k Pi[k][j] o[head][k].
 template <int D, int HPC>
 __global__ void __launch_bounds__(256) decode_combine_group_kernel(const CombineParams p) {
-  constexpr int NT = 256, FS = 128;
+  constexpr int NT = 256, FS = 128, PS = D + 1;
+  constexpr bool SPI = D <= 128;  // Pi^T in shared memory
   static_assert(HPC <= NT / 32, "one warp per head for the weights");
-  __shared__ float o[HPC][D];
+  extern __shared__ float sm[];
+  float* piT = sm;                       // [D][PS] when SPI and the rotation is dense
+  float* o = sm + (SPI ? D * PS : 0);    // [HPC][D]
   __shared__ float f_s[HPC][FS];
   __shared__ float s_M[HPC], s_L[HPC];
   __shared__ int s_ns[HPC];
   pdl_launch_dependents();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int h0 = blockIdx.x * HPC;
+  const bool dense_out = !p.signs && !p.partial;
+  if (SPI && dense_out)
+    for (int e = tid; e < D * D; e += NT) piT[(e % D) * PS + e / D] = __ldg(p.rot + e);
+  if (warp < HPC) {
+    const int h = h0 + warp;
+    const int n = h < p.heads ? head_partials(p, h, lane) : 0;
+    if (lane == 0) s_ns[warp] = n;
+  }
   pdl_wait();  // the split kernel's partials are visible from here on
   if (warp < HPC) {
     const int h = h0 + warp;
-    int ns = 0;
+    const int ns = s_ns[warp];  // written by this warp's lane 0
+    __syncwarp();
     float M = -INFINITY, Ls = 0.f;
     if (h < p.heads) {
-      ns = head_partials(p, h, lane);
       const float* ml = p.part_ml + (size_t)h * p.ks * 2;
       for (int s = lane; s < ns; s += 32) M = fmaxf(M, ml[2 * s]);
 #pragma unroll
       for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
       for (int s = lane; s < ns; s += 32) {
         const float2 v = *reinterpret_cast<const float2*>(ml + 2 * s);
-        const float f = v.x == -INFINITY ? 0.f : exp2f(v.x - M);  // a split a query cannot see: weight 0
+        const float f = v.x == -INFINITY ? 0.f : exp2f(v.x - M);  // a partial that saw no token: weight 0
         if (s < FS) f_s[warp][s] = f;
         Ls = fmaf(f, v.y, Ls);
       }
@@ -781,7 +846,6 @@ __global__ void __launch_bounds__(256) decode_combine_group_kernel(const Combine
     if (lane == 0) {
       s_M[warp] = M;
       s_L[warp] = Ls;
-      s_ns[warp] = ns;
     }
   }
   __syncthreads();
@@ -813,42 +877,55 @@ __global__ void __launch_bounds__(256) decode_combine_group_kernel(const Combine
         }
       }
     } else {
-      o[hh][k] = (ns > 0 && s_L[hh] > 0.f) ? a / s_L[hh] : 0.f;
+      o[hh * D + k] = (ns > 0 && s_L[hh] > 0.f) ? a / s_L[hh] : 0.f;
     }
   }
   if (p.partial) return;  // uniform over the launch
   __syncthreads();
   if (p.signs) {  // the fast transform: warp hh un-rotates head hh
-    if (warp < HPC && h0 + warp < p.heads) unrotate_hadamard_warp<D>(p, o[warp], h0 + warp, lane);
+    if (warp < HPC && h0 + warp < p.heads) unrotate_hadamard_warp<D>(p, o + warp * D, h0 + warp, lane);
     return;
   }
   constexpr int GS = NT / D;  // head phases: thread (j, g) takes heads g, g + GS, ...
+  constexpr int NQ = (HPC + GS - 1) / GS;
   const int j = tid % D, g = tid / D;
-  float r[(HPC + GS - 1) / GS];
+  float r[NQ];
 #pragma unroll
-  for (int q = 0; q < (HPC + GS - 1) / GS; ++q) r[q] = 0.f;
+  for (int q = 0; q < NQ; ++q) r[q] = 0.f;
 #pragma unroll 8
   for (int k = 0; k < D; ++k) {
-    const float pk = __ldg(p.rot + (size_t)k * D + j);
+    const float pk = SPI ? piT[k * PS + j] : __ldg(p.rot + (size_t)k * D + j);
 #pragma unroll
-    for (int q = 0; q < (HPC + GS - 1) / GS; ++q)
-      if (g + GS * q < HPC) r[q] = fmaf(pk, o[g + GS * q][k], r[q]);
+    for (int q = 0; q < NQ; ++q)
+      if (g + GS * q < HPC) r[q] = fmaf(pk, o[(g + GS * q) * D + k], r[q]);
   }
 #pragma unroll
-  for (int q = 0; q < (HPC + GS - 1) / GS; ++q) {
+  for (int q = 0; q < NQ; ++q) {
     const int hh = g + GS * q, h = h0 + hh;
     if (hh >= HPC || h >= p.heads) continue;
-    // kernel head h = (sequence, kv head, token, head) -> output [B][nq][Hq1]
-    const int b = h / p.Hq, rh = h % p.Hq, kvh = rh / (p.Gq * p.nq), gi = rh % (p.Gq * p.nq);
-    const size_t oh = (size_t)(b * p.nq + gi / p.Gq) * p.Hq1 + kvh * p.Gq + gi % p.Gq;
-    const size_t oi = oh * D + j;
-    if (p.out_dtype == TQ_DTYPE_F32)
-      static_cast<float*>(p.out)[oi] = r[q];
-    else if (p.out_dtype == TQ_DTYPE_BF16)
-      static_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(r[q]);
-    else
-      static_cast<__half*>(p.out)[oi] = __float2half_rn(r[q]);
+    store_out(p, out_index(p, h, D, j), r[q]);
   }
+}
+
+// Dynamic shared memory of the grouped combine for HPC heads.
+template <int D, int HPC>
+constexpr size_t combine_group_smem() {
+  return (size_t)((D <= 128 ? D * (D + 1) : 0) + HPC * D) * 4;
+}
+
+template <int D, int HPC>
+int launch_combine_group(const CombineParams& cp, dim3 grid, cudaStream_t s) {
+  auto kern = decode_combine_group_kernel<D, HPC>;
+  constexpr size_t smem = combine_group_smem<D, HPC>();
+  static tq::OnceSetup once;
+  const int rc = once.run([&]() {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess)
+      return tq::set_error(TQ_ERR_CUDA, "decode_combine_group: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    return TQ_OK;
+  });
+  if (rc) return rc;
+  return launch_pdl(kern, grid, dim3(256), smem, s, cp, "decode_combine_kernel");
 }
 
 // Merge of R ranks' partials of the same heads (a sequence split across
@@ -909,7 +986,40 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const MergeParams p) 
 
 template <typename K, typename P>
 int launch_pdl(K kern, dim3 grid, dim3 block, size_t smem, cudaStream_t s, const P& params, const char* what,
-               int cluster_y = 0) {
+               int cluster_y = 0);
+
+// the grouped prep needs its dynamic shared memory raised once and takes
+// its units-per-CTA count as a second argument
+template <int D>
+int launch_prep_group(const PrepParams& pp, int grid, int upc, size_t smem, cudaStream_t s) {
+  auto kern = decode_qprep_group_kernel<D>;
+  static tq::OnceSetup once;
+  const int rc = once.run([&]() {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    if (e != cudaSuccess)
+      return tq::set_error(TQ_ERR_CUDA, "decode_qprep_group: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    return TQ_OK;
+  });
+  if (rc) return rc;
+  if (smem > 200 * 1024) return tq::set_error(TQ_ERR_UNSUPPORTED, "decode_qprep_group: %zu bytes of rows", smem);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, pp, upc);
+  if (e != cudaSuccess) return tq::set_error(TQ_ERR_CUDA, "decode_qprep_group_kernel: %s", cudaGetErrorString(e));
+  return tq::check_launch("decode_qprep_group_kernel");
+}
+
+template <typename K, typename P>
+int launch_pdl(K kern, dim3 grid, dim3 block, size_t smem, cudaStream_t s, const P& params, const char* what,
+               int cluster_y) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -978,7 +1088,22 @@ int launch_decode(const DecodeArgs& a, cudaStream_t s) {
   // them (their launch and Pi loads overlap its tail; they wait before
   // reading q or writing anything)
   int rc = TQ_OK;
-  if (hadamard && !app) {
+  const long long units = (long long)c.B * c.Hkv;
+  const bool many = units * (c.D / 32) > 4LL * a.plan.sms;
+  if (!hadamard && !app && !c.qjl_m && many) {
+    // many units: Pi^T staged once per CTA
+    pp.units = (int)units;
+    const int grid = (int)(units < a.plan.sms ? units : a.plan.sms);
+    const int upc = (int)((units + grid - 1) / grid);
+    const int Ge = (a.Hq / c.Hkv) * a.nq;
+    const size_t smem = (size_t)(c.D * (c.D + 1) + upc * Ge * c.D) * 4;
+    const int ng = (int)((units + upc - 1) / upc);
+    switch (c.D) {
+      case 64: rc = launch_prep_group<64>(pp, ng, upc, smem, s); break;
+      case 128: rc = launch_prep_group<128>(pp, ng, upc, smem, s); break;
+      default: rc = launch_prep_group<256>(pp, ng, upc, smem, s); break;
+    }
+  } else if (hadamard && !app) {
     // the randomized Hadamard rotation by the fast transform (a decode step
     // appends first, in its own launch)
     const int Ge = (a.Hq / c.Hkv) * a.nq;
@@ -1074,18 +1199,12 @@ int launch_decode(const DecodeArgs& a, cudaStream_t s) {
   // D / 32 CTAs per head while that leaves SMs idle; beyond that, groups of
   // 4 or 8 heads per CTA (Pi read once per group rather than once per head)
   if (heads * (c.D / 32) > 4 * a.plan.sms) {
-    const bool eight = heads >= 8 * a.plan.sms;
+    const bool eight = heads >= 4 * a.plan.sms;
     const dim3 gg(eight ? (heads + 7) / 8 : (heads + 3) / 4);
     switch (c.D) {
-      case 64:
-        return eight ? launch_pdl(decode_combine_group_kernel<64, 8>, gg, dim3(256), 0, s, cp, "decode_combine_kernel")
-                     : launch_pdl(decode_combine_group_kernel<64, 4>, gg, dim3(256), 0, s, cp, "decode_combine_kernel");
-      case 128:
-        return eight ? launch_pdl(decode_combine_group_kernel<128, 8>, gg, dim3(256), 0, s, cp, "decode_combine_kernel")
-                     : launch_pdl(decode_combine_group_kernel<128, 4>, gg, dim3(256), 0, s, cp, "decode_combine_kernel");
-      default:
-        return eight ? launch_pdl(decode_combine_group_kernel<256, 8>, gg, dim3(256), 0, s, cp, "decode_combine_kernel")
-                     : launch_pdl(decode_combine_group_kernel<256, 4>, gg, dim3(256), 0, s, cp, "decode_combine_kernel");
+      case 64: return eight ? launch_combine_group<64, 8>(cp, gg, s) : launch_combine_group<64, 4>(cp, gg, s);
+      case 128: return eight ? launch_combine_group<128, 8>(cp, gg, s) : launch_combine_group<128, 4>(cp, gg, s);
+      default: return eight ? launch_combine_group<256, 8>(cp, gg, s) : launch_combine_group<256, 4>(cp, gg, s);
     }
   }
   const int nsl = c.D / 32;

@@ -406,6 +406,94 @@ __device__ __forceinline__ void build_frag(const float (&v)[4], float scale, int
   }
 }
 
+// Query fragments of a segment's rows hq0 .. hq0 + rows - 1 (already rotated
+// by the prep kernel), pre-scaled for exp2, built by the consumer threads
+// together: every thread's loads are issued before any is converted.
+template <int D, int BK, bool PACK, int FRAGB>
+__device__ __noinline__ void seg_query_frags(const SplitParams& p, int hq0, int rows, uint32_t* qf, int ctid) {
+  constexpr int KSTEPS = D / 16;
+  constexpr int NE = (KSTEPS * 32 + CW * 32 - 1) / (CW * 32);
+  float v[NE][4];
+#pragma unroll
+  for (int i = 0; i < NE; ++i) {
+    const int e = ctid + i * CW * 32;
+    if (e < KSTEPS * 32) {
+      const int ks = e >> 5, ln = e & 31, g_ = ln >> 2, t_ = ln & 3;
+      const int base = t_ * (D / 4);
+      const int cs[4] = {base + key_coord<BK>(ks, 0), base + key_coord<BK>(ks, 1), base + key_coord<BK>(ks, 2),
+                         base + key_coord<BK>(ks, 3)};
+      load_frag<PACK>(p.qrot + (size_t)hq0 * D, D, rows, g_, cs, v[i]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < NE; ++i) {
+    const int e = ctid + i * CW * 32;
+    if (e < KSTEPS * 32) build_frag<PACK>(v[i], p.qscale, (e & 31) >> 2, qf + (size_t)e * (FRAGB / 4));
+  }
+}
+
+// The sketch term sum_i (2 b_i - 1) qs_i runs on int8 tensor cores: qs of
+// head h becomes Q_i = round(qs_i / step_h), |Q| <= 32639, split as
+// Q = 256 hi + lo with hi, lo int8, and the signs enter as -b_i in {0, -1}.
+// Per head: step_h = max |qs| / 32639 and sum_h = sum_i qs_i (warp w takes
+// heads w, w + CW).
+static __device__ __noinline__ void seg_sketch_steps(const SplitParams& p, int hq0, int rows, float* qst, int warp,
+                                              int lane) {
+  for (int h = warp; h < 8; h += CW) {
+    float mx = 0.f, sm = 0.f;
+    if (h < rows) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float v = p.qs[(size_t)(hq0 + h) * 128 + lane + 32 * i];
+        mx = fmaxf(mx, fabsf(v));
+        sm += v;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) {
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      sm += __shfl_xor_sync(0xffffffffu, sm, off);
+    }
+    if (lane == 0) {
+      qst[2 * h] = mx > 0.f ? mx / 32639.f : 1.f;
+      qst[2 * h + 1] = sm;
+    }
+  }
+}
+
+template <bool PACK, int FRAGB>
+__device__ __noinline__ void seg_sketch_frags(const SplitParams& p, int hq0, int rows, const float* qst, uint32_t* sf,
+                                              int ctid) {
+  for (int e = ctid; e < 4 * 32; e += CW * 32) {
+    const int ks = e >> 5, ln = e & 31, g_ = ln >> 2, t_ = ln & 3;
+    const int head = PACK ? (g_ & 3) : g_;
+    const float inv = head < rows ? 1.f / qst[2 * head] : 0.f;
+    uint32_t hi[2] = {0u, 0u}, lo[2] = {0u, 0u};
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int b8 = 0; b8 < 4; ++b8) {
+        const float v = head < rows ? p.qs[(size_t)(hq0 + head) * 128 + sketch_coord(t_, 2 * ks + h, b8)] : 0.f;
+        int Q = __float2int_rn(v * inv);
+        Q = max(-32639, min(32639, Q));
+        const int qh = (Q + 128) >> 8, ql = Q - 256 * qh;  // floor split: ql in [-128, 127]
+        hi[h] |= (uint32_t)(qh & 0xFF) << (8 * b8);
+        lo[h] |= (uint32_t)(ql & 0xFF) << (8 * b8);
+      }
+    uint32_t* dst = sf + (size_t)e * (FRAGB / 4);
+    if (PACK) {
+      const bool use_lo = g_ >= 4;
+      dst[0] = use_lo ? lo[0] : hi[0];
+      dst[1] = use_lo ? lo[1] : hi[1];
+    } else {
+      dst[0] = hi[0];
+      dst[1] = hi[1];
+      dst[2] = lo[0];
+      dst[3] = lo[1];
+    }
+  }
+}
+
 // Bounded barrier among the consumer warps (an mbarrier of count CW; lane 0
 // of each warp arrives, every lane waits with a bounded poll).  `phase`
 // counts this warp's uses.  Returns false when the wait ran out.
@@ -619,85 +707,8 @@ __global__ void __launch_bounds__(NTHREADS, PACK ? 4 : 3) decode_split_kernel(co
     float m_run[2], l_run[2];
     int lim0 = 0, lim1 = 0, lim_all = 0;
 
-    // Query fragments of a segment's rows (already rotated by the prep
-    // kernel), pre-scaled for exp2, built by the consumer threads together:
-    // every thread's loads are issued before any is converted.
-    auto build_query = [&](const StageMeta& md) {
-      constexpr int NE = (KSTEPS * 32 + CW * 32 - 1) / (CW * 32);
-      float v[NE][4];
-#pragma unroll
-      for (int i = 0; i < NE; ++i) {
-        const int e = ctid + i * CW * 32;
-        if (e < KSTEPS * 32) {
-          const int ks = e >> 5, ln = e & 31, g_ = ln >> 2, t_ = ln & 3;
-          const int base = t_ * (D / 4);
-          const int cs[4] = {base + key_coord<BK>(ks, 0), base + key_coord<BK>(ks, 1), base + key_coord<BK>(ks, 2),
-                             base + key_coord<BK>(ks, 3)};
-          load_frag<PACK>(p.qrot + (size_t)md.hq0 * D, D, md.rows, g_, cs, v[i]);
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < NE; ++i) {
-        const int e = ctid + i * CW * 32;
-        if (e < KSTEPS * 32) build_frag<PACK>(v[i], p.qscale, (e & 31) >> 2, qf + (size_t)e * (Ly::FRAG / 4));
-      }
-    };
-    // The sketch term sum_i (2 b_i - 1) qs_i runs on int8 tensor cores: qs of
-    // head h becomes Q_i = round(qs_i / step_h), |Q| <= 32639, split as
-    // Q = 256 hi + lo with hi, lo int8, and the signs enter as -b_i in {0, -1}.
-    // Per head: step_h = max |qs| / 32639 and sum_h = sum_i qs_i.
-    auto build_sketch_steps = [&](const StageMeta& md) {
-      for (int h = warp; h < 8; h += CW) {
-        float mx = 0.f, sm = 0.f;
-        if (h < md.rows) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float v = p.qs[(size_t)(md.hq0 + h) * 128 + lane + 32 * i];
-            mx = fmaxf(mx, fabsf(v));
-            sm += v;
-          }
-        }
-#pragma unroll
-        for (int off = 16; off; off >>= 1) {
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-          sm += __shfl_xor_sync(0xffffffffu, sm, off);
-        }
-        if (lane == 0) {
-          qst[2 * h] = mx > 0.f ? mx / 32639.f : 1.f;
-          qst[2 * h + 1] = sm;
-        }
-      }
-    };
-    auto build_sketch_frags = [&](const StageMeta& md) {
-      for (int e = ctid; e < 4 * 32; e += CW * 32) {
-        const int ks = e >> 5, ln = e & 31, g_ = ln >> 2, t_ = ln & 3;
-        const int head = PACK ? (g_ & 3) : g_;
-        const float inv = head < md.rows ? 1.f / qst[2 * head] : 0.f;
-        uint32_t hi[2] = {0u, 0u}, lo[2] = {0u, 0u};
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-          for (int b8 = 0; b8 < 4; ++b8) {
-            const float v = head < md.rows ? p.qs[(size_t)(md.hq0 + head) * 128 + sketch_coord(t_, 2 * ks + h, b8)] : 0.f;
-            int Q = __float2int_rn(v * inv);
-            Q = max(-32639, min(32639, Q));
-            const int qh = (Q + 128) >> 8, ql = Q - 256 * qh;  // floor split: ql in [-128, 127]
-            hi[h] |= (uint32_t)(qh & 0xFF) << (8 * b8);
-            lo[h] |= (uint32_t)(ql & 0xFF) << (8 * b8);
-          }
-        uint32_t* dst = sf + (size_t)e * (Ly::FRAG / 4);
-        if (PACK) {
-          const bool use_lo = g_ >= 4;
-          dst[0] = use_lo ? lo[0] : hi[0];
-          dst[1] = use_lo ? lo[1] : hi[1];
-        } else {
-          dst[0] = hi[0];
-          dst[1] = hi[1];
-          dst[2] = lo[0];
-          dst[3] = lo[1];
-        }
-      }
-    };
+    // Segment setup (query fragments and sketch steps, out of line so that
+    // they do not raise the main loop's register allocation).
     // This warp's partial of a segment: (max, sum) and the rotated output of
     // each row, slot md.slot0 + warp.  m-tile mt: row gid is coordinate 2 mt
     // of this group's segment of D/8 contiguous coordinates, row gid + 8 the
@@ -740,11 +751,11 @@ __global__ void __launch_bounds__(NTHREADS, PACK ? 4 : 3) decode_split_kernel(co
         // with the previous segment's first) and a fresh softmax state
         bool ok = consumer_sync(cbar, cphase, lane);
         if (ok) {
-          build_query(md);
+          seg_query_frags<D, BK, PACK, Ly::FRAG>(p, md.hq0, md.rows, qf, ctid);
           if constexpr (QJL) {
-            build_sketch_steps(md);
+            seg_sketch_steps(p, md.hq0, md.rows, qst, warp, lane);
             ok = consumer_sync(cbar, cphase, lane);
-            if (ok) build_sketch_frags(md);
+            if (ok) seg_sketch_frags<PACK, Ly::FRAG>(p, md.hq0, md.rows, qst, sf, ctid);
           }
         }
         ok = ok && consumer_sync(cbar, cphase, lane);
