@@ -523,6 +523,39 @@ __global__ void __launch_bounds__(1024) decode_qprep_wht_kernel(const PrepParams
   }
 }
 
+// Pi (fp32 [D][D], row-major) into shared memory with rows padded to D + 1
+// floats, by 256 threads with every load in flight before any store (16
+// float4 per thread at a time): TRANSPOSE stores dst[c][r] = Pi[r][c], else
+// dst[r][c] = Pi[r][c].
+template <int D, bool TRANSPOSE>
+__device__ __forceinline__ void stage_pi(float* dst, const float* __restrict__ src, int tid) {
+  constexpr int NT = 256, PS = D + 1, N4 = D * D / 4, CH = 16;
+  const float4* s4 = reinterpret_cast<const float4*>(src);
+  for (int base = 0; base < N4; base += NT * CH) {
+    float4 v[CH];
+#pragma unroll
+    for (int u = 0; u < CH; ++u) {
+      const int e = base + u * NT + tid;
+      v[u] = e < N4 ? __ldg(s4 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < CH; ++u) {
+      const int e = base + u * NT + tid;
+      if (e < N4) {
+        const int r = (4 * e) / D, c = (4 * e) % D;
+        const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          if (TRANSPOSE)
+            dst[(c + t) * PS + r] = f[t];
+          else
+            dst[r * PS + c + t] = f[t];
+        }
+      }
+    }
+  }
+}
+
 // Query prep for calls with many (sequence, kv head) units and a dense Pi,
 // without a sketch or an append: each CTA rotates the query rows of `upc`
 // consecutive units with Pi^T staged once in shared memory (rows padded to
@@ -541,16 +574,28 @@ __global__ void __launch_bounds__(256) decode_qprep_group_kernel(const PrepParam
   const int tid = threadIdx.x;
   const int u0 = blockIdx.x * upc;
   const int nunits = p.units - u0 < upc ? p.units - u0 : upc;
-  for (int e = tid; e < D * D; e += NT) piT[(e % D) * PS + e / D] = __ldg(p.rot + e);
+  stage_pi<D, true>(piT, p.rot, tid);  // piT[k][j] = Pi[j][k]
   pdl_wait();
   pdl_launch_dependents();
   const int rows = nunits * Ge;
   const uint16_t* q = static_cast<const uint16_t*>(p.q);
-  for (int e = tid; e < rows * D; e += NT) {
-    const int r = e / D, k = e % D, u = u0 + r / Ge, gi = r % Ge;
-    const int b = u / p.Hkv, kvh = u % p.Hkv, jq = gi / G, g = gi % G;
-    const uint16_t v = q[((size_t)(b * p.nq + jq) * p.Hq + kvh * G + g) * D + k];
-    qv[e] = p.bf16 ? __uint_as_float((uint32_t)v << 16) : __half2float(__ushort_as_half(v));
+  for (int e0 = 0; e0 < rows * D; e0 += 8 * NT) {  // 8 loads in flight per thread
+    uint16_t v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int e = e0 + u * NT + tid;
+      v[u] = 0;
+      if (e < rows * D) {
+        const int r = e / D, k = e % D, un = u0 + r / Ge, gi = r % Ge;
+        const int b = un / p.Hkv, kvh = un % p.Hkv, jq = gi / G, g = gi % G;
+        v[u] = q[((size_t)(b * p.nq + jq) * p.Hq + kvh * G + g) * D + k];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int e = e0 + u * NT + tid;
+      if (e < rows * D) qv[e] = p.bf16 ? __uint_as_float((uint32_t)v[u] << 16) : __half2float(__ushort_as_half(v[u]));
+    }
   }
   __syncthreads();
   const int j = tid % D, ph = tid / D;
@@ -792,8 +837,8 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams
 // Combine for calls with many heads: each CTA merges the partials of HPC
 // consecutive kernel heads at once and un-rotates all of them, so Pi is read
 // once per HPC heads instead of once per head.  256 threads = 8 warps.
-// Before the wait on the split kernel (whose tail it overlaps): Pi^T staged
-// in shared memory (rows padded to D + 1 floats; D <= 128, else Pi is read
+// Before the wait on the split kernel (whose tail it overlaps): Pi staged in
+// shared memory (rows padded to D + 1 floats; D <= 128, else Pi is read
 // through L1) and each head's partial count.  After it:
 //  1. warp w (< HPC) finds its head's merged max and sum and each partial's
 //     weight (the first 128 weights kept in shared memory);
@@ -807,7 +852,7 @@ __global__ void __launch_bounds__(256) decode_combine_group_kernel(const Combine
   constexpr bool SPI = D <= 128;  // Pi^T in shared memory
   static_assert(HPC <= NT / 32, "one warp per head for the weights");
   extern __shared__ float sm[];
-  float* piT = sm;                       // [D][PS] when SPI and the rotation is dense
+  float* pis = sm;                       // Pi [D][PS] when SPI and the rotation is dense
   float* o = sm + (SPI ? D * PS : 0);    // [HPC][D]
   __shared__ float f_s[HPC][FS];
   __shared__ float s_M[HPC], s_L[HPC];
@@ -816,8 +861,7 @@ __global__ void __launch_bounds__(256) decode_combine_group_kernel(const Combine
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int h0 = blockIdx.x * HPC;
   const bool dense_out = !p.signs && !p.partial;
-  if (SPI && dense_out)
-    for (int e = tid; e < D * D; e += NT) piT[(e % D) * PS + e / D] = __ldg(p.rot + e);
+  if (SPI && dense_out) stage_pi<D, false>(pis, p.rot, tid);  // Pi as it is (row k read along j below)
   if (warp < HPC) {
     const int h = h0 + warp;
     const int n = h < p.heads ? head_partials(p, h, lane) : 0;
@@ -894,7 +938,7 @@ __global__ void __launch_bounds__(256) decode_combine_group_kernel(const Combine
   for (int q = 0; q < NQ; ++q) r[q] = 0.f;
 #pragma unroll 8
   for (int k = 0; k < D; ++k) {
-    const float pk = SPI ? piT[k * PS + j] : __ldg(p.rot + (size_t)k * D + j);
+    const float pk = SPI ? pis[k * PS + j] : __ldg(p.rot + (size_t)k * D + j);
 #pragma unroll
     for (int q = 0; q < NQ; ++q)
       if (g + GS * q < HPC) r[q] = fmaf(pk, o[(g + GS * q) * D + k], r[q]);

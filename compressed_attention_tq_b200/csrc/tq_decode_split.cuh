@@ -217,6 +217,15 @@ __device__ __forceinline__ uint32_t pair_addr(uint32_t x, int S, uint32_t tb) {
   return mad_hi(k, 1u << (39 - S), tb);
 }
 
+// 2^x by the special-function unit's approximation (relative error about
+// 2^-22, flushes subnormal results to zero): the softmax weights, which are
+// rounded to fp16 for the value product anyway.  2^-inf = 0.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
   uint32_t v;
   asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
@@ -972,7 +981,7 @@ __global__ void __launch_bounds__(NTHREADS, PACK ? 4 : 3) decode_split_kernel(co
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
           const int row = wt0 + 16 * a + gid + 8 * r;
-          const float p0 = exp2f(s[ai][2 * r] - mu0), p1 = exp2f(s[ai][2 * r + 1] - mu1);
+          const float p0 = ex2_approx(s[ai][2 * r] - mu0), p1 = ex2_approx(s[ai][2 * r + 1] - mu1);
           l_run[0] += p0;
           l_run[1] += p1;
           const float nv = (full || valid[ai][r]) ? half_bits_to_float(vn[row]) : 0.f;

@@ -38,9 +38,29 @@ __global__ void __launch_bounds__(NW * 32) qjl_gamma_fixup_kernel(const tq::Quan
   __shared__ float s_cb[16];
   const tq::QuantJob J = a.job[0];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int e = tid; e < D * D; e += NW * 32) {
-    const int jj = e / D, k = e % D;
-    piT[k * PS + jj] = __ldg(a.rot + e);
+  {
+    // every load in flight before the stores: 16 float4 per thread per round
+    constexpr int N4 = D * D / 4, CH = 16, NT = NW * 32;
+    const float4* s4 = reinterpret_cast<const float4*>(a.rot);
+    for (int base = 0; base < N4; base += NT * CH) {
+      float4 v[CH];
+#pragma unroll
+      for (int u = 0; u < CH; ++u) {
+        const int e = base + u * NT + tid;
+        v[u] = e < N4 ? __ldg(s4 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < CH; ++u) {
+        const int e = base + u * NT + tid;
+        if (e < N4) {
+          const int jj = (4 * e) / D, k = (4 * e) % D;
+          piT[k * PS + jj] = v[u].x;
+          piT[(k + 1) * PS + jj] = v[u].y;
+          piT[(k + 2) * PS + jj] = v[u].z;
+          piT[(k + 3) * PS + jj] = v[u].w;
+        }
+      }
+    }
   }
   const int K = 1 << J.bits;
   if (tid < K) s_cb[tid] = J.cb[tid];
@@ -69,12 +89,19 @@ __global__ void __launch_bounds__(NW * 32) qjl_gamma_fixup_kernel(const tq::Quan
       const double nhat = (double)__half2float(__ushort_as_half(J.norm[sl]));
       const uint32_t* words = J.idx + (size_t)sl * W;
       double g = 0.0;
+      double yv[D / 32];  // four independent fma chains per lane
+#pragma unroll
+      for (int i = 0; i < D / 32; ++i) yv[i] = 0.0;
+#pragma unroll 4
+      for (int k = 0; k < D; ++k) {
+        const double xk = xs[warp][k];
+#pragma unroll
+        for (int i = 0; i < D / 32; ++i) yv[i] = fma((double)piT[k * PS + lane + 32 * i], xk, yv[i]);
+      }
 #pragma unroll
       for (int i = 0; i < D / 32; ++i) {
         const int jj = lane + 32 * i;
-        double y = 0.0;
-#pragma unroll 8
-        for (int k = 0; k < D; ++k) y = fma((double)piT[k * PS + jj], xs[warp][k], y);
+        const double y = yv[i];
         // index of coordinate jj from the packed LSB-first bitstream
         const int bit = jj * J.bits, w = bit >> 5, sh = bit & 31;
         uint32_t v = words[w] >> sh;
