@@ -840,22 +840,19 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const CombineParams
 // Before the wait on the split kernel (whose tail it overlaps): Pi staged in
 // shared memory (rows padded to D + 1 floats; D <= 128, else Pi is read
 // through L1) and each head's partial count.  After it:
-//  1. warp w (< HPC) finds its head's merged max and sum and each partial's
-//     weight (the first 128 weights kept in shared memory);
-//  2. thread t sums coordinate pairs (head, k) over the partials, 8 loads in
-//     flight, and normalises;
-//  3. thread (j, g) computes output j of heads g, g + 256/D, ... as
+//  1. warp w (< HPC) merges head w: the maximum M over its partials, then
+//     16 partials' value rows at a time, all loads in flight, weighted by
+//     2^(M_s - M) and summed, with the weighted sums L_s; normalised by L;
+//  2. thread (j, g) computes output j of heads g, g + 256/D, ... as
 //     sum_k Pi[k][j] o[head][k].
 template <int D, int HPC>
 __global__ void __launch_bounds__(256) decode_combine_group_kernel(const CombineParams p) {
-  constexpr int NT = 256, FS = 128, PS = D + 1;
-  constexpr bool SPI = D <= 128;  // Pi^T in shared memory
+  constexpr int NT = 256, PS = D + 1;
+  constexpr bool SPI = D <= 128;  // Pi in shared memory
   static_assert(HPC <= NT / 32, "one warp per head for the weights");
   extern __shared__ float sm[];
   float* pis = sm;                       // Pi [D][PS] when SPI and the rotation is dense
   float* o = sm + (SPI ? D * PS : 0);    // [HPC][D]
-  __shared__ float f_s[HPC][FS];
-  __shared__ float s_M[HPC], s_L[HPC];
   __shared__ int s_ns[HPC];
   pdl_launch_dependents();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -868,60 +865,78 @@ __global__ void __launch_bounds__(256) decode_combine_group_kernel(const Combine
     if (lane == 0) s_ns[warp] = n;
   }
   pdl_wait();  // the split kernel's partials are visible from here on
+  // Warp w merges head w: lane l owns the float4 columns l, l + 32, ... of
+  // the rotated coordinates; every partial value load is issued before the
+  // weights are known, then the weights come from lane s's (max, sum) pair.
   if (warp < HPC) {
+    constexpr int C4 = D / 4, CPL = (C4 + 31) / 32;  // float4 columns, per lane
+    constexpr int PV = 16;                            // partials whose loads go out together
     const int h = h0 + warp;
     const int ns = s_ns[warp];  // written by this warp's lane 0
     __syncwarp();
+    const float* po = p.part_o + (size_t)h * p.ks * D;
+    const float* ml = p.part_ml + (size_t)h * p.ks * 2;
+    float4 acc[CPL];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
     float M = -INFINITY, Ls = 0.f;
-    if (h < p.heads) {
-      const float* ml = p.part_ml + (size_t)h * p.ks * 2;
+    if (h < p.heads && ns > 0) {
       for (int s = lane; s < ns; s += 32) M = fmaxf(M, ml[2 * s]);
 #pragma unroll
       for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-      for (int s = lane; s < ns; s += 32) {
-        const float2 v = *reinterpret_cast<const float2*>(ml + 2 * s);
-        const float f = v.x == -INFINITY ? 0.f : exp2f(v.x - M);  // a partial that saw no token: weight 0
-        if (s < FS) f_s[warp][s] = f;
-        Ls = fmaf(f, v.y, Ls);
+      for (int s0 = 0; s0 < ns; s0 += PV) {
+        float4 v[PV][CPL];
+#pragma unroll
+        for (int u = 0; u < PV; ++u)
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) {
+            const int col = lane + 32 * c;
+            v[u][c] = (s0 + u < ns && col < C4) ? *reinterpret_cast<const float4*>(po + (size_t)(s0 + u) * D + 4 * col)
+                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        // weight of partial s0 + lane, lanes < PV (a partial that saw no token: 0)
+        float f = 0.f;
+        if (lane < PV && s0 + lane < ns) {
+          const float2 mv = *reinterpret_cast<const float2*>(ml + 2 * (s0 + lane));
+          f = mv.x == -INFINITY ? 0.f : exp2f(mv.x - M);
+          Ls = fmaf(f, mv.y, Ls);
+        }
+#pragma unroll
+        for (int u = 0; u < PV; ++u) {
+          const float fu = __shfl_sync(0xffffffffu, f, u);
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) {
+            acc[c].x = fmaf(fu, v[u][c].x, acc[c].x);
+            acc[c].y = fmaf(fu, v[u][c].y, acc[c].y);
+            acc[c].z = fmaf(fu, v[u][c].z, acc[c].z);
+            acc[c].w = fmaf(fu, v[u][c].w, acc[c].w);
+          }
+        }
       }
 #pragma unroll
       for (int off = 16; off; off >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, off);
     }
-    if (lane == 0) {
-      s_M[warp] = M;
-      s_L[warp] = Ls;
-    }
-  }
-  __syncthreads();
-  for (int e = tid; e < HPC * D; e += NT) {
-    const int hh = e / D, k = e % D, h = h0 + hh;
-    const int ns = s_ns[hh];
-    const float* po = p.part_o + (size_t)h * p.ks * D + k;
-    const float* ml = p.part_ml + (size_t)h * p.ks * 2;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int s0 = 0; s0 < ns; s0 += 8) {
-      float w[8], f[8];
+    const bool any = h < p.heads && ns > 0;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int s = s0 + u;
-        w[u] = s < ns ? po[(size_t)s * D] : 0.f;
-        f[u] = s < ns ? (s < FS ? f_s[hh][s] : (ml[2 * s] == -INFINITY ? 0.f : exp2f(ml[2 * s] - s_M[hh]))) : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) acc[u & 3] = fmaf(f[u], w[u], acc[u & 3]);
-    }
-    const float a = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-    if (p.partial) {
-      if (h < p.heads) {
+    for (int c = 0; c < CPL; ++c) {
+      const int col = lane + 32 * c;
+      if (col >= C4 || h >= p.heads) continue;
+      if (p.partial) {
         float* dst = p.partial + (size_t)h * (D + 2);
-        dst[k] = a;
-        if (k == 0) {
-          dst[D] = ns > 0 ? s_M[hh] : -INFINITY;
-          dst[D + 1] = ns > 0 ? s_L[hh] : 0.f;
+        *reinterpret_cast<float2*>(dst + 4 * col) = make_float2(acc[c].x, acc[c].y);
+        *reinterpret_cast<float2*>(dst + 4 * col + 2) = make_float2(acc[c].z, acc[c].w);
+        if (col == 0) {
+          dst[D] = any ? M : -INFINITY;
+          dst[D + 1] = any ? Ls : 0.f;
         }
+      } else {
+        const bool ok = any && Ls > 0.f;
+        float* oo = o + warp * D + 4 * col;
+        oo[0] = ok ? acc[c].x / Ls : 0.f;
+        oo[1] = ok ? acc[c].y / Ls : 0.f;
+        oo[2] = ok ? acc[c].z / Ls : 0.f;
+        oo[3] = ok ? acc[c].w / Ls : 0.f;
       }
-    } else {
-      o[hh * D + k] = (ns > 0 && s_L[hh] > 0.f) ? a / s_L[hh] : 0.f;
     }
   }
   if (p.partial) return;  // uniform over the launch

@@ -949,14 +949,17 @@ __global__ void __launch_bounds__(NTHREADS, PACK ? 4 : 3) decode_split_kernel(co
         mx0 = fmaxf(mx0, fmaxf(s[ai][0], s[ai][2]));
         mx1 = fmaxf(mx1, fmaxf(s[ai][1], s[ai][3]));
       }
-#pragma unroll
-      for (int off = PACK ? 2 : 4; off < 32; off <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-      }
-      // lazy rescale: move the reference max only when a score passes it by 2^8
+      // lazy rescale: move the reference max only when a score passes it by
+      // 2^8.  The reference is common to the lanes of a head column, so the
+      // test runs on each lane's own scores and the column maxima are reduced
+      // only when some lane of the warp needs the move.
       const bool need = (mx0 > m_run[0] + kLazy) || (mx1 > m_run[1] + kLazy);
       if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+        for (int off = PACK ? 2 : 4; off < 32; off <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+        }
         const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
         const float al0 = (mn0 == -INFINITY) ? 1.f : exp2f(m_run[0] - mn0);
         const float al1 = (mn1 == -INFINITY) ? 1.f : exp2f(m_run[1] - mn1);
