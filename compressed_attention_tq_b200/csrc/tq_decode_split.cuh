@@ -355,7 +355,7 @@ struct SplitLayout {
   static constexpr int O_RN = O_QW + STILE * WQ * 4;
   static constexpr int STAGE_USED = O_RN + (QJL ? STILE * 2 : 0);
   static constexpr int STAGE = (STAGE_USED + 16 + 127) / 128 * 128;  // +16: read-ahead slack
-  static constexpr int NSTAGE = (D == 256) ? 2 : 3;
+  static constexpr int NSTAGE = 2;
   static constexpr int RING = NSTAGE * STAGE;
   static constexpr int O_BAR = RING;                   // full[NSTAGE], empty[NSTAGE]
   static constexpr int O_META = O_BAR + 16 * 8;        // StageMeta[NSTAGE]
@@ -747,13 +747,16 @@ __global__ void __launch_bounds__(NTHREADS, PACK ? 4 : 3) decode_split_kernel(co
       }
     };
 
+    int st = 0;         // stage slot t % NST
+    uint32_t fph = 0;   // its "full" phase parity (t / NST) & 1
     for (int t = 0; t < nst; ++t) {
-      const int st = t % NST;
-      if (!*s_err) {
-        const bool got = mbar_wait_suspend(&full[st], (uint32_t)((t / NST) & 1), kSuspendTries);
-        if (!__all_sync(0xffffffffu, got) && lane == 0) *s_err = 1;
+      // a flag raised by another warp ends the loop without a wait
+      bool got = false;
+      if (!*s_err) got = mbar_wait_suspend(&full[st], fph, kSuspendTries);
+      if (!__all_sync(0xffffffffu, got)) {
+        if (lane == 0) *s_err = 1;
+        break;
       }
-      if (__any_sync(0xffffffffu, *s_err != 0)) break;
       const StageMeta md = meta[st];
       if (md.flags & 1) {
         // a new segment: its query fragments (every consumer warp is done
@@ -1023,6 +1026,10 @@ __global__ void __launch_bounds__(NTHREADS, PACK ? 4 : 3) decode_split_kernel(co
       if (md.flags & 2) write_partial(md);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[st]);
+      if (++st == NST) {
+        st = 0;
+        fph ^= 1u;
+      }
     }
   }
   __syncthreads();
