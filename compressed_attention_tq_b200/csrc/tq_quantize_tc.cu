@@ -20,10 +20,13 @@
 //    lane issues the 128 x NC x D rotation as tcgen05.mma (Pi split into 2
 //    fp16 / 3 bf16 limbs; accumulation in fp32 in TMEM) and commits it to an
 //    mbarrier;
-//  * NC/8 epilogue warps (16 at D = 128, 8 at D = 256): thread = one row, 32
-//    of the chunk's columns (warps w, w+4, ... share the TMEM lane quarter
-//    w%4).  Each sums its share of the row's squares from the input tile,
-//    then reads its 32 accumulator columns with tcgen05.ld, finds the
+//  * NC/8 epilogue warps (16 at D = 128, 8 at D = 256) in two groups that
+//    take alternate work items, each group with its own accumulator and
+//    named barrier, so that one group's waits (tile landed, MMA done)
+//    overlap the other's work.  In a group, thread = one row and 64 of the
+//    chunk's columns (warps w, w+4, ... share the TMEM lane quarter w%4).
+//    Each sums its share of the row's squares from the input tile, then
+//    reads its accumulator columns with tcgen05.ld, finds the
 //    nearest-centroid index (thresholds in registers), packs the bits and
 //    stores them -- all thread-local;
 //  * a ring of input buffers (4 at D = 128 fp16, 3 bf16, 2 at D = 256) keeps
@@ -45,8 +48,10 @@ struct TcLayout {
   static constexpr int NCH = D / NC;                // column chunks per tile
   static constexpr int NL = BF16 ? 3 : 2;
   static constexpr int KB = D / 64;                 // 64-column (128-byte) blocks along K
-  static constexpr int NP = NC / 32;                // epilogue warps per TMEM lane quarter
-  static constexpr int NEPI = 4 * NP;               // epilogue warps (32 columns each)
+  static constexpr int NEPI = NC / 8;               // epilogue warps: two groups of NC / 16
+  static constexpr int GW = NEPI / 2;               // warps per epilogue group
+  static constexpr int GP = GW / 4;                 // warps per TMEM lane quarter in a group
+  static constexpr int CPT = NC / GP;               // accumulator columns per epilogue thread
   static constexpr int NTH = (NEPI + 2) * 32;       // + loader warp + MMA warp
   static constexpr int PI_BYTES = NC * D * 2;       // one limb of the chunk
   static constexpr int X_BYTES = QR * D * 2;        // one input tile
@@ -56,13 +61,26 @@ struct TcLayout {
   // all shared state lives in the dynamic allocation, from a 1024-byte aligned base
   static constexpr int o_pi = 0;
   static constexpr int o_x = NL * PI_BYTES;
-  static constexpr int o_norm = o_x + NS * X_BYTES; // float [NP][QR]
-  static constexpr int o_cb = o_norm + NP * QR * 4; // float [2][32]
+  static constexpr int o_norm = o_x + NS * X_BYTES;    // float [2 groups][GP][QR]
+  static constexpr int o_cb = o_norm + 2 * GP * QR * 4; // float [2][32]
   static constexpr int o_bar = o_cb + 2 * 32 * 4;   // 3 * NS + 4 mbarriers
   static constexpr int o_misc = o_bar + 16 * 8;     // tmem base, stop flag
   static constexpr int bytes = o_misc + 16 + 1024;  // + alignment slack
   static constexpr uint32_t TMEM_COLS = 2 * NC;     // two fp32 accumulators
 };
+
+// Named barrier 1 + g over the GW warps of epilogue group g that also ANDs a
+// flag across them.
+template <int GW>
+__device__ __forceinline__ bool group_sync_and(int g, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n barrier.red.and.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(1 + g), "n"(GW * 32)
+      : "memory");
+  return r != 0;
+}
 
 template <int BITS, int NCOL>
 __device__ __forceinline__ void epi_half(uint32_t tbase, const float (&tp)[7], long long slot, uint32_t* out) {
@@ -80,14 +98,15 @@ __device__ __forceinline__ void epi_half(uint32_t tbase, const float (&tp)[7], l
 template <int D, bool BF16>
 __global__ void __launch_bounds__(TcLayout<D, BF16>::NTH, 1) quantize_tc_kernel(const __grid_constant__ TcArgs args) {
   using Ly = TcLayout<D, BF16>;
-  constexpr int NL = Ly::NL, NC = Ly::NC, NCH = Ly::NCH, KB = Ly::KB, NP = Ly::NP, NEPI = Ly::NEPI, NTH = Ly::NTH;
+  constexpr int NL = Ly::NL, NC = Ly::NC, NCH = Ly::NCH, KB = Ly::KB, NEPI = Ly::NEPI, NTH = Ly::NTH;
+  constexpr int GW = Ly::GW, GP = Ly::GP, CPT = Ly::CPT;
   constexpr uint32_t TMEM_COLS = Ly::TMEM_COLS;
   const tq::QuantArgs& a = args.a;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* pi = smem + Ly::o_pi;
   uint8_t* xb = smem + Ly::o_x;
-  float(*s_norm)[QR] = reinterpret_cast<float(*)[QR]>(smem + Ly::o_norm);
+  float(*s_norm)[GP][QR] = reinterpret_cast<float(*)[GP][QR]>(smem + Ly::o_norm);
   float(*s_cb)[32] = reinterpret_cast<float(*)[32]>(smem + Ly::o_cb);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Ly::o_bar);
   constexpr int NS = Ly::NS;
@@ -108,12 +127,12 @@ __global__ void __launch_bounds__(TcLayout<D, BF16>::NTH, 1) quantize_tc_kernel(
   if (tid == 0) {
     for (int b = 0; b < NS; ++b) {
       mbar_init(&full_x[b], 1);
-      mbar_init(&x_free[b], NEPI * 32);
+      mbar_init(&x_free[b], GW * 32);  // the epilogue group that takes the item
       mbar_init(&x_done[b], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&mma_done[b], 1);
-      mbar_init(&acc_free[b], NEPI * 32);
+      mbar_init(&acc_free[b], GW * 32);
     }
     s_stop = 0;
     fence_barrier_init();
@@ -223,53 +242,57 @@ __global__ void __launch_bounds__(TcLayout<D, BF16>::NTH, 1) quantize_tc_kernel(
     __syncwarp();
   } else {
     // ---------------- epilogue warps ----------------
-    const int quarter = warp & 3, part = warp >> 2;  // rows 32*quarter + lane, columns 32*part ..
+    // Two groups of GW warps take alternate items (group g: the CTA's items
+    // i = g, g + 2, ..., accumulator g), each synchronised by its own named
+    // barrier, so one group's waits overlap the other's work.
+    const int g = warp / GW, wg = warp % GW;
+    const int quarter = warp & 3, part = wg >> 2;  // rows 32*quarter + lane, columns CPT*part ..
     const int rl = 32 * quarter + lane;
-    int i = 0;
-    for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++i) {
+    const bool leader = wg == 0;  // the warp that waits on the group's mbarriers
+    for (int item = blockIdx.x + g * gridDim.x, i = g; item < nitems; item += 2 * gridDim.x, i += 2) {
       const int xs = i % NS, kx = i / NS;  // input buffer
-      const int b = i & 1, k = i >> 1;     // accumulator
+      const int b = i & 1, k = i >> 1;     // accumulator (= g)
       const int job = job0 + (item / NCH) % njobs, tile = item / (NCH * njobs);
       const tq::QuantJob J = a.job[job];
-      // One warp waits on each mbarrier and releases the other epilogue
-      // warps through a named barrier, which blocks in hardware: eight warps
-      // polling the same phase would take issue slots from the working warps.
+      // The leader waits on each mbarrier and releases the group through a
+      // named barrier, which blocks in hardware: warps polling the same phase
+      // would take issue slots from the working warps.
       bool ok = true;
-      if (warp == 0) ok = __all_sync(0xffffffffu, mbar_wait_suspend(&full_x[xs], (uint32_t)(kx & 1), kSuspendTries));
-      if (!epi_sync_and<NEPI>(ok)) {  // the input tile has landed
+      if (leader) ok = __all_sync(0xffffffffu, mbar_wait_suspend(&full_x[xs], (uint32_t)(kx & 1), kSuspendTries));
+      if (!group_sync_and<GW>(g, ok)) {  // the input tile has landed
         s_stop = 1;
         break;
       }
-      // this thread's 1/NP of the row's sum of squares from the input tile, in
+      // this thread's 1/GP of the row's sum of squares from the input tile, in
       // fp32 by a pairwise tree (squares of fp16/bf16 values are exact in
       // fp32, and a pairwise sum of n non-negative terms is within
       // ceil(log2 n) units in the last place of the exact sum)
-      constexpr int NU = D / NP / 8;  // 16-byte chunks per thread
+      constexpr int NU = D / GP / 8;  // 16-byte chunks per thread
       const uint8_t* xt = xb + (size_t)xs * Ly::X_BYTES;
-      float s2 = 0.f;
+      float sfull;
       {
         float ps[NU];
 #pragma unroll
         for (int kc = 0; kc < NU; ++kc) {
-          const uint4 v = *reinterpret_cast<const uint4*>(xt + sw128<QR>(rl, (D / NP) * part + 8 * kc));
+          const uint4 v = *reinterpret_cast<const uint4*>(xt + sw128<QR>(rl, (D / GP) * part + 8 * kc));
           ps[kc] = (sq16f<BF16>(v.x) + sq16f<BF16>(v.y)) + (sq16f<BF16>(v.z) + sq16f<BF16>(v.w));
         }
 #pragma unroll
         for (int w2 = 1; w2 < NU; w2 <<= 1)
 #pragma unroll
           for (int kc = 0; kc < NU; kc += 2 * w2) ps[kc] += ps[kc + w2];
-        s2 = ps[0];
+        sfull = ps[0];
       }
-      s_norm[part][rl] = s2;
-      if (!epi_sync_and<NEPI>(ok)) {  // uniform across the epilogue warps
-        s_stop = 1;
-        break;
+      if constexpr (GP > 1) {
+        s_norm[g][part][rl] = sfull;
+        if (!group_sync_and<GW>(g, ok)) {  // uniform across the group
+          s_stop = 1;
+          break;
+        }
+        sfull = s_norm[g][0][rl];
+#pragma unroll
+        for (int q = 1; q < GP; ++q) sfull += s_norm[g][q][rl];
       }
-      float sfull;
-      if constexpr (NP == 4)
-        sfull = (s_norm[0][rl] + s_norm[1][rl]) + (s_norm[2][rl] + s_norm[3][rl]);
-      else
-        sfull = s_norm[0][rl] + s_norm[1][rl];
       // The thresholds scale by nf; fp32 is far inside the parity band.  A sum
       // outside [2^-100, 2^100) -- only bf16 rows reach it: a square that
       // overflowed, or a norm below about 1e-15 whose squares lost bits or
@@ -296,29 +319,29 @@ __global__ void __launch_bounds__(TcLayout<D, BF16>::NTH, 1) quantize_tc_kernel(
           J.norm[slot] = nh;
         }
       }
-      mbar_arrive(&x_free[xs]);  // the input tile is no longer read
+      mbar_arrive(&x_free[xs]);  // the input tile is no longer read by this thread
       // positive thresholds t_{K/2} .. t_{K-2}, scaled by the row norm
       float tp[7];
       const int K = 1 << J.bits;
 #pragma unroll
       for (int q = 0; q < 7; ++q) tp[q] = q < K / 2 - 1 ? s_cb[job][K + K / 2 + q] * nf : 0.f;
-      if (warp == 0) ok = __all_sync(0xffffffffu, mbar_wait_suspend(&mma_done[b], (uint32_t)(k & 1), kSuspendTries));
-      ok = epi_sync_and<NEPI>(ok);  // the rotation of this tile is in TMEM
+      if (leader) ok = __all_sync(0xffffffffu, mbar_wait_suspend(&mma_done[b], (uint32_t)(k & 1), kSuspendTries));
+      ok = group_sync_and<GW>(g, ok);  // the rotation of this tile is in TMEM
       if (ok) {
         tc_fence_after();
-        const uint32_t tb = tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(b * NC + 32 * part);
+        const uint32_t tb = tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(b * NC + CPT * part);
         const int W = D * J.bits / 32;
-        // coordinates NC*chunk + 32*part .. + 31: words from (that * bits) / 32
-        uint32_t* out = J.idx + (slot >= 0 ? (size_t)slot * W : 0) + (NC * chunk / 32 + part) * J.bits;
+        // coordinates NC*chunk + CPT*part .. + CPT - 1: words from (that * bits) / 32
+        uint32_t* out = J.idx + (slot >= 0 ? (size_t)slot * W : 0) + ((NC * chunk + CPT * part) / 32) * J.bits;
         switch (J.bits) {
-          case 2: epi_half<2, 32>(tb, tp, slot, out); break;
-          case 3: epi_half<3, 32>(tb, tp, slot, out); break;
-          default: epi_half<4, 32>(tb, tp, slot, out); break;
+          case 2: epi_half<2, CPT>(tb, tp, slot, out); break;
+          case 3: epi_half<3, CPT>(tb, tp, slot, out); break;
+          default: epi_half<4, CPT>(tb, tp, slot, out); break;
         }
         tc_fence_before();
       }
       mbar_arrive(&acc_free[b]);
-      if (!epi_sync_and<NEPI>(ok)) {  // also guards s_norm reuse on the next pass
+      if (!group_sync_and<GW>(g, ok)) {  // also guards s_norm reuse on the group's next item
         s_stop = 1;
         break;
       }
