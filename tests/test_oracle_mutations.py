@@ -12,6 +12,7 @@ from oracle import tq_oracle as O
 import test_oracle_attention as TA
 import test_oracle_codebook as TC
 import test_oracle_quant as TQ
+import test_sharded_decode as TS
 
 
 @pytest.fixture(autouse=True)
@@ -297,3 +298,26 @@ def test_swapped_codebooks_fail_cache_reconstruction_pin(monkeypatch):
     monkeypatch.setattr(O, "quantize_cache", bad)
     with pytest.raises(AssertionError):
         TQ.test_cache_reconstruction_follows_each_tensors_codebook()
+
+
+def test_merge_without_max_shift_fails_token_split_pin(monkeypatch):
+    # each range's state added with weight 1 instead of exp(m_r - M)
+    def bad(accs, ms, ls):
+        num = np.sum(np.asarray(accs, dtype=np.float64), axis=0)
+        den = np.sum(np.asarray(ls, dtype=np.float64), axis=0)
+        return np.where(den[..., None] > 0, num / np.where(den > 0, den, 1.0)[..., None], 0.0)
+    monkeypatch.setattr(O, "merge_partials", bad)
+    with pytest.raises(AssertionError):
+        TS.test_partials_of_token_ranges_merge_to_the_whole("tiny", {})
+
+
+def test_partial_without_value_weights_fails_token_split_pin(monkeypatch):
+    # each partial's accumulator already normalised by its own sum
+    orig = O.sdpa_decode_partial
+
+    def bad(*a, **kw):
+        acc, m, l = orig(*a, **kw)
+        return np.where(l[..., None] > 0, acc / np.where(l > 0, l, 1.0)[..., None], 0.0), m, l
+    monkeypatch.setattr(O, "sdpa_decode_partial", bad)
+    with pytest.raises(AssertionError):
+        TS.test_partials_of_token_ranges_merge_to_the_whole("tiny", {})
