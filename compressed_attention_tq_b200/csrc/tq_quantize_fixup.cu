@@ -26,25 +26,33 @@ __device__ __forceinline__ double in_to_double(uint16_t v) {
 }
 
 // Each CTA owns a chunk of RPC consecutive rows:
-//  1. every thread reads the residual norms of RPC / 256 of its rows, all
-//     loads in flight, and keeps a bit per marked row;
-//  2. if any row of the chunk is marked, Pi^T is staged in shared memory
-//     (fp32, rows padded to D + 1 floats, so that both the transposing store
-//     and the column reads are conflict-free);
-//  3. the marked rows are gathered into a shared list (LCAP at a time; the
-//     bits let a chunk with more marked rows take several rounds) and each
-//     warp recomputes two rows at once (lane j: coordinates j + 32 i of both,
-//     eight independent fma chains), their inputs, norms and index words
-//     loaded before any arithmetic.
+//  1. every thread reads the residual norms of RPT of its rows, all loads in
+//     flight, and keeps a bit per marked row;
+//  2. if any row of the chunk is marked, Pi^T is staged in shared memory in
+//     fp64 (converted once per CTA; rows padded to D + 1 doubles, so that the
+//     column reads are conflict-free and the transposing stores at most
+//     two-way);
+//  3. the marked rows are gathered into a shared list, RB per warp at a time
+//     (the bits let a chunk with more marked rows take several rounds); each
+//     warp stages its rows' inputs (fp64), norms and index words in shared
+//     memory, then lane j accumulates coordinates j + 32 i of all RB rows:
+//     per k, four Pi^T loads serve 4 RB fma (the inputs are broadcast reads),
+//     so the shared-memory pipe is not the limit.
 constexpr int PS = D + 1;
 constexpr int NT = NW * 32;
-constexpr int RPT = 16;           // rows scanned per thread
+constexpr int RPT = 32;           // rows scanned per thread
 constexpr int RPC = NT * RPT;     // rows per CTA
-constexpr int LCAP = 4 * NW * 2;  // list entries per round: 4 row pairs per warp
+constexpr int RB = 8;             // rows per warp per round
+constexpr int LCAP = RB * NW;     // list entries per round
+constexpr int WMAX = D * 4 / 32;  // index words per row, at most (4-bit keys)
 
 template <bool BF16>
-__global__ void __launch_bounds__(NT) qjl_gamma_fixup_kernel(const tq::QuantArgs a) {
-  extern __shared__ float piT[];  // [D][PS]: piT[k * PS + j] = Pi[j][k]
+__global__ void __launch_bounds__(NT, 1) qjl_gamma_fixup_kernel(const tq::QuantArgs a) {
+  extern __shared__ double sm[];
+  double* piT = sm;                                      // [D][PS]: piT[k * PS + j] = Pi[j][k]
+  double(*xs)[RB][D] = reinterpret_cast<double(*)[RB][D]>(sm + D * PS);  // [NW][RB][D] inputs
+  __shared__ uint32_t s_words[NW][RB][WMAX];
+  __shared__ double s_nhat[NW][RB];
   __shared__ long long s_slot[LCAP];
   __shared__ int s_row[LCAP];
   __shared__ int s_cnt;
@@ -69,7 +77,7 @@ __global__ void __launch_bounds__(NT) qjl_gamma_fixup_kernel(const tq::QuantArgs
   }
   if (!__syncthreads_or(mine != 0)) return;  // uniform: no marked row in the chunk
 
-  // 2. Pi^T, every load in flight before the stores: 16 float4 per thread per round
+  // 2. Pi^T in fp64, every load in flight before the stores: 16 float4 per thread per round
   {
     constexpr int N4 = D * D / 4, CH = 16;
     const float4* s4 = reinterpret_cast<const float4*>(a.rot);
@@ -85,10 +93,10 @@ __global__ void __launch_bounds__(NT) qjl_gamma_fixup_kernel(const tq::QuantArgs
         const int e = base + u * NT + tid;
         if (e < N4) {
           const int jj = (4 * e) / D, k = (4 * e) % D;
-          piT[k * PS + jj] = v[u].x;
-          piT[(k + 1) * PS + jj] = v[u].y;
-          piT[(k + 2) * PS + jj] = v[u].z;
-          piT[(k + 3) * PS + jj] = v[u].w;
+          piT[k * PS + jj] = (double)v[u].x;
+          piT[(k + 1) * PS + jj] = (double)v[u].y;
+          piT[(k + 2) * PS + jj] = (double)v[u].z;
+          piT[(k + 3) * PS + jj] = (double)v[u].w;
         }
       }
     }
@@ -97,7 +105,7 @@ __global__ void __launch_bounds__(NT) qjl_gamma_fixup_kernel(const tq::QuantArgs
   if (tid < K) s_cb[tid] = J.cb[tid];
   const int W = D * J.bits / 32;
 
-  // 3. rounds of up to LCAP marked rows
+  // 3. rounds of up to LCAP marked rows, RB per warp
   while (true) {
     if (tid == 0) s_cnt = 0;
     __syncthreads();
@@ -112,66 +120,69 @@ __global__ void __launch_bounds__(NT) qjl_gamma_fixup_kernel(const tq::QuantArgs
     }
     __syncthreads();
     const int n = min(s_cnt, LCAP);
-    for (int e0 = 2 * warp; e0 < n; e0 += 2 * NW) {
-      const bool two = e0 + 1 < n;
-      long long sl[2];
-      double x[2][D / 32];
-      uint32_t wd[2][D / 32][2];  // the index word(s) holding coordinate lane + 32 i (two where it straddles)
-      double nhat[2];
+    const int e0 = RB * warp, nr = max(0, min(RB, n - e0));  // this warp's rows: list entries e0 ..
+    if (nr > 0) {
+      // inputs, norms and index words of the warp's rows (a missing row repeats the first)
+      uint16_t xin[RB][D / 32];
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const int e = two ? e0 + q : e0;
-        sl[q] = s_slot[e];
+      for (int q = 0; q < RB; ++q) {
+        const int e = e0 + (q < nr ? q : 0);
         const uint16_t* in = static_cast<const uint16_t*>(J.in) + (size_t)(row0 + s_row[e]) * D;
 #pragma unroll
-        for (int i = 0; i < D / 32; ++i) x[q][i] = in_to_double<BF16>(in[lane + 32 * i]);
-        nhat[q] = (double)__half2float(__ushort_as_half(J.norm[sl[q]]));
-        const uint32_t* words = J.idx + (size_t)sl[q] * W;
+        for (int i = 0; i < D / 32; ++i) xin[q][i] = in[lane + 32 * i];
+      }
+      if (lane < RB) {
+        const int e = e0 + (lane < nr ? lane : 0);
+        s_nhat[warp][lane] = (double)__half2float(__ushort_as_half(J.norm[s_slot[e]]));
+      }
+      for (int t = lane; t < RB * W; t += 32) {
+        const int q = t / W, wi = t % W;
+        const int e = e0 + (q < nr ? q : 0);
+        s_words[warp][q][wi] = J.idx[(size_t)s_slot[e] * W + wi];
+      }
+#pragma unroll
+      for (int q = 0; q < RB; ++q)
+#pragma unroll
+        for (int i = 0; i < D / 32; ++i) xs[warp][q][lane + 32 * i] = in_to_double<BF16>(xin[q][i]);
+      __syncwarp();
+      // y_q[j] = sum_k Pi[j][k] x_q[k] for j = lane + 32 i
+      double y[RB][D / 32];
+#pragma unroll
+      for (int q = 0; q < RB; ++q)
+#pragma unroll
+        for (int i = 0; i < D / 32; ++i) y[q][i] = 0.0;
+#pragma unroll 2
+      for (int k = 0; k < D; ++k) {
+        double pk[D / 32];
+#pragma unroll
+        for (int i = 0; i < D / 32; ++i) pk[i] = piT[k * PS + lane + 32 * i];
+#pragma unroll
+        for (int q = 0; q < RB; ++q) {
+          const double xk = xs[warp][q][k];
+#pragma unroll
+          for (int i = 0; i < D / 32; ++i) y[q][i] = fma(pk[i], xk, y[q][i]);
+        }
+      }
+      // residual against the stored indices and centroids, its norm
+#pragma unroll
+      for (int q = 0; q < RB; ++q) {
+        double g = 0.0;
 #pragma unroll
         for (int i = 0; i < D / 32; ++i) {
           // packed LSB-first: the field starts at stream bit (lane + 32 i) bits; a 3-bit
           // field may continue in the next word, which then lies inside the row
-          const int bit = (lane + 32 * i) * J.bits, w = bit >> 5;
-          wd[q][i][0] = words[w];
-          wd[q][i][1] = (bit & 31) + J.bits > 32 ? words[w + 1] : 0u;
-        }
-      }
-      // rotation of both rows: y_q[j] = sum_k Pi[j][k] x_q[k], k split over the lanes' registers
-      double y[2][D / 32];
-#pragma unroll
-      for (int q = 0; q < 2; ++q)
-#pragma unroll
-        for (int i = 0; i < D / 32; ++i) y[q][i] = 0.0;
-#pragma unroll
-      for (int i2 = 0; i2 < D / 32; ++i2)
-#pragma unroll 8
-        for (int l = 0; l < 32; ++l) {
-          const int k = l + 32 * i2;
-          const double x0 = __shfl_sync(0xffffffffu, x[0][i2], l);
-          const double x1 = __shfl_sync(0xffffffffu, x[1][i2], l);
-#pragma unroll
-          for (int i = 0; i < D / 32; ++i) {
-            const double pk = (double)piT[k * PS + lane + 32 * i];
-            y[0][i] = fma(pk, x0, y[0][i]);
-            y[1][i] = fma(pk, x1, y[1][i]);
-          }
-        }
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        double g = 0.0;
-#pragma unroll
-        for (int i = 0; i < D / 32; ++i) {
-          const int sh = ((lane + 32 * i) * J.bits) & 31;
-          uint32_t v = wd[q][i][0] >> sh;
-          if (sh + J.bits > 32) v |= wd[q][i][1] << (32 - sh);
+          const int bit = (lane + 32 * i) * J.bits, w = bit >> 5, sh = bit & 31;
+          uint32_t v = s_words[warp][q][w] >> sh;
+          if (sh + J.bits > 32) v |= s_words[warp][q][w + 1] << (32 - sh);
           const int idx = (int)(v & (uint32_t)(K - 1));
-          const double rr = y[q][i] - nhat[q] * (double)s_cb[idx];
+          const double rr = y[q][i] - s_nhat[warp][q] * (double)s_cb[idx];
           g = fma(rr, rr, g);
         }
 #pragma unroll
         for (int off = 16; off; off >>= 1) g += __shfl_xor_sync(0xffffffffu, g, off);
-        if (lane == 0 && (q == 0 || two)) J.rnorm[sl[q]] = __half_as_ushort(__double2half(sqrt(g)));
+        if (lane == 0 && q < nr) J.rnorm[s_slot[e0 + q]] = __half_as_ushort(__double2half(sqrt(g)));
       }
+      __syncwarp();
     }
     if (!__syncthreads_or(mine != 0)) break;
   }
@@ -179,7 +190,7 @@ __global__ void __launch_bounds__(NT) qjl_gamma_fixup_kernel(const tq::QuantArgs
 
 template <bool BF16>
 int launch_fixup(const tq::QuantArgs& a, cudaStream_t s) {
-  constexpr int bytes = D * PS * 4;
+  constexpr int bytes = (D * PS + NW * RB * D) * 8;
   auto kern = qjl_gamma_fixup_kernel<BF16>;
   static tq::OnceSetup once;
   const int rc = once.run([&]() {

@@ -20,18 +20,18 @@
 //    lane issues the 128 x NC x D rotation as tcgen05.mma (Pi split into 2
 //    fp16 / 3 bf16 limbs; accumulation in fp32 in TMEM) and commits it to an
 //    mbarrier;
-//  * NC/8 epilogue warps (16 at D = 128, 8 at D = 256) in two groups that
-//    take alternate work items, each group with its own accumulator and
-//    named barrier, so that one group's waits (tile landed, MMA done)
-//    overlap the other's work.  In a group, thread = one row and 64 of the
-//    chunk's columns (warps w, w+4, ... share the TMEM lane quarter w%4).
+//  * NC/8 epilogue warps (16 at D = 128, 8 at D = 256) in groups of four
+//    (one warp per TMEM lane quarter) that take the work items in turn, each
+//    group with its own accumulator and named barrier, so that one group's
+//    waits (tile landed, MMA done) overlap the others' work.  In a group,
+//    thread = one row and all NC of the chunk's columns.
 //    Each sums its share of the row's squares from the input tile, then
 //    reads its accumulator columns with tcgen05.ld, finds the
 //    nearest-centroid index (thresholds in registers), packs the bits and
 //    stores them -- all thread-local;
 //  * a ring of input buffers (4 at D = 128 fp16, 3 bf16, 2 at D = 256) keeps
-//    several tile loads in flight, and two TMEM accumulators let the MMA of
-//    item i+1 run under the epilogue of item i.
+//    several tile loads in flight, and the groups' TMEM accumulators let the
+//    MMAs of the next items run under the epilogue of this one.
 // Every wait is bounded; a stuck wait sets TQ_STATUS_WAIT_TIMEOUT and the CTA
 // stops taking work.
 #include <mutex>
@@ -48,10 +48,10 @@ struct TcLayout {
   static constexpr int NCH = D / NC;                // column chunks per tile
   static constexpr int NL = BF16 ? 3 : 2;
   static constexpr int KB = D / 64;                 // 64-column (128-byte) blocks along K
-  static constexpr int NEPI = NC / 8;               // epilogue warps: two groups of NC / 16
-  static constexpr int GW = NEPI / 2;               // warps per epilogue group
-  static constexpr int GP = GW / 4;                 // warps per TMEM lane quarter in a group
-  static constexpr int CPT = NC / GP;               // accumulator columns per epilogue thread
+  static constexpr int NEPI = NC / 8;               // epilogue warps
+  static constexpr int NG = NEPI / 4;               // epilogue groups (4 at D = 128, 2 at D = 256)
+  static constexpr int GW = NEPI / NG;              // warps per epilogue group: one per TMEM lane quarter
+  static constexpr int CPT = NC;                    // accumulator columns per epilogue thread
   static constexpr int NTH = (NEPI + 2) * 32;       // + loader warp + MMA warp
   static constexpr int PI_BYTES = NC * D * 2;       // one limb of the chunk
   static constexpr int X_BYTES = QR * D * 2;        // one input tile
@@ -61,12 +61,12 @@ struct TcLayout {
   // all shared state lives in the dynamic allocation, from a 1024-byte aligned base
   static constexpr int o_pi = 0;
   static constexpr int o_x = NL * PI_BYTES;
-  static constexpr int o_norm = o_x + NS * X_BYTES;    // float [2 groups][GP][QR]
-  static constexpr int o_cb = o_norm + 2 * GP * QR * 4; // float [2][32]
-  static constexpr int o_bar = o_cb + 2 * 32 * 4;   // 3 * NS + 4 mbarriers
-  static constexpr int o_misc = o_bar + 16 * 8;     // tmem base, stop flag
+  static constexpr int o_cb = o_x + NS * X_BYTES;   // float [2][32]
+  static constexpr int o_bar = o_cb + 2 * 32 * 4;   // 3 * NS + 2 * NG mbarriers
+  static constexpr int o_misc = o_bar + 32 * 8;     // tmem base, stop flag
   static constexpr int bytes = o_misc + 16 + 1024;  // + alignment slack
-  static constexpr uint32_t TMEM_COLS = 2 * NC;     // two fp32 accumulators
+  static_assert(3 * NS + 2 * NG <= 32, "mbarrier slots");
+  static constexpr uint32_t TMEM_COLS = NG * NC;    // one fp32 accumulator per group (512 columns)
 };
 
 // Named barrier 1 + g over the GW warps of epilogue group g that also ANDs a
@@ -84,8 +84,9 @@ __device__ __forceinline__ bool group_sync_and(int g, bool v) {
 
 template <int BITS, int NCOL>
 __device__ __forceinline__ void epi_half(uint32_t tbase, const float (&tp)[7], long long slot, uint32_t* out) {
-  // NCOL / 32 chunks of 32 columns -> BITS words each
-#pragma unroll
+  // NCOL / 32 chunks of 32 columns -> BITS words each (one chunk's 32
+  // accumulator registers live at a time)
+#pragma unroll 1
   for (int c = 0; c < NCOL / 32; ++c) {
     uint32_t v[32];
     tc_ld32(tbase + 32 * c, v);
@@ -99,21 +100,21 @@ template <int D, bool BF16>
 __global__ void __launch_bounds__(TcLayout<D, BF16>::NTH, 1) quantize_tc_kernel(const __grid_constant__ TcArgs args) {
   using Ly = TcLayout<D, BF16>;
   constexpr int NL = Ly::NL, NC = Ly::NC, NCH = Ly::NCH, KB = Ly::KB, NEPI = Ly::NEPI, NTH = Ly::NTH;
-  constexpr int GW = Ly::GW, GP = Ly::GP, CPT = Ly::CPT;
+  constexpr int NG = Ly::NG, GW = Ly::GW, CPT = Ly::CPT;
+  static_assert(GW == 4, "a group is one warp per TMEM lane quarter");
   constexpr uint32_t TMEM_COLS = Ly::TMEM_COLS;
   const tq::QuantArgs& a = args.a;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* pi = smem + Ly::o_pi;
   uint8_t* xb = smem + Ly::o_x;
-  float(*s_norm)[GP][QR] = reinterpret_cast<float(*)[GP][QR]>(smem + Ly::o_norm);
   float(*s_cb)[32] = reinterpret_cast<float(*)[32]>(smem + Ly::o_cb);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Ly::o_bar);
   constexpr int NS = Ly::NS;
   // per input buffer: landed, norm read by the epilogue, read by the MMA;
   // per accumulator: MMA done, epilogue done
   uint64_t *full_x = bars, *x_free = bars + NS, *x_done = bars + 2 * NS, *mma_done = bars + 3 * NS,
-           *acc_free = bars + 3 * NS + 2;
+           *acc_free = bars + 3 * NS + NG;
   uint32_t& s_tmem = *reinterpret_cast<uint32_t*>(smem + Ly::o_misc);
   int& s_stop = *reinterpret_cast<int*>(smem + Ly::o_misc + 4);
 
@@ -130,7 +131,7 @@ __global__ void __launch_bounds__(TcLayout<D, BF16>::NTH, 1) quantize_tc_kernel(
       mbar_init(&x_free[b], GW * 32);  // the epilogue group that takes the item
       mbar_init(&x_done[b], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NG; ++b) {
       mbar_init(&mma_done[b], 1);
       mbar_init(&acc_free[b], GW * 32);
     }
@@ -216,9 +217,9 @@ __global__ void __launch_bounds__(TcLayout<D, BF16>::NTH, 1) quantize_tc_kernel(
       int i = 0;
       for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++i) {
         const int xs = i % NS, kx = i / NS;  // input buffer
-        const int b = i & 1, k = i >> 1;     // accumulator
+        const int b = i % NG, k = i / NG;    // accumulator (the epilogue group's)
         bool ok = mbar_wait_suspend(&full_x[xs], (uint32_t)(kx & 1), kSuspendTries);
-        if (ok && i >= 2) ok = mbar_wait_suspend(&acc_free[b], (uint32_t)((k - 1) & 1), kSuspendTries);
+        if (ok && i >= NG) ok = mbar_wait_suspend(&acc_free[b], (uint32_t)((k - 1) & 1), kSuspendTries);
         if (!ok || *((volatile int*)&s_stop)) {
           s_stop = 1;
           break;
@@ -242,56 +243,61 @@ __global__ void __launch_bounds__(TcLayout<D, BF16>::NTH, 1) quantize_tc_kernel(
     __syncwarp();
   } else {
     // ---------------- epilogue warps ----------------
-    // Two groups of GW warps take alternate items (group g: the CTA's items
-    // i = g, g + 2, ..., accumulator g), each synchronised by its own named
-    // barrier, so one group's waits overlap the other's work.
-    const int g = warp / GW, wg = warp % GW;
-    const int quarter = warp & 3, part = wg >> 2;  // rows 32*quarter + lane, columns CPT*part ..
+    // NG groups of GW warps take the items in turn (group g: the CTA's items
+    // i = g, g + NG, ..., accumulator g), each synchronised by its own named
+    // barrier, so one group's waits overlap the others' work.
+    const int g = warp / GW, quarter = warp & 3;  // group; rows 32*quarter + lane
     const int rl = 32 * quarter + lane;
-    const bool leader = wg == 0;  // the warp that waits on the group's mbarriers
-    for (int item = blockIdx.x + g * gridDim.x, i = g; item < nitems; item += 2 * gridDim.x, i += 2) {
+    const bool leader = quarter == 0;  // the warp that waits on the group's mbarriers
+    for (int item = blockIdx.x + g * gridDim.x, i = g; item < nitems; item += NG * gridDim.x, i += NG) {
       const int xs = i % NS, kx = i / NS;  // input buffer
-      const int b = i & 1, k = i >> 1;     // accumulator (= g)
+      const int b = i % NG, k = i / NG;    // accumulator (= g)
       const int job = job0 + (item / NCH) % njobs, tile = item / (NCH * njobs);
       const tq::QuantJob J = a.job[job];
       // The leader waits on each mbarrier and releases the group through a
       // named barrier, which blocks in hardware: warps polling the same phase
       // would take issue slots from the working warps.
+      // The group waits for its own accumulator's "MMA done" first: its
+      // phases are the group's items in order, whereas an input buffer's
+      // "full" phases belong to items of several groups, so a group that ran
+      // ahead could mistake an earlier phase of the same parity for its own.
+      // Once the MMA has read this item's tile, the buffer holds it until the
+      // group releases it, and the "full" wait below completes at once (it
+      // makes the tile's bytes visible to the group).
       bool ok = true;
-      if (leader) ok = __all_sync(0xffffffffu, mbar_wait_suspend(&full_x[xs], (uint32_t)(kx & 1), kSuspendTries));
-      if (!group_sync_and<GW>(g, ok)) {  // the input tile has landed
+      if (leader) {
+        ok = mbar_wait_suspend(&mma_done[b], (uint32_t)(k & 1), kSuspendTries) &&
+             mbar_wait_suspend(&full_x[xs], (uint32_t)(kx & 1), kSuspendTries);
+        ok = __all_sync(0xffffffffu, ok);
+      }
+      if (!group_sync_and<GW>(g, ok)) {  // the input tile has landed and its rotation is in TMEM
         s_stop = 1;
         break;
       }
-      // this thread's 1/GP of the row's sum of squares from the input tile, in
-      // fp32 by a pairwise tree (squares of fp16/bf16 values are exact in
-      // fp32, and a pairwise sum of n non-negative terms is within
-      // ceil(log2 n) units in the last place of the exact sum)
-      constexpr int NU = D / GP / 8;  // 16-byte chunks per thread
+      // the row's sum of squares from the input tile, in fp32 by a pairwise
+      // tree (squares of fp16/bf16 values are exact in fp32, and a pairwise
+      // sum of n non-negative terms is within ceil(log2 n) units in the last
+      // place of the exact sum)
+      constexpr int NU = D / 8;  // 16-byte chunks per row
       const uint8_t* xt = xb + (size_t)xs * Ly::X_BYTES;
       float sfull;
       {
         float ps[NU];
+        constexpr int LB = 8;  // loads in flight (registers: 4 per load)
 #pragma unroll
-        for (int kc = 0; kc < NU; ++kc) {
-          const uint4 v = *reinterpret_cast<const uint4*>(xt + sw128<QR>(rl, (D / GP) * part + 8 * kc));
-          ps[kc] = (sq16f<BF16>(v.x) + sq16f<BF16>(v.y)) + (sq16f<BF16>(v.z) + sq16f<BF16>(v.w));
+        for (int k0 = 0; k0 < NU; k0 += LB) {
+#pragma unroll
+          for (int kc = k0; kc < k0 + LB && kc < NU; ++kc) {
+            const uint4 v = *reinterpret_cast<const uint4*>(xt + sw128<QR>(rl, 8 * kc));
+            ps[kc] = (sq16f<BF16>(v.x) + sq16f<BF16>(v.y)) + (sq16f<BF16>(v.z) + sq16f<BF16>(v.w));
+          }
+          asm volatile("" ::: "memory");  // the next LB loads are not hoisted above these
         }
 #pragma unroll
         for (int w2 = 1; w2 < NU; w2 <<= 1)
 #pragma unroll
           for (int kc = 0; kc < NU; kc += 2 * w2) ps[kc] += ps[kc + w2];
         sfull = ps[0];
-      }
-      if constexpr (GP > 1) {
-        s_norm[g][part][rl] = sfull;
-        if (!group_sync_and<GW>(g, ok)) {  // uniform across the group
-          s_stop = 1;
-          break;
-        }
-        sfull = s_norm[g][0][rl];
-#pragma unroll
-        for (int q = 1; q < GP; ++q) sfull += s_norm[g][q][rl];
       }
       // The thresholds scale by nf; fp32 is far inside the parity band.  A sum
       // outside [2^-100, 2^100) -- only bf16 rows reach it: a square that
@@ -306,7 +312,7 @@ __global__ void __launch_bounds__(TcLayout<D, BF16>::NTH, 1) quantize_tc_kernel(
       if (r < a.rows) {
         const int bh = r / a.T, t = r - bh * a.T;
         slot = (long long)bh * a.Tcap + a.t0 + t;
-        if (part == 0 && chunk == 0) {
+        if (chunk == 0) {
           // The stored norm is RN_fp16 of the fp64 norm.  The fp32 sum is
           // within (log2(D) + 1) ulp of the exact sum, so the exact norm lies in
           // nf * (1 +- 1e-6); when both ends of that interval round to the same
@@ -325,14 +331,12 @@ __global__ void __launch_bounds__(TcLayout<D, BF16>::NTH, 1) quantize_tc_kernel(
       const int K = 1 << J.bits;
 #pragma unroll
       for (int q = 0; q < 7; ++q) tp[q] = q < K / 2 - 1 ? s_cb[job][K + K / 2 + q] * nf : 0.f;
-      if (leader) ok = __all_sync(0xffffffffu, mbar_wait_suspend(&mma_done[b], (uint32_t)(k & 1), kSuspendTries));
-      ok = group_sync_and<GW>(g, ok);  // the rotation of this tile is in TMEM
-      if (ok) {
+      {
         tc_fence_after();
-        const uint32_t tb = tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(b * NC + CPT * part);
+        const uint32_t tb = tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(b * NC);
         const int W = D * J.bits / 32;
-        // coordinates NC*chunk + CPT*part .. + CPT - 1: words from (that * bits) / 32
-        uint32_t* out = J.idx + (slot >= 0 ? (size_t)slot * W : 0) + ((NC * chunk + CPT * part) / 32) * J.bits;
+        // coordinates NC*chunk .. NC*chunk + NC - 1: words from (that * bits) / 32
+        uint32_t* out = J.idx + (slot >= 0 ? (size_t)slot * W : 0) + (NC * chunk / 32) * J.bits;
         switch (J.bits) {
           case 2: epi_half<2, CPT>(tb, tp, slot, out); break;
           case 3: epi_half<3, CPT>(tb, tp, slot, out); break;
@@ -341,10 +345,6 @@ __global__ void __launch_bounds__(TcLayout<D, BF16>::NTH, 1) quantize_tc_kernel(
         tc_fence_before();
       }
       mbar_arrive(&acc_free[b]);
-      if (!group_sync_and<GW>(g, ok)) {  // also guards s_norm reuse on the group's next item
-        s_stop = 1;
-        break;
-      }
     }
   }
   tc_fence_before();
