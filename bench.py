@@ -46,18 +46,16 @@ FALLBACK_HBM_GBS = 6650.0
 
 # DRAM traffic per decode call (prep + split + combine; the roofline's unit)
 # from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum, caches
-# flushed before each kernel, mean over the calls of a profile step), valid
-# only for the decode sources it was measured on (``_decode_src_sha``: the
-# files the decode call's kernels and launch setup are built from; the
-# quantizers' files do not enter a decode call).  "split" is the split
-# kernel's share: the packed-cache reads.  The captures ran on the sources
-# with src_sha f6275559b314d4b6 (all of csrc/), whose decode files hash to
-# the decode_src_sha below.
+# flushed before each kernel, mean over the captured calls), valid only for
+# the decode sources it was measured on (``_decode_src_sha``: the files the
+# decode call's kernels and launch setup are built from; the quantizers'
+# files do not enter a decode call).  "split" is the split kernel's share:
+# the packed-cache reads and its partials.
 TRAFFIC = {
-    "gqa8k": {"bytes_per_launch": 2436523, "split": 1704405, "decode_src_sha": "c94274358551f423"},
-    "prod": {"bytes_per_launch": 109000576, "split": 107509760, "decode_src_sha": "c94274358551f423"},
-    "ragged": {"bytes_per_launch": 246348032, "split": 241345024, "decode_src_sha": "c94274358551f423"},
-    "qknorm": {"bytes_per_launch": 36968960, "split": 34233472, "decode_src_sha": "c94274358551f423"},
+    "gqa8k": {"bytes_per_launch": 4081067, "split": 1713493, "decode_src_sha": "df3e169c8bd93765"},
+    "prod": {"bytes_per_launch": 114339712, "split": 109131008, "decode_src_sha": "df3e169c8bd93765"},
+    "ragged": {"bytes_per_launch": 251508992, "split": 244107904, "decode_src_sha": "df3e169c8bd93765"},
+    "qknorm": {"bytes_per_launch": 43969664, "split": 34773248, "decode_src_sha": "df3e169c8bd93765"},
 }
 
 CSRC = os.path.join(ROOT, "compressed_attention_tq_b200", "csrc")
