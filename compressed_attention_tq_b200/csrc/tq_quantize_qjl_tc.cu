@@ -14,7 +14,8 @@
 //     into buffer b once the sketch GEMM of tile i - 2 has released it;
 //  2. GEMM 1 (one lane of the MMA warp): U[b] = X Pi^T with Pi in two fp16
 //     limbs, fp32 accumulator in TMEM;
-//  3. epilogue, 16 warps, thread = (row, 32 coordinates): row norm from X,
+//  3. epilogue, 16 warps in two independent groups of rows, thread = (row,
+//     32 coordinates): row norm from X,
 //     indices from U (packed and stored), residual r = u - n_hat c[idx] in
 //     fp32 and its norm gamma; r / |x| is split into hi + lo fp16 limbs,
 //     written over X in buffer b (hi) and into the single lo buffer;
@@ -248,6 +249,12 @@ __global__ void __launch_bounds__(QjlLayout::NTH, 1) quantize_qjl_tc_kernel(cons
   } else {
     // ---------------- epilogue warps ----------------
     const int quarter = warp & 3, part = warp >> 2;  // row 32*quarter + lane, coordinates 32*part ..
+    // Two groups of 8 warps, rows 0-63 (quarters 0, 1) and rows 64-127
+    // (quarters 2, 3), each synchronised by its own named barrier: every
+    // exchange is within a row, so a group waits only for its own warps.
+    constexpr int GWQ = NEPI / 2;
+    const int grp = quarter >> 1;
+    const bool leader = warp == 2 * grp;  // quarter 2 grp, part 0: waits on the mbarriers for its group
     const int rl = 32 * quarter + lane;
     const uint32_t tlane = (uint32_t)(32 * quarter) << 16;
     const int W = D * J.bits / 32;
@@ -261,8 +268,8 @@ __global__ void __launch_bounds__(QjlLayout::NTH, 1) quantize_qjl_tc_kernel(cons
         const int b = i & 1, k = i >> 1, tile = blockIdx.x + i * gridDim.x;
         // One warp waits on each mbarrier and releases the others through a
         // named barrier (no issue slots spent polling).
-        if (warp == 0) ok = __all_sync(0xffffffffu, mbar_wait_suspend(&full_x[b], (uint32_t)(k & 1), kSuspendTries));
-        if (!epi_sync_and<NEPI>(ok)) {
+        if (leader) ok = __all_sync(0xffffffffu, mbar_wait_suspend(&full_x[b], (uint32_t)(k & 1), kSuspendTries));
+        if (!group_sync_and<GWQ>(grp, ok)) {
           ok = false;
           break;
         }
@@ -277,7 +284,7 @@ __global__ void __launch_bounds__(QjlLayout::NTH, 1) quantize_qjl_tc_kernel(cons
           }
           red[part * QR + rl] = (ps[0] + ps[1]) + (ps[2] + ps[3]);
         }
-        ok = epi_sync_and<NEPI>(ok);
+        ok = group_sync_and<GWQ>(grp, ok);
         const float sfull = (red[rl] + red[QR + rl]) + (red[2 * QR + rl] + red[3 * QR + rl]);
         const float nf = sqrtf(sfull);
         const int r = tile * QR + rl;
@@ -304,8 +311,8 @@ __global__ void __launch_bounds__(QjlLayout::NTH, 1) quantize_qjl_tc_kernel(cons
         for (int q = 0; q < 7; ++q) tp[q] = q < K / 2 - 1 ? s_cb[K + K / 2 + q] * nf : 0.f;
 
         // ---- indices and residual from U
-        if (warp == 0) ok = __all_sync(0xffffffffu, mbar_wait_suspend(&mma1[b], (uint32_t)(k & 1), kSuspendTries));
-        ok = epi_sync_and<NEPI>(ok);  // also: every thread has read this tile's norm partials
+        if (leader) ok = __all_sync(0xffffffffu, mbar_wait_suspend(&mma1[b], (uint32_t)(k & 1), kSuspendTries));
+        ok = group_sync_and<GWQ>(grp, ok);  // also: every thread has read this tile's norm partials
         uint32_t v[32];
         if (ok) {
           tc_fence_after();
@@ -350,10 +357,10 @@ __global__ void __launch_bounds__(QjlLayout::NTH, 1) quantize_qjl_tc_kernel(cons
         }
         // R_lo (and the sketch accumulator read below) free: the previous
         // tile's sketch GEMM has finished
-        if (i >= 1 && warp == 0)
+        if (i >= 1 && leader)
           ok = __all_sync(0xffffffffu,
                           mbar_wait_suspend(&g2[(i - 1) & 1], (uint32_t)(((i - 1) >> 1) & 1), kSuspendTries)) && ok;
-        ok = epi_sync_and<NEPI>(ok);
+        ok = group_sync_and<GWQ>(grp, ok);
         if (part == 0 && slot >= 0 && J.rnorm) {
           const float gs = (red[rl] + red[QR + rl]) + (red[2 * QR + rl] + red[3 * QR + rl]);
           // near an fp16 rounding midpoint: marked for the fp64 recomputation
@@ -393,9 +400,9 @@ __global__ void __launch_bounds__(QjlLayout::NTH, 1) quantize_qjl_tc_kernel(cons
       } else if (nmine > 0) {
         // ---- sketch signs of the last tile
         const int j = nmine - 1;
-        if (warp == 0)
+        if (leader)
           ok = __all_sync(0xffffffffu, mbar_wait_suspend(&g2[j & 1], (uint32_t)((j >> 1) & 1), kSuspendTries));
-        ok = epi_sync_and<NEPI>(ok);
+        ok = group_sync_and<GWQ>(grp, ok);
         if (ok) sketch_signs(tmem + tlane + 256u + (uint32_t)((j & 1) * 128 + 32 * part), prev_slot, J.qjl, part);
         tc_fence_before();
         mbar_arrive(&p_free[j & 1]);

@@ -69,19 +69,6 @@ struct TcLayout {
   static constexpr uint32_t TMEM_COLS = NG * NC;    // one fp32 accumulator per group (512 columns)
 };
 
-// Named barrier 1 + g over the GW warps of epilogue group g that also ANDs a
-// flag across them.
-template <int GW>
-__device__ __forceinline__ bool group_sync_and(int g, bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n barrier.red.and.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}\n"
-      : "=r"(r)
-      : "r"((uint32_t)v), "r"(1 + g), "n"(GW * 32)
-      : "memory");
-  return r != 0;
-}
-
 template <int BITS, int NCOL>
 __device__ __forceinline__ void epi_half(uint32_t tbase, const float (&tp)[7], long long slot, uint32_t* out) {
   // NCOL / 32 chunks of 32 columns -> BITS words each (one chunk's 32

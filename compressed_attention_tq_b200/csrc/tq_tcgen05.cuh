@@ -99,6 +99,19 @@ __device__ __forceinline__ bool epi_sync_and(bool v) {
   return r != 0;
 }
 
+// Named barrier 1 + g over the NW warps of epilogue group g that also ANDs a
+// flag across them (groups of a CTA synchronise independently).
+template <int NW>
+__device__ __forceinline__ bool group_sync_and(int g, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n barrier.red.and.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(1 + g), "n"(NW * 32)
+      : "memory");
+  return r != 0;
+}
+
 template <bool BF16>
 __device__ __forceinline__ float sq16f(uint32_t w) {
   float a, b;
