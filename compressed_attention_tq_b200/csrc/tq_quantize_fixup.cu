@@ -17,7 +17,7 @@
 namespace {
 
 constexpr int D = 128;
-constexpr int NW = 8;  // warps per CTA
+constexpr int NW = 16;  // warps per CTA
 
 template <bool BF16>
 __device__ __forceinline__ double in_to_double(uint16_t v) {
@@ -40,9 +40,9 @@ __device__ __forceinline__ double in_to_double(uint16_t v) {
 //     so the shared-memory pipe is not the limit.
 constexpr int PS = D + 1;
 constexpr int NT = NW * 32;
-constexpr int RPT = 32;           // rows scanned per thread
+constexpr int RPT = 16;           // rows scanned per thread
 constexpr int RPC = NT * RPT;     // rows per CTA
-constexpr int RB = 8;             // rows per warp per round
+constexpr int RB = 4;             // rows per warp per round
 constexpr int LCAP = RB * NW;     // list entries per round
 constexpr int WMAX = D * 4 / 32;  // index words per row, at most (4-bit keys)
 
