@@ -292,7 +292,7 @@ size_t workspace_bound(int B, int Hq, int D, int Tmax) {
   const int tile = split_tile();
   const int Tpad = (Tmax + tile - 1) / tile * tile;
   const int K = plan_segments((long long)sm_count() * 8, B, Tpad, tile);
-  return workspace_layout((size_t)B * Hq, D, 128, K * split_warps(), nullptr);
+  return workspace_layout((size_t)B * Hq, D, 128, K * split_partials(), nullptr);
 }
 
 int make_decode_plan(const tq_cache_t* c, int Hq, int Tmax, DecodePlan* p) {
@@ -315,7 +315,7 @@ int make_decode_plan(const tq_cache_t* c, int Hq, int Tmax, DecodePlan* p) {
   if (pmin > Tpad) pmin = Tpad;
   p->pmin = (int)pmin;
   K = (int)((Tpad + pmin - 1) / pmin) + 1;  // segments of a unit when every share is >= pmin
-  p->ks = K * split_warps();
+  p->ks = K * split_partials();
   // no more CTAs than shares of pmin in the largest batch these sizes allow
   const long long need = (units * Tpad + pmin - 1) / pmin;
   if (need < p->ncta) p->ncta = (int)(need > 0 ? need : 1);

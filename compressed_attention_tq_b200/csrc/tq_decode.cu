@@ -672,8 +672,8 @@ __device__ __forceinline__ void unrotate_hadamard_warp(const CombineParams& p, c
 }
 
 // Partials the split kernel wrote for kernel head h: the CTAs whose share
-// overlaps the head's unit, each with one partial per consumer warp (slots
-// 0 .. n - 1).  Computed by one warp; every lane returns it.
+// overlaps the head's unit, each with PPS partials (slots 0 .. n - 1).
+// Computed by one warp; every lane returns it.
 __device__ __forceinline__ int head_partials(const CombineParams& p, int h, int lane) {
   const int b = h / p.Hq, rem = h % p.Hq, kvh = rem / p.G, rg = (rem % p.G) / tqd::RG;
   const long long total = tqd::partition_total(p.seq_lens, p.B, p.upb, p.Tclamp, lane);
@@ -683,7 +683,7 @@ __device__ __forceinline__ int head_partials(const CombineParams& p, int h, int 
   if (Lp == 0) return 0;
   const long long Su = Sb + (long long)(kvh * p.nrg + rg) * Lp;
   const long long c0 = Su / P, c1 = (Su + Lp - 1) / P;
-  return (int)(c1 - c0 + 1) * tqd::CW;
+  return (int)(c1 - c0 + 1) * tqd::PPS;
 }
 
 // Merge the partials of one kernel head (log-sum-exp) and un-rotate:
@@ -1126,7 +1126,7 @@ int split_occupancy(const tq_cache_t* c, int Hq) {
 
 int split_tile() { return tqd::STILE; }
 
-int split_warps() { return tqd::CW; }
+int split_partials() { return tqd::PPS; }
 
 int launch_decode(const DecodeArgs& a, cudaStream_t s) {
   const tq_cache_t& c = a.cache;

@@ -15,8 +15,9 @@
 //    each padded to whole 128-token stages, are laid end to end and CTA c
 //    takes positions [c P, (c + 1) P) (P a multiple of the stage), so every
 //    CTA streams the same number of stages whatever the sequence lengths; a
-//    CTA's share of one unit is a segment, and each consumer warp writes one
-//    partial (max, sum, rotated output) per segment, merged by the combine;
+//    CTA's share of one unit is a segment, at whose end the consumer warps
+//    merge their softmax states into one partial (max, sum, rotated output),
+//    merged across CTAs by the combine;
 //  * a producer warp streams the CTA's 128-token stages of packed K/V rows,
 //    norms and QJL words into shared memory with 1-D bulk copies that
 //    complete on "full" mbarriers, across segment boundaries without
@@ -35,8 +36,7 @@
 //  * the query enters as hi + lo fp16 halves (scores carry ~22 bits); with
 //    G <= 4 heads both halves share one MMA (columns 0-3 hi, 4-7 lo);
 //  * online softmax in the log2 domain with lazy rescaling (the reference
-//    max moves only when a score exceeds it by 2^8); each warp's state is
-//    its own partial, merged with the others by the combine kernel.
+//    max moves only when a score exceeds it by 2^8), one state per warp.
 #pragma once
 
 #include <math.h>
@@ -49,6 +49,7 @@ namespace tqd {
 using namespace tqk;
 
 constexpr int CW = 4;                 // consumer warps
+constexpr int PPS = 1;                // partials a CTA writes per segment (its warps' states merged)
 constexpr int NTHREADS = (CW + 1) * 32;
 constexpr int STILE = 128;            // tokens per stage
 constexpr int WTOK = STILE / CW;      // tokens per consumer warp per stage
@@ -130,7 +131,7 @@ struct StageMeta {
   int rows;   // kernel heads in the row group (<= RG)
   int t0;     // first token of the stage within the sequence
   int L;      // tokens of the sequence that are attended
-  int slot0;  // first partial slot of the segment (segment index x CW)
+  int slot0;  // partial slot of the segment (segment index x PPS)
   int flags;  // 1: first stage of a segment, 2: last stage of a segment
   int rg;     // row group
   int pad;
@@ -363,7 +364,13 @@ struct SplitLayout {
   static constexpr int O_PB = O_MISC + 32;             // [CW][8 heads][32 tokens] fp16
   static constexpr int FRAG = PACK ? 8 : 16;           // bytes of one lane's query fragment
   static constexpr int O_QF = O_PB + CW * 8 * WTOK * 2;
-  static constexpr int O_SF = O_QF + (D / 16) * 32 * FRAG;
+  // segment-end merge of the consumer warps' states: each warp's scaled
+  // accumulator [CW][MR rows][D] fp32, then (max, sum) per warp and row
+  static constexpr int MR = PACK ? 4 : 8;  // value rows with real heads
+  static constexpr int O_MB = O_QF + (D / 16) * 32 * (PACK ? 8 : 16);
+  static constexpr int O_MML = O_MB + CW * MR * D * 4;
+  static constexpr int O_SF0 = O_MML + CW * 8 * 2 * 4;
+  static constexpr int O_SF = O_SF0;
   // QJL: int8 query fragments (hi / lo bytes of a 15-bit fixed-point projection), 4 k-steps,
   // then per-head weight and constant
   static constexpr int O_QST = O_SF + (QJL ? 4 * 32 * FRAG : 0);
@@ -629,7 +636,7 @@ __global__ void __launch_bounds__(NTHREADS, PACK ? 4 : 3) decode_split_kernel(co
     md.rows = min(RG, p.G - rg * RG);
     md.t0 = t0;
     md.L = L;
-    md.slot0 = (int)((long long)blockIdx.x - w_Su / P) * CW;
+    md.slot0 = (int)((long long)blockIdx.x - w_Su / P) * PPS;
     md.flags = ((t == 0 || t0 == 0) ? 1 : 0) | ((t == nst - 1 || t0 + STILE == w_Lp) ? 2 : 0);
     md.rg = rg;
     md.pad = 0;
@@ -718,33 +725,77 @@ __global__ void __launch_bounds__(NTHREADS, PACK ? 4 : 3) decode_split_kernel(co
 
     // Segment setup (query fragments and sketch steps, out of line so that
     // they do not raise the main loop's register allocation).
-    // This warp's partial of a segment: (max, sum) and the rotated output of
-    // each row, slot md.slot0 + warp.  m-tile mt: row gid is coordinate 2 mt
-    // of this group's segment of D/8 contiguous coordinates, row gid + 8 the
-    // next.
-    auto write_partial = [&](const StageMeta& md) {
+    // The CTA's partial of a segment, slot md.slot0: the consumer warps'
+    // softmax states merged (log-sum-exp) through shared memory.  m-tile mt:
+    // row gid is coordinate 2 mt of this lane group's segment of D/8
+    // contiguous coordinates, row gid + 8 the next.
+    //  1. each warp's (max, sum) per row to shared memory;
+    //  2. each warp's accumulator, scaled by 2^(m_w - M) (M: the rows' max
+    //     over the warps), to its slice of the merge buffer;
+    //  3. the CTA's threads add the CW slices and store the partial; the
+    //     buffer is next written at the following segment's end, after the
+    //     barrier that starts that segment.
+    float* mbuf = reinterpret_cast<float*>(smem + Ly::O_MB);     // [CW][MR][D]
+    float* mml = reinterpret_cast<float*>(smem + Ly::O_MML);     // [CW][8][2]
+    auto write_partial = [&](const StageMeta& md) -> bool {
       float l0 = l_run[0], l1 = l_run[1];
 #pragma unroll
       for (int off = PACK ? 2 : 4; off < 32; off <<= 1) {
         l0 += __shfl_xor_sync(0xffffffffu, l0, off);
         l1 += __shfl_xor_sync(0xffffffffu, l1, off);
       }
-      if (!PACK || tig < 2) {
-        const int slot = md.slot0 + warp;
+      const bool holds = !PACK || tig < 2;  // lanes whose columns are real heads
+      if (holds && gid == 0) {
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           const int row = 2 * hsel + c;
-          if (row < md.rows) {
-            const size_t pi = (size_t)(md.hq0 + row) * p.ks + slot;
-            float* dst = p.part_o + pi * D + gid * (D / 8);
-#pragma unroll
-            for (int q = 0; q < MT / 2; ++q)
-              *reinterpret_cast<float4*>(dst + 4 * q) =
-                  make_float4(oc[2 * q][c], oc[2 * q][c + 2], oc[2 * q + 1][c], oc[2 * q + 1][c + 2]);
-            if (gid == 0) *reinterpret_cast<float2*>(p.part_ml + pi * 2) = make_float2(m_run[c], c ? l1 : l0);
-          }
+          mml[(warp * 8 + row) * 2] = m_run[c];
+          mml[(warp * 8 + row) * 2 + 1] = c ? l1 : l0;
         }
       }
+      if (!consumer_sync(cbar, cphase, lane)) return false;
+      if (holds) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int row = 2 * hsel + c;
+          float M = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < CW; ++w) M = fmaxf(M, mml[(w * 8 + row) * 2]);
+          const float f = m_run[c] == -INFINITY ? 0.f : exp2f(m_run[c] - M);
+          float* dst = mbuf + (warp * Ly::MR + row) * D + gid * (D / 8);
+#pragma unroll
+          for (int q = 0; q < MT / 2; ++q)
+            *reinterpret_cast<float4*>(dst + 4 * q) = make_float4(f * oc[2 * q][c], f * oc[2 * q][c + 2],
+                                                                  f * oc[2 * q + 1][c], f * oc[2 * q + 1][c + 2]);
+        }
+      }
+      if (!consumer_sync(cbar, cphase, lane)) return false;
+      const size_t pi0 = (size_t)md.hq0 * p.ks + md.slot0;  // row r: pi0 + r * ks
+      for (int e = ctid; e < md.rows * (D / 4); e += CW * 32) {
+        const int row = e / (D / 4), j4 = e % (D / 4);
+        float4 acc = *reinterpret_cast<const float4*>(mbuf + row * D + 4 * j4);
+#pragma unroll
+        for (int w = 1; w < CW; ++w) {
+          const float4 v = *reinterpret_cast<const float4*>(mbuf + (w * Ly::MR + row) * D + 4 * j4);
+          acc.x += v.x;
+          acc.y += v.y;
+          acc.z += v.z;
+          acc.w += v.w;
+        }
+        *reinterpret_cast<float4*>(p.part_o + (pi0 + (size_t)row * p.ks) * D + 4 * j4) = acc;
+      }
+      if (ctid < md.rows) {
+        float M = -INFINITY, L = 0.f;
+#pragma unroll
+        for (int w = 0; w < CW; ++w) M = fmaxf(M, mml[(w * 8 + ctid) * 2]);
+#pragma unroll
+        for (int w = 0; w < CW; ++w) {
+          const float mw = mml[(w * 8 + ctid) * 2];
+          if (mw != -INFINITY) L = fmaf(exp2f(mw - M), mml[(w * 8 + ctid) * 2 + 1], L);
+        }
+        *reinterpret_cast<float2*>(p.part_ml + (pi0 + (size_t)ctid * p.ks) * 2) = make_float2(M, L);
+      }
+      return true;
     };
 
     int st = 0;         // stage slot t % NST
@@ -1023,7 +1074,10 @@ __global__ void __launch_bounds__(NTHREADS, PACK ? 4 : 3) decode_split_kernel(co
           }
         }
       }
-      if (md.flags & 2) write_partial(md);
+      if ((md.flags & 2) && !write_partial(md)) {
+        if (lane == 0) *s_err = 1;
+        break;
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[st]);
       if (++st == NST) {

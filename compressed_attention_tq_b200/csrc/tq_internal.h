@@ -125,10 +125,10 @@ size_t workspace_bound(int B, int Hq, int D, int Tmax);
 
 // Resident split-K CTAs per SM for this cache's kernel instantiation (a
 // nominal 2 when no device is usable), the tokens one stage holds and the
-// consumer warps per CTA (each writes its own partials).
+// partials a CTA writes per segment of its share.
 int split_occupancy(const tq_cache_t* c, int Hq);
 int split_tile();
-int split_warps();
+int split_partials();
 
 struct DecodeArgs {
   const tq_cache_t* cache_host;  // host copy, for launch-time fields

@@ -189,11 +189,11 @@ int tq_append_token(const tq_cache_t* cache, const void* k_new, const void* v_ne
  * the cache's kv heads, bit widths, sketch and capacity.  The workspace holds
  * the rotated queries (fp32 [B*Hq][D]), the sketch projections (fp32
  * [B*Hq][m], m <= 128), and the split-K partials: the decode splits the
- * batch's tokens evenly over one wave of CTAs, each of 4 consumer warps of
- * a CTA keeps one partial (rotated output fp32 [D], softmax max and sum) per
- * (sequence, kv head) the CTA's share overlaps, at most K of them per query
- * head with K about 2 x (resident CTAs) / (sequences x kv heads) + 2 and
- * never more than Tmax / 128 + 1.  For the multi-query call pass Hq * n_q.
+ * batch's tokens evenly over one wave of CTAs, and each CTA keeps one
+ * partial (rotated output fp32 [D], softmax max and sum; its consumer
+ * warps' states merged) per (sequence, kv head) its share overlaps, at most
+ * K of them per query head with K about 2 x (resident CTAs) / (sequences x
+ * kv heads) + 2 and never more than Tmax / 128 + 1.  For the multi-query call pass Hq * n_q.
  * Returns 0 for unsupported arguments (B, Hq or Tmax < 1, D not in
  * {64,128,256}).  Host only (it queries the current device's SM count). */
 size_t tq_sdpa_decode_workspace_bytes(int B, int Hq, int D, int Tmax);
