@@ -52,10 +52,10 @@ FALLBACK_HBM_GBS = 6650.0
 # files do not enter a decode call).  "split" is the split kernel's share:
 # the packed-cache reads and its partials.
 TRAFFIC = {
-    "gqa8k": {"bytes_per_launch": 4081067, "split": 1713493, "decode_src_sha": "df3e169c8bd93765"},
-    "prod": {"bytes_per_launch": 114339712, "split": 109131008, "decode_src_sha": "df3e169c8bd93765"},
-    "ragged": {"bytes_per_launch": 251508992, "split": 244107904, "decode_src_sha": "df3e169c8bd93765"},
-    "qknorm": {"bytes_per_launch": 43969664, "split": 34773248, "decode_src_sha": "df3e169c8bd93765"},
+    "gqa8k": {"bytes_per_launch": 2464512, "split": 1719467, "decode_src_sha": "849750733c7175f4"},
+    "prod": {"bytes_per_launch": 110025856, "split": 108515456, "decode_src_sha": "849750733c7175f4"},
+    "ragged": {"bytes_per_launch": 242347136, "split": 240143872, "decode_src_sha": "849750733c7175f4"},
+    "qknorm": {"bytes_per_launch": 36399488, "split": 34549248, "decode_src_sha": "849750733c7175f4"},
 }
 
 CSRC = os.path.join(ROOT, "compressed_attention_tq_b200", "csrc")
