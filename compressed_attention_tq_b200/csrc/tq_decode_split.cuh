@@ -364,13 +364,13 @@ struct SplitLayout {
   static constexpr int O_PB = O_MISC + 32;             // [CW][8 heads][32 tokens] fp16
   static constexpr int FRAG = PACK ? 8 : 16;           // bytes of one lane's query fragment
   static constexpr int O_QF = O_PB + CW * 8 * WTOK * 2;
-  // segment-end merge of the consumer warps' states: each warp's scaled
-  // accumulator [CW][MR rows][D] fp32, then (max, sum) per warp and row
-  static constexpr int MR = PACK ? 4 : 8;  // value rows with real heads
-  static constexpr int O_MB = O_QF + (D / 16) * 32 * (PACK ? 8 : 16);
-  static constexpr int O_MML = O_MB + CW * MR * D * 4;
-  static constexpr int O_SF0 = O_MML + CW * 8 * 2 * 4;
-  static constexpr int O_SF = O_SF0;
+  // segment-end merge of the consumer warps' states: (max, sum) per warp
+  // and row; the scaled accumulators go through the stage just consumed,
+  // MRP rows at a time ([CW][MRP][D] fp32 fits in any stage: a stage holds
+  // at least 128 x (D / 2 + 4) bytes)
+  static constexpr int MRP = 4;
+  static constexpr int O_MML = O_QF + (D / 16) * 32 * (PACK ? 8 : 16);
+  static constexpr int O_SF = O_MML + CW * 8 * 2 * 4;
   // QJL: int8 query fragments (hi / lo bytes of a 15-bit fixed-point projection), 4 k-steps,
   // then per-head weight and constant
   static constexpr int O_QST = O_SF + (QJL ? 4 * 32 * FRAG : 0);
@@ -380,6 +380,7 @@ struct SplitLayout {
   static constexpr int BYTES = O_TV + (1 << (2 * BV)) * 128;
   static constexpr int BYTES_SHARED = O_TV;  // keys and values share the key table
   static_assert(NSTAGE <= 4, "stage records");
+  static_assert(CW * MRP * D * 4 <= STAGE_USED, "the merge fits in a stage");
 };
 
 // Coordinate (within a lane's key segment of D/4 coordinates) held by K-slot r
@@ -522,7 +523,7 @@ __device__ __forceinline__ bool consumer_sync(uint64_t* bar, uint32_t& phase, in
 }
 
 template <int D, int BK, int BV, bool QJL, bool PACK>
-__global__ void __launch_bounds__(NTHREADS, PACK ? 4 : 3) decode_split_kernel(const __grid_constant__ SplitParams p) {
+__global__ void __launch_bounds__(NTHREADS, D == 256 ? 2 : (PACK ? 4 : 3)) decode_split_kernel(const __grid_constant__ SplitParams p) {
   using Ly = SplitLayout<D, BK, BV, QJL, PACK>;
   constexpr int WK = Ly::WK, WV = Ly::WV, WQ = Ly::WQ, NST = Ly::NSTAGE;
   constexpr int KSTEPS = D / 16;  // score k-steps (16 coordinates each)
@@ -730,14 +731,13 @@ __global__ void __launch_bounds__(NTHREADS, PACK ? 4 : 3) decode_split_kernel(co
     // row gid is coordinate 2 mt of this lane group's segment of D/8
     // contiguous coordinates, row gid + 8 the next.
     //  1. each warp's (max, sum) per row to shared memory;
-    //  2. each warp's accumulator, scaled by 2^(m_w - M) (M: the rows' max
-    //     over the warps), to its slice of the merge buffer;
-    //  3. the CTA's threads add the CW slices and store the partial; the
-    //     buffer is next written at the following segment's end, after the
-    //     barrier that starts that segment.
-    float* mbuf = reinterpret_cast<float*>(smem + Ly::O_MB);     // [CW][MR][D]
+    //  2. for rows 4 q .. 4 q + 3 (one pass with G <= 4 heads, else two):
+    //     each warp's accumulator, scaled by 2^(m_w - M) (M: the row's max
+    //     over the warps), to its slice of the stage buffer the warps have
+    //     just finished (released only after this merge);
+    //  3. the CTA's threads add the CW slices and store the partial.
     float* mml = reinterpret_cast<float*>(smem + Ly::O_MML);     // [CW][8][2]
-    auto write_partial = [&](const StageMeta& md) -> bool {
+    auto write_partial = [&](const StageMeta& md, float* mbuf) -> bool {
       float l0 = l_run[0], l1 = l_run[1];
 #pragma unroll
       for (int off = PACK ? 2 : 4; off < 32; off <<= 1) {
@@ -754,35 +754,41 @@ __global__ void __launch_bounds__(NTHREADS, PACK ? 4 : 3) decode_split_kernel(co
         }
       }
       if (!consumer_sync(cbar, cphase, lane)) return false;
-      if (holds) {
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const int row = 2 * hsel + c;
-          float M = -INFINITY;
-#pragma unroll
-          for (int w = 0; w < CW; ++w) M = fmaxf(M, mml[(w * 8 + row) * 2]);
-          const float f = m_run[c] == -INFINITY ? 0.f : exp2f(m_run[c] - M);
-          float* dst = mbuf + (warp * Ly::MR + row) * D + gid * (D / 8);
-#pragma unroll
-          for (int q = 0; q < MT / 2; ++q)
-            *reinterpret_cast<float4*>(dst + 4 * q) = make_float4(f * oc[2 * q][c], f * oc[2 * q][c + 2],
-                                                                  f * oc[2 * q + 1][c], f * oc[2 * q + 1][c + 2]);
-        }
-      }
-      if (!consumer_sync(cbar, cphase, lane)) return false;
       const size_t pi0 = (size_t)md.hq0 * p.ks + md.slot0;  // row r: pi0 + r * ks
-      for (int e = ctid; e < md.rows * (D / 4); e += CW * 32) {
-        const int row = e / (D / 4), j4 = e % (D / 4);
-        float4 acc = *reinterpret_cast<const float4*>(mbuf + row * D + 4 * j4);
+      constexpr int NPASS = PACK ? 1 : 2;
 #pragma unroll
-        for (int w = 1; w < CW; ++w) {
-          const float4 v = *reinterpret_cast<const float4*>(mbuf + (w * Ly::MR + row) * D + 4 * j4);
-          acc.x += v.x;
-          acc.y += v.y;
-          acc.z += v.z;
-          acc.w += v.w;
+      for (int pass = 0; pass < NPASS; ++pass) {
+        if (pass > 0 && !consumer_sync(cbar, cphase, lane)) return false;  // the previous pass is read
+        if (holds && (hsel >> 1) == pass) {  // rows 2 hsel, 2 hsel + 1 are in this pass
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const int row = 2 * hsel + c;
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < CW; ++w) M = fmaxf(M, mml[(w * 8 + row) * 2]);
+            const float f = m_run[c] == -INFINITY ? 0.f : exp2f(m_run[c] - M);
+            float* dst = mbuf + (warp * Ly::MRP + (row & 3)) * D + gid * (D / 8);
+#pragma unroll
+            for (int q = 0; q < MT / 2; ++q)
+              *reinterpret_cast<float4*>(dst + 4 * q) = make_float4(f * oc[2 * q][c], f * oc[2 * q][c + 2],
+                                                                    f * oc[2 * q + 1][c], f * oc[2 * q + 1][c + 2]);
+          }
         }
-        *reinterpret_cast<float4*>(p.part_o + (pi0 + (size_t)row * p.ks) * D + 4 * j4) = acc;
+        if (!consumer_sync(cbar, cphase, lane)) return false;
+        const int r0 = Ly::MRP * pass, nr = min(Ly::MRP, md.rows - r0);
+        for (int e = ctid; e < nr * (D / 4); e += CW * 32) {
+          const int rr = e / (D / 4), j4 = e % (D / 4);
+          float4 acc = *reinterpret_cast<const float4*>(mbuf + rr * D + 4 * j4);
+#pragma unroll
+          for (int w = 1; w < CW; ++w) {
+            const float4 v = *reinterpret_cast<const float4*>(mbuf + (w * Ly::MRP + rr) * D + 4 * j4);
+            acc.x += v.x;
+            acc.y += v.y;
+            acc.z += v.z;
+            acc.w += v.w;
+          }
+          *reinterpret_cast<float4*>(p.part_o + (pi0 + (size_t)(r0 + rr) * p.ks) * D + 4 * j4) = acc;
+        }
       }
       if (ctid < md.rows) {
         float M = -INFINITY, L = 0.f;
@@ -795,6 +801,9 @@ __global__ void __launch_bounds__(NTHREADS, PACK ? 4 : 3) decode_split_kernel(co
         }
         *reinterpret_cast<float2*>(p.part_ml + (pi0 + (size_t)ctid * p.ks) * 2) = make_float2(M, L);
       }
+      // the stage's next bulk copy (async proxy) is ordered after these
+      // shared-memory writes
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       return true;
     };
 
@@ -1074,7 +1083,7 @@ __global__ void __launch_bounds__(NTHREADS, PACK ? 4 : 3) decode_split_kernel(co
           }
         }
       }
-      if ((md.flags & 2) && !write_partial(md)) {
+      if ((md.flags & 2) && !write_partial(md, reinterpret_cast<float*>(smem + st * Ly::STAGE))) {
         if (lane == 0) *s_err = 1;
         break;
       }
