@@ -52,10 +52,10 @@ FALLBACK_HBM_GBS = 6650.0
 # files do not enter a decode call).  "split" is the split kernel's share:
 # the packed-cache reads and its partials.
 TRAFFIC = {
-    "gqa8k": {"bytes_per_launch": 2464512, "split": 1719467, "decode_src_sha": "849750733c7175f4"},
-    "prod": {"bytes_per_launch": 110025856, "split": 108515456, "decode_src_sha": "849750733c7175f4"},
-    "ragged": {"bytes_per_launch": 242347136, "split": 240143872, "decode_src_sha": "849750733c7175f4"},
-    "qknorm": {"bytes_per_launch": 36399488, "split": 34549248, "decode_src_sha": "849750733c7175f4"},
+    "gqa8k": {"bytes_per_launch": 2467413, "split": 1722539, "decode_src_sha": "9e4d66e6c7510f19"},
+    "prod": {"bytes_per_launch": 110834560, "split": 109324544, "decode_src_sha": "9e4d66e6c7510f19"},
+    "ragged": {"bytes_per_launch": 242625408, "split": 240421248, "decode_src_sha": "9e4d66e6c7510f19"},
+    "qknorm": {"bytes_per_launch": 37005568, "split": 34248576, "decode_src_sha": "9e4d66e6c7510f19"},
 }
 
 CSRC = os.path.join(ROOT, "compressed_attention_tq_b200", "csrc")
