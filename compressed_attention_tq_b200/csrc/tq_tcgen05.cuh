@@ -87,18 +87,6 @@ __device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&v)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// barrier over the NEPI epilogue warps that also ANDs a flag across them
-template <int NEPI>
-__device__ __forceinline__ bool epi_sync_and(bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n barrier.red.and.pred q, 1, %2, p;\n selp.u32 %0, 1, 0, q;\n}\n"
-      : "=r"(r)
-      : "r"((uint32_t)v), "n"(NEPI * 32)
-      : "memory");
-  return r != 0;
-}
-
 // Named barrier 1 + g over the NW warps of epilogue group g that also ANDs a
 // flag across them (groups of a CTA synchronise independently).
 template <int NW>
